@@ -1,0 +1,187 @@
+"""fp64 CPU oracle of the dynamic short convolution (test infrastructure).
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  It shares no code with the CUDA library; the
+arithmetic lives in ``dsc_oracle.c`` (plain loops over the definitions, see
+that file's header for the formulas and their sources), and this module only
+compiles it, marshals numpy arrays and returns fp64 results.
+
+Inputs are numpy arrays in storage form: ``float32`` (fp32), ``uint16``
+(bf16 bit patterns) or ``float64``.  Every output is fp64.
+"""
+
+from __future__ import annotations
+
+import ctypes as C
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dsc_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+F32, BF16, F64 = 0, 1, 2
+HEADWISE, LOWRANK, STATIC = 0, 1, 2
+Y, DX, DW, DZ, DU, DWS, W_TAP = 0, 1, 2, 3, 4, 5, 6
+
+_lock = threading.Lock()
+_lib = None
+
+
+class Problem(C.Structure):
+    _fields_ = [("B", C.c_int64), ("T", C.c_int64), ("D", C.c_int64), ("W", C.c_int64),
+                ("H", C.c_int64), ("R", C.c_int64), ("residual", C.c_int64)]
+
+    @property
+    def G(self):
+        return self.D // self.H
+
+
+class _In(C.Structure):
+    _fields_ = [("p", C.c_void_p), ("dt", C.c_int64)]
+
+
+class _Filter(C.Structure):
+    _fields_ = [("kind", C.c_int64), ("w", _In), ("z", _In), ("U", _In)]
+
+
+def problem(B, T, D, W, H=1, R=0, residual=1) -> Problem:
+    if D % H:
+        raise ValueError("D must be a multiple of H")
+    return Problem(B, T, D, W, H, R, residual)
+
+
+def problem_of(wl) -> Problem:
+    """Problem of a ``synth.workloads.Workload``."""
+    return problem(wl.B, wl.T, wl.D, wl.W, wl.H, wl.R, wl.residual)
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile the oracle with gcc (plain IEEE fp64: no fast-math, no contraction)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        tmp = out + f".tmp{os.getpid()}"
+        subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-ffp-contract=off", "-fno-fast-math",
+                        "-shared", "-fPIC", src, "-o", tmp, "-lm"], check=True)
+        os.replace(tmp, out)
+    return out
+
+
+def load(path: str | None = None):
+    """Load (building if needed) the oracle library; ``path`` selects another build."""
+    global _lib
+    if path is not None:
+        return _bind(C.CDLL(path))
+    with _lock:
+        if _lib is None:
+            _lib = _bind(C.CDLL(build()))
+    return _lib
+
+
+def _bind(lib):
+    P = C.POINTER(Problem)
+    d = C.POINTER(C.c_double)
+    lib.orc_max_threads.restype = C.c_int
+    lib.orc_lowrank_filters.argtypes = [P, _In, _In, d]
+    lib.orc_forward.argtypes = [P, C.c_int64, _In, _In, d]
+    lib.orc_backward.argtypes = [P, C.c_int64, _In, _In, _In, d, d]
+    lib.orc_lowrank_grads.argtypes = [P, _In, _In, d, d, d]
+    lib.orc_sample.argtypes = [P, C.POINTER(_Filter), _In, _In, C.c_int64, C.c_int64,
+                               C.POINTER(C.c_int64), d]
+    for f in ("orc_lowrank_filters", "orc_forward", "orc_backward", "orc_lowrank_grads", "orc_sample"):
+        getattr(lib, f).restype = None
+    return lib
+
+
+def max_threads() -> int:
+    return load().orc_max_threads()
+
+
+def _in(a: np.ndarray | None) -> _In:
+    if a is None:
+        return _In(None, F64)
+    if not a.flags.c_contiguous:
+        raise ValueError("oracle inputs must be C-contiguous")
+    dt = {np.dtype(np.float32): F32, np.dtype(np.uint16): BF16, np.dtype(np.float64): F64}[a.dtype]
+    return _In(a.ctypes.data, dt)
+
+
+def _out(shape) -> np.ndarray:
+    return np.empty(shape, dtype=np.float64)
+
+
+def _dp(a: np.ndarray):
+    return a.ctypes.data_as(C.POINTER(C.c_double))
+
+
+def forward_headwise(P: Problem, x, w, lib=None) -> np.ndarray:
+    lib = lib or load()
+    y = _out((P.B, P.T, P.D))
+    lib.orc_forward(C.byref(P), HEADWISE, _in(w), _in(x), _dp(y))
+    return y
+
+
+def backward_headwise(P: Problem, x, w, dy, lib=None):
+    """Returns (dx [B,T,D], dw [B,T,G,W])."""
+    lib = lib or load()
+    dx = _out((P.B, P.T, P.D))
+    dw = _out((P.B, P.T, P.G, P.W))
+    lib.orc_backward(C.byref(P), HEADWISE, _in(w), _in(x), _in(dy), _dp(dx), _dp(dw))
+    return dx, dw
+
+
+def forward_static(P: Problem, x, ws, lib=None) -> np.ndarray:
+    lib = lib or load()
+    y = _out((P.B, P.T, P.D))
+    lib.orc_forward(C.byref(P), STATIC, _in(ws), _in(x), _dp(y))
+    return y
+
+
+def backward_static(P: Problem, x, ws, dy, lib=None):
+    """Returns (dx [B,T,D], dws [D,W])."""
+    lib = lib or load()
+    dx = _out((P.B, P.T, P.D))
+    dws = _out((P.D, P.W))
+    lib.orc_backward(C.byref(P), STATIC, _in(ws), _in(x), _in(dy), _dp(dx), _dp(dws))
+    return dx, dws
+
+
+def lowrank_filters(P: Problem, z, U, lib=None) -> np.ndarray:
+    """w [B,T,G,W] = z . U, materialised in fp64."""
+    lib = lib or load()
+    w = _out((P.B, P.T, P.G, P.W))
+    lib.orc_lowrank_filters(C.byref(P), _in(z), _in(U), _dp(w))
+    return w
+
+
+def forward_lowrank(P: Problem, x, z, U, lib=None) -> np.ndarray:
+    """Filters w = zU, then the head-wise forward with them."""
+    lib = lib or load()
+    w = lowrank_filters(P, z, U, lib)
+    return forward_headwise(P, x, w, lib)
+
+
+def backward_lowrank(P: Problem, x, z, U, dy, lib=None):
+    """Returns (dx [B,T,D], dz [B,T,R], dU [R,G*W], dw [B,T,G,W])."""
+    lib = lib or load()
+    w = lowrank_filters(P, z, U, lib)
+    dx, dw = backward_headwise(P, x, w, dy, lib)
+    dz = _out((P.B, P.T, P.R))
+    dU = _out((P.R, P.G * P.W))
+    lib.orc_lowrank_grads(C.byref(P), _in(z), _in(U), _dp(dw), _dp(dz), _dp(dU))
+    return dx, dz, dU, dw
+
+
+def sample(P: Problem, kind: int, what: int, idx, *, x=None, dy=None, w=None, z=None, U=None, lib=None):
+    """Evaluate single output elements; ``idx`` is an int64 array [n, <=4]."""
+    lib = lib or load()
+    idx = np.asarray(idx, dtype=np.int64)
+    q = np.zeros((idx.shape[0], 4), dtype=np.int64)
+    q[:, :idx.shape[1]] = idx
+    F = _Filter(kind, _in(w), _in(z), _in(U))
+    out = _out((idx.shape[0],))
+    lib.orc_sample(C.byref(P), C.byref(F), _in(x), _in(dy), what, idx.shape[0],
+                   q.ctypes.data_as(C.POINTER(C.c_int64)), _dp(out))
+    return out

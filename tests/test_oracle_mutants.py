@@ -1,0 +1,135 @@
+"""Plant plausible mistakes in a copy of the oracle and check that the pins
+catch every one of them.  Mutations are text edits of a temporary copy of
+``oracle/dsc_oracle.c``; the committed oracle is never touched.  Every
+mutant stays in bounds (it only changes which in-range element is read or
+how terms combine), so a failing pin shows up as a wrong value.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SRC = os.path.join(os.path.dirname(HERE), "oracle", "dsc_oracle.c")
+
+MUTANTS = {
+    "strided groups instead of consecutive": ("int64_t g = c / P->H;", "int64_t g = c % G;"),
+    "residual dropped in dx": ("double acc = P->residual ? xval(P, dy, b, s, c) : 0.0;", "double acc = 0.0;"),
+    "dx uses w(s) instead of w(s+k)": ("acc += tap(P, F, b, s + k, c, k)", "acc += tap(P, F, b, s, c, k)"),
+    "dw ignores the lag": ("++c)\n        s += xval(P, dy, b, t, c) * xval(P, x, b, t - k, c);",
+                           "++c)\n        s += xval(P, dy, b, t, c) * xval(P, x, b, t, c);"),
+    "U read transposed in zU": ("* P->R + r) * val(F->U, r * GW + g * P->W + k);",
+                                "* P->R + r) * val(F->U, (g * P->W + k) * P->R + r);"),
+    "causal boundary off by one": ("if (t - k >= 0) s += tap", "if (t - k > 0) s += tap"),
+    "conv term sign flipped": ("s += tap(P, F, b, t, c, k) * xval(P, x, b, t - k, c);",
+                               "s -= tap(P, F, b, t, c, k) * xval(P, x, b, t - k, c);"),
+    "dz drops the rank index of U": ("s += dw[n * GW + j] * val(U, r * GW + j);", "s += dw[n * GW + j] * val(U, j);"),
+    "dU skips the first token": ("for (int64_t n = 0; n < NT; ++n) s += val(z,", "for (int64_t n = 1; n < NT; ++n) s += val(z,"),
+    "static dw reads the wrong lag": ("for (int64_t t = k; t < P->T; ++t)\n            s += xval(P, dy, b, t, c) * xval(P, x, b, t - k, c);",
+                                      "for (int64_t t = k; t < P->T; ++t)\n            s += xval(P, dy, b, t, c) * xval(P, x, b, t - (k > 0), c);"),
+    "static taps in reverse order": ("if (F->kind == ORC_STATIC) return val(F->w, c * P->W + k);",
+                                     "if (F->kind == ORC_STATIC) return val(F->w, c * P->W + (P->W - 1 - k));"),
+}
+
+
+def _pins(lib):
+    """A compact run of the pins; returns the names of those that fail."""
+    rng = np.random.default_rng(5)
+    fails = []
+
+    def check(name, ok):
+        if not ok:
+            fails.append(name)
+
+    with open(os.path.join(HERE, "golden", "handworked.json")) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        p = oracle.problem(c["B"], c["T"], c["D"], c["W"], c["H"], c["R"], c["residual"])
+        x, dy = np.array(c["x"], float), np.array(c["dy"], float)
+        if c["variant"] == "headwise":
+            w = np.array(c["w"], float)
+            dx, dw = oracle.backward_headwise(p, x, w, dy, lib=lib)
+            check("golden", np.array_equal(oracle.forward_headwise(p, x, w, lib=lib), c["y"])
+                  and np.array_equal(dx, c["dx"]) and np.array_equal(dw, c["dw"]))
+        elif c["variant"] == "lowrank":
+            z, U = np.array(c["z"], float), np.array(c["U"], float)
+            dx, dz, dU, _ = oracle.backward_lowrank(p, x, z, U, dy, lib=lib)
+            check("golden", np.array_equal(oracle.forward_lowrank(p, x, z, U, lib=lib), c["y"])
+                  and np.array_equal(dx, c["dx"]) and np.array_equal(dz, c["dz"]) and np.array_equal(dU, c["dU"]))
+        else:
+            ws = np.array(c["ws"], float)
+            dx, dws = oracle.backward_static(p, x, ws, dy, lib=lib)
+            check("golden", np.array_equal(oracle.forward_static(p, x, ws, lib=lib), c["y"])
+                  and np.array_equal(dx, c["dx"]) and np.array_equal(dws, c["dws"]))
+
+    # static vs torch conv1d and its autograd
+    B, T, D, W = 2, 9, 4, 3
+    p = oracle.problem(B, T, D, W, 1, 0, 1)
+    x, ws, dy = rng.standard_normal((B, T, D)), rng.standard_normal((D, W)), rng.standard_normal((B, T, D))
+    xt, wt = torch.tensor(x, requires_grad=True), torch.tensor(ws, requires_grad=True)
+    ref = torch.nn.functional.conv1d(xt.transpose(1, 2), wt.flip(-1)[:, None, :], groups=D, padding=W - 1)
+    ref = ref[..., :T].transpose(1, 2) + xt
+    ref.backward(torch.tensor(dy))
+    dx, dws = oracle.backward_static(p, x, ws, dy, lib=lib)
+    check("static-conv1d", np.allclose(oracle.forward_static(p, x, ws, lib=lib), ref.detach().numpy(), atol=1e-12)
+          and np.allclose(dx, xt.grad.numpy(), atol=1e-12) and np.allclose(dws, wt.grad.numpy(), atol=1e-11))
+
+    # matrix form and exact differences, head-wise and low-rank
+    B, T, D, W, H, R = 2, 7, 6, 3, 2, 4
+    G = D // H
+    p = oracle.problem(B, T, D, W, H, R, 1)
+    x, dy = rng.standard_normal((B, T, D)), rng.standard_normal((B, T, D))
+    w, z, U = rng.standard_normal((B, T, G, W)), rng.standard_normal((B, T, R)), rng.standard_normal((R, G * W))
+    y = oracle.forward_headwise(p, x, w, lib=lib)
+    dx, dw = oracle.backward_headwise(p, x, w, dy, lib=lib)
+    ok = True
+    for b in range(B):
+        for c in range(D):
+            A = np.eye(T)
+            for t in range(T):
+                for k in range(W):
+                    if t - k >= 0:
+                        A[t, t - k] += w[b, t, c // H, k]
+            ok &= np.allclose(y[b, :, c], A @ x[b, :, c], atol=1e-12)
+            ok &= np.allclose(dx[b, :, c], A.T @ dy[b, :, c], atol=1e-12)
+    check("matrix-form", ok)
+
+    def fd(f, arg, grad):
+        a, g = arg.reshape(-1), grad.reshape(-1)
+        for i in range(a.size):
+            o = a[i]
+            a[i] = o + 0.5
+            lp = f()
+            a[i] = o - 0.5
+            lm = f()
+            a[i] = o
+            if abs(lp - lm - g[i]) > 1e-9 * (1 + abs(g[i])):
+                return False
+        return True
+
+    check("fd-headwise", fd(lambda: np.sum(dy * oracle.forward_headwise(p, x, w, lib=lib)), w, dw))
+    dxl, dz, dU, _ = oracle.backward_lowrank(p, x, z, U, dy, lib=lib)
+    fl = lambda: np.sum(dy * oracle.forward_lowrank(p, x, z, U, lib=lib))
+    check("fd-lowrank", fd(fl, z, dz) and fd(fl, U, dU) and fd(fl, x, dxl))
+    return fails
+
+
+def test_unmutated_copy_passes(tmp_path):
+    lib = oracle.load(oracle.build(force=True, out=str(tmp_path / "ok.so")))
+    assert _pins(lib) == []
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_pins_catch_mutant(name, tmp_path):
+    old, new = MUTANTS[name]
+    src = open(SRC).read()
+    assert src.count(old) == 1, f"mutation site not unique/present: {old!r}"
+    path = tmp_path / "mutant.c"
+    path.write_text(src.replace(old, new))
+    lib = oracle.load(oracle.build(force=True, src=str(path), out=str(tmp_path / "mutant.so")))
+    assert _pins(lib), f"no pin caught the mutant '{name}'"

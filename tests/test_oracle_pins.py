@@ -1,0 +1,330 @@
+"""Pins of the fp64 oracle to things other than itself.
+
+Each check below would catch a plausible slip in the oracle (a dropped term,
+a wrong sign, a wrong tap/lag index, a transposed operand, a wrong channel to
+group mapping):
+
+* hand-worked values (tests/golden/handworked.json);
+* the convolution written as a banded T x T matrix per (batch, channel):
+  y = (rI + A) x, hence dx = (rI + A)^T dy by linear algebra;
+* exact central differences of L = <dy, y>, which is linear in each of x, w,
+  z and U separately, so the difference quotient is exact up to rounding;
+* the static filter against torch.nn.functional.conv1d (a library routine)
+  and its autograd gradients in fp64;
+* the equivalences between the parameterisations (head-wise H vs per-channel,
+  constant-in-time vs static, full-rank identity U vs head-wise);
+* special cases (zero filter, delta filter, W = 1, T = 1, T < W).
+"""
+
+import itertools
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+RNG = np.random.default_rng(1234)
+
+
+def rand(*shape):
+    return RNG.standard_normal(shape)
+
+
+def P(B, T, D, W, H=1, R=0, residual=1):
+    return oracle.problem(B, T, D, W, H, R, residual)
+
+
+def banded(wch, T, W):
+    """A[t, t-k] = wch[t, k] for one (batch, channel): the causal conv as a matrix."""
+    A = np.zeros((T, T))
+    for t in range(T):
+        for k in range(W):
+            if t - k >= 0:
+                A[t, t - k] = wch[t, k]
+    return A
+
+
+# ---------------------------------------------------------------- golden ---
+
+def _golden_cases():
+    with open(os.path.join(HERE, "golden", "handworked.json")) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
+def test_handworked_golden(case):
+    c = case
+    p = P(c["B"], c["T"], c["D"], c["W"], c["H"], c["R"], c["residual"])
+    x = np.array(c["x"], dtype=np.float64)
+    dy = np.array(c["dy"], dtype=np.float64)
+    if c["variant"] == "headwise":
+        w = np.array(c["w"], dtype=np.float64)
+        np.testing.assert_array_equal(oracle.forward_headwise(p, x, w), c["y"])
+        dx, dw = oracle.backward_headwise(p, x, w, dy)
+        np.testing.assert_array_equal(dx, c["dx"])
+        np.testing.assert_array_equal(dw, c["dw"])
+    elif c["variant"] == "lowrank":
+        z = np.array(c["z"], dtype=np.float64)
+        U = np.array(c["U"], dtype=np.float64)
+        np.testing.assert_array_equal(oracle.forward_lowrank(p, x, z, U), c["y"])
+        dx, dz, dU, _ = oracle.backward_lowrank(p, x, z, U, dy)
+        np.testing.assert_array_equal(dx, c["dx"])
+        np.testing.assert_array_equal(dz, c["dz"])
+        np.testing.assert_array_equal(dU, c["dU"])
+    else:
+        ws = np.array(c["ws"], dtype=np.float64)
+        np.testing.assert_array_equal(oracle.forward_static(p, x, ws), c["y"])
+        dx, dws = oracle.backward_static(p, x, ws, dy)
+        np.testing.assert_array_equal(dx, c["dx"])
+        np.testing.assert_array_equal(dws, c["dws"])
+
+
+# ----------------------------------------------------------- matrix form ---
+
+def _shapes():
+    out = []
+    for T, D, W in [(1, 1, 1), (1, 3, 4), (2, 4, 3), (3, 2, 5), (5, 6, 2), (9, 4, 4), (16, 8, 3), (7, 6, 5)]:
+        for H in [h for h in range(1, D + 1) if D % h == 0]:
+            out.append((T, D, W, H))
+    return out
+
+
+@pytest.mark.parametrize("T,D,W,H", _shapes())
+@pytest.mark.parametrize("residual", [0, 1])
+def test_matrix_form_headwise(T, D, W, H, residual):
+    B, G = 2, D // H
+    p = P(B, T, D, W, H, 0, residual)
+    x, w, dy = rand(B, T, D), rand(B, T, G, W), rand(B, T, D)
+    y = oracle.forward_headwise(p, x, w)
+    dx, _ = oracle.backward_headwise(p, x, w, dy)
+    for b, c in itertools.product(range(B), range(D)):
+        M = residual * np.eye(T) + banded(w[b, :, c // H, :], T, W)
+        np.testing.assert_allclose(y[b, :, c], M @ x[b, :, c], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(dx[b, :, c], M.T @ dy[b, :, c], rtol=0, atol=1e-12)
+
+
+# -------------------------------------------- exact central differences ---
+
+def _loss_grad_check(f, arg, grad, eps=0.5, n_probe=None):
+    """f is linear in `arg`: (f(a+eps e) - f(a-eps e)) / 2eps = grad . e exactly."""
+    flat = arg.reshape(-1)
+    gflat = grad.reshape(-1)
+    idx = range(flat.size) if n_probe is None else RNG.choice(flat.size, n_probe, replace=False)
+    for i in idx:
+        old = flat[i]
+        flat[i] = old + eps
+        lp = f()
+        flat[i] = old - eps
+        lm = f()
+        flat[i] = old
+        assert abs((lp - lm) / (2 * eps) - gflat[i]) <= 1e-9 * (1 + abs(gflat[i])), i
+
+
+@pytest.mark.parametrize("T,D,W,H", [(6, 4, 3, 2), (5, 6, 4, 3), (3, 2, 5, 1), (8, 8, 2, 8)])
+def test_fd_headwise(T, D, W, H):
+    B = 2
+    p = P(B, T, D, W, H)
+    x, w, dy = rand(B, T, D), rand(B, T, D // H, W), rand(B, T, D)
+    dx, dw = oracle.backward_headwise(p, x, w, dy)
+    f = lambda: float(np.sum(dy * oracle.forward_headwise(p, x, w)))
+    _loss_grad_check(f, x, dx)
+    _loss_grad_check(f, w, dw)
+
+
+@pytest.mark.parametrize("T,D,W,H,R", [(6, 4, 3, 2, 3), (5, 6, 4, 1, 2), (4, 8, 2, 4, 5), (3, 3, 4, 3, 1)])
+def test_fd_lowrank(T, D, W, H, R):
+    B = 2
+    p = P(B, T, D, W, H, R)
+    x, z, U, dy = rand(B, T, D), rand(B, T, R), rand(R, (D // H) * W), rand(B, T, D)
+    dx, dz, dU, _ = oracle.backward_lowrank(p, x, z, U, dy)
+    f = lambda: float(np.sum(dy * oracle.forward_lowrank(p, x, z, U)))
+    _loss_grad_check(f, x, dx)
+    _loss_grad_check(f, z, dz)
+    _loss_grad_check(f, U, dU)
+
+
+def test_adjoint_dw():
+    """<dy, conv(x; v)> = <dw(x, dy), v> for a random filter direction v."""
+    B, T, D, W, H = 3, 11, 12, 4, 3
+    p0 = P(B, T, D, W, H, 0, residual=0)
+    p1 = P(B, T, D, W, H, 0, residual=1)
+    x, dy, w = rand(B, T, D), rand(B, T, D), rand(B, T, D // H, W)
+    _, dw = oracle.backward_headwise(p1, x, w, dy)
+    for _ in range(5):
+        v = rand(B, T, D // H, W)
+        lhs = np.sum(dy * oracle.forward_headwise(p0, x, v))
+        assert abs(lhs - np.sum(dw * v)) < 1e-10 * (1 + abs(lhs))
+
+
+# ------------------------------------------ static filter vs torch conv1d ---
+
+@pytest.mark.parametrize("T,D,W,residual", [(1, 3, 4, 1), (3, 5, 4, 0), (17, 8, 4, 1), (9, 6, 2, 1), (12, 4, 8, 0), (6, 2, 1, 1)])
+def test_static_vs_torch_conv1d(T, D, W, residual):
+    B = 2
+    p = P(B, T, D, W, 1, 0, residual)
+    x, ws, dy = rand(B, T, D), rand(D, W), rand(B, T, D)
+    y = oracle.forward_static(p, x, ws)
+    dx, dws = oracle.backward_static(p, x, ws, dy)
+
+    xt = torch.tensor(x, requires_grad=True)
+    wt = torch.tensor(ws, requires_grad=True)
+    # conv1d is a cross-correlation: reversed taps make weight[..., W-1-k] hit x_{t-k}.
+    ref = torch.nn.functional.conv1d(xt.transpose(1, 2), wt.flip(-1)[:, None, :], groups=D, padding=W - 1)
+    ref = ref[..., :T].transpose(1, 2) + residual * xt
+    ref.backward(torch.tensor(dy))
+    np.testing.assert_allclose(y, ref.detach().numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dx, xt.grad.numpy(), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(dws, wt.grad.numpy(), rtol=0, atol=1e-11)
+
+
+# ------------------------------------------------------- equivalences ---
+
+@pytest.mark.parametrize("H", [1, 2, 3, 6])
+def test_constant_filters_equal_static(H):
+    B, T, D, W = 2, 10, 6, 4
+    G = D // H
+    p = P(B, T, D, W, H)
+    wg = rand(G, W)
+    w = np.broadcast_to(wg, (B, T, G, W)).copy()
+    ws = np.repeat(wg, H, axis=0)  # channel c uses group c // H
+    x, dy = rand(B, T, D), rand(B, T, D)
+    np.testing.assert_allclose(oracle.forward_headwise(p, x, w), oracle.forward_static(P(B, T, D, W), x, ws), atol=1e-12)
+    dx_h, dw_h = oracle.backward_headwise(p, x, w, dy)
+    dx_s, dws = oracle.backward_static(P(B, T, D, W), x, ws, dy)
+    np.testing.assert_allclose(dx_h, dx_s, atol=1e-12)
+    np.testing.assert_allclose(dw_h.sum(axis=(0, 1)), dws.reshape(G, H, W).sum(axis=1), atol=1e-10)
+
+
+@pytest.mark.parametrize("D,H", [(6, 2), (6, 3), (8, 4), (4, 4)])
+def test_headwise_equals_replicated_per_channel(D, H):
+    B, T, W = 2, 9, 3
+    G = D // H
+    x, dy, w = rand(B, T, D), rand(B, T, D), rand(B, T, G, W)
+    w1 = np.repeat(w, H, axis=2)  # per-channel filters: channel c takes group c // H
+    pH, p1 = P(B, T, D, W, H), P(B, T, D, W, 1)
+    np.testing.assert_allclose(oracle.forward_headwise(pH, x, w), oracle.forward_headwise(p1, x, w1), atol=1e-12)
+    dxH, dwH = oracle.backward_headwise(pH, x, w, dy)
+    dx1, dw1 = oracle.backward_headwise(p1, x, w1, dy)
+    np.testing.assert_allclose(dxH, dx1, atol=1e-12)
+    np.testing.assert_allclose(dwH, dw1.reshape(B, T, G, H, W).sum(axis=3), atol=1e-12)
+
+
+@pytest.mark.parametrize("D,H,W", [(4, 1, 3), (6, 2, 2), (6, 3, 4)])
+def test_lowrank_full_rank_identity_equals_headwise(D, H, W):
+    B, T = 2, 7
+    G = D // H
+    R = G * W
+    w = rand(B, T, G, W)
+    z = w.reshape(B, T, R).copy()
+    U = np.eye(R)
+    x, dy = rand(B, T, D), rand(B, T, D)
+    p = P(B, T, D, W, H, R)
+    np.testing.assert_allclose(oracle.lowrank_filters(p, z, U), w, atol=1e-14)
+    np.testing.assert_allclose(oracle.forward_lowrank(p, x, z, U), oracle.forward_headwise(p, x, w), atol=1e-12)
+    dx, dz, dU, dwl = oracle.backward_lowrank(p, x, z, U, dy)
+    dxh, dwh = oracle.backward_headwise(p, x, w, dy)
+    np.testing.assert_allclose(dx, dxh, atol=1e-12)
+    np.testing.assert_allclose(dz, dwh.reshape(B, T, R), atol=1e-12)
+    # with U = I, dU[r, j] = sum over tokens of w[., r] * dw[., j]
+    np.testing.assert_allclose(dU, np.einsum("nr,nj->rj", w.reshape(-1, R), dwh.reshape(-1, R)), atol=1e-10)
+
+
+# ---------------------------------------------------------- special cases ---
+
+def test_zero_filter_is_identity():
+    B, T, D, W, H = 2, 8, 6, 4, 2
+    p = P(B, T, D, W, H)
+    x, dy = rand(B, T, D), rand(B, T, D)
+    w = np.zeros((B, T, D // H, W))
+    np.testing.assert_array_equal(oracle.forward_headwise(p, x, w), x)
+    np.testing.assert_array_equal(oracle.backward_headwise(p, x, w, dy)[0], dy)
+
+
+@pytest.mark.parametrize("j", [0, 1, 3])
+def test_delta_filter_shifts(j):
+    B, T, D, W = 1, 9, 3, 4
+    p = P(B, T, D, W, 1)
+    x = rand(B, T, D)
+    w = np.zeros((B, T, D, W))
+    w[..., j] = 1.0
+    shifted = np.zeros_like(x)
+    shifted[:, j:] = x[:, :T - j]
+    np.testing.assert_allclose(oracle.forward_headwise(p, x, w), x + shifted, atol=1e-15)
+
+
+def test_width_one_is_scaling():
+    B, T, D = 2, 5, 4
+    p = P(B, T, D, 1, 1)
+    x, w, dy = rand(B, T, D), rand(B, T, D, 1), rand(B, T, D)
+    np.testing.assert_allclose(oracle.forward_headwise(p, x, w), (1 + w[..., 0]) * x, atol=1e-14)
+    dx, dw = oracle.backward_headwise(p, x, w, dy)
+    np.testing.assert_allclose(dx, (1 + w[..., 0]) * dy, atol=1e-14)
+    np.testing.assert_allclose(dw[..., 0], dy * x, atol=1e-14)
+
+
+@pytest.mark.parametrize("T", [1, 2])
+def test_short_sequences_only_reach_back_to_zero(T):
+    B, D, W = 2, 4, 5
+    p = P(B, T, D, W, 2)
+    x, w, dy = rand(B, T, D), rand(B, T, 2, W), rand(B, T, D)
+    y = oracle.forward_headwise(p, x, w)
+    wc = np.repeat(w, 2, axis=2)
+    np.testing.assert_allclose(y[:, 0], x[:, 0] * (1 + wc[:, 0, :, 0]), atol=1e-14)
+    _, dw = oracle.backward_headwise(p, x, w, dy)
+    for t in range(T):
+        assert np.all(dw[:, t, :, t + 1:] == 0)
+
+
+def test_batches_are_independent():
+    B, T, D, W, H = 3, 6, 4, 3, 2
+    p = P(B, T, D, W, H)
+    x, w, dy = rand(B, T, D), rand(B, T, D // H, W), rand(B, T, D)
+    y = oracle.forward_headwise(p, x, w)
+    for b in range(B):
+        yb = oracle.forward_headwise(P(1, T, D, W, H), x[b:b + 1].copy(), w[b:b + 1].copy())
+        np.testing.assert_array_equal(y[b:b + 1], yb)
+
+
+# ------------------------------------------ storage dtypes and sampling ---
+
+def test_bf16_and_f32_inputs_read_exactly():
+    import synth
+
+    B, T, D, W, H = 1, 6, 8, 4, 2
+    p = P(B, T, D, W, H)
+    x32 = rand(B, T, D).astype(np.float32)
+    w32 = rand(B, T, D // H, W).astype(np.float32)
+    xb, wb = synth.f32_to_bf16_bits(x32), synth.f32_to_bf16_bits(w32)
+    ref = oracle.forward_headwise(p, synth.to_f64(xb, "bf16"), synth.to_f64(wb, "bf16"))
+    np.testing.assert_array_equal(oracle.forward_headwise(p, xb, wb), ref)
+    np.testing.assert_array_equal(oracle.forward_headwise(p, x32, w32),
+                                  oracle.forward_headwise(p, x32.astype(np.float64), w32.astype(np.float64)))
+
+
+def test_sample_matches_full():
+    B, T, D, W, H, R = 2, 7, 6, 3, 2, 4
+    p = P(B, T, D, W, H, R)
+    x, z, U, dy = rand(B, T, D), rand(B, T, R), rand(R, (D // H) * W), rand(B, T, D)
+    y = oracle.forward_lowrank(p, x, z, U)
+    dx, dz, dU, dw = oracle.backward_lowrank(p, x, z, U, dy)
+    wf = oracle.lowrank_filters(p, z, U)
+    kw = dict(x=x, dy=dy, z=z, U=U)
+    bt = np.array(list(itertools.product(range(B), range(T))))
+    pts = np.array([(b, t, c) for b, t in bt for c in range(D)])
+    np.testing.assert_allclose(oracle.sample(p, oracle.LOWRANK, oracle.Y, pts, **kw), y.reshape(-1), atol=1e-12)
+    np.testing.assert_allclose(oracle.sample(p, oracle.LOWRANK, oracle.DX, pts, **kw), dx.reshape(-1), atol=1e-12)
+    pg = np.array([(b, t, g, k) for b, t in bt for g in range(D // H) for k in range(W)])
+    np.testing.assert_allclose(oracle.sample(p, oracle.LOWRANK, oracle.DW, pg, **kw), dw.reshape(-1), atol=1e-12)
+    np.testing.assert_allclose(oracle.sample(p, oracle.LOWRANK, oracle.W_TAP, pg, **kw), wf.reshape(-1), atol=1e-12)
+    pr = np.array([(b, t, r) for b, t in bt for r in range(R)])
+    np.testing.assert_allclose(oracle.sample(p, oracle.LOWRANK, oracle.DZ, pr, **kw), dz.reshape(-1), atol=1e-12)
+    pu = np.array([(r, g, k) for r in range(R) for g in range(D // H) for k in range(W)])
+    np.testing.assert_allclose(oracle.sample(p, oracle.LOWRANK, oracle.DU, pu, **kw), dU.reshape(-1), atol=1e-11)
+    ws = rand(D, W)
+    _, dws = oracle.backward_static(p, x, ws, dy)
+    pc = np.array([(c, k) for c in range(D) for k in range(W)])
+    np.testing.assert_allclose(oracle.sample(p, oracle.STATIC, oracle.DWS, pc, x=x, dy=dy, w=ws), dws.reshape(-1), atol=1e-11)
