@@ -1,0 +1,502 @@
+#!/usr/bin/env python
+"""Throughput of the dynamic short convolution's training hot path on B200.
+
+One step = the forward and the backward of the convolution over one batch of
+the named workload (default: the Q/K/V placement with head-wise filters,
+B=8, T=2048, D=6144, W=4, H=16, bf16 with fp32 accumulation), called through
+the C ABI of libdsc.so on torch's current stream with inputs resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+    python bench.py --impl reference ...     # the fp64 CPU oracle, same line
+
+Prints ONE JSON line (rank 0).  `value` is whole-job tokens/s: every rank
+processes its own batch (data parallel, no exchange on this path: "weak"
+scaling), the time is the max over ranks of the device-measured time of K
+steps.  Also reported: the roofline of the dominant kernel (the backward)
+against the measured HBM copy bandwidth, the oracle on the host cores as a
+CPU baseline, the same metric end to end with host buffers (H2D of the
+inputs and D2H of all outputs inside the timed region), SM clocks sampled
+during the timed region, and the number of library kernels launched.
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "tokens/s and achieved HBM GB/s (fwd+bwd, bf16, W=4) vs B200 roofline"
+FALLBACK_HBM_GBS = 6650.0
+L2_BYTES = 126 * 2 ** 20
+
+
+# ------------------------------------------------------------ rank helpers ---
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def rank_workload(wl, rank: int):
+    """Each rank draws its own batch (seed = base seed + rank)."""
+    return wl.with_(seed=wl.seed + rank)
+
+
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank_step: int, world: int, steps: int, max_ms: float) -> float:
+    return tokens_per_rank_step * world * steps / (max_ms / 1e3)
+
+
+# ------------------------------------------------------- algorithmic bytes ---
+
+def step_bytes(wl):
+    """Algorithmic HBM bytes of one forward and one backward launch (each
+    tensor read or written once; w/z never materialised for low-rank)."""
+    s = 2 if wl.dtype == "bf16" else 4
+    N, D, GW, R = wl.B * wl.T, wl.D, (wl.D // wl.H) * wl.W, wl.R
+    if wl.variant == "headwise":
+        return N * (2 * D + GW) * s, N * (3 * D + 2 * GW) * s
+    if wl.variant == "lowrank":
+        u = R * GW * s
+        return N * (2 * D + R) * s + u, N * (3 * D + 2 * R) * s + u + 4 * R * GW
+    return N * 2 * D * s + D * wl.W * s, N * 3 * D * s + D * wl.W * s + 4 * D * wl.W
+
+
+def hbm_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def source_digest():
+    """sha256 of the kernel sources, to match ncu traffic figures to a build."""
+    import glob
+
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "input_dependent_short_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(os.path.basename(p).encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str, digest: str):
+    """DRAM bytes per launch from profiles/traffic.txt, if taken on this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    try:
+        with open(path) as f:
+            for line in f:
+                parts = line.split("|")
+                if len(parts) >= 4 and not line.startswith("#"):
+                    k, w, d, b = (p.strip() for p in parts[:4])
+                    if k == kernel and w == workload and d == digest:
+                        return float(b)
+    except OSError:
+        pass
+    return None
+
+
+# ------------------------------------------------------------------ clocks ---
+
+class ClockSampler:
+    """SM clock and throttle reasons via NVML, sampled every 5 ms (read only)."""
+
+    REASONS = {
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4,
+        "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, index: int):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # noqa: BLE001
+            self.nv = None
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:  # noqa: BLE001
+                pass
+            time.sleep(0.005)
+
+    def __enter__(self):
+        if self.nv:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------- the step ---
+
+class Step:
+    """Pre-allocated device buffers and the two C-ABI calls of one step."""
+
+    def __init__(self, wl, host, device):
+        import torch
+
+        from input_dependent_short_b200 import _lib, ops
+
+        self.wl, self.L = wl, _lib
+        self.dev = device
+        td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
+        import synth
+
+        self.h = {k: synth.to_torch(v, wl.dtype).pin_memory() for k, v in host.items()}
+        self.d = {k: v.to(device) for k, v in self.h.items()}
+        x = self.d["x"]
+        self.out = {"y": torch.empty_like(x), "dx": torch.empty_like(x)}
+        if wl.variant == "headwise":
+            self.out["dw"] = torch.empty_like(self.d["w"])
+            self.p = ops.problem(x, wl.W, wl.H, 0, bool(wl.residual))
+        elif wl.variant == "lowrank":
+            self.out["dz"] = torch.empty_like(self.d["z"])
+            self.out["dU"] = torch.empty(self.d["U"].shape, dtype=torch.float32, device=device)
+            self.p = ops.problem(x, wl.W, wl.H, wl.R, bool(wl.residual))
+        else:
+            self.out["dws"] = torch.empty(self.d["ws"].shape, dtype=torch.float32, device=device)
+            self.p = ops.problem(x, wl.W, 1, 0, bool(wl.residual))
+        lib = _lib.lib()
+        self.nfw = self.nbw = 0
+        if wl.variant == "lowrank":
+            self.nfw = lib.dsc_fwd_lowrank_workspace_bytes(self.p)
+            self.nbw = lib.dsc_bwd_lowrank_workspace_bytes(self.p)
+        elif wl.variant == "static":
+            self.nbw = lib.dsc_bwd_static_workspace_bytes(self.p)
+        self.fws = torch.empty(max(self.nfw, 16), dtype=torch.uint8, device=device)
+        self.bws = torch.empty(max(self.nbw, 16), dtype=torch.uint8, device=device)
+        self.out_h = {k: torch.empty(v.shape, dtype=v.dtype).pin_memory() for k, v in self.out.items()}
+        self.td = td
+
+    def fwd(self, stream):
+        d, o, L = self.d, self.out, self.L
+        if self.wl.variant == "headwise":
+            L.call("dsc_fwd_headwise", self.p, d["x"].data_ptr(), d["w"].data_ptr(), o["y"].data_ptr(), stream)
+        elif self.wl.variant == "lowrank":
+            L.call("dsc_fwd_lowrank", self.p, d["x"].data_ptr(), d["z"].data_ptr(), d["U"].data_ptr(),
+                   o["y"].data_ptr(), self.fws.data_ptr(), self.nfw, stream)
+        else:
+            L.call("dsc_fwd_static", self.p, d["x"].data_ptr(), d["ws"].data_ptr(), o["y"].data_ptr(), stream)
+
+    def bwd(self, stream):
+        d, o, L = self.d, self.out, self.L
+        if self.wl.variant == "headwise":
+            L.call("dsc_bwd_headwise", self.p, d["x"].data_ptr(), d["w"].data_ptr(), d["dy"].data_ptr(),
+                   o["dx"].data_ptr(), o["dw"].data_ptr(), stream)
+        elif self.wl.variant == "lowrank":
+            L.call("dsc_bwd_lowrank", self.p, d["x"].data_ptr(), d["z"].data_ptr(), d["U"].data_ptr(),
+                   d["dy"].data_ptr(), o["dx"].data_ptr(), o["dz"].data_ptr(), o["dU"].data_ptr(),
+                   self.bws.data_ptr(), self.nbw, stream)
+        else:
+            L.call("dsc_bwd_static", self.p, d["x"].data_ptr(), d["ws"].data_ptr(), d["dy"].data_ptr(),
+                   o["dx"].data_ptr(), o["dws"].data_ptr(), self.bws.data_ptr(), self.nbw, stream)
+
+    def h2d(self):
+        for k, v in self.h.items():
+            self.d[k].copy_(v, non_blocking=True)
+
+    def d2h(self):
+        for k, v in self.out.items():
+            self.out_h[k].copy_(v, non_blocking=True)
+
+    def bytes_in(self):
+        return sum(v.numel() * v.element_size() for v in self.h.values())
+
+    def bytes_out(self):
+        return sum(v.numel() * v.element_size() for v in self.out.values())
+
+
+# ----------------------------------------------------------------- our arm ---
+
+def run_dsc(args, wl0):
+    import torch
+    import torch.distributed as dist
+
+    import synth  # noqa: F401
+    from synth import workloads as wls
+
+    world, rank, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = rank_workload(wl0, rank)
+    host = wls.make_inputs(wl)
+    step = Step(wl, host, dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+
+    for _ in range(args.warmup):
+        step.fwd(stream)
+        step.bwd(stream)
+    torch.cuda.synchronize(dev)
+
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    lib = step.L.lib()
+    n0 = lib.dsc_launch_count()
+    with ClockSampler(local) as clocks:
+        start.record()
+        for i in range(K):
+            ev[i][0].record()
+            step.fwd(stream)
+            ev[i][1].record()
+            step.bwd(stream)
+            ev[i][2].record()
+        end.record()
+        end.synchronize()
+    torch.cuda.synchronize(dev)
+    launches = lib.dsc_launch_count() - n0
+    if world > 1:
+        dist.barrier()
+    ms_local = start.elapsed_time(end)
+    fwd_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
+    bwd_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(K))
+    ms = max_over_ranks(ms_local, world, dev)
+
+    # end to end: inputs from pinned host memory, every output back to the host
+    Ke = max(3, min(args.e2e_steps, K))
+    for _ in range(2):
+        step.h2d(); step.fwd(stream); step.bwd(stream); step.d2h()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(Ke):
+        step.h2d()
+        step.fwd(stream)
+        step.bwd(stream)
+        step.d2h()
+    e1.record()
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+
+    tokens = wl.B * wl.T
+    fb, bb = step_bytes(wl)
+    peak, peak_src = hbm_peak()
+    digest = source_digest()
+    bwd_gbs = bb / (bwd_ms / 1e3) / 1e9
+    fwd_gbs = fb / (fwd_ms / 1e3) / 1e9
+    step_gbs = (fb + bb) / (ms / K / 1e3) / 1e9
+    kname = {"headwise": "k_stream_bwd", "static": "k_stream_bwd", "lowrank": "lowrank_bwd"}[wl.variant]
+    traffic = ncu_traffic(kname, wl0.name, digest)
+
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC,
+            "value": job_tokens_per_s(tokens, world, K, ms),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": K,
+            "warmup": args.warmup,
+            "ms_per_step": ms / K,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+            "accumulate": "f32",
+            "data": "synthetic (seeded normals, seed = rank)",
+            "config": {
+                "workload": wl0.name, "variant": wl.variant, "B": wl.B, "T": wl.T, "D": wl.D, "W": wl.W,
+                "H": wl.H, "R": wl.R, "residual": wl.residual, "pass": "forward + backward",
+                "global_batch": wl.B * world, "seq_len": wl.T, "parallelism": f"dp{world}",
+                "l2": "inputs larger than L2 (x, dy, y, dx are %.0f MB each; L2 126 MB), no flush"
+                      % (tokens * wl.D * (2 if wl.dtype == "bf16" else 4) / 1e6),
+            },
+            "hbm_gbs_step": step_gbs,
+            "kernels": {
+                "fwd": {"us": fwd_ms * 1e3, "alg_bytes": fb, "gbs": fwd_gbs, "frac": fwd_gbs / peak},
+                "bwd": {"us": bwd_ms * 1e3, "alg_bytes": bb, "gbs": bwd_gbs, "frac": bwd_gbs / peak},
+            },
+            "roofline": {
+                "kernel": kname, "bound": "hbm", "achieved": bwd_gbs, "peak": peak, "unit": "GB/s",
+                "frac": bwd_gbs / peak, "traffic": traffic, "peak_source": peak_src + " (hbm_gbs, copy)",
+                "frac_of_8000": bwd_gbs / 8000.0, "step_frac": step_gbs / peak,
+            },
+            "e2e": {"value": job_tokens_per_s(tokens, world, Ke, e2e_ms), "unit": "tokens/s",
+                    "h2d_bytes_per_step": step.bytes_in(), "d2h_bytes_per_step": step.bytes_out(),
+                    "steps": Ke, "ms_per_step": e2e_ms / Ke},
+            "gpu_launches": launches,
+            "clocks": clocks.summary(),
+            "source_digest": digest,
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result, host, wl
+
+
+# ----------------------------------------------------------- CPU baselines ---
+
+def oracle_pass(wl, t):
+    import oracle
+
+    if wl.variant == "headwise":
+        P = oracle.problem_of(wl)
+        oracle.forward_headwise(P, t["x"], t["w"])
+        oracle.backward_headwise(P, t["x"], t["w"], t["dy"])
+    elif wl.variant == "lowrank":
+        P = oracle.problem_of(wl)
+        oracle.forward_lowrank(P, t["x"], t["z"], t["U"])
+        oracle.backward_lowrank(P, t["x"], t["z"], t["U"], t["dy"])
+    else:
+        P = oracle.problem(wl.B, wl.T, wl.D, wl.W, 1, 0, wl.residual)
+        oracle.forward_static(P, t["x"], t["ws"])
+        oracle.backward_static(P, t["x"], t["ws"], t["dy"])
+
+
+def sample_of(wl, host, tokens):
+    """The first `tokens` tokens of batch row 0 (a causal prefix: the same
+    per-token work as the full workload)."""
+    T = max(1, min(wl.T, tokens))
+    sub = wl.with_(B=1, T=T)
+    t = {}
+    for k, v in host.items():
+        if k in ("x", "dy", "w", "z"):
+            t[k] = v[:1, :T].copy()
+        else:
+            t[k] = v
+    return sub, t
+
+
+def cpu_baseline(wl, host, seconds=10.0):
+    import oracle
+
+    sub, t = sample_of(wl, host, 2048)
+    n = 0
+    t0 = time.perf_counter()
+    while True:
+        oracle_pass(sub, t)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": n * sub.B * sub.T / el, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+            "sample": f"{n} passes of fwd+bwd over the first {sub.T} tokens of batch row 0 "
+                      f"({sub.D} channels, fp64 oracle, {el:.1f} s)"}
+
+
+def run_reference(args, wl0):
+    """The fp64 oracle on the host cores, same metric and config."""
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return None
+    import oracle
+    from synth import workloads as wls
+
+    oracle.build()
+    tokens = args.ref_tokens
+    sub0 = wl0.with_(B=1, T=min(wl0.T, tokens))
+    host = wls.make_inputs(sub0)
+    sub, t = sample_of(sub0, host, tokens)
+    for _ in range(args.warmup):
+        oracle_pass(sub, t)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_pass(sub, t)
+    el = time.perf_counter() - t0
+    v = args.steps * sub.T / el
+    cores = oracle.max_threads()
+    return {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / args.steps * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl0.name, "variant": wl0.variant, "pass": "forward + backward",
+                   "sample_tokens_per_step": sub.T},
+        "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                         "sample": f"each step: fwd+bwd over the first {sub.T} tokens of one sequence"},
+        "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=500)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["dsc", "reference"], default="dsc")
+    ap.add_argument("--workload", default="qkv-headwise")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--ref-tokens", type=int, default=256)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    from synth import workloads as wls
+
+    if args.workload in wls.NAMED:
+        wl0 = wls.NAMED[args.workload]
+    else:
+        matches = [w for w in wls.sweep_workloads() if w.name.replace(" ", "-") == args.workload]
+        if not matches:
+            ap.error(f"unknown workload {args.workload}")
+        wl0 = matches[0]
+
+    if args.impl == "reference":
+        res = run_reference(args, wl0)
+    else:
+        res, host, wl = run_dsc(args, wl0)
+        if res is not None:
+            world = res["n_gpus"]
+            if world == 1 and not args.no_cpu_baseline:
+                res["cpu_baseline"] = cpu_baseline(wl, host, args.cpu_seconds)
+            else:
+                res["cpu_baseline"] = None
+    if res is not None:
+        print(json.dumps(res), flush=True)
+
+
+if __name__ == "__main__":
+    main()

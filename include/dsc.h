@@ -1,0 +1,136 @@
+/*
+ * dsc.h -- C ABI of the B200 (sm_100a) dynamic short convolution library
+ * (libdsc.so).
+ *
+ * The operation (from "Dynamic Short Convolutions Improve Transformers",
+ * technical summary, Methodology: "Mechanism", "Parameterisation",
+ * "Placement"; and the authors' thread, on static short convolutions):
+ *
+ *   y[b,t,c] = r*x[b,t,c] + sum_{k=0}^{W-1} w(t)_k[c] * x[b,t-k,c]
+ *
+ * a causal depthwise convolution of width W whose filter is chosen per token;
+ * terms with t-k < 0 are zero and every batch row is an independent sequence.
+ * r is the residual flag (the pages place the op as X = X + conv(X)).  The
+ * filter of channel c at token t is:
+ *   head-wise:  w[b,t,c/H,k]                (one filter per H consecutive
+ *                                            channels, w is [B,T,G,W], G=D/H)
+ *   low-rank:   sum_r z[b,t,r] * U[r, (c/H)*W + k]
+ *               (z [B,T,R], U [R, G*W]; the product is formed on chip and the
+ *                full filter tensor is never written to memory)
+ *   static:     ws[c,k]                     (ws [D,W], the same at every t)
+ *
+ * Backward (the gradients of the definition above; the pages' kernels are
+ * training kernels but print no formula):
+ *   dx[b,s,c]   = r*dy[b,s,c] + sum_{k, s+k<T} w(s+k)_k[c] * dy[b,s+k,c]
+ *   dw[b,t,g,k] = sum_{c in group g} dy[b,t,c] * x[b,t-k,c]     (0 if t < k)
+ *   dz[b,t,r]   = sum_{g,k} dw[b,t,g,k] * U[r, g*W+k]
+ *   dU[r,g*W+k] = sum_{b,t} z[b,t,r] * dw[b,t,g,k]
+ *   dws[c,k]    = sum_{b,t} dy[b,t,c] * x[b,t-k,c]
+ *
+ * Conventions shared by every entry point
+ *  - All tensor arguments are caller-owned DEVICE pointers, dense row-major
+ *    in the shapes above (last index fastest), base address 16-byte aligned
+ *    (else DSC_ERR_MISALIGNED).  Outputs must not alias inputs.
+ *  - dtype DSC_BF16: x, w, z, U, ws, dy and the outputs y, dx, dw, dz are
+ *    bf16; arithmetic is fp32; dU and dws are fp32.  DSC_F32: everything fp32.
+ *  - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *    call only enqueues work on that stream and returns; it never
+ *    synchronises and never allocates device memory.  Scratch memory, where a
+ *    call needs it, is passed in by the caller (`workspace`); its size comes
+ *    from the matching *_workspace_bytes query, it must stay untouched until
+ *    the stream has passed the call, and it may be NULL when the query
+ *    returns 0.
+ *  - Validation: B,T >= 1; D >= 1; 1 <= W <= 8; H >= 1 with D % H == 0;
+ *    low-rank 1 <= R <= 256; non-NULL tensor pointers; else
+ *    DSC_ERR_INVALID_ARG.  Nothing is launched when validation fails.
+ *  - A failed launch returns DSC_ERR_CUDA (cudaGetLastError() is left set
+ *    for the caller to inspect).
+ *  - Kernels that wait on on-chip barriers wait a bounded time; on expiry
+ *    they record DSC_ERR_TIMEOUT in a device status word and return.
+ *    dsc_check() reads and clears it.
+ */
+#ifndef DSC_H
+#define DSC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifndef DSC_API
+#define DSC_API __attribute__((visibility("default")))
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DSC_OK = 0,
+    DSC_ERR_INVALID_ARG = 1,
+    DSC_ERR_UNSUPPORTED = 2,
+    DSC_ERR_MISALIGNED = 3,
+    DSC_ERR_CUDA = 4,
+    DSC_ERR_TIMEOUT = 5
+} dsc_status;
+
+typedef enum { DSC_F32 = 0, DSC_BF16 = 1 } dsc_dtype;
+
+/* Problem shape.  H: channels per shared filter (G = D/H groups).  R: rank
+ * of the low-rank factorisation (ignored by the other variants).  residual:
+ * 1 adds x to y and dy to dx, 0 does not. */
+typedef struct {
+    int64_t B, T, D, W, H, R;
+    int32_t dtype;    /* dsc_dtype */
+    int32_t residual;
+} dsc_problem;
+
+/* Head-wise forward: x [B,T,D], w [B,T,G,W] -> y [B,T,D]. */
+DSC_API dsc_status dsc_fwd_headwise(const dsc_problem *p, const void *x, const void *w, void *y, void *stream);
+
+/* Head-wise backward: x, w, dy -> dx [B,T,D], dw [B,T,G,W]. */
+DSC_API dsc_status dsc_bwd_headwise(const dsc_problem *p, const void *x, const void *w, const void *dy, void *dx, void *dw,
+                            void *stream);
+
+/* Bytes of scratch the low-rank forward / backward need for this problem
+ * (0 when the fused kernels apply). */
+DSC_API size_t dsc_fwd_lowrank_workspace_bytes(const dsc_problem *p);
+DSC_API size_t dsc_bwd_lowrank_workspace_bytes(const dsc_problem *p);
+
+/* Low-rank forward: x [B,T,D], z [B,T,R], U [R,G*W] -> y [B,T,D]. */
+DSC_API dsc_status dsc_fwd_lowrank(const dsc_problem *p, const void *x, const void *z, const void *U, void *y,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
+/* Low-rank backward: x, z, U, dy -> dx [B,T,D], dz [B,T,R], dU [R,G*W] fp32
+ * (dU is overwritten, not accumulated into). */
+DSC_API dsc_status dsc_bwd_lowrank(const dsc_problem *p, const void *x, const void *z, const void *U, const void *dy,
+                           void *dx, void *dz, float *dU, void *workspace, size_t workspace_bytes, void *stream);
+
+/* Static-filter forward: x [B,T,D], ws [D,W] -> y [B,T,D]. */
+DSC_API dsc_status dsc_fwd_static(const dsc_problem *p, const void *x, const void *ws, void *y, void *stream);
+
+/* Scratch bytes of the static backward (per-tile partial filter gradients). */
+DSC_API size_t dsc_bwd_static_workspace_bytes(const dsc_problem *p);
+
+/* Static-filter backward: x, ws, dy -> dx [B,T,D], dws [D,W] fp32
+ * (overwritten).  Deterministic: partial sums are reduced in a fixed order. */
+DSC_API dsc_status dsc_bwd_static(const dsc_problem *p, const void *x, const void *ws, const void *dy, void *dx, float *dws,
+                          void *workspace, size_t workspace_bytes, void *stream);
+
+/* Synchronise `stream`, then return and clear the device status word of the
+ * current device: DSC_OK, DSC_ERR_TIMEOUT, or DSC_ERR_CUDA if the stream
+ * reported an error. */
+DSC_API dsc_status dsc_check(void *stream);
+
+/* Static description of a status code. */
+DSC_API const char *dsc_status_string(dsc_status s);
+
+/* Number of kernels this library has launched in this process so far (all
+ * devices, all streams).  Lets a caller count the launches of a region. */
+DSC_API uint64_t dsc_launch_count(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+DSC_API int dsc_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DSC_H */

@@ -1,0 +1,246 @@
+// C entry points of libdsc.so: argument checks, then dispatch to the kernels.
+// The contract of every function is in include/dsc.h.
+#include <atomic>
+#include <mutex>
+
+#include "kernels.cuh"
+
+namespace dsc {
+
+static std::atomic<uint64_t> g_launches{0};
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static dsc_status validate(const dsc_problem *p, bool lowrank) {
+    if (!p) return DSC_ERR_INVALID_ARG;
+    if (p->B < 1 || p->T < 1 || p->D < 1 || p->W < 1 || p->W > 8 || p->H < 1) return DSC_ERR_INVALID_ARG;
+    if (p->D % p->H) return DSC_ERR_INVALID_ARG;
+    if (p->dtype != DSC_F32 && p->dtype != DSC_BF16) return DSC_ERR_INVALID_ARG;
+    if (p->T > (int64_t)1 << 30 || p->B > (int64_t)1 << 30) return DSC_ERR_UNSUPPORTED;
+    if (lowrank && (p->R < 1 || p->R > 256)) return DSC_ERR_INVALID_ARG;
+    return DSC_OK;
+}
+
+static dsc_status check_ptrs(std::initializer_list<const void *> ptrs) {
+    for (const void *q : ptrs)
+        if (!q) return DSC_ERR_INVALID_ARG;
+    for (const void *q : ptrs)
+        if (!aligned16(q)) return DSC_ERR_MISALIGNED;
+    return DSC_OK;
+}
+
+static int sm_count() {
+    static std::mutex mu;
+    static int cache[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+        cudaGetLastError();
+        return 148;
+    }
+    std::lock_guard<std::mutex> g(mu);
+    if (!cache[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+            cudaGetLastError();
+            n = 148;
+        }
+        cache[dev] = n;
+    }
+    return cache[dev];
+}
+
+static Ctx ctx(void *stream) { return Ctx{static_cast<cudaStream_t>(stream), sm_count()}; }
+
+static int vec_of(const dsc_problem &p) { return p.dtype == DSC_BF16 ? 8 : 4; }
+
+static dsc_status done(cudaError_t e) { return e == cudaSuccess ? DSC_OK : DSC_ERR_CUDA; }
+
+static GenArgs gen_args(const dsc_problem &p, int wmode) {
+    GenArgs a{};
+    a.B = p.B; a.T = p.T; a.D = p.D; a.H = p.H; a.G = p.D / p.H;
+    a.W = (int)p.W;
+    a.residual = p.residual ? 1 : 0;
+    a.wmode = wmode;
+    return a;
+}
+
+static dsc_problem static_view(const dsc_problem &p) {
+    dsc_problem q = p;
+    q.H = 1;  // one filter per channel
+    return q;
+}
+
+static size_t lr_generic_fwd_bytes(const dsc_problem &p) {
+    return (size_t)(p.B * p.T) * (size_t)((p.D / p.H) * p.W) * sizeof(float);
+}
+
+}  // namespace dsc
+
+using namespace dsc;
+
+extern "C" {
+
+int dsc_version(void) { return 100; }
+
+uint64_t dsc_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+const char *dsc_status_string(dsc_status s) {
+    switch (s) {
+    case DSC_OK: return "ok";
+    case DSC_ERR_INVALID_ARG: return "invalid argument";
+    case DSC_ERR_UNSUPPORTED: return "unsupported problem";
+    case DSC_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+    case DSC_ERR_CUDA: return "CUDA error";
+    case DSC_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+dsc_status dsc_fwd_headwise(const dsc_problem *p, const void *x, const void *w, void *y, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_ptrs({x, w, y});
+    if (s != DSC_OK) return s;
+    const Ctx c = ctx(stream);
+    HwArgs a{};
+    if (stream_map(*p, vec_of(*p), a.m)) {
+        a.x = x; a.w = w; a.y = y;
+        return done(launch_hw_fwd(c, *p, a));
+    }
+    GenArgs g = gen_args(*p, WMODE_HEADWISE);
+    g.x = x; g.w = w; g.y = y;
+    return done(launch_gen_fwd(c, *p, g, false));
+}
+
+dsc_status dsc_bwd_headwise(const dsc_problem *p, const void *x, const void *w, const void *dy, void *dx, void *dw,
+                            void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_ptrs({x, w, dy, dx, dw});
+    if (s != DSC_OK) return s;
+    const Ctx c = ctx(stream);
+    HwArgs a{};
+    if (stream_map(*p, vec_of(*p), a.m)) {
+        a.x = x; a.w = w; a.dy = dy; a.dx = dx; a.dw = dw;
+        return done(launch_hw_bwd(c, *p, a));
+    }
+    GenArgs g = gen_args(*p, WMODE_HEADWISE);
+    g.x = x; g.w = w; g.dy = dy; g.dx = dx; g.dw = dw;
+    cudaError_t e = launch_gen_dx(c, *p, g, false);
+    if (e == cudaSuccess) e = launch_gen_dw(c, *p, g, false);
+    return done(e);
+}
+
+dsc_status dsc_fwd_static(const dsc_problem *p, const void *x, const void *ws, void *y, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_ptrs({x, ws, y});
+    if (s != DSC_OK) return s;
+    const dsc_problem q = static_view(*p);
+    const Ctx c = ctx(stream);
+    HwArgs a{};
+    if (stream_map(q, vec_of(q), a.m)) {
+        a.x = x; a.w = ws; a.y = y;
+        return done(launch_st_fwd(c, q, a));
+    }
+    GenArgs g = gen_args(q, WMODE_STATIC);
+    g.x = x; g.w = ws; g.y = y;
+    return done(launch_gen_fwd(c, q, g, false));
+}
+
+size_t dsc_bwd_static_workspace_bytes(const dsc_problem *p) {
+    if (validate(p, false) != DSC_OK) return 0;
+    const dsc_problem q = static_view(*p);
+    StreamMap m;
+    size_t parts;
+    if (stream_map(q, vec_of(q), m)) parts = st_partial_count(ctx(nullptr), q);
+    else parts = (size_t)(q.B * ((q.T + 63) / 64));
+    return parts * (size_t)(q.D * q.W) * sizeof(float);
+}
+
+dsc_status dsc_bwd_static(const dsc_problem *p, const void *x, const void *ws, const void *dy, void *dx, float *dws,
+                          void *workspace, size_t workspace_bytes, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_ptrs({x, ws, dy, dx, dws, workspace});
+    if (s != DSC_OK) return s;
+    if (workspace_bytes < dsc_bwd_static_workspace_bytes(p)) return DSC_ERR_INVALID_ARG;
+    const dsc_problem q = static_view(*p);
+    const Ctx c = ctx(stream);
+    HwArgs a{};
+    if (stream_map(q, vec_of(q), a.m)) {
+        a.x = x; a.w = ws; a.dy = dy; a.dx = dx;
+        a.partial = static_cast<float *>(workspace);
+        return done(launch_st_bwd(c, q, a, dws));
+    }
+    GenArgs g = gen_args(q, WMODE_STATIC);
+    g.x = x; g.w = ws; g.dy = dy; g.dx = dx;
+    cudaError_t e = launch_gen_dx(c, q, g, false);
+    if (e == cudaSuccess) e = launch_gen_dws(c, q, g, dws, static_cast<float *>(workspace), 0);
+    return done(e);
+}
+
+size_t dsc_fwd_lowrank_workspace_bytes(const dsc_problem *p) {
+    if (validate(p, true) != DSC_OK) return 0;
+    if (lowrank_fused_ok(*p)) return 0;
+    return lr_generic_fwd_bytes(*p);
+}
+
+size_t dsc_bwd_lowrank_workspace_bytes(const dsc_problem *p) {
+    if (validate(p, true) != DSC_OK) return 0;
+    if (lowrank_fused_ok(*p)) return lr_bwd_fused_ws_bytes(ctx(nullptr), *p);
+    return 2 * lr_generic_fwd_bytes(*p);
+}
+
+dsc_status dsc_fwd_lowrank(const dsc_problem *p, const void *x, const void *z, const void *U, void *y,
+                           void *workspace, size_t workspace_bytes, void *stream) {
+    dsc_status s = validate(p, true);
+    if (s == DSC_OK) s = check_ptrs({x, z, U, y});
+    if (s != DSC_OK) return s;
+    const Ctx c = ctx(stream);
+    if (lowrank_fused_ok(*p)) return done(launch_lr_fwd_fused(c, *p, x, z, U, y));
+    // Unfused fallback: filters w = zU in the workspace, then the per-channel kernel.
+    if (!workspace) return DSC_ERR_INVALID_ARG;
+    if (!aligned16(workspace)) return DSC_ERR_MISALIGNED;
+    if (workspace_bytes < lr_generic_fwd_bytes(*p)) return DSC_ERR_INVALID_ARG;
+    float *wf = static_cast<float *>(workspace);
+    cudaError_t e = launch_lr_filters(c, *p, z, U, wf);
+    GenArgs g = gen_args(*p, WMODE_HEADWISE);
+    g.x = x; g.w = wf; g.y = y;
+    if (e == cudaSuccess) e = launch_gen_fwd(c, *p, g, true);
+    return done(e);
+}
+
+dsc_status dsc_bwd_lowrank(const dsc_problem *p, const void *x, const void *z, const void *U, const void *dy,
+                           void *dx, void *dz, float *dU, void *workspace, size_t workspace_bytes, void *stream) {
+    dsc_status s = validate(p, true);
+    if (s == DSC_OK) s = check_ptrs({x, z, U, dy, dx, dz, dU});
+    if (s != DSC_OK) return s;
+    const size_t need = dsc_bwd_lowrank_workspace_bytes(p);
+    if (need && (!workspace || workspace_bytes < need)) return DSC_ERR_INVALID_ARG;
+    if (need && !aligned16(workspace)) return DSC_ERR_MISALIGNED;
+    const Ctx c = ctx(stream);
+    if (lowrank_fused_ok(*p)) return done(launch_lr_bwd_fused(c, *p, x, z, U, dy, dx, dz, dU, workspace, workspace_bytes));
+    // Unfused fallback: w = zU and dw in the workspace; dz = dw U^T; dU = z^T dw.
+    const int64_t N = p->B * p->T, GW = (p->D / p->H) * p->W;
+    float *wf = static_cast<float *>(workspace);
+    float *dwf = wf + N * GW;
+    const bool bf = p->dtype == DSC_BF16;
+    cudaError_t e = launch_lr_filters(c, *p, z, U, wf);
+    GenArgs g = gen_args(*p, WMODE_HEADWISE);
+    g.x = x; g.w = wf; g.dy = dy; g.dx = dx; g.dw = dwf;
+    if (e == cudaSuccess) e = launch_gen_dx(c, *p, g, true);
+    if (e == cudaSuccess) e = launch_gen_dw(c, *p, g, true);
+    if (e == cudaSuccess)  // dz[n][r] = sum_j dw[n][j] U[r][j]
+        e = launch_gemm(c, (int)N, (int)p->R, (int)GW, dwf, true, GW, 1, U, !bf, GW, 1, dz, !bf, p->R, bf);
+    if (e == cudaSuccess)  // dU[r][j] = sum_n z[n][r] dw[n][j]
+        e = launch_gemm(c, (int)p->R, (int)GW, (int)N, z, !bf, 1, p->R, dwf, true, 1, GW, dU, true, GW, bf);
+    return done(e);
+}
+
+dsc_status dsc_check(void *stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSC_ERR_CUDA;
+    const int st = take_device_status(static_cast<cudaStream_t>(stream));
+    if (st < 0) return DSC_ERR_CUDA;
+    return static_cast<dsc_status>(st);
+}
+
+}  // extern "C"

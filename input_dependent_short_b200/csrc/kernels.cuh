@@ -1,0 +1,84 @@
+// Launch interface between the C entry points (api.cu) and the kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace dsc {
+
+// Mapping of the time-streaming kernels.  Each thread owns one 16-byte vector
+// of channels (V = 8 bf16 or 4 fp32) and walks Tt consecutive tokens of one
+// sequence.  A warp covers CW channels starting at wc*CW; lane l owns channels
+// wc*CW + l*V .. +V-1 and is active when l < lanes_used and the channel is < D.
+// When H is a multiple of V, the L = H/V consecutive lanes of one filter group
+// reduce the group's filter gradient with shuffles; when V is a multiple of H a
+// lane owns GPT = V/H whole groups.
+struct StreamMap {
+    int64_t B, T, D, H, G;
+    int W;
+    int Tt, nTiles, nWc, CW, lanes_used, L, gpt;
+    int64_t n_warps;
+    int residual;
+};
+
+struct HwArgs {
+    StreamMap m;
+    const void *x, *w, *dy;
+    void *y, *dx, *dw;
+    float *partial;  // static filter-gradient partials [B*nTiles][D][W]
+};
+
+// Generic per-channel kernels (any D, H, W <= 8); `wmode` selects the filter.
+enum { WMODE_HEADWISE = 0, WMODE_STATIC = 1 };
+
+struct GenArgs {
+    int64_t B, T, D, H, G;
+    int W, Tt, nTiles, residual, wmode;
+    const void *x, *w, *dy;
+    void *y, *dx, *dw;
+    float *partial;
+};
+
+struct Ctx {
+    cudaStream_t stream;
+    int sms;
+};
+
+// conv_stream.cu
+bool stream_map(const dsc_problem &p, int V, StreamMap &m);
+void finish_map(StreamMap &m, int64_t target_warps);
+cudaError_t launch_hw_fwd(const Ctx &c, const dsc_problem &p, HwArgs a);
+cudaError_t launch_hw_bwd(const Ctx &c, const dsc_problem &p, HwArgs a);
+cudaError_t launch_st_fwd(const Ctx &c, const dsc_problem &p, HwArgs a);
+cudaError_t launch_st_bwd(const Ctx &c, const dsc_problem &p, HwArgs a, float *dws);
+size_t st_partial_count(const Ctx &c, const dsc_problem &p);
+
+// generic.cu (w may be a fp32 workspace: `w_f32`)
+cudaError_t launch_gen_fwd(const Ctx &c, const dsc_problem &p, GenArgs a, bool w_f32);
+cudaError_t launch_gen_dx(const Ctx &c, const dsc_problem &p, GenArgs a, bool w_f32);
+cudaError_t launch_gen_dw(const Ctx &c, const dsc_problem &p, GenArgs a, bool out_f32);
+cudaError_t launch_gen_dws(const Ctx &c, const dsc_problem &p, GenArgs a, float *dws, float *partial, int tile);
+cudaError_t launch_lr_filters(const Ctx &c, const dsc_problem &p, const void *z, const void *U, float *wf);
+// C[i][j] = sum_k A[i*sai + k*sak] * B[j*sbj + k*sbk], fp32 accumulate.
+cudaError_t launch_gemm(const Ctx &c, int M, int N, int K, const void *A, bool a_f32, int64_t sai, int64_t sak,
+                        const void *B, bool b_f32, int64_t sbj, int64_t sbk, void *C, bool c_f32, int64_t ldc,
+                        bool bf16_io);
+cudaError_t launch_reduce_partials(const Ctx &c, const float *partial, int64_t S, int64_t n, float *out);
+
+// lowrank.cu (fused kernels)
+bool lowrank_fused_ok(const dsc_problem &p);
+cudaError_t launch_lr_fwd_fused(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U,
+                                void *y);
+cudaError_t launch_lr_bwd_fused(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U,
+                                const void *dy, void *dx, void *dz, float *dU, void *ws, size_t ws_bytes);
+size_t lr_bwd_fused_ws_bytes(const Ctx &c, const dsc_problem &p);
+
+int resident_blocks(const void *kernel, int threads, size_t smem);
+
+// Records one kernel launch (api.cu keeps the process-wide count).
+void count_launch();
+
+// Status word of kernels with bounded waits (lowrank.cu): returns the
+// recorded dsc_status of the current device and clears it.
+int take_device_status(cudaStream_t stream);
+
+}  // namespace dsc

@@ -1,0 +1,181 @@
+"""PyTorch-facing binding of libdsc.so.
+
+Each function has the name of the C entry point it calls and only marshals
+arguments: it checks shapes/dtypes/devices, allocates the outputs (and any
+scratch the library asks for) with torch on the tensors' device, and passes
+raw device pointers plus torch's current CUDA stream.  Every step of the
+computation runs in the library's CUDA kernels.
+
+Layouts (row-major, contiguous): x, dy, y, dx [B,T,D]; head-wise w, dw
+[B,T,G,W] with G = D/H; low-rank z, dz [B,T,R] and U [R,G*W]; static
+ws [D,W].  dtypes: all bf16 or all fp32; dU and dws are fp32.
+"""
+
+from __future__ import annotations
+
+import torch
+
+from ._lib import DSC_BF16, DSC_F32, DscProblem, call, lib
+
+_DT = {torch.bfloat16: DSC_BF16, torch.float32: DSC_F32}
+
+
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(dev: torch.device):
+    return torch.cuda.current_stream(dev).cuda_stream
+
+
+def _check(*ts: torch.Tensor, dtype=None):
+    dev = ts[0].device
+    if dev.type != "cuda":
+        raise ValueError("libdsc operates on CUDA tensors")
+    for t in ts:
+        if t.device != dev:
+            raise ValueError("all tensors must be on the same device")
+        if not t.is_contiguous():
+            raise ValueError("tensors must be contiguous")
+        if dtype is not None and t.dtype != dtype:
+            raise ValueError(f"expected {dtype}, got {t.dtype}")
+    return dev
+
+
+def problem(x: torch.Tensor, W: int, H: int, R: int = 0, residual: bool = True) -> DscProblem:
+    B, T, D = x.shape
+    if x.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    return DscProblem(B, T, D, W, H, R, _DT[x.dtype], int(bool(residual)))
+
+
+# ----------------------------------------------------------------- head-wise ---
+
+def dsc_fwd_headwise(x, w, residual=True):
+    """y = r*x + causal per-token conv of x with head-wise filters w [B,T,G,W]."""
+    dev = _check(x, w, dtype=x.dtype)
+    B, T, D = x.shape
+    G, W = w.shape[2], w.shape[3]
+    if w.shape[:2] != (B, T) or D % G:
+        raise ValueError("w must be [B,T,G,W] with G dividing D")
+    p = problem(x, W, D // G, 0, residual)
+    y = torch.empty_like(x)
+    with torch.cuda.device(dev):
+        call("dsc_fwd_headwise", p, _ptr(x), _ptr(w), _ptr(y), _stream(dev))
+    return y
+
+
+def dsc_bwd_headwise(x, w, dy, residual=True):
+    """Returns (dx, dw)."""
+    dev = _check(x, w, dy, dtype=x.dtype)
+    B, T, D = x.shape
+    G, W = w.shape[2], w.shape[3]
+    p = problem(x, W, D // G, 0, residual)
+    dx = torch.empty_like(x)
+    dw = torch.empty_like(w)
+    with torch.cuda.device(dev):
+        call("dsc_bwd_headwise", p, _ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), _stream(dev))
+    return dx, dw
+
+
+# ------------------------------------------------------------------ low-rank ---
+
+def _lr_problem(x, z, U, H, residual):
+    B, T, D = x.shape
+    R = z.shape[-1]
+    if z.shape != (B, T, R) or U.shape[0] != R or D % H or U.shape[1] % (D // H):
+        raise ValueError("expected z [B,T,R] and U [R,(D/H)*W]")
+    W = U.shape[1] // (D // H)
+    return problem(x, W, H, R, residual)
+
+
+def dsc_fwd_lowrank(x, z, U, H=1, residual=True):
+    """y with filters w(t) = z_t U formed on chip (U is [R, (D/H)*W])."""
+    dev = _check(x, z, U, dtype=x.dtype)
+    p = _lr_problem(x, z, U, H, residual)
+    y = torch.empty_like(x)
+    n = lib().dsc_fwd_lowrank_workspace_bytes(p)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
+    with torch.cuda.device(dev):
+        call("dsc_fwd_lowrank", p, _ptr(x), _ptr(z), _ptr(U), _ptr(y), _ptr(ws), n, _stream(dev))
+    return y
+
+
+def dsc_bwd_lowrank(x, z, U, dy, H=1, residual=True):
+    """Returns (dx, dz, dU); dU is fp32."""
+    dev = _check(x, z, U, dy, dtype=x.dtype)
+    p = _lr_problem(x, z, U, H, residual)
+    dx = torch.empty_like(x)
+    dz = torch.empty_like(z)
+    dU = torch.empty(U.shape, dtype=torch.float32, device=dev)
+    n = lib().dsc_bwd_lowrank_workspace_bytes(p)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
+    with torch.cuda.device(dev):
+        call("dsc_bwd_lowrank", p, _ptr(x), _ptr(z), _ptr(U), _ptr(dy), _ptr(dx), _ptr(dz), _ptr(dU),
+             _ptr(ws), n, _stream(dev))
+    return dx, dz, dU
+
+
+# -------------------------------------------------------------------- static ---
+
+def dsc_fwd_static(x, ws, residual=False):
+    """Depthwise causal conv with one fixed filter per channel, ws [D,W]."""
+    dev = _check(x, ws, dtype=x.dtype)
+    p = problem(x, ws.shape[1], 1, 0, residual)
+    y = torch.empty_like(x)
+    with torch.cuda.device(dev):
+        call("dsc_fwd_static", p, _ptr(x), _ptr(ws), _ptr(y), _stream(dev))
+    return y
+
+
+def dsc_bwd_static(x, ws, dy, residual=False):
+    """Returns (dx, dws); dws is fp32."""
+    dev = _check(x, ws, dy, dtype=x.dtype)
+    p = problem(x, ws.shape[1], 1, 0, residual)
+    dx = torch.empty_like(x)
+    dws = torch.empty(ws.shape, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        n = lib().dsc_bwd_static_workspace_bytes(p)
+        scratch = torch.empty(max(n, 16), dtype=torch.uint8, device=dev)
+        call("dsc_bwd_static", p, _ptr(x), _ptr(ws), _ptr(dy), _ptr(dx), _ptr(dws), _ptr(scratch), n,
+             _stream(dev))
+    return dx, dws
+
+
+def dsc_check(device=None):
+    """Synchronise the current stream and raise if a kernel recorded a timeout."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else torch.device(device).index)
+    with torch.cuda.device(dev):
+        call("dsc_check", _stream(dev))
+
+
+# ------------------------------------------------------------------ autograd ---
+
+class DynamicShortConvHeadwise(torch.autograd.Function):
+    """Autograd wrapper: forward and backward are the library's kernels."""
+
+    @staticmethod
+    def forward(ctx, x, w, residual=True):
+        ctx.save_for_backward(x, w)
+        ctx.residual = residual
+        return dsc_fwd_headwise(x, w, residual)
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, w = ctx.saved_tensors
+        dx, dw = dsc_bwd_headwise(x, w, dy.contiguous(), ctx.residual)
+        return dx, dw, None
+
+
+class DynamicShortConvLowRank(torch.autograd.Function):
+    @staticmethod
+    def forward(ctx, x, z, U, H=1, residual=True):
+        ctx.save_for_backward(x, z, U)
+        ctx.H, ctx.residual = H, residual
+        return dsc_fwd_lowrank(x, z, U, H, residual)
+
+    @staticmethod
+    def backward(ctx, dy):
+        x, z, U = ctx.saved_tensors
+        dx, dz, dU = dsc_bwd_lowrank(x, z, U, dy.contiguous(), ctx.H, ctx.residual)
+        return dx, dz, dU.to(U.dtype), None, None

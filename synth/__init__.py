@@ -28,6 +28,7 @@ Storage: fp32 tensors are ``numpy.float32`` arrays, bf16 tensors are
 from __future__ import annotations
 
 import math
+import os
 
 import numpy as np
 
@@ -41,7 +42,7 @@ BF16 = "bf16"
 # Tensor ids of the stream keys (one stream per tensor role).
 TID_X, TID_W, TID_Z, TID_U, TID_DY, TID_WS = 1, 2, 3, 4, 5, 6
 
-_CHUNK = 1 << 22
+_CHUNK = 1 << 21
 
 
 def _mix64(z: np.ndarray) -> np.ndarray:
@@ -72,10 +73,14 @@ def splitmix_outputs(key: int, first: int, count: int) -> np.ndarray:
 
 
 def normals_f64(seed: int, tensor_id: int, n: int, start: int = 0) -> np.ndarray:
-    """Standard normals for elements start .. start+n-1 of one tensor, in fp64."""
+    """Standard normals for elements start .. start+n-1 of one tensor, in fp64.
+
+    Chunks are drawn on a thread pool; every element depends only on its
+    index, so the result does not depend on the chunking or thread count."""
     key = stream_key(seed, tensor_id)
     out = np.empty(n, dtype=np.float64)
-    for lo in range(0, n, _CHUNK):
+
+    def fill(lo):
         m = min(_CHUNK, n - lo)
         raw = splitmix_outputs(key, 2 * (start + lo), 2 * m)
         a = raw[0::2]
@@ -83,6 +88,16 @@ def normals_f64(seed: int, tensor_id: int, n: int, start: int = 0) -> np.ndarray
         u1 = ((a >> np.uint64(11)) + np.uint64(1)).astype(np.float64) * (2.0 ** -53)
         u2 = (b >> np.uint64(11)).astype(np.float64) * (2.0 ** -53)
         out[lo:lo + m] = np.sqrt(-2.0 * np.log(u1)) * np.cos(2.0 * math.pi * u2)
+
+    starts = range(0, n, _CHUNK)
+    if n <= _CHUNK:
+        for lo in starts:
+            fill(lo)
+    else:
+        from concurrent.futures import ThreadPoolExecutor
+
+        with ThreadPoolExecutor(max_workers=min(8, os.cpu_count() or 1)) as ex:
+            list(ex.map(fill, starts))
     return out
 
 

@@ -1,0 +1,109 @@
+"""The C ABI on a machine without a GPU: the library loads, exports every
+entry point include/dsc.h declares, and rejects bad arguments before any CUDA
+call (so these checks make no compute call)."""
+
+import ctypes as C
+import os
+import re
+import subprocess
+
+import pytest
+
+from input_dependent_short_b200 import _lib
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADERS = [os.path.join(ROOT, "include", f) for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")]
+
+
+def declared():
+    names = set()
+    for h in HEADERS:
+        src = open(h).read()
+        names |= set(re.findall(r"DSC_API\s+[\w\s\*]+?\b(dsc_\w+)\s*\(", src))
+    return names
+
+
+def test_header_declares_the_entry_points():
+    d = declared()
+    for n in ["dsc_fwd_headwise", "dsc_bwd_headwise", "dsc_fwd_lowrank", "dsc_bwd_lowrank", "dsc_fwd_static",
+              "dsc_bwd_static", "dsc_check", "dsc_status_string"]:
+        assert n in d
+
+
+def test_library_exports_every_declared_symbol():
+    L = _lib.lib()
+    out = subprocess.run(["nm", "-D", "--defined-only", _lib.LIB_PATH], capture_output=True, text=True, check=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    for n in declared():
+        assert n in exported, n
+        assert getattr(L, n) is not None
+    # nothing but the declared C ABI is exported
+    assert {e for e in exported if e.startswith("dsc_")} == declared()
+
+
+def test_every_binding_signature_is_declared():
+    assert set(_lib._SIGS) == declared()
+
+
+def test_version_and_status_strings():
+    assert _lib.lib().dsc_version() >= 100
+    assert _lib.status_string(_lib.DSC_OK) == "ok"
+    assert "aligned" in _lib.status_string(_lib.DSC_ERR_MISALIGNED)
+    assert "timed out" in _lib.status_string(_lib.DSC_ERR_TIMEOUT)
+    assert _lib.status_string(99) == "unknown status"
+
+
+def P(B=1, T=8, D=16, W=4, H=1, R=0, dtype=1, residual=1):
+    return _lib.DscProblem(B, T, D, W, H, R, dtype, residual)
+
+
+GOOD = 0x10000  # a 16-byte aligned, never dereferenced address
+
+
+@pytest.mark.parametrize("bad", [dict(B=0), dict(T=0), dict(D=0), dict(W=0), dict(W=9), dict(H=0), dict(D=10, H=4),
+                                 dict(dtype=7)])
+def test_invalid_problem_rejected(bad):
+    L = _lib.lib()
+    p = P(**bad)
+    assert L.dsc_fwd_headwise(C.byref(p), GOOD, GOOD, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_bwd_headwise(C.byref(p), GOOD, GOOD, GOOD, GOOD, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_fwd_static(C.byref(p), GOOD, GOOD, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_bwd_static_workspace_bytes(C.byref(p)) == 0
+
+
+@pytest.mark.parametrize("R", [0, 257])
+def test_invalid_rank_rejected(R):
+    L = _lib.lib()
+    p = P(R=R)
+    assert L.dsc_fwd_lowrank(C.byref(p), GOOD, GOOD, GOOD, GOOD, None, 0, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_bwd_lowrank(C.byref(p), GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, None, 0, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_fwd_lowrank_workspace_bytes(C.byref(p)) == 0
+
+
+def test_null_problem_and_pointers_rejected():
+    L = _lib.lib()
+    assert L.dsc_fwd_headwise(None, GOOD, GOOD, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
+    p = P()
+    assert L.dsc_fwd_headwise(C.byref(p), None, GOOD, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_bwd_headwise(C.byref(p), GOOD, GOOD, GOOD, GOOD, None, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_bwd_static(C.byref(p), GOOD, GOOD, GOOD, GOOD, GOOD, None, 0, None) == _lib.DSC_ERR_INVALID_ARG
+
+
+def test_misaligned_pointers_rejected():
+    L = _lib.lib()
+    p = P()
+    assert L.dsc_fwd_headwise(C.byref(p), GOOD + 2, GOOD, GOOD, None) == _lib.DSC_ERR_MISALIGNED
+    assert L.dsc_fwd_static(C.byref(p), GOOD, GOOD, GOOD + 8, None) == _lib.DSC_ERR_MISALIGNED
+    p.R = 4
+    assert L.dsc_fwd_lowrank(C.byref(p), GOOD, GOOD + 4, GOOD, GOOD, None, 0, None) == _lib.DSC_ERR_MISALIGNED
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+
+    from input_dependent_short_b200 import ops
+
+    x = torch.zeros(1, 4, 8, dtype=torch.bfloat16)
+    w = torch.zeros(1, 4, 8, 4, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        ops.dsc_fwd_headwise(x, w)

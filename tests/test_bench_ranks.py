@@ -1,0 +1,62 @@
+"""The N>1 path of bench.py on CPU: two gloo ranks, each with its own batch,
+the timing reduced as the max over ranks and the job value aggregated over
+ranks (data parallel; the path has no exchange step)."""
+
+import os
+import socket
+
+import torch.multiprocessing as mp
+
+import bench
+from synth import workloads as wls
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _rank(rank, world, port, q):
+    import torch.distributed as dist
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world),
+                      LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    wl = bench.rank_workload(wls.TINY_F32, rank)
+    t = wls.make_inputs(wl)
+    ms = 10.0 + 5.0 * rank  # rank 1 is the slow one
+    mx = bench.max_over_ranks(ms, world, "cpu")
+    q.put((rank, wl.seed, float(t["x"].reshape(-1)[0]), mx, bench.dist_env()))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_ranks_shard_batches_and_take_the_max_time():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = sorted(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    (r0, s0, x0, m0, env0), (r1, s1, x1, m1, env1) = out
+    assert (s0, s1) == (0, 1)          # each rank draws its own batch
+    assert x0 != x1
+    assert m0 == m1 == 15.0            # max over ranks
+    assert env0 == (2, 0, 0) and env1 == (2, 1, 1)
+    # whole-job tokens/s = all ranks' tokens / the slowest rank's time
+    assert bench.job_tokens_per_s(1000, 2, 10, 15.0) == 1000 * 2 * 10 / 0.015
+
+
+def test_algorithmic_bytes_of_the_headline_workload():
+    fb, bb = bench.step_bytes(wls.QKV_HEADWISE)
+    N, D, GW = 8 * 2048, 6144, 384 * 4
+    assert fb == N * (4 * D + 2 * GW)
+    assert bb == N * (6 * D + 4 * GW)
+    assert fb + bb == 1_157_627_904
