@@ -115,6 +115,30 @@ DSC_API size_t dsc_bwd_static_workspace_bytes(const dsc_problem *p);
 DSC_API dsc_status dsc_bwd_static(const dsc_problem *p, const void *x, const void *ws, const void *dy, void *dx, float *dws,
                           void *workspace, size_t workspace_bytes, void *stream);
 
+/* Size of the scratch array built into the library for
+ * dsc_bwd_static_noalloc (16 MiB per device that loads the library). */
+#define DSC_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+
+/* Static-filter backward that allocates nothing and takes no workspace.
+ * The paper has no counterpart: this exists for callers that cannot hand the
+ * library scratch memory -- plugin or custom-op interfaces that pass an
+ * operator only its inputs and outputs, and services that allocate all device
+ * memory at start-up and must not call cudaMalloc/cudaFree afterwards.
+ * Same arguments, results and errors as dsc_bwd_static, except:
+ *  - its scratch is an array of DSC_NOALLOC_SCRATCH_BYTES inside the library,
+ *    one per device, held from library load until process exit; a problem
+ *    whose scratch (dsc_bwd_static_workspace_bytes) exceeds that size is
+ *    rejected with DSC_ERR_UNSUPPORTED before anything is launched;
+ *  - the first call with a given device current looks the array's device
+ *    address up (cudaGetSymbolAddress); make that first call before any
+ *    stream capture on that device;
+ *  - all calls on a device share the one array: calls whose work overlaps on
+ *    the GPU (different streams without ordering between them) race and give
+ *    wrong results.  Each call writes every scratch element it reads, so the
+ *    array needs no clearing between calls. */
+DSC_API dsc_status dsc_bwd_static_noalloc(const dsc_problem *p, const void *x, const void *ws, const void *dy,
+                                          void *dx, float *dws, void *stream);
+
 /* Synchronise `stream`, then return and clear the device status word of the
  * current device: DSC_OK, DSC_ERR_TIMEOUT, or DSC_ERR_CUDA if the stream
  * reported an error. */
