@@ -178,6 +178,73 @@ template <typename T, int N> __device__ __forceinline__ void store_row(T *p, con
     for (int i = 0; i < N; ++i) p[i] = from_f<T>(f[i]);
 }
 
+// ------------------------------------------------------------ f32 pairs ---
+// sm_100 executes fma/mul/add on pairs of fp32 values in one instruction
+// (fma.rn.f32x2): each lane of the pair is an ordinary fp32 operation with
+// round-to-nearest, so results equal the scalar ones.
+
+typedef unsigned long long u64;
+
+__device__ __forceinline__ u64 mk2(float lo, float hi) {
+    u64 r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float lo2(u64 v) {
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+    (void)b;
+    return a;
+}
+__device__ __forceinline__ float hi2(u64 v) {
+    float a, b;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+    (void)a;
+    return b;
+}
+__device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {
+    u64 d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ u64 mul2(u64 a, u64 b) {
+    u64 d;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ u64 add2(u64 a, u64 b) {
+    u64 d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// 16 bytes of T <-> P pairs of fp32 (pair p holds channels 2p and 2p+1).
+template <typename T> struct Pairs;
+template <> struct Pairs<bf16> {
+    static constexpr int P = 4;
+    __device__ __forceinline__ static void unpack(const uint4 &u, u64 (&p)[4]) {
+        p[0] = mk2(bf_lo(u.x), bf_hi(u.x));
+        p[1] = mk2(bf_lo(u.y), bf_hi(u.y));
+        p[2] = mk2(bf_lo(u.z), bf_hi(u.z));
+        p[3] = mk2(bf_lo(u.w), bf_hi(u.w));
+    }
+    __device__ __forceinline__ static uint4 pack(const u64 (&p)[4]) {
+        return make_uint4(pack_bf2(lo2(p[0]), hi2(p[0])), pack_bf2(lo2(p[1]), hi2(p[1])),
+                          pack_bf2(lo2(p[2]), hi2(p[2])), pack_bf2(lo2(p[3]), hi2(p[3])));
+    }
+};
+template <> struct Pairs<float> {
+    static constexpr int P = 2;
+    __device__ __forceinline__ static void unpack(const uint4 &u, u64 (&p)[2]) {
+        p[0] = mk2(__uint_as_float(u.x), __uint_as_float(u.y));
+        p[1] = mk2(__uint_as_float(u.z), __uint_as_float(u.w));
+    }
+    __device__ __forceinline__ static uint4 pack(const u64 (&p)[2]) {
+        return make_uint4(__float_as_uint(lo2(p[0])), __float_as_uint(hi2(p[0])), __float_as_uint(lo2(p[1])),
+                          __float_as_uint(hi2(p[1])));
+    }
+};
+
 // Sum of v over the L consecutive lanes of this lane's segment (segments start
 // at multiples of L and lie inside the warp); the result is valid on the
 // segment's first lane.  Any 1 <= L <= 32.

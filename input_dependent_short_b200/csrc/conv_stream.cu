@@ -14,8 +14,10 @@
 //    sequence; the W-1 previous x rows live in registers (a sliding window),
 //    so x is read once, plus a (W-1)-row halo at the tile start (an L2 hit:
 //    the neighbouring tile streams the same rows at the same time);
-//  - loads of U_LD consecutive tokens are issued together before any of them
-//    is used, so each thread keeps several 16-byte requests in flight;
+//  - each thread keeps its next tokens' loads in flight through a private
+//    ring of shared-memory slots filled by cp.async (see "async copy ring");
+//  - the arithmetic runs on fp32 pairs (fma.rn.f32x2), two channels per
+//    instruction, and the residual is folded into tap 0 (w_0 + 1);
 //  - backward walks forward in time too: dx rows are finished W-1 tokens
 //    late from an accumulator window (row s collects w(s+k)_k dy_{s+k} as
 //    token s+k streams by), and the tile runs W-1 tokens past its end (right
@@ -29,8 +31,6 @@
 namespace dsc {
 
 constexpr int STREAM_THREADS = 256;
-
-__host__ __device__ constexpr int ld_batch(int wwords) { return wwords >= 16 ? 2 : (wwords >= 8 ? 4 : 8); }
 
 struct Pos {
     int64_t b;
@@ -56,226 +56,431 @@ __device__ __forceinline__ bool locate(const StreamMap &m, Pos &q) {
     return true;
 }
 
+// ------------------------------------------------------- async copy ring ---
+// Each thread streams its own tokens through a private ring of NS slots in
+// shared memory, filled with cp.async (LDGSTS) NS-1 tokens ahead of use, so
+// its next tokens' loads stay in flight while it computes without holding
+// registers.  A thread only reads slots it filled itself, so cp.async.wait_group
+// is the only synchronisation needed (no barriers, no spin loops).
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N> __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+__device__ __forceinline__ uint4 lds16(uint32_t a) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
+    return r;
+}
+
+constexpr int gcd_c(int a, int b) { return b == 0 ? a : gcd_c(b, a % b); }
+
+// The filter taps a thread needs per token (NW elements of T).  The start of
+// every such row is a multiple of AL = gcd(16, row bytes): the base pointer is
+// 16-byte aligned and both the token stride G*W and a thread's group offset
+// are multiples of the row length.  Rows with AL >= 4 travel through the ring
+// with cp.async; 2-byte aligned rows (odd W, bf16, one group per thread) are
+// read into a register ring instead.
+template <typename T, int NW> struct FiltRow {
+    static constexpr int BYTES = NW * (int)sizeof(T);
+    static constexpr int AL = gcd_c(16, BYTES);
+    static constexpr bool IN_SMEM = AL >= 4;
+    static constexpr int SLOTS = IN_SMEM ? (BYTES + 15) / 16 : 0;  // 16-byte ring slots
+    static constexpr int WORDS = (BYTES + 3) / 4;
+
+    __device__ __forceinline__ static void copy(uint32_t dst, uint32_t stride, const char *src) {
+        if constexpr (AL == 16) {
+#pragma unroll
+            for (int i = 0; i < BYTES / 16; ++i) cp_async16(dst + i * stride, src + 16 * i);
+        } else if constexpr (AL == 8) {
+#pragma unroll
+            for (int i = 0; i < BYTES / 8; ++i) cp_async8(dst + (i / 2) * stride + 8 * (i % 2), src + 8 * i);
+        } else if constexpr (AL == 4) {
+#pragma unroll
+            for (int i = 0; i < BYTES / 4; ++i) cp_async4(dst + (i / 4) * stride + 4 * (i % 4), src + 4 * i);
+        }
+    }
+
+    // Read back the words of a row that went through the ring.
+    __device__ __forceinline__ static void read(uint32_t src, uint32_t stride, uint32_t (&w)[WORDS]) {
+#pragma unroll
+        for (int i = 0; i < SLOTS; ++i) {
+            uint4 v = lds16(src + i * stride);
+            if (4 * i + 0 < WORDS) w[4 * i + 0] = v.x;
+            if (4 * i + 1 < WORDS) w[4 * i + 1] = v.y;
+            if (4 * i + 2 < WORDS) w[4 * i + 2] = v.z;
+            if (4 * i + 3 < WORDS) w[4 * i + 3] = v.w;
+        }
+    }
+
+    // Direct read of a row with plain loads (element by element).
+    __device__ __forceinline__ static void load_direct(const char *src, uint32_t (&w)[WORDS]) {
+        if constexpr (sizeof(T) == 4) {
+#pragma unroll
+            for (int i = 0; i < NW; ++i) w[i] = __ldg(reinterpret_cast<const uint32_t *>(src) + i);
+        } else {
+            const unsigned short *q = reinterpret_cast<const unsigned short *>(src);
+#pragma unroll
+            for (int i = 0; i < WORDS; ++i) w[i] = 0u;
+#pragma unroll
+            for (int i = 0; i < NW; ++i) w[i >> 1] |= (uint32_t)__ldg(q + i) << (16 * (i & 1));
+        }
+    }
+
+    __device__ __forceinline__ static float get(const uint32_t (&w)[WORDS], int i) {
+        if constexpr (sizeof(T) == 4) return __uint_as_float(w[i]);
+        else return (i & 1) ? bf_hi(w[i >> 1]) : bf_lo(w[i >> 1]);
+    }
+};
+
+// Ring depth (tokens) for a given number of 16-byte slots per token, keeping
+// the ring at <= 96 KB for a 256-thread block (two blocks per SM).
+__host__ __device__ constexpr int ring_depth(int slots) {
+    return slots * 16 * 8 <= 384 ? 8 : (384 / (slots * 16) < 2 ? 2 : 384 / (slots * 16));
+}
+
+template <typename T, int W, int GPT, bool WS, bool BWD> struct StreamCfg {
+    static constexpr int V = VecOf<T>::V;
+    static constexpr int NW = WS ? V * W : GPT * W;  // filter taps per token per thread
+    static constexpr int CPG = WS ? 1 : V / GPT;      // channels sharing one filter inside a thread
+    static constexpr int WIN = W - 1;
+    using F = FiltRow<T, NW>;
+    static constexpr bool WRING = !WS && F::IN_SMEM;  // filter rows through the shared ring
+    static constexpr bool WREG = !WS && !F::IN_SMEM;  // filter rows through a register ring
+    static constexpr int SUB = (BWD ? 2 : 1) + (WRING ? F::SLOTS : 0);  // 16-byte slots per token
+    static constexpr int NS = ring_depth(SUB);
+    static constexpr size_t SMEM = (size_t)NS * SUB * 16 * STREAM_THREADS;
+    // Blocks per SM the register budget is sized for: the narrow head-wise
+    // filters fit 3 (forward) / 2 (backward) blocks of 256 threads; wider or
+    // per-channel (static) filters need more registers per thread.
+    static constexpr int MINB = BWD ? ((!WS && W <= 4) || (WS && W <= 2) ? 2 : 1)
+                                    : ((!WS && W <= 4) ? 3 : (W <= 3 ? 2 : 1));
+};
+
+template <typename T, int W, int GPT, bool WS, bool BWD>
+size_t stream_smem() { return StreamCfg<T, W, GPT, WS, BWD>::SMEM; }
+
+template <bool B> struct BoolC { static constexpr bool value = B; };
+
+// Tap k of the filters of channel pair p (channels 2p, 2p+1 of the thread's
+// vector) as an fp32 pair; `add` is added to both (the residual on tap 0).
+template <typename F, int W, int CPG>
+__device__ __forceinline__ u64 tap2(const uint32_t (&wv)[F::WORDS], int p, int k, float add = 0.f) {
+    const int g0 = (2 * p) / CPG, g1 = (2 * p + 1) / CPG;
+    const float a = F::get(wv, g0 * W + k) + add;
+    if (g0 == g1) return mk2(a, a);
+    return mk2(a, F::get(wv, g1 * W + k) + add);
+}
+
+// Sum part[k] (k < N) over the L lanes of a filter group; afterwards the
+// group's first lane holds the sums (every lane, when L is a power of two).
+template <int N>
+__device__ __forceinline__ void group_reduce(float (&part)[N], int L, int pos) {
+    if ((L & (L - 1)) == 0) {
+        for (int o = 1; o < L; o <<= 1)
+#pragma unroll
+            for (int k = 0; k < N; ++k) part[k] += __shfl_xor_sync(FULL_MASK, part[k], o);
+    } else {
+        for (int o = 1; o < L; o <<= 1)
+#pragma unroll
+            for (int k = 0; k < N; ++k) {
+                const float t = __shfl_down_sync(FULL_MASK, part[k], o);
+                if (pos + o < L) part[k] += t;
+            }
+    }
+}
+
 // ---------------------------------------------------------------- forward ---
 
-// WSTATIC = false: head-wise filters w[b,t,g,k] read per token.
-// WSTATIC = true : static filters ws[c,k] read once per thread.
-template <typename T, int W, int GPT, bool WSTATIC>
-__global__ void __launch_bounds__(STREAM_THREADS) k_stream_fwd(const HwArgs a) {
-    constexpr int V = VecOf<T>::V;
-    constexpr int NW = WSTATIC ? V * W : GPT * W;  // filter taps a thread needs per token
-    constexpr int CPG = WSTATIC ? 1 : V / GPT;      // channels per filter (within the thread)
-    constexpr int UL = ld_batch(Row<T, NW>::WORDS);
-    constexpr int WIN = W > 1 ? W - 1 : 1;
+// WS = false: head-wise filters w[b,t,g,k] read per token.
+// WS = true : static filters ws[c,k] read once per thread.
+template <typename T, int W, int GPT, bool WS>
+__global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, false>::MINB)) k_stream_fwd(const HwArgs a) {
+    using C = StreamCfg<T, W, GPT, WS, false>;
+    using F = typename C::F;
+    using PR = Pairs<T>;
+    constexpr int P = PR::P, NS = C::NS, WIN = C::WIN, XW = WIN > 0 ? WIN : 1, CPG = C::CPG;
+    extern __shared__ uint4 ring[];
     const StreamMap &m = a.m;
     Pos q;
-    if (!locate<V>(m, q) || !q.active) return;
+    if (!locate<VecOf<T>::V>(m, q) || !q.active) return;
 
-    const int64_t row0 = q.b * m.T;
-    const T *xb = static_cast<const T *>(a.x) + row0 * m.D + q.c0;
-    T *yb = static_cast<T *>(a.y) + row0 * m.D + q.c0;
-    const T *wb = WSTATIC ? static_cast<const T *>(a.w) + q.c0 * W
-                          : static_cast<const T *>(a.w) + row0 * m.G * W + (q.c0 / m.H) * W;
-    const int64_t wstride = WSTATIC ? 0 : m.G * W;
-
-    Row<T, NW> wst;
-    if constexpr (WSTATIC) wst.load(wb);
-
-    float win[WIN][V];
-#pragma unroll
-    for (int j = 0; j < WIN; ++j) {
-        const int t = q.t_start - 1 - j;
-        if (W > 1 && t >= 0) {
-            unpack(ld16(xb + (int64_t)t * m.D), win[j]);
-        } else {
-#pragma unroll
-            for (int v = 0; v < V; ++v) win[j][v] = 0.f;
-        }
-    }
+    const int n = q.t_end - q.t_start;
+    const int64_t xstep = m.D * (int64_t)sizeof(T);
+    const int64_t wstep = WS ? 0 : m.G * W * (int64_t)sizeof(T);
+    const int64_t row = q.b * m.T + q.t_start;
+    const char *xp = static_cast<const char *>(a.x) + (row * m.D + q.c0) * (int64_t)sizeof(T);
+    char *yp = static_cast<char *>(a.y) + (row * m.D + q.c0) * (int64_t)sizeof(T);
+    const char *wp = WS ? static_cast<const char *>(a.w) + q.c0 * W * (int64_t)sizeof(T)
+                        : static_cast<const char *>(a.w) + (row * m.G + q.c0 / m.H) * W * (int64_t)sizeof(T);
     const float res = m.residual ? 1.f : 0.f;
 
-    for (int t = q.t_start; t < q.t_end; t += UL) {
-        uint4 xr[UL];
-        Row<T, NW> wr[UL];
+    const uint32_t base = (uint32_t)__cvta_generic_to_shared(ring) + 16u * threadIdx.x;
+    constexpr uint32_t SUBSTRIDE = 16u * STREAM_THREADS;
+    auto slot = [&](int s, int sub) { return base + (uint32_t)(s * C::SUB + sub) * SUBSTRIDE; };
+
+    u64 wsp[WS ? P : 1][WS ? W : 1];  // static filters as pairs (tap 0 carries the residual)
+    if constexpr (WS) {
+        uint32_t wst[F::WORDS];
+        F::load_direct(wp, wst);
 #pragma unroll
-        for (int u = 0; u < UL; ++u) {
-            if (t + u < q.t_end) {
-                xr[u] = ld16(xb + (int64_t)(t + u) * m.D);
-                if constexpr (!WSTATIC) wr[u].load(wb + (int64_t)(t + u) * wstride);
-            } else {
-                xr[u] = make_uint4(0, 0, 0, 0);
-                if constexpr (!WSTATIC) wr[u].zero();
-            }
-        }
+        for (int pp = 0; pp < P; ++pp)
 #pragma unroll
-        for (int u = 0; u < UL; ++u) {
-            const Row<T, NW> &wv = WSTATIC ? wst : wr[u];
-            float xc[V], acc[V];
-            unpack(xr[u], xc);
-#pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const int f = WSTATIC ? v * W : (v / CPG) * W;
-                float s = res * xc[v];
-                s = fmaf(wv.get(f), xc[v], s);
-#pragma unroll
-                for (int k = 1; k < W; ++k) s = fmaf(wv.get(f + k), win[k - 1][v], s);
-                acc[v] = s;
-            }
-            if (t + u < q.t_end) st16(yb + (int64_t)(t + u) * m.D, pack(acc));
-#pragma unroll
-            for (int j = WIN - 1; j > 0; --j)
-#pragma unroll
-                for (int v = 0; v < V; ++v) win[j][v] = win[j - 1][v];
-#pragma unroll
-            for (int v = 0; v < V; ++v) win[0][v] = xc[v];
-        }
+            for (int k = 0; k < W; ++k) wsp[pp][k] = tap2<F, W, CPG>(wst, pp, k, k == 0 ? res : 0.f);
     }
+    uint32_t wreg[C::WREG ? NS : 1][F::WORDS];
+
+    auto issue = [&](int i, int s, bool full) {
+        if (full || i < n) {
+            cp_async16(slot(s, 0), xp + i * xstep);
+            if constexpr (C::WRING) F::copy(slot(s, 1), SUBSTRIDE, wp + i * wstep);
+            if constexpr (C::WREG) F::load_direct(wp + i * wstep, wreg[s]);
+        }
+        cp_commit();
+    };
+
+    u64 xs[XW][P];  // xs[j] = x[t-1-j]
+#pragma unroll
+    for (int j = 0; j < XW; ++j) {
+        const int t = q.t_start - 1 - j;
+        if (WIN > 0 && t >= 0) PR::unpack(ld16(xp - (int64_t)(1 + j) * xstep), xs[j]);
+        else
+#pragma unroll
+            for (int pp = 0; pp < P; ++pp) xs[j][pp] = 0ull;
+    }
+#pragma unroll
+    for (int j = 0; j < NS - 1; ++j) issue(j, j, false);
+
+    auto group = [&](int i0, auto fulltag) {
+        constexpr bool FULL = decltype(fulltag)::value;
+#pragma unroll
+        for (int u = 0; u < NS; ++u) {
+            const int i = i0 + u;
+            if (!FULL && i >= n) break;
+            issue(i + NS - 1, (u + NS - 1) % NS, FULL);
+            cp_wait<NS - 1>();
+            u64 xc[P], acc[P];
+            PR::unpack(lds16(slot(u, 0)), xc);
+            uint32_t wv[F::WORDS];
+            if constexpr (C::WRING) F::read(slot(u, 1), SUBSTRIDE, wv);
+            if constexpr (C::WREG)
+#pragma unroll
+                for (int k = 0; k < F::WORDS; ++k) wv[k] = wreg[u][k];
+#pragma unroll
+            for (int pp = 0; pp < P; ++pp) {
+                u64 s = mul2(WS ? wsp[pp][0] : tap2<F, W, CPG>(wv, pp, 0, res), xc[pp]);
+#pragma unroll
+                for (int k = 1; k < W; ++k) s = fma2(WS ? wsp[pp][k] : tap2<F, W, CPG>(wv, pp, k), xs[k - 1][pp], s);
+                acc[pp] = s;
+            }
+            st16(yp + i * xstep, PR::pack(acc));
+#pragma unroll
+            for (int j = XW - 1; j > 0; --j)
+#pragma unroll
+                for (int pp = 0; pp < P; ++pp) xs[j][pp] = xs[j - 1][pp];
+#pragma unroll
+            for (int pp = 0; pp < P; ++pp) xs[0][pp] = xc[pp];
+        }
+    };
+    int i0 = 0;
+    for (; i0 + 2 * NS - 1 <= n; i0 += NS) group(i0, BoolC<true>{});
+    for (; i0 < n; i0 += NS) group(i0, BoolC<false>{});
+    cp_wait<0>();
 }
 
 // --------------------------------------------------------------- backward ---
 
-template <typename T, int W, int GPT, bool WSTATIC>
-__global__ void __launch_bounds__(STREAM_THREADS) k_stream_bwd(const HwArgs a) {
-    constexpr int V = VecOf<T>::V;
-    constexpr int NW = WSTATIC ? V * W : GPT * W;
-    constexpr int CPG = WSTATIC ? 1 : V / GPT;
-    constexpr int UL = ld_batch(Row<T, NW>::WORDS) > 4 ? 4 : ld_batch(Row<T, NW>::WORDS);
-    constexpr int WIN = W > 1 ? W - 1 : 1;
+template <typename T, int W, int GPT, bool WS>
+__global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true>::MINB)) k_stream_bwd(const HwArgs a) {
+    using C = StreamCfg<T, W, GPT, WS, true>;
+    using F = typename C::F;
+    using PR = Pairs<T>;
+    constexpr int P = PR::P, NS = C::NS, WIN = C::WIN, XW = WIN > 0 ? WIN : 1, CPG = C::CPG;
+    constexpr int PPG = CPG >= 2 ? CPG / 2 : 1;  // channel pairs per filter group (CPG >= 2)
+    extern __shared__ uint4 ring[];
     const StreamMap &m = a.m;
     Pos q;
-    if (!locate<V>(m, q)) return;  // whole warp out of range
+    if (!locate<VecOf<T>::V>(m, q)) return;  // whole warp out of range; partial warps stay for the shuffles
+    // Inactive lanes (no channels of their own) stream channel 0 of the same rows: in bounds, never
+    // stored, and never in a filter group with an active lane.
     const bool act = q.active;
     const int L = m.L;
-    const int pos = q.lane % (L > 0 ? L : 1);
+    const int pos = q.lane % L;
 
-    const int64_t row0 = q.b * m.T;
+    const int n = q.t_end - q.t_start;                                   // tokens owned
+    const int nl = (int)(min((int64_t)q.t_end + WIN, m.T) - q.t_start);  // tokens with dy and w
+    const int niter = n + WIN;                                            // tokens streamed
     const int64_t c0 = act ? q.c0 : 0;
-    const T *xb = static_cast<const T *>(a.x) + row0 * m.D + c0;
-    const T *dyb = static_cast<const T *>(a.dy) + row0 * m.D + c0;
-    T *dxb = static_cast<T *>(a.dx) + row0 * m.D + c0;
-    const int64_t g0 = c0 / m.H;
-    const T *wb = WSTATIC ? static_cast<const T *>(a.w) + c0 * W
-                          : static_cast<const T *>(a.w) + row0 * m.G * W + g0 * W;
-    T *dwb = WSTATIC ? nullptr : static_cast<T *>(a.dw) + row0 * m.G * W + g0 * W;
-    const int64_t wstride = WSTATIC ? 0 : m.G * W;
-
-    Row<T, NW> wst;
-    if constexpr (WSTATIC) {
-        if (act) wst.load(wb); else wst.zero();
-    }
-    float dws[WSTATIC ? V : 1][WSTATIC ? W : 1];
-    if constexpr (WSTATIC) {
-#pragma unroll
-        for (int v = 0; v < V; ++v)
-#pragma unroll
-            for (int k = 0; k < W; ++k) dws[v][k] = 0.f;
-    }
-
-    float xw[WIN][V];   // xw[j] = x[t-1-j]
-    float acc[WIN][V];  // acc[j] = partial dx of row t-1-j
-#pragma unroll
-    for (int j = 0; j < WIN; ++j) {
-        const int t = q.t_start - 1 - j;
-        if (W > 1 && act && t >= 0) {
-            unpack(ld16(xb + (int64_t)t * m.D), xw[j]);
-        } else {
-#pragma unroll
-            for (int v = 0; v < V; ++v) xw[j][v] = 0.f;
-        }
-#pragma unroll
-        for (int v = 0; v < V; ++v) acc[j][v] = 0.f;
-    }
+    const int64_t xstep = m.D * (int64_t)sizeof(T);
+    const int64_t wstep = WS ? 0 : m.G * W * (int64_t)sizeof(T);
+    const int64_t row = q.b * m.T + q.t_start;
+    const char *xp = static_cast<const char *>(a.x) + (row * m.D + c0) * (int64_t)sizeof(T);
+    const char *dyp = static_cast<const char *>(a.dy) + (row * m.D + c0) * (int64_t)sizeof(T);
+    char *dxp = static_cast<char *>(a.dx) + (row * m.D + c0) * (int64_t)sizeof(T);
+    const char *wp = WS ? static_cast<const char *>(a.w) + c0 * W * (int64_t)sizeof(T)
+                        : static_cast<const char *>(a.w) + (row * m.G + c0 / m.H) * W * (int64_t)sizeof(T);
+    char *dwp = WS ? nullptr : static_cast<char *>(a.dw) + (row * m.G + c0 / m.H) * W * (int64_t)sizeof(T);
     const float res = m.residual ? 1.f : 0.f;
-    const int t_stop = q.t_end + W - 1;  // right halo: W-1 extra tokens finish the last rows
-    const int t_lim = (int)min((int64_t)t_stop, m.T);
 
-    for (int t = q.t_start; t < t_stop; t += UL) {
-        uint4 xr[UL], dr[UL];
-        Row<T, NW> wr[UL];
+    const uint32_t base = (uint32_t)__cvta_generic_to_shared(ring) + 16u * threadIdx.x;
+    constexpr uint32_t SUBSTRIDE = 16u * STREAM_THREADS;
+    auto slot = [&](int s, int sub) { return base + (uint32_t)(s * C::SUB + sub) * SUBSTRIDE; };
+
+    u64 wsp[WS ? P : 1][WS ? W : 1];
+    u64 dws[WS ? P : 1][WS ? W : 1];
+    if constexpr (WS) {
+        uint32_t wst[F::WORDS];
+        F::load_direct(wp, wst);
 #pragma unroll
-        for (int u = 0; u < UL; ++u) {
-            const int tt = t + u;
-            xr[u] = (act && tt < q.t_end) ? ld16(xb + (int64_t)tt * m.D) : make_uint4(0, 0, 0, 0);
-            dr[u] = (act && tt < t_lim) ? ld16(dyb + (int64_t)tt * m.D) : make_uint4(0, 0, 0, 0);
-            if constexpr (!WSTATIC) {
-                if (act && tt < t_lim) wr[u].load(wb + (int64_t)tt * wstride); else wr[u].zero();
+        for (int pp = 0; pp < P; ++pp)
+#pragma unroll
+            for (int k = 0; k < W; ++k) {
+                wsp[pp][k] = tap2<F, W, CPG>(wst, pp, k, k == 0 ? res : 0.f);
+                dws[pp][k] = 0ull;
             }
+    }
+    uint32_t wreg[C::WREG ? NS : 1][F::WORDS];
+
+    auto issue = [&](int i, int s, bool full) {
+        if (full || i < n) cp_async16(slot(s, 0), xp + i * xstep);
+        if (full || i < nl) {
+            cp_async16(slot(s, 1), dyp + i * xstep);
+            if constexpr (C::WRING) F::copy(slot(s, 2), SUBSTRIDE, wp + i * wstep);
+            if constexpr (C::WREG) F::load_direct(wp + i * wstep, wreg[s]);
         }
+        cp_commit();
+    };
+
+    u64 xs[XW][P];   // xs[j] = x[t-1-j]
+    u64 acc[XW][P];  // acc[j] = partial dx of row t-1-j
 #pragma unroll
-        for (int u = 0; u < UL; ++u) {
-            const int tt = t + u;
-            const Row<T, NW> &wv = WSTATIC ? wst : wr[u];
-            float xc[V], dyc[V], r0[V];
-            unpack(xr[u], xc);
-            unpack(dr[u], dyc);
-            const bool main = tt < q.t_end;
-            // dx: token tt feeds row tt-k through tap k of w(tt).
+    for (int j = 0; j < XW; ++j) {
+        const int t = q.t_start - 1 - j;
+        if (WIN > 0 && t >= 0) PR::unpack(ld16(xp - (int64_t)(1 + j) * xstep), xs[j]);
+        else
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                const int f = WSTATIC ? v * W : (v / CPG) * W;
-                r0[v] = fmaf(wv.get(f), dyc[v], main ? res * dyc[v] : 0.f);
+            for (int pp = 0; pp < P; ++pp) xs[j][pp] = 0ull;
 #pragma unroll
-                for (int k = 1; k < W; ++k) acc[k - 1][v] = fmaf(wv.get(f + k), dyc[v], acc[k - 1][v]);
+        for (int pp = 0; pp < P; ++pp) acc[j][pp] = 0ull;
+    }
+#pragma unroll
+    for (int j = 0; j < NS - 1; ++j) issue(j, j, false);
+
+    auto group = [&](int i0, auto fulltag) {
+        constexpr bool FULL = decltype(fulltag)::value;
+#pragma unroll
+        for (int u = 0; u < NS; ++u) {
+            const int i = i0 + u;
+            if (!FULL && i >= niter) break;
+            issue(i + NS - 1, (u + NS - 1) % NS, FULL);
+            cp_wait<NS - 1>();
+            const bool hx = FULL || i < n, hd = FULL || i < nl;
+            u64 xc[P], dyc[P], r0[P];
+            uint32_t wv[F::WORDS];
+            if (hx) PR::unpack(lds16(slot(u, 0)), xc);
+            else
+#pragma unroll
+                for (int pp = 0; pp < P; ++pp) xc[pp] = 0ull;
+            if (hd) {
+                PR::unpack(lds16(slot(u, 1)), dyc);
+                if constexpr (C::WRING) F::read(slot(u, 2), SUBSTRIDE, wv);
+                if constexpr (C::WREG)
+#pragma unroll
+                    for (int k = 0; k < F::WORDS; ++k) wv[k] = wreg[u][k];
+            } else {
+#pragma unroll
+                for (int pp = 0; pp < P; ++pp) dyc[pp] = 0ull;
+#pragma unroll
+                for (int k = 0; k < F::WORDS; ++k) wv[k] = 0u;
             }
-            // row tt-(W-1) is complete
-            const int done = tt - (W - 1);
-            if (act && done >= q.t_start && done < q.t_end) {
-                if constexpr (W > 1) st16(dxb + (int64_t)done * m.D, pack(acc[WIN - 1]));
-                else st16(dxb + (int64_t)done * m.D, pack(r0));
+            // dx: token i feeds row i-k through tap k of w(i); row i itself starts
+            // with the residual (rows past the tile are never stored).
+#pragma unroll
+            for (int pp = 0; pp < P; ++pp) {
+                r0[pp] = mul2(WS ? wsp[pp][0] : tap2<F, W, CPG>(wv, pp, 0, res), dyc[pp]);
+#pragma unroll
+                for (int k = 1; k < W; ++k)
+                    acc[k - 1][pp] = fma2(WS ? wsp[pp][k] : tap2<F, W, CPG>(wv, pp, k), dyc[pp], acc[k - 1][pp]);
             }
-            // dw(tt)_k = sum over the group's channels of dy_tt * x_{tt-k}
-            if (tt < q.t_end) {
-                if constexpr (WSTATIC) {
+            if (act && i >= WIN) {  // row i-WIN is complete
+                if constexpr (W > 1) st16(dxp + (i - WIN) * xstep, PR::pack(acc[XW - 1]));
+                else st16(dxp + (i - WIN) * xstep, PR::pack(r0));
+            }
+            // dw(i)_k = sum over the group's channels of dy_i * x_{i-k}
+            if (FULL || i < n) {
+                if constexpr (WS) {
 #pragma unroll
-                    for (int v = 0; v < V; ++v) {
-                        dws[v][0] = fmaf(dyc[v], xc[v], dws[v][0]);
+                    for (int pp = 0; pp < P; ++pp)
 #pragma unroll
-                        for (int k = 1; k < W; ++k) dws[v][k] = fmaf(dyc[v], xw[k - 1][v], dws[v][k]);
-                    }
+                        for (int k = 0; k < W; ++k) dws[pp][k] = fma2(dyc[pp], k == 0 ? xc[pp] : xs[k - 1][pp], dws[pp][k]);
+                } else if constexpr (CPG == 1) {
+                    float part[GPT * W];
+#pragma unroll
+                    for (int pp = 0; pp < P; ++pp)
+#pragma unroll
+                        for (int k = 0; k < W; ++k) {
+                            const u64 d = mul2(dyc[pp], k == 0 ? xc[pp] : xs[k - 1][pp]);
+                            part[(2 * pp) * W + k] = lo2(d);
+                            part[(2 * pp + 1) * W + k] = hi2(d);
+                        }
+                    if (act) store_row<T, GPT * W>(reinterpret_cast<T *>(dwp + i * wstep), part);
                 } else {
                     float part[GPT * W];
 #pragma unroll
-                    for (int gi = 0; gi < GPT; ++gi) {
+                    for (int gi = 0; gi < GPT; ++gi)
 #pragma unroll
                         for (int k = 0; k < W; ++k) {
-                            float s = 0.f;
+                            u64 s2 = mul2(dyc[gi * PPG], k == 0 ? xc[gi * PPG] : xs[k - 1][gi * PPG]);
 #pragma unroll
-                            for (int v = gi * CPG; v < (gi + 1) * CPG; ++v) s = fmaf(dyc[v], k == 0 ? xc[v] : xw[k - 1][v], s);
-                            part[gi * W + k] = s;
+                            for (int pp = gi * PPG + 1; pp < (gi + 1) * PPG; ++pp)
+                                s2 = fma2(dyc[pp], k == 0 ? xc[pp] : xs[k - 1][pp], s2);
+                            part[gi * W + k] = lo2(s2) + hi2(s2);
                         }
-                    }
                     if (GPT == 1 && L > 1) {
-#pragma unroll
-                        for (int k = 0; k < W; ++k) part[k] = segment_sum(part[k], L, pos);
-                        if (act && pos == 0) store_row<T, GPT * W>(dwb + (int64_t)tt * wstride, part);
+                        group_reduce<GPT * W>(part, L, pos);
+                        if (act && pos == 0) store_row<T, GPT * W>(reinterpret_cast<T *>(dwp + i * wstep), part);
                     } else if (act) {
-                        store_row<T, GPT * W>(dwb + (int64_t)tt * wstride, part);
+                        store_row<T, GPT * W>(reinterpret_cast<T *>(dwp + i * wstep), part);
                     }
                 }
             }
-            // shift windows
 #pragma unroll
-            for (int j = WIN - 1; j > 0; --j)
+            for (int j = XW - 1; j > 0; --j)
 #pragma unroll
-                for (int v = 0; v < V; ++v) {
-                    acc[j][v] = acc[j - 1][v];
-                    xw[j][v] = xw[j - 1][v];
+                for (int pp = 0; pp < P; ++pp) {
+                    acc[j][pp] = acc[j - 1][pp];
+                    xs[j][pp] = xs[j - 1][pp];
                 }
 #pragma unroll
-            for (int v = 0; v < V; ++v) {
-                acc[0][v] = r0[v];
-                xw[0][v] = xc[v];
+            for (int pp = 0; pp < P; ++pp) {
+                acc[0][pp] = r0[pp];
+                xs[0][pp] = xc[pp];
             }
         }
-    }
-    if constexpr (WSTATIC) {
+    };
+    int i0 = 0;
+    for (; i0 + 2 * NS - 1 <= n; i0 += NS) group(i0, BoolC<true>{});
+    for (; i0 < niter; i0 += NS) group(i0, BoolC<false>{});
+    cp_wait<0>();
+    if constexpr (WS) {
         if (act) {
             const int64_t s = q.b * m.nTiles + q.t_start / m.Tt;
             float *pp = a.partial + (s * m.D + c0) * W;
 #pragma unroll
-            for (int v = 0; v < V; ++v)
+            for (int p2 = 0; p2 < P; ++p2)
 #pragma unroll
-                for (int k = 0; k < W; ++k) pp[v * W + k] = dws[v][k];
+                for (int k = 0; k < W; ++k) {
+                    pp[(2 * p2) * W + k] = lo2(dws[p2][k]);
+                    pp[(2 * p2 + 1) * W + k] = hi2(dws[p2][k]);
+                }
         }
     }
 }
@@ -324,14 +529,14 @@ bool stream_map(const dsc_problem &p, int V, StreamMap &m) {
     return true;
 }
 
-// Pick the tile length so that all warps are resident at once (one wave),
-// with at least 32 tokens per tile to keep the (W-1)-row halo small.
+// Pick the tile length so that all warps are resident at once (exactly one
+// wave): the largest number of time tiles whose warps all fit on the GPU.
 void finish_map(StreamMap &m, int64_t target_warps) {
     const int64_t cols = m.B * m.nWc;
-    int64_t tt = (m.T * cols + target_warps - 1) / target_warps;
-    tt = ((tt + 7) / 8) * 8;
-    if (tt < 32) tt = 32;
-    if (tt > m.T) tt = m.T;
+    int64_t tiles = target_warps / cols;
+    if (tiles < 1) tiles = 1;
+    if (tiles > m.T) tiles = m.T;
+    const int64_t tt = (m.T + tiles - 1) / tiles;
     m.Tt = (int)tt;
     m.nTiles = (int)((m.T + tt - 1) / tt);
     m.n_warps = m.B * m.nTiles * (int64_t)m.nWc;
@@ -343,14 +548,28 @@ static const void *stream_kernel() {
     else return (const void *)k_stream_fwd<T, W, GPT, WS>;
 }
 
+// Dynamic shared memory of one instantiation, set up once (thread-safe).
+template <typename T, int W, int GPT, bool WS, bool BWD>
+static size_t stream_setup(int &per_sm_warps) {
+    static const size_t smem = stream_smem<T, W, GPT, WS, BWD>();
+    static const int blocks = [] {
+        const void *k = stream_kernel<T, W, GPT, WS, BWD>();
+        cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        cudaGetLastError();
+        return resident_blocks(k, STREAM_THREADS, smem);
+    }();
+    per_sm_warps = blocks * (STREAM_THREADS / 32);
+    return smem;
+}
+
 template <typename T, int W, int GPT, bool WS, bool BWD>
 static cudaError_t run_stream(const Ctx &c, HwArgs a) {
-    const void *k = stream_kernel<T, W, GPT, WS, BWD>();
-    const int per_sm = resident_blocks(k, STREAM_THREADS, 0) * (STREAM_THREADS / 32);
+    int per_sm = 0;
+    const size_t smem = stream_setup<T, W, GPT, WS, BWD>(per_sm);
     finish_map(a.m, (int64_t)per_sm * c.sms);
     const int64_t blocks = (a.m.n_warps + STREAM_THREADS / 32 - 1) / (STREAM_THREADS / 32);
-    if constexpr (BWD) { k_stream_bwd<T, W, GPT, WS><<<(unsigned)blocks, STREAM_THREADS, 0, c.stream>>>(a); count_launch(); }
-    else { k_stream_fwd<T, W, GPT, WS><<<(unsigned)blocks, STREAM_THREADS, 0, c.stream>>>(a); count_launch(); }
+    if constexpr (BWD) { k_stream_bwd<T, W, GPT, WS><<<(unsigned)blocks, STREAM_THREADS, smem, c.stream>>>(a); count_launch(); }
+    else { k_stream_fwd<T, W, GPT, WS><<<(unsigned)blocks, STREAM_THREADS, smem, c.stream>>>(a); count_launch(); }
     return cudaGetLastError();
 }
 
@@ -401,23 +620,26 @@ cudaError_t launch_st_bwd(const Ctx &c, const dsc_problem &p, HwArgs a, float *d
     return launch_reduce_partials(c, a.partial, st_partial_count(c, p), p.D * p.W, dws);
 }
 
+template <typename T, int W> static int64_t st_tiles_w(const Ctx &c, StreamMap m) {
+    int per_sm = 0;
+    stream_setup<T, W, 1, true, true>(per_sm);
+    finish_map(m, (int64_t)per_sm * c.sms);
+    return m.B * m.nTiles;
+}
+
 template <typename T> static int64_t st_tiles(const Ctx &c, const dsc_problem &p) {
     StreamMap m;
     stream_map(p, VecOf<T>::V, m);
-    const void *k = nullptr;
     switch (p.W) {
-    case 1: k = stream_kernel<T, 1, 1, true, true>(); break;
-    case 2: k = stream_kernel<T, 2, 1, true, true>(); break;
-    case 3: k = stream_kernel<T, 3, 1, true, true>(); break;
-    case 4: k = stream_kernel<T, 4, 1, true, true>(); break;
-    case 5: k = stream_kernel<T, 5, 1, true, true>(); break;
-    case 6: k = stream_kernel<T, 6, 1, true, true>(); break;
-    case 7: k = stream_kernel<T, 7, 1, true, true>(); break;
-    default: k = stream_kernel<T, 8, 1, true, true>(); break;
+    case 1: return st_tiles_w<T, 1>(c, m);
+    case 2: return st_tiles_w<T, 2>(c, m);
+    case 3: return st_tiles_w<T, 3>(c, m);
+    case 4: return st_tiles_w<T, 4>(c, m);
+    case 5: return st_tiles_w<T, 5>(c, m);
+    case 6: return st_tiles_w<T, 6>(c, m);
+    case 7: return st_tiles_w<T, 7>(c, m);
+    default: return st_tiles_w<T, 8>(c, m);
     }
-    const int per_sm = resident_blocks(k, STREAM_THREADS, 0) * (STREAM_THREADS / 32);
-    finish_map(m, (int64_t)per_sm * c.sms);
-    return m.B * m.nTiles;
 }
 
 // Number of partial gradients the static backward writes (fast path).
