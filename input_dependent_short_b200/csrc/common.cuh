@@ -191,15 +191,13 @@ __device__ __forceinline__ u64 mk2(float lo, float hi) {
     return r;
 }
 __device__ __forceinline__ float lo2(u64 v) {
-    float a, b;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-    (void)b;
+    float a;
+    asm("{ .reg .f32 hi; mov.b64 {%0, hi}, %1; }" : "=f"(a) : "l"(v));
     return a;
 }
 __device__ __forceinline__ float hi2(u64 v) {
-    float a, b;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
-    (void)a;
+    float b;
+    asm("{ .reg .f32 lo; mov.b64 {lo, %0}, %1; }" : "=f"(b) : "l"(v));
     return b;
 }
 __device__ __forceinline__ u64 fma2(u64 a, u64 b, u64 c) {

@@ -293,3 +293,35 @@ SWEEP = [w for w in wls.sweep_workloads() if (w.variant, w.W, w.H, w.R) in {
 @pytest.mark.parametrize("wl", SWEEP, ids=lambda w: w.name.replace(" ", "-"))
 def test_sweep_workloads_sampled(wl):
     sampled_check(wl, n=256)
+
+
+@pytest.mark.parametrize("shape", [(4, 4096, 8192, 4, 64, 64), (2, 2048, 6144, 4, 1, 32)],
+                         ids=["all-linear-shape", "qkv-shape"])
+def test_lowrank_fused_materialises_no_filters(shape):
+    """The fused low-rank kernels never hold w = zU or dw in device memory: the
+    forward needs no workspace, the backward's workspace (per-range dU partials
+    and an fp32 dz accumulator) is far smaller than the filter tensor, and the
+    peak allocation grows by the outputs and that workspace only."""
+    import ctypes as C
+
+    from input_dependent_short_b200 import _lib
+
+    B, T, D, W, H, R = shape
+    o = ops()
+    wl = W_("lr-mem", LOWRANK, B, T, D, W, H, R)
+    t = wls.make_inputs(wl)
+    x, dy, z, U = (to_dev(t[k], "bf16") for k in ("x", "dy", "z", "U"))
+    p = o.problem(x, W, H, R)
+    L = _lib.lib()
+    filters = B * T * (D // H) * W * 4
+    ws = L.dsc_bwd_lowrank_workspace_bytes(C.byref(p))
+    assert L.dsc_fwd_lowrank_workspace_bytes(C.byref(p)) == 0
+    assert ws < filters / 3
+    torch.cuda.synchronize()
+    base = torch.cuda.memory_allocated()
+    torch.cuda.reset_peak_memory_stats()
+    y = o.dsc_fwd_lowrank(x, z, U, H)
+    dx, dz, dU = o.dsc_bwd_lowrank(x, z, U, dy, H)
+    torch.cuda.synchronize()
+    outputs = sum(v.numel() * v.element_size() for v in (y, dx, dz, dU))
+    assert torch.cuda.max_memory_allocated() - base <= outputs + ws + (1 << 20)
