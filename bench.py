@@ -93,14 +93,20 @@ def hbm_peak():
         return FALLBACK_HBM_GBS, "fallback"
 
 
-def source_digest():
-    """sha256 of the kernel sources, to match ncu traffic figures to a build."""
-    import glob
+KERNEL_SOURCES = {
+    "headwise": ("conv_stream.cu", "common.cuh", "kernels.cuh"),
+    "static": ("conv_stream.cu", "common.cuh", "kernels.cuh"),
+    "lowrank": ("lowrank.cu", "common.cuh", "kernels.cuh"),
+}
 
+
+def source_digest(variant: str) -> str:
+    """sha256 of the sources of a variant's kernels, to match ncu traffic
+    figures (profiles/traffic.txt) to the build they were taken on."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "input_dependent_short_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
-            h.update(os.path.basename(p).encode() + f.read())
+    for name in KERNEL_SOURCES[variant]:
+        with open(os.path.join(ROOT, "input_dependent_short_b200", "csrc", name), "rb") as f:
+            h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
 
 
@@ -324,11 +330,11 @@ def run_dsc(args, wl0):
     tokens = wl.B * wl.T
     fb, bb = step_bytes(wl)
     peak, peak_src = hbm_peak()
-    digest = source_digest()
+    digest = source_digest(wl.variant)
     bwd_gbs = bb / (bwd_ms / 1e3) / 1e9
     fwd_gbs = fb / (fwd_ms / 1e3) / 1e9
     step_gbs = (fb + bb) / (ms / K / 1e3) / 1e9
-    kname = {"headwise": "k_stream_bwd", "static": "k_stream_bwd", "lowrank": "lowrank_bwd"}[wl.variant]
+    kname = {"headwise": "k_stream_bwd", "static": "k_stream_bwd", "lowrank": "k_lr_bwd"}[wl.variant]
     traffic = ncu_traffic(kname, wl0.name, digest)
 
     result = None
