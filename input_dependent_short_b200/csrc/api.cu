@@ -180,12 +180,13 @@ dsc_status dsc_bwd_static(const dsc_problem *p, const void *x, const void *ws, c
 
 size_t dsc_fwd_lowrank_workspace_bytes(const dsc_problem *p) {
     if (validate(p, true) != DSC_OK) return 0;
-    if (lowrank_fused_ok(*p)) return 0;
+    if (lowrank_tc_ok(*p) || lowrank_fused_ok(*p)) return 0;
     return lr_generic_fwd_bytes(*p);
 }
 
 size_t dsc_bwd_lowrank_workspace_bytes(const dsc_problem *p) {
     if (validate(p, true) != DSC_OK) return 0;
+    if (lowrank_tc_bwd_ok(*p, sm_count())) return lr_tc_bwd_ws_bytes(*p, sm_count());
     if (lowrank_fused_ok(*p)) return lr_bwd_fused_ws_bytes(ctx(nullptr), *p);
     return 2 * lr_generic_fwd_bytes(*p);
 }
@@ -196,6 +197,7 @@ dsc_status dsc_fwd_lowrank(const dsc_problem *p, const void *x, const void *z, c
     if (s == DSC_OK) s = check_ptrs({x, z, U, y});
     if (s != DSC_OK) return s;
     const Ctx c = ctx(stream);
+    if (lowrank_tc_ok(*p)) return done(launch_lr_fwd_tc(c, *p, x, z, U, y));
     if (lowrank_fused_ok(*p)) return done(launch_lr_fwd_fused(c, *p, x, z, U, y));
     // Unfused fallback: filters w = zU in the workspace, then the per-channel kernel.
     if (!workspace) return DSC_ERR_INVALID_ARG;
@@ -218,6 +220,8 @@ dsc_status dsc_bwd_lowrank(const dsc_problem *p, const void *x, const void *z, c
     if (need && (!workspace || workspace_bytes < need)) return DSC_ERR_INVALID_ARG;
     if (need && !aligned16(workspace)) return DSC_ERR_MISALIGNED;
     const Ctx c = ctx(stream);
+    if (lowrank_tc_bwd_ok(*p, c.sms))
+        return done(launch_lr_bwd_tc(c, *p, x, z, U, dy, dx, dz, dU, workspace, workspace_bytes));
     if (lowrank_fused_ok(*p)) return done(launch_lr_bwd_fused(c, *p, x, z, U, dy, dx, dz, dU, workspace, workspace_bytes));
     // Unfused fallback: w = zU and dw in the workspace; dz = dw U^T; dU = z^T dw.
     const int64_t N = p->B * p->T, GW = (p->D / p->H) * p->W;
@@ -239,8 +243,9 @@ dsc_status dsc_bwd_lowrank(const dsc_problem *p, const void *x, const void *z, c
 dsc_status dsc_check(void *stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSC_ERR_CUDA;
     const int st = take_device_status(static_cast<cudaStream_t>(stream));
-    if (st < 0) return DSC_ERR_CUDA;
-    return static_cast<dsc_status>(st);
+    const int st_tc = take_tc_status(static_cast<cudaStream_t>(stream));
+    if (st < 0 || st_tc < 0) return DSC_ERR_CUDA;
+    return static_cast<dsc_status>(st ? st : st_tc);
 }
 
 }  // extern "C"

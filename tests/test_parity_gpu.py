@@ -149,6 +149,15 @@ LOWRANK_SHAPES = [
     (1, 40, 48, 8, 1, 3),
     (2, 3, 64, 4, 8, 1),
     (1, 70, 40, 5, 5, 7),
+    # shapes the tensor-core kernels take in bf16 (W in {1,2,4,8}, H | 64, D % 32H == 0)
+    (2, 300, 256, 4, 8, 16),
+    (1, 200, 2048, 2, 64, 32),
+    (2, 129, 64, 8, 2, 48),
+    (1, 128, 32, 1, 1, 20),
+    (1, 131, 1024, 4, 32, 64),
+    (1, 140, 512, 4, 16, 16),
+    (2, 150, 2048, 4, 64, 32),
+    (1, 260, 256, 8, 8, 24),
 ]
 
 
