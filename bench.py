@@ -96,7 +96,8 @@ def hbm_peak():
 KERNEL_SOURCES = {
     "headwise": ("conv_stream.cu", "common.cuh", "kernels.cuh"),
     "static": ("conv_stream.cu", "common.cuh", "kernels.cuh"),
-    "lowrank": ("lowrank.cu", "common.cuh", "kernels.cuh"),
+    "lowrank": ("lowrank_tc_fwd.cu", "lowrank_tc_bwd.cu", "lowrank_tc.cuh", "tc.cuh", "lowrank.cu", "common.cuh",
+                "kernels.cuh"),
 }
 
 

@@ -144,6 +144,15 @@ DSC_API dsc_status dsc_bwd_static_noalloc(const dsc_problem *p, const void *x, c
  * reported an error. */
 DSC_API dsc_status dsc_check(void *stream);
 
+/* Failure-detection self-test.  Launches one single-thread kernel that waits
+ * on an on-chip barrier nothing completes, with the same bounded wait as the
+ * tensor-core kernels but a limit of about 10 million cycles (~5 ms).  The
+ * wait gives up, records DSC_ERR_TIMEOUT in the device status word and the
+ * kernel returns, leaving the context usable; the next dsc_check() on the
+ * stream returns DSC_ERR_TIMEOUT and clears the word.  Returns DSC_OK once
+ * the kernel is launched, DSC_ERR_CUDA if the launch failed. */
+DSC_API dsc_status dsc_selftest_timeout(void *stream);
+
 /* Static description of a status code. */
 DSC_API const char *dsc_status_string(dsc_status s);
 

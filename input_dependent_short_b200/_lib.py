@@ -42,6 +42,7 @@ _SIGS = {
     "dsc_bwd_static": (C.c_int, [_P, _v, _v, _v, _v, _v, _v, C.c_size_t, _v]),
     "dsc_bwd_static_noalloc": (C.c_int, [_P, _v, _v, _v, _v, _v, _v]),
     "dsc_check": (C.c_int, [_v]),
+    "dsc_selftest_timeout": (C.c_int, [_v]),
     "dsc_status_string": (C.c_char_p, [C.c_int]),
     "dsc_version": (C.c_int, []),
     "dsc_launch_count": (C.c_uint64, []),

@@ -240,6 +240,10 @@ dsc_status dsc_bwd_lowrank(const dsc_problem *p, const void *x, const void *z, c
     return done(e);
 }
 
+dsc_status dsc_selftest_timeout(void *stream) {
+    return launch_wait_selftest(static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSC_OK : DSC_ERR_CUDA;
+}
+
 dsc_status dsc_check(void *stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSC_ERR_CUDA;
     const int st = take_device_status(static_cast<cudaStream_t>(stream));

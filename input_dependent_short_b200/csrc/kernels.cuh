@@ -72,10 +72,11 @@ cudaError_t launch_lr_bwd_fused(const Ctx &c, const dsc_problem &p, const void *
                                 const void *dy, void *dx, void *dz, float *dU, void *ws, size_t ws_bytes);
 size_t lr_bwd_fused_ws_bytes(const Ctx &c, const dsc_problem &p);
 
-// lowrank_tc.cu (tensor-core kernels, bf16)
+// lowrank_tc_fwd.cu, lowrank_tc_bwd.cu (tensor-core kernels, bf16)
 bool lowrank_tc_ok(const dsc_problem &p);
 cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U, void *y);
 int take_tc_status(cudaStream_t stream);
+cudaError_t launch_wait_selftest(cudaStream_t stream);
 bool lowrank_tc_bwd_ok(const dsc_problem &p, int sms);
 size_t lr_tc_bwd_ws_bytes(const dsc_problem &p, int sms);
 cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U,

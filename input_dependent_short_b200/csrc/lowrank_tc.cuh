@@ -1,0 +1,120 @@
+// Shared pieces of the tensor-core low-rank kernels (lowrank_tc_fwd.cu,
+// lowrank_tc_bwd.cu): the problem map, the kernel arguments, tensor-map
+// encoding and small device helpers.
+//
+// "Dynamic Short Convolutions Improve Transformers", technical summary,
+// Methodology, "Parameterisation" 1 (rank-R factorisation of the filter
+// generator, w[b,t,g,k] = sum_r z[b,t,r] U[r, g*W + k]) and "Efficient
+// training implementation" (the fused kernels form zU on chip and convolve at
+// once; the filter tensor never reaches HBM).
+//
+// Used for bf16 with R a multiple of 8 up to 64, W in {1, 2, 4, 8}, H a
+// divisor of 64 and D a multiple of 32*H; the CUDA-core kernels cover every
+// other shape.
+#pragma once
+
+#include <cuda.h>
+
+#include "kernels.cuh"
+#include "tc.cuh"
+
+namespace dsc {
+namespace lrtc {
+
+constexpr int TC_M = 128;                            // tokens per tile (TMEM lanes)
+constexpr int TC_GROUPS = 32;                        // filter groups per forward unit block
+constexpr long long TC_WAIT_LIMIT = 2000000000ll;    // ~1 s of clock cycles
+
+struct TcMap {
+    int64_t B, T, D, H, R, GW;
+    int W, RP;           // RP: R padded to a multiple of 16
+    int tilesPerSeq;     // tiles of 128 tokens per sequence
+    int lgH;             // log2 H
+    int residual;
+    // forward: item = (tile, block of CF channels) -> NF TMEM columns; sub-tiles of SF channels
+    int CF, NF, SF, nSubF, nBlkF, NSF;
+    int64_t nItemsF;
+    // backward: block of CB channels = GB groups -> W*GB = 128 filter columns;
+    // sub-tiles of SB channels; CTA = (range of tiles) x (group of CPC blocks)
+    int CB, GB, SB, nSubB, nBlkB;
+    int CPC, nGroups, nRanges, tilesPerRange;
+    int NSB, DWB, NOP;   // sub-tile ring slots, dw tile buffers, operand buffers
+    int64_t totalTiles;
+};
+
+struct TcArgs {
+    TcMap m;
+    const bf16 *x, *z, *U, *dy;
+    bf16 *y, *dx, *dz;
+    float *dU, *dz_acc, *dU_part;
+    bf16 *Up;  // backward: U with the columns of each block in tap-major order
+};
+
+// Fills the common part of the map; false when the tensor-core kernels do not take the shape.
+bool tc_map(const dsc_problem &p, TcMap &m);
+
+// bf16 tensor map of `rank` dimensions (innermost first): extents `dims`,
+// byte strides of dimensions 1.. in `strides_bytes`, box `box`, zeros outside.
+bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
+              const uint32_t *box, CUtensorMapSwizzle swz, CUtensorMapL2promotion l2);
+
+// Status word of the backward's bounded waits (read and cleared).
+int take_tc_bwd_status(cudaStream_t stream);
+
+__host__ __device__ constexpr uint32_t up1024(uint32_t v) { return (v + 1023u) & ~1023u; }
+
+// 32 lanes x N consecutive fp32 TMEM columns (N = 1, 2, 4 or a multiple of 8).
+template <int N> __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
+    uint32_t r[N];
+    if constexpr (N == 1) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
+    } else if constexpr (N == 2) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
+    } else if constexpr (N == 4) {
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+                     : "r"(taddr));
+    } else {
+        static_assert(N % 8 == 0, "TMEM loads of 8 columns at a time");
+#pragma unroll
+        for (int i = 0; i < N / 8; ++i)
+            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                         : "=r"(r[8 * i]), "=r"(r[8 * i + 1]), "=r"(r[8 * i + 2]), "=r"(r[8 * i + 3]),
+                           "=r"(r[8 * i + 4]), "=r"(r[8 * i + 5]), "=r"(r[8 * i + 6]), "=r"(r[8 * i + 7])
+                         : "r"(taddr + 8 * i));
+    }
+#pragma unroll
+    for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ uint4 lds16(uint32_t a) {
+    uint4 r;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "r"(a));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t word_of(const uint4 &v, int i) {
+    return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// acc + a.lo*b.lo and acc + a.hi*b.hi straight from packed bf16 words
+// (exact bf16 products, fp32 round-to-nearest adds).
+__device__ __forceinline__ float fma_bf16_lo(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{ .reg .b16 al, ah, bl, bh;\n\t mov.b32 {al, ah}, %1;\n\t mov.b32 {bl, bh}, %2;\n\t"
+        " fma.rn.f32.bf16 %0, al, bl, %3; }"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+__device__ __forceinline__ float fma_bf16_hi(uint32_t a, uint32_t b, float c) {
+    float d;
+    asm("{ .reg .b16 al, ah, bl, bh;\n\t mov.b32 {al, ah}, %1;\n\t mov.b32 {bl, bh}, %2;\n\t"
+        " fma.rn.f32.bf16 %0, ah, bh, %3; }"
+        : "=f"(d)
+        : "r"(a), "r"(b), "f"(c));
+    return d;
+}
+
+}  // namespace lrtc
+}  // namespace dsc

@@ -1,0 +1,746 @@
+// Tensor-core backward of the low-rank dynamic short convolution (sm_100a).
+//
+// "Dynamic Short Convolutions Improve Transformers", technical summary,
+// Methodology, "Parameterisation" 1 and "Efficient training implementation"
+// (the backward forms the filters on chip as the forward does):
+//   dx[t,c]   = (w[t,g,0] + r) dy[t,c] + sum_{k>=1} w[t+k,g,k] dy[t+k,c]
+//   dw[t,g,k] = sum_{c in g} dy[t,c] x[t-k,c]
+//   dz[t,:]   = sum_{g,k} dw[t,g,k] U[:, g*W+k]      dU[:, g*W+k] = sum_t z[t,:] dw[t,g,k]
+// (g = g(c) the channel's group; x, dy zero outside [0, T)).
+//
+// Block = GB = 128/W groups = CB = GB*H channels; U's columns of a block are
+// first reordered tap-major (U_perm, column k*GB + g) by a small kernel, so
+// that per tap k one MMA  z[t0+k .. t0+k+127] . U_perm[:, k-th GB columns]
+// puts w[t+k, g, k] -- the filter dx of token t needs -- on TMEM lane t: the
+// shift by k tokens is only a start address in the z tile (which holds 136
+// rows).  Work item = (tile of 128 tokens, block).  Per item:
+//   W MMAs        filters into one of two TMEM buffers (128 columns);
+//   epilogue      per sub-tile of SB channels: dx (stored) and dw (bf16,
+//                 tap-major, into a [128 x 128] shared tile);
+//   2 x 8 MMAs    dz[tile] += dw . U_perm^T   (TMEM, over the CTA's blocks),
+//                 dU[block] += dw^T . z        (TMEM, over the CTA's tiles).
+// CTA = (range of tiles) x (group of CPC blocks); dz leaves TMEM after a
+// tile's last block (bf16, or fp32 adds into an accumulator when several
+// block groups exist), dU after the range (directly, or as a per-range
+// partial summed by a finalize kernel).
+//
+// Warp roles (576 threads): warp 16 TMA producer, warp 17 TMEM owner and MMA
+// issuer, warps 0-15 epilogue (thread part p of token t: VPT 8-channel
+// vectors of each sub-tile).  Groups wider than a part's channels (PPG parts
+// per group) add their dw partial sums through a small exchange buffer.
+#include "lowrank_tc.cuh"
+
+namespace dsc {
+
+// Status word of the backward's bounded waits on each device.
+__device__ int g_dsc_status_tcb = 0;
+
+namespace lrtc {
+
+int take_tc_bwd_status(cudaStream_t stream) {
+    int v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_dsc_status_tcb, sizeof v, 0, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return -1;
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_dsc_status_tcb, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, stream) !=
+        cudaSuccess)
+        return -1;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return -1;
+    return v;
+}
+
+namespace {
+
+constexpr int TB_EPI = 512;              // epilogue threads
+constexpr int TB_THREADS = TB_EPI + 64;  // + producer warp + MMA warp
+constexpr int TB_MAXNS = 8;              // most sub-tiles in flight
+constexpr int TB_SMEM = 220 * 1024;
+constexpr int TB_NB = 128;               // filter columns per block (W * GB)
+constexpr int TB_ZROWS = 136;            // z rows per tile: 128 + up to 7 for the shifted filters
+constexpr uint32_t TB_ZR = TB_ZROWS * 16;  // bytes per 8-wide k-chunk of the z tile
+
+struct BwdSmem {
+    uint32_t zbytes, ubytes, opsize, dw, dwsize, xch, ring, boxb, slot, bars, tmem, total;
+    __host__ __device__ BwdSmem(const TcMap &m, int nop, int ns, int dwb, bool xchg) {
+        const int rb = m.SB == 32 ? 64 : 128;
+        boxb = up1024((uint32_t)(rb * (TC_M + m.W - 1)));
+        slot = 2 * boxb;  // x box + dy box
+        zbytes = (uint32_t)(m.RP / 8) * TB_ZR;
+        ubytes = (uint32_t)(m.RP * TB_NB * 2);
+        opsize = up1024(zbytes + ubytes);
+        dw = (uint32_t)nop * opsize;
+        dwsize = (uint32_t)(TC_M * TB_NB * 2);
+        xch = dw + (uint32_t)dwb * dwsize;
+        ring = up1024(xch + (xchg ? (uint32_t)(2 * 4 * TC_M * m.W * 4) : 0u));
+        bars = ring + (uint32_t)ns * slot;
+        tmem = bars + (17 + 2 * TB_MAXNS) * 8;
+        total = tmem + 16 + 1024;  // + slack to align the base to 1024 bytes
+    }
+};
+
+// OPF[3] OPE[3] WF[2] WE[2] DWF[2] DWE[2] DZF[2] DZE[2] DUF XF[MAXNS] XE[MAXNS]
+struct BwdBars {
+    uint32_t base;
+    __device__ uint32_t opf(int b) const { return base + 8u * (uint32_t)b; }
+    __device__ uint32_t ope(int b) const { return base + 24u + 8u * (uint32_t)b; }
+    __device__ uint32_t wf(int b) const { return base + 48u + 8u * (uint32_t)b; }
+    __device__ uint32_t we(int b) const { return base + 64u + 8u * (uint32_t)b; }
+    __device__ uint32_t dwf(int b) const { return base + 80u + 8u * (uint32_t)b; }
+    __device__ uint32_t dwe(int b) const { return base + 96u + 8u * (uint32_t)b; }
+    __device__ uint32_t dzf(int b) const { return base + 112u + 8u * (uint32_t)b; }
+    __device__ uint32_t dze(int b) const { return base + 128u + 8u * (uint32_t)b; }
+    __device__ uint32_t duf() const { return base + 144u; }
+    __device__ uint32_t xf(int s) const { return base + 152u + 8u * (uint32_t)s; }
+    __device__ uint32_t xe(int s) const { return base + 152u + 8u * TB_MAXNS + 8u * (uint32_t)s; }
+};
+
+// Items of a CTA in order (tile-major, block-minor), advanced without divisions.
+struct BwdWalk {
+    int tl, cl, t0, b, blk;
+    __device__ void init(const TcMap &m, int64_t tile_lo, int chunk_lo) {
+        tl = 0;
+        cl = 0;
+        b = (int)(tile_lo / m.tilesPerSeq);
+        t0 = (int)(tile_lo % m.tilesPerSeq) * TC_M;
+        blk = chunk_lo;
+    }
+    __device__ void next(const TcMap &m, int chunk_lo, int ncl) {
+        if (++cl == ncl) {
+            cl = 0;
+            ++tl;
+            t0 += TC_M;
+            if (t0 >= m.T) {
+                t0 = 0;
+                ++b;
+            }
+        }
+        blk = chunk_lo + cl;
+    }
+};
+
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(TB_EPI) : "memory"); }
+
+__device__ __forceinline__ void red_add_v4(float *p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
+
+// Stores n = 1, 2, 4, 8 or 16 consecutive bf16 values (from fp32) at a dw tile address.
+template <int N> __device__ __forceinline__ void st_dw(unsigned char *p, const float *v) {
+    if constexpr (N == 1) {
+        *reinterpret_cast<bf16 *>(p) = __float2bfloat16_rn(v[0]);
+    } else if constexpr (N == 2) {
+        *reinterpret_cast<uint32_t *>(p) = pack_bf2(v[0], v[1]);
+    } else if constexpr (N == 4) {
+        *reinterpret_cast<uint2 *>(p) = make_uint2(pack_bf2(v[0], v[1]), pack_bf2(v[2], v[3]));
+    } else if constexpr (N == 8) {
+        *reinterpret_cast<uint4 *>(p) =
+            make_uint4(pack_bf2(v[0], v[1]), pack_bf2(v[2], v[3]), pack_bf2(v[4], v[5]), pack_bf2(v[6], v[7]));
+    } else {
+        static_assert(N == 16, "dw run length");
+        st_dw<8>(p, v);
+        st_dw<8>(p + 128, v + 8);  // the next core matrix along the columns
+    }
+}
+
+// One sub-tile of the epilogue for token t_loc, thread part `part`.
+//   VPT vectors of 8 channels; GPT groups among the thread's 8*VPT channels
+//   (1 when the group is wider: PPG parts then share it).
+template <int W, int VPT, int GPT, int PPG, int RB>
+__device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
+                                            unsigned char *dwt, float *xch, int part, int t_loc, int s, bf16 *dxrow,
+                                            bool store, float res) {
+    constexpr int WIN = W - 1;
+    constexpr int CT = 8 * VPT;                      // the thread's channels
+    constexpr int GPV = GPT >= VPT ? GPT / VPT : 1;  // groups inside one vector
+    constexpr int CPG = 8 / GPV;                     // a group's channels inside one vector
+    const int cs0 = part * CT;                       // sub-tile channel of the thread's first vector
+    const int ci0 = s * m.SB + cs0;                  // block channel
+    const int g0 = ci0 >> m.lgH;                     // block group of the thread's first channel
+    // filters w[t+k, g0 .. g0+GPT-1, k] (tap-major TMEM columns k*GB + g)
+    float wt[W][GPT];
+#pragma unroll
+    for (int k = 0; k < W; ++k) tmem_ld<GPT>(tb + (uint32_t)(k * m.GB + g0), wt[k]);
+    const unsigned char *xb = xs;          // x rows t0-WIN .. t0+127
+    const unsigned char *yb = xs + boxb;   // dy rows t0 .. t0+127+WIN
+    uint4 dyv[VPT][W];
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+        const int cs = cs0 + 8 * v;
+        const int bo = (cs % (RB / 2)) / 8;
+#pragma unroll
+        for (int k = 0; k < W; ++k) dyv[v][k] = *reinterpret_cast<const uint4 *>(yb + tc::swz<RB>(t_loc + k, bo));
+    }
+    tc::tmem_wait_ld();
+#pragma unroll
+    for (int g = 0; g < GPT; ++g) wt[0][g] += res;
+    // dx
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+        float dxv[8];
+#pragma unroll
+        for (int pp = 0; pp < 4; ++pp) {
+            const int ga = GPT >= VPT ? v * GPV + (2 * pp) / CPG : (v * GPT) / VPT;
+            const int gb = GPT >= VPT ? v * GPV + (2 * pp + 1) / CPG : (v * GPT) / VPT;
+            if constexpr (GPV == 1) {
+                u64 acc2 = 0ull;
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    const uint32_t word = word_of(dyv[v][k], pp);
+                    const u64 dp = mk2(bf_lo(word), bf_hi(word));
+                    const float wk = wt[k][ga];
+                    acc2 = k == 0 ? mul2(mk2(wk, wk), dp) : fma2(mk2(wk, wk), dp, acc2);
+                }
+                dxv[2 * pp] = lo2(acc2);
+                dxv[2 * pp + 1] = hi2(acc2);
+            } else {
+                float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    const uint32_t word = word_of(dyv[v][k], pp);
+                    a0 = k == 0 ? wt[k][ga] * bf_lo(word) : fmaf(wt[k][ga], bf_lo(word), a0);
+                    a1 = k == 0 ? wt[k][gb] * bf_hi(word) : fmaf(wt[k][gb], bf_hi(word), a1);
+                }
+                dxv[2 * pp] = a0;
+                dxv[2 * pp + 1] = a1;
+            }
+        }
+        if (store)
+            st16(dxrow + ci0 + 8 * v, make_uint4(pack_bf2(dxv[0], dxv[1]), pack_bf2(dxv[2], dxv[3]),
+                                                 pack_bf2(dxv[4], dxv[5]), pack_bf2(dxv[6], dxv[7])));
+    }
+    // dw[t, g, k] over the thread's channels
+    float pk[W][GPT];
+#pragma unroll
+    for (int k = 0; k < W; ++k)
+#pragma unroll
+        for (int g = 0; g < GPT; ++g) pk[k][g] = 0.f;
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+        const int cs = cs0 + 8 * v;
+        const int bo = (cs % (RB / 2)) / 8;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            const uint4 xv = *reinterpret_cast<const uint4 *>(xb + tc::swz<RB>(t_loc + WIN - k, bo));
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+                const uint32_t dyw = word_of(dyv[v][0], wd), xwd = word_of(xv, wd);
+                const int ga = GPT >= VPT ? v * GPV + (2 * wd) / CPG : (v * GPT) / VPT;
+                const int gb = GPT >= VPT ? v * GPV + (2 * wd + 1) / CPG : (v * GPT) / VPT;
+                pk[k][ga] = fma_bf16_lo(dyw, xwd, pk[k][ga]);
+                pk[k][gb] = fma_bf16_hi(dyw, xwd, pk[k][gb]);
+            }
+        }
+    }
+    if constexpr (PPG == 1) {
+#pragma unroll
+        for (int k = 0; k < W; ++k)
+            st_dw<GPT>(dwt + tc::core_off(t_loc, k * m.GB + g0, TB_NB), pk[k]);
+    } else {
+        // parts p0 .. p0+PPG-1 share the group; part p finishes the taps k = p (mod PPG)
+        float *mine = xch + ((s & 1) * 4 * TC_M + part * TC_M + t_loc) * W;
+#pragma unroll
+        for (int k = 0; k < W; ++k) mine[k] = pk[k][0];
+        epi_bar();
+        const int p0 = part - part % PPG;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            if (k % PPG != part % PPG) continue;
+            float tot = 0.f;
+#pragma unroll
+            for (int q = 0; q < PPG; ++q) tot += xch[((s & 1) * 4 * TC_M + (p0 + q) * TC_M + t_loc) * W + k];
+            st_dw<1>(dwt + tc::core_off(t_loc, k * m.GB + g0, TB_NB), &tot);
+        }
+    }
+}
+
+template <int W, int VPT, int GPT, int PPG>
+__global__ void __launch_bounds__(TB_THREADS, 1)
+    k_lr_tc_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmdy,
+                const __grid_constant__ CUtensorMap tmz, const __grid_constant__ CUtensorMap tmu, const TcArgs a) {
+    constexpr int WIN = W - 1;
+    constexpr int RB = VPT == 1 ? 64 : 128;  // box row bytes (32 or 64 channels)
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const TcMap &m = a.m;
+    const int NS = m.NSB, NOP = m.NOP, DWB = m.DWB;
+    const BwdSmem S(m, NOP, NS, DWB, PPG > 1);
+    const int group = blockIdx.x % m.nGroups;
+    const int range = blockIdx.x / m.nGroups;
+    const int chunk_lo = group * m.CPC;
+    const int ncl = min(m.CPC, m.nBlkB - chunk_lo);
+    const int64_t tile_lo = (int64_t)range * m.tilesPerRange;
+    const int ntl = (int)min((int64_t)m.tilesPerRange, m.totalTiles - tile_lo);
+    if (ncl <= 0 || ntl <= 0) return;
+    const int nI = ntl * ncl;
+    const int nG = nI * m.nSubB;
+
+    const uint32_t sraw = tc::smem_u32(smem_raw);
+    const uint32_t sbase = (sraw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - sraw);
+    const BwdBars bars{sbase + S.bars};
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int kz = m.R / 8;  // z k-chunks loaded per item; kz .. RP/8-1 stay zero
+    const uint32_t col_dz = 2 * TB_NB, col_dU = 2 * TB_NB + 2 * m.RP;
+
+    if (tid == 0) {
+        for (int i = 0; i < 3; ++i) {
+            tc::mbar_init(bars.opf(i), 1);
+            tc::mbar_init(bars.ope(i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(bars.wf(i), 1);
+            tc::mbar_init(bars.we(i), TB_EPI / 32);
+            tc::mbar_init(bars.dwf(i), TB_EPI / 32);
+            tc::mbar_init(bars.dwe(i), 1);
+            tc::mbar_init(bars.dzf(i), 1);
+            tc::mbar_init(bars.dze(i), TB_EPI / 32);
+        }
+        tc::mbar_init(bars.duf(), 1);
+        for (int i = 0; i < NS; ++i) {
+            tc::mbar_init(bars.xf(i), 1);
+            tc::mbar_init(bars.xe(i), TB_EPI / 32);
+        }
+        tc::fence_mbar_init();
+    }
+    // zero the padded k-chunks of every z buffer (read by the MMAs, never loaded)
+    const int zpad = (m.RP / 8 - kz) * TB_ZROWS;
+    for (int i = tid; i < NOP * zpad; i += TB_THREADS) {
+        const int b = i / zpad, r = i % zpad;
+        *reinterpret_cast<uint4 *>(smem + (uint32_t)b * S.opsize + (uint32_t)kz * TB_ZR + (uint32_t)r * 16) =
+            make_uint4(0, 0, 0, 0);
+    }
+    tc::fence_proxy_async();
+    if (warp == 17) tc::tmem_alloc(sbase + S.tmem, 512);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + S.tmem);
+    bool timed_out = false;
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+        if (!timed_out && !tc::mbar_wait(bar, parity, TC_WAIT_LIMIT)) timed_out = true;  // sticky: later waits skip
+    };
+
+    if (warp == 16) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tc::tma_prefetch_desc(&tmx);
+            tc::tma_prefetch_desc(&tmdy);
+            tc::tma_prefetch_desc(&tmz);
+            tc::tma_prefetch_desc(&tmu);
+            BwdWalk it;
+            it.init(m, tile_lo, chunk_lo);
+            int ob = 0, slot = 0, l = 0;
+            uint32_t oph = 0, xph = 0;
+            for (int li = 0; li < nI; ++li, it.next(m, chunk_lo, ncl)) {
+                if (li >= NOP) wait(bars.ope(ob), oph ^ 1u);
+                const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
+                tc::mbar_expect_tx(bars.opf(ob), (uint32_t)kz * TB_ZR + S.ubytes);
+                for (int j = 0; j < kz; ++j) tc::tma_load_3d(zb + (uint32_t)j * TB_ZR, &tmz, 8 * j, it.t0, it.b, bars.opf(ob));
+                for (int j = 0; j < TB_NB / 8; ++j)
+                    tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), &tmu, it.blk * TB_NB + 8 * j, 0, bars.opf(ob));
+                if (++ob == NOP) {
+                    ob = 0;
+                    oph ^= 1u;
+                }
+                for (int s = 0; s < m.nSubB; ++s, ++l) {
+                    if (l >= NS) wait(bars.xe(slot), xph ^ 1u);
+                    const uint32_t xb = sbase + S.ring + (uint32_t)slot * S.slot;
+                    tc::mbar_expect_tx(bars.xf(slot), (uint32_t)(2 * RB * (TC_M + WIN)));
+                    const int c = it.blk * m.CB + s * m.SB;
+                    tc::tma_load_3d(xb, &tmx, c, it.t0 - WIN, it.b, bars.xf(slot));
+                    tc::tma_load_3d(xb + S.boxb, &tmdy, c, it.t0, it.b, bars.xf(slot));
+                    if (++slot == NS) {
+                        slot = 0;
+                        xph ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 17) {
+        // ----------------------------------------------------------------- MMA
+        if (lane == 0) {
+            const uint32_t id_w = tc::idesc_bf16(TC_M, m.GB, 0, 1);
+            const uint32_t id_dz = tc::idesc_bf16(TC_M, m.RP, 0, 0);
+            const uint32_t id_dU = tc::idesc_bf16(TC_M, m.RP, 1, 1);
+            // dz / dU of item j (its dw tile is complete), then release its buffers
+            int fob = 0, fdb = 0, ftl = 0, fcl = 0;
+            uint32_t fdph = 0;
+            auto finish = [&](void) {
+                wait(bars.dwf(fdb), fdph);
+                tc::fence_after_sync();
+                const int tp = ftl & 1;
+                if (fcl == 0 && ftl >= 2) wait(bars.dze(tp), (uint32_t)(((ftl - 2) >> 1) & 1));
+                tc::fence_after_sync();
+                const uint32_t zb = sbase + (uint32_t)fob * S.opsize, ub = zb + S.zbytes;
+                const uint32_t dwb = sbase + S.dw + (uint32_t)fdb * S.dwsize;
+                for (int ks = 0; ks < TB_NB / 16; ++ks) {
+                    const uint64_t ad = tc::smem_desc(dwb + (uint32_t)ks * 256u, 128, (TB_NB / 8) * 128);
+                    const uint64_t bd = tc::smem_desc(ub + (uint32_t)(ks * 2 * m.RP * 16), (uint32_t)(m.RP * 16), 128);
+                    tc::mma_bf16(tmem + col_dz + (uint32_t)(tp * m.RP), ad, bd, id_dz, (fcl > 0 || ks > 0) ? 1u : 0u);
+                }
+                for (int ks = 0; ks < TC_M / 16; ++ks) {
+                    const uint64_t ad = tc::smem_desc(dwb + (uint32_t)ks * 2u * ((TB_NB / 8) * 128), (TB_NB / 8) * 128, 128);
+                    const uint64_t bd = tc::smem_desc(zb + (uint32_t)ks * 256u, 128, TB_ZR);
+                    tc::mma_bf16(tmem + col_dU + (uint32_t)(fcl * m.RP), ad, bd, id_dU, (ftl > 0 || ks > 0) ? 1u : 0u);
+                }
+                tc::mma_commit(bars.dwe(fdb));
+                tc::mma_commit(bars.ope(fob));
+                if (fcl == ncl - 1) tc::mma_commit(bars.dzf(tp));
+                if (++fob == NOP) fob = 0;
+                if (++fdb == DWB) {
+                    fdb = 0;
+                    fdph ^= 1u;
+                }
+                if (++fcl == ncl) {
+                    fcl = 0;
+                    ++ftl;
+                }
+            };
+            int ob = 0;
+            uint32_t oph = 0;
+            for (int li = 0; li < nI; ++li) {
+                const int b = li & 1;
+                wait(bars.opf(ob), oph);
+                if (li >= 2) wait(bars.we(b), (uint32_t)(((li - 2) >> 1) & 1));
+                tc::fence_after_sync();
+                const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
+                for (int k = 0; k < W; ++k)
+                    for (int ks = 0; ks < m.RP / 16; ++ks) {
+                        const uint64_t ad = tc::smem_desc(zb + (uint32_t)(k * 16) + (uint32_t)ks * 2u * TB_ZR, TB_ZR, 128);
+                        const uint64_t bd = tc::smem_desc(ub + (uint32_t)((k * m.GB / 8) * m.RP * 16) + (uint32_t)ks * 256u,
+                                                          128, (uint32_t)(m.RP * 16));
+                        tc::mma_bf16(tmem + (uint32_t)(b * TB_NB + k * m.GB), ad, bd, id_w, ks > 0 ? 1u : 0u);
+                    }
+                tc::mma_commit(bars.wf(b));
+                if (++ob == NOP) {
+                    ob = 0;
+                    oph ^= 1u;
+                }
+                if (li >= 1) finish();
+            }
+            finish();
+            tc::mma_commit(bars.duf());
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int t_loc = tid & (TC_M - 1), part = tid >> 7, quarter = warp & 3;
+        const float res = m.residual ? 1.f : 0.f;
+        const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
+        float *xch = reinterpret_cast<float *>(smem + S.xch);
+        // dz of CTA-local tile j (its last block's MMAs are done) leaves TMEM
+        auto dz_out = [&](int j, int bseq, int t0) {
+            const int tp = j & 1;
+            wait(bars.dzf(tp), (uint32_t)((j >> 1) & 1));
+            tc::fence_after_sync();
+            const int t = t0 + t_loc;
+            for (int r = 8 * part; r < m.RP; r += 32) {  // 8-column chunks, dealt round the parts
+                float v[8];
+                tmem_ld<8>(tlane + col_dz + (uint32_t)(tp * m.RP + r), v);
+                tc::tmem_wait_ld();
+                if (t < m.T && r < m.R) {  // R is a multiple of 8
+                    const int64_t o = ((int64_t)bseq * m.T + t) * m.R + r;
+                    if (m.nGroups == 1) {
+                        st16(a.dz + o, make_uint4(pack_bf2(v[0], v[1]), pack_bf2(v[2], v[3]), pack_bf2(v[4], v[5]),
+                                                  pack_bf2(v[6], v[7])));
+                    } else {
+                        red_add_v4(a.dz_acc + o, v[0], v[1], v[2], v[3]);
+                        red_add_v4(a.dz_acc + o + 4, v[4], v[5], v[6], v[7]);
+                    }
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bars.dze(tp));
+        };
+        BwdWalk it;
+        it.init(m, tile_lo, chunk_lo);
+        int slot = 0, db = 0, pb = 0, pt0 = 0;
+        uint32_t xph = 0, dph = 0;
+        for (int li = 0; li < nI; ++li) {
+            const int b = li & 1;
+            const int t = it.t0 + t_loc;
+            if (li >= 1 && it.cl == 0) dz_out(it.tl - 1, pb, pt0);  // previous tile done
+            wait(bars.wf(b), (uint32_t)((li >> 1) & 1));
+            if (li >= DWB) wait(bars.dwe(db), dph ^ 1u);
+            tc::fence_after_sync();
+            const uint32_t tb = tlane + (uint32_t)(b * TB_NB);
+            unsigned char *dwt = smem + S.dw + (uint32_t)db * S.dwsize;
+            bf16 *dxrow = a.dx + ((int64_t)it.b * m.T + t) * m.D + (int64_t)it.blk * m.CB;
+            for (int s = 0; s < m.nSubB; ++s) {
+                wait(bars.xf(slot), xph);
+                bwd_subtile<W, VPT, GPT, PPG, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, xch, part,
+                                                  t_loc, s, dxrow, t < m.T, res);
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bars.xe(slot));
+                if (++slot == NS) {
+                    slot = 0;
+                    xph ^= 1u;
+                }
+            }
+            tc::fence_proxy_async();  // dw tile (generic stores) -> MMA operand
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) {
+                tc::mbar_arrive(bars.dwf(db));
+                tc::mbar_arrive(bars.we(b));
+            }
+            if (++db == DWB) {
+                db = 0;
+                dph ^= 1u;
+            }
+            pb = it.b;
+            pt0 = it.t0;
+            it.next(m, chunk_lo, ncl);
+        }
+        dz_out(ntl - 1, pb, pt0);
+        // dU of the CTA's blocks over its tile range: TMEM lane = block column k*GB + g
+        wait(bars.duf(), 0);
+        tc::fence_after_sync();
+        const int k = t_loc / m.GB, gl = t_loc % m.GB;
+        for (int cl = 0; cl < ncl; ++cl) {
+            const int64_t col = (int64_t)(chunk_lo + cl) * TB_NB + gl * W + k;
+            for (int r8 = 8 * part; r8 < m.RP; r8 += 32) {  // 8-column chunks, dealt round the parts
+                float v[8];
+                tmem_ld<8>(tlane + col_dU + (uint32_t)(cl * m.RP + r8), v);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const int r = r8 + j;
+                    if (r < m.R) {
+                        if (m.nRanges == 1) a.dU[(int64_t)r * m.GW + col] = v[j];
+                        else a.dU_part[((int64_t)range * m.R + r) * m.GW + col] = v[j];
+                    }
+                }
+            }
+        }
+    }
+
+    // teardown: every load and MMA this CTA issued has landed before the
+    // shared memory and TMEM are given back (bounded, also after a time-out)
+    if (warp == 16 && lane == 0) {
+        for (int s = 0; s < NS && s < nG; ++s) {
+            const int lastl = s + ((nG - 1 - s) / NS) * NS;
+            tc::mbar_wait(bars.xf(s), (uint32_t)((lastl / NS) & 1), TC_WAIT_LIMIT);
+        }
+    }
+    if (warp == 17 && lane == 0) tc::mbar_wait(bars.duf(), 0, TC_WAIT_LIMIT);
+    if (timed_out) atomicExch(&g_dsc_status_tcb, (int)DSC_ERR_TIMEOUT);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 17) tc::tmem_dealloc(tmem, 512);
+}
+
+// U_perm[r][blk*128 + k*GB + g] = U[r][(blk*GB + g)*W + k]
+__global__ void k_uperm(const bf16 *U, bf16 *Up, int64_t R, int64_t GW, int W, int GB) {
+    const int64_t n = R * GW;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / GW, j = i % GW;
+        const int64_t blk = j / TB_NB;
+        const int rem = (int)(j % TB_NB);
+        const int k = rem / GB, g = rem % GB;
+        Up[i] = U[r * GW + (blk * GB + g) * W + k];
+    }
+}
+
+__global__ void k_tc_zero(float *p, int64_t n) {
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) p[i] = 0.f;
+}
+
+// dU = sum of the per-range partials (fixed order); dz = the fp32 accumulator in bf16.
+__global__ void k_tc_finalize(const TcArgs a) {
+    const TcMap &m = a.m;
+    const int64_t nU = m.nRanges > 1 ? m.R * m.GW : 0;
+    const int64_t nz = m.nGroups > 1 ? m.B * m.T * m.R : 0;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nU + nz; i += (int64_t)gridDim.x * blockDim.x) {
+        if (i < nU) {
+            float sacc = 0.f;
+            for (int q = 0; q < m.nRanges; ++q) sacc += a.dU_part[(int64_t)q * m.R * m.GW + i];
+            a.dU[i] = sacc;
+        } else {
+            a.dz[i - nU] = __float2bfloat16_rn(a.dz_acc[i - nU]);
+        }
+    }
+}
+
+// Backward plan.  Blocks of GB = 128/W groups; TMEM holds two filter buffers
+// (2 x 128 columns), two dz accumulators (2 x RP) and one dU accumulator per
+// block of the CTA (RP each).  Among the block-group sizes that fit, take the
+// one with the fewest items on the busiest SM, then the least partial-sum
+// traffic (dU partials of the token ranges, dz contributions of the block
+// groups).  Shared memory: operand buffers (3 when items are short), dw tiles
+// (2 when items are short), the exchange buffer, and as deep a sub-tile ring
+// as fits.
+bool tc_bwd_plan(TcMap &m, int sms) {
+    m.GB = TB_NB / m.W;
+    m.CB = (int)(m.GB * m.H);
+    if (m.D % m.CB) return false;
+    m.SB = m.CB < 64 ? m.CB : 64;
+    if (m.SB < 32) return false;
+    m.nSubB = m.CB / m.SB;
+    m.nBlkB = (int)(m.D / m.CB);
+    m.totalTiles = m.B * (int64_t)m.tilesPerSeq;
+    const int cpc_max = (512 - 2 * TB_NB - 2 * m.RP) / m.RP;
+    if (cpc_max < 1) return false;
+    double best_work = -1, best_cost = 0;
+    for (int cpc = 1; cpc <= cpc_max && cpc <= m.nBlkB; ++cpc) {
+        const int ng = (m.nBlkB + cpc - 1) / cpc;
+        int64_t nr = sms / ng;
+        if (nr < 1) nr = 1;
+        if (nr > m.totalTiles) nr = m.totalTiles;
+        const int64_t tpr = (m.totalTiles + nr - 1) / nr;
+        const int64_t waves = (ng * nr + sms - 1) / sms;
+        const double work = (double)waves * tpr * cpc;  // items on the busiest SM
+        const double nz = (double)m.B * m.T * m.R;
+        const double cost = (nr > 1 ? 2.0 * nr * m.R * m.GW : 0.0) + (ng > 1 ? (2.0 + 0.25 * ng) * nz : 0.0);
+        if (best_work < 0 || work < best_work * 0.97 || (work <= best_work * 1.03 && cost < best_cost)) {
+            best_work = work;
+            best_cost = cost;
+            m.CPC = cpc;
+            m.nGroups = ng;
+            m.nRanges = (int)nr;
+        }
+    }
+    m.tilesPerRange = (int)((m.totalTiles + m.nRanges - 1) / m.nRanges);
+    m.nRanges = (int)((m.totalTiles + m.tilesPerRange - 1) / m.tilesPerRange);
+    const int vpt = m.SB / 32, ct = 8 * vpt;
+    const bool xchg = m.H > ct;
+    const bool short_items = m.nSubB < 4;
+    const int nop = short_items ? 3 : 2, dwb = short_items ? 2 : 1;
+    for (m.NSB = TB_MAXNS; m.NSB >= 2; --m.NSB) {
+        m.NOP = nop;
+        m.DWB = dwb;
+        if (BwdSmem(m, nop, m.NSB, dwb, xchg).total <= TB_SMEM) return true;
+    }
+    return false;
+}
+
+size_t up_bytes(const TcMap &m) { return ((size_t)m.R * m.GW * 2 + 255) & ~(size_t)255; }
+
+size_t tc_bwd_ws_bytes(const TcMap &m) {
+    size_t n = up_bytes(m);
+    if (m.nRanges > 1) n += (size_t)m.nRanges * m.R * m.GW * 4;
+    if (m.nGroups > 1) n += (size_t)m.B * m.T * m.R * 4;
+    return n;
+}
+
+struct BwdMaps {
+    CUtensorMap x, dy, z, u;
+};
+
+bool bwd_maps(const TcArgs &a, BwdMaps &f) {
+    const TcMap &m = a.m;
+    const int rb = m.SB == 32 ? 64 : 128;
+    const uint64_t xd[3] = {(uint64_t)m.D, (uint64_t)m.T, (uint64_t)m.B};
+    const uint64_t xs[2] = {(uint64_t)m.D * 2, (uint64_t)(m.T * m.D * 2)};
+    const uint32_t xb[3] = {(uint32_t)(rb / 2), (uint32_t)(TC_M + m.W - 1), 1};
+    const uint64_t zd[3] = {(uint64_t)m.R, (uint64_t)m.T, (uint64_t)m.B};
+    const uint64_t zs[2] = {(uint64_t)m.R * 2, (uint64_t)(m.T * m.R * 2)};
+    const uint32_t zb[3] = {8, (uint32_t)TB_ZROWS, 1};
+    const uint64_t ud[2] = {(uint64_t)m.GW, (uint64_t)m.R};
+    const uint64_t us[1] = {(uint64_t)m.GW * 2};
+    const uint32_t ub[2] = {8, (uint32_t)m.RP};
+    const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    return make_map(&f.x, a.x, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
+           make_map(&f.dy, a.dy, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
+           make_map(&f.z, a.z, 3, zd, zs, zb, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
+           make_map(&f.u, a.Up, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
+}
+
+template <int W, int VPT, int GPT, int PPG>
+cudaError_t launch_bwd(const Ctx &c, const TcArgs &a) {
+    const BwdSmem S(a.m, a.m.NOP, a.m.NSB, a.m.DWB, PPG > 1);
+    static const cudaError_t attr = cudaFuncSetAttribute(k_lr_tc_bwd<W, VPT, GPT, PPG>,
+                                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TB_SMEM);
+    if (attr != cudaSuccess) return attr;
+    if (S.total > TB_SMEM) return cudaErrorInvalidValue;
+    BwdMaps f;
+    if (!bwd_maps(a, f)) return cudaErrorNotSupported;
+    // the whole of TMEM per CTA: enough shared memory that no second CTA shares the SM
+    const uint32_t smem = S.total < 120 * 1024 ? 120 * 1024 : S.total;
+    k_lr_tc_bwd<W, VPT, GPT, PPG><<<(unsigned)(a.m.nGroups * a.m.nRanges), TB_THREADS, smem, c.stream>>>(f.x, f.dy, f.z,
+                                                                                                       f.u, a);
+    count_launch();
+    return cudaGetLastError();
+}
+
+// Thread channels per sub-tile: CT = 8*VPT (SB = 32 or 64, four parts).
+template <int W, int VPT> cudaError_t bwd_by_h(const Ctx &c, const TcArgs &a) {
+    constexpr int CT = 8 * VPT;
+    switch (a.m.H) {
+    case 1: if constexpr (CT * W <= 32) return launch_bwd<W, VPT, CT, 1>(c, a); break;
+    case 2: if constexpr (CT / 2 * W <= 32) return launch_bwd<W, VPT, CT / 2, 1>(c, a); break;
+    case 4: return launch_bwd<W, VPT, CT / 4, 1>(c, a);
+    case 8: return launch_bwd<W, VPT, CT / 8, 1>(c, a);
+    case 16: if constexpr (CT >= 16) return launch_bwd<W, VPT, 1, 1>(c, a); else return launch_bwd<W, VPT, 1, 2>(c, a);
+    case 32: return launch_bwd<W, VPT, 1, 32 / CT>(c, a);
+    case 64: return launch_bwd<W, VPT, 1, 64 / CT>(c, a);
+    }
+    return cudaErrorNotSupported;
+}
+
+template <int W> cudaError_t bwd_by_vpt(const Ctx &c, const TcArgs &a) {
+    return a.m.SB == 32 ? bwd_by_h<W, 1>(c, a) : bwd_by_h<W, 2>(c, a);
+}
+
+}  // namespace
+}  // namespace lrtc
+
+bool lowrank_tc_bwd_ok(const dsc_problem &p, int sms) {
+    lrtc::TcMap m;
+    return lrtc::tc_map(p, m) && lrtc::tc_bwd_plan(m, sms);
+}
+
+size_t lr_tc_bwd_ws_bytes(const dsc_problem &p, int sms) {
+    lrtc::TcMap m;
+    if (!lrtc::tc_map(p, m) || !lrtc::tc_bwd_plan(m, sms)) return 0;
+    return lrtc::tc_bwd_ws_bytes(m);
+}
+
+cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U,
+                             const void *dy, void *dx, void *dz, float *dU, void *ws, size_t ws_bytes) {
+    using namespace lrtc;
+    TcArgs a{};
+    if (!tc_map(p, a.m) || !tc_bwd_plan(a.m, c.sms)) return cudaErrorNotSupported;
+    if (!ws || ws_bytes < tc_bwd_ws_bytes(a.m)) return cudaErrorInvalidValue;
+    a.x = static_cast<const bf16 *>(x);
+    a.z = static_cast<const bf16 *>(z);
+    a.U = static_cast<const bf16 *>(U);
+    a.dy = static_cast<const bf16 *>(dy);
+    a.dx = static_cast<bf16 *>(dx);
+    a.dz = static_cast<bf16 *>(dz);
+    a.dU = dU;
+    unsigned char *w = static_cast<unsigned char *>(ws);
+    a.Up = reinterpret_cast<bf16 *>(w);
+    w += up_bytes(a.m);
+    if (a.m.nRanges > 1) {
+        a.dU_part = reinterpret_cast<float *>(w);
+        w += (size_t)a.m.nRanges * a.m.R * a.m.GW * 4;
+    }
+    const int64_t nUp = a.m.R * a.m.GW;
+    k_uperm<<<(unsigned)min((int64_t)1024, (nUp + 255) / 256), 256, 0, c.stream>>>(a.U, a.Up, a.m.R, a.m.GW, a.m.W,
+                                                                                   a.m.GB);
+    count_launch();
+    if (a.m.nGroups > 1) {
+        a.dz_acc = reinterpret_cast<float *>(w);
+        const int64_t n = a.m.B * a.m.T * a.m.R;
+        k_tc_zero<<<(unsigned)min((int64_t)1024, (n + 255) / 256), 256, 0, c.stream>>>(a.dz_acc, n);
+        count_launch();
+    }
+    cudaError_t e = cudaErrorNotSupported;
+    switch (a.m.W) {
+    case 1: e = bwd_by_vpt<1>(c, a); break;
+    case 2: e = bwd_by_vpt<2>(c, a); break;
+    case 4: e = bwd_by_vpt<4>(c, a); break;
+    case 8: e = bwd_by_vpt<8>(c, a); break;
+    }
+    if (e != cudaSuccess) return e;
+    if (a.m.nRanges > 1 || a.m.nGroups > 1) {
+        const int64_t n = (a.m.nRanges > 1 ? a.m.R * a.m.GW : 0) + (a.m.nGroups > 1 ? a.m.B * a.m.T * a.m.R : 0);
+        k_tc_finalize<<<(unsigned)min((int64_t)2048, (n + 255) / 256), 256, 0, c.stream>>>(a);
+        count_launch();
+    }
+    return cudaGetLastError();
+}
+
+}  // namespace dsc

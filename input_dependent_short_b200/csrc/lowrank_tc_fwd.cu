@@ -1,0 +1,560 @@
+// Tensor-core forward of the low-rank dynamic short convolution (sm_100a).
+//
+// "Dynamic Short Convolutions Improve Transformers", technical summary,
+// Methodology, "Parameterisation" 1 and "Efficient training implementation":
+//     y[b,t,c] = r x[b,t,c] + sum_k w[b,t,g(c),k] x[b,t-k,c],
+//     w[b,t,g,k] = sum_r z[b,t,r] U[r, g*W + k],
+// with the filters formed on chip (tcgen05 MMA into tensor memory) and never
+// written to HBM.
+//
+// Item = (tile of 128 tokens, block of CF channels); the block's filters are
+// NF = CF/H*W TMEM columns (NF <= 256) formed by one zU MMA.  TMEM holds two
+// such buffers, so the MMA of item i+1 runs while item i's outputs are formed.
+// A CTA takes a contiguous range of (item, sub-tile) pairs, so every CTA gets
+// the same number of sub-tiles; an item split between two CTAs has its MMA
+// issued by both.  Warp roles (576 threads):
+//   warp 16    TMA producer: z tile and U block of each item (two buffers),
+//              x sub-tiles of SF channels x (128 + W-1) rows (a ring of NS);
+//   warp 17    TMEM owner and MMA issuer;
+//   warps 0-15 epilogue: thread part p of token t forms y for VPT 8-channel
+//              vectors of each sub-tile from its own TMEM lane.
+// Every hand-off is an mbarrier (full / empty pairs); nothing waits on the
+// whole block inside the loop.
+//
+// Operand layouts written by TMA (no swizzle, 8-element boxes):
+//   z tile  (A, K-major):  element (t, k) at (k/8)*2048 + t*16 + (k%8)*2
+//   U block (B, MN-major): element (k, n) at (n/8)*(RP*16) + k*16 + (n%8)*2
+// x sub-tiles: boxes of 64 channels (128-byte rows, 128-byte swizzle) or of
+// 32 channels (64-byte rows, 64-byte swizzle).
+#include "lowrank_tc.cuh"
+
+namespace dsc {
+
+// Status word of the forward's bounded waits on each device: 0 = OK,
+// otherwise the dsc_status of a wait that gave up.
+__device__ int g_dsc_status_tcf = 0;
+
+int take_tc_status(cudaStream_t stream) {
+    int v = 0;
+    if (cudaMemcpyFromSymbolAsync(&v, g_dsc_status_tcf, sizeof v, 0, cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return -1;
+    const int zero = 0;
+    if (cudaMemcpyToSymbolAsync(g_dsc_status_tcf, &zero, sizeof zero, 0, cudaMemcpyHostToDevice, stream) !=
+        cudaSuccess)
+        return -1;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return -1;
+    const int vb = lrtc::take_tc_bwd_status(stream);
+    if (vb < 0) return -1;
+    return v ? v : vb;
+}
+
+// One thread waits on an mbarrier that nothing arrives at; the bounded wait
+// gives up and the time-out is recorded as in the tensor-core kernels.
+__global__ void k_wait_selftest(long long limit) {
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t a = tc::smem_u32(&bar);
+    tc::mbar_init(a, 1);
+    tc::fence_mbar_init();
+    if (!tc::mbar_wait(a, 0, limit)) atomicExch(&g_dsc_status_tcf, (int)DSC_ERR_TIMEOUT);
+}
+
+cudaError_t launch_wait_selftest(cudaStream_t stream) {
+    k_wait_selftest<<<1, 1, 0, stream>>>(10000000ll);
+    count_launch();
+    return cudaGetLastError();
+}
+
+namespace lrtc {
+
+// ------------------------------------------------------------------ common ---
+
+bool tc_map(const dsc_problem &p, TcMap &m) {
+    if (p.dtype != DSC_BF16) return false;
+    if (p.R < 8 || p.R > 64 || p.R % 8) return false;  // 16-byte z rows
+    if (!(p.W == 1 || p.W == 2 || p.W == 4 || p.W == 8)) return false;
+    if (p.H > 64 || (64 % p.H) != 0) return false;
+    if (p.D % (TC_GROUPS * p.H)) return false;
+    m = TcMap{};
+    m.B = p.B; m.T = p.T; m.D = p.D; m.H = p.H; m.R = p.R; m.W = (int)p.W;
+    m.GW = (p.D / p.H) * p.W;
+    m.RP = (int)((p.R + 15) / 16) * 16;
+    m.tilesPerSeq = (int)((p.T + TC_M - 1) / TC_M);
+    m.lgH = 0;
+    while ((1 << m.lgH) < m.H) ++m.lgH;
+    m.residual = p.residual ? 1 : 0;
+    return true;
+}
+
+// cuTensorMapEncodeTiled, looked up once through the runtime.
+using EncodeTiled = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                 const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiled encode_fn() {
+    static EncodeTiled fn = [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &p, 12000, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            p = nullptr;
+        return reinterpret_cast<EncodeTiled>(p);
+    }();
+    return fn;
+}
+
+bool make_map(CUtensorMap *map, const void *base, int rank, const uint64_t *dims, const uint64_t *strides_bytes,
+              const uint32_t *box, CUtensorMapSwizzle swz, CUtensorMapL2promotion l2) {
+    const EncodeTiled fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t gd[5], gs[4];
+    cuuint32_t bd[5], es[5];
+    for (int i = 0; i < rank; ++i) {
+        gd[i] = dims[i];
+        bd[i] = box[i];
+        es[i] = 1;
+        if (i + 1 < rank) gs[i] = strides_bytes[i];
+    }
+    return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, (cuuint32_t)rank, const_cast<void *>(base), gd, gs, bd, es,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, l2, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+namespace {
+
+// ----------------------------------------------------------------- forward ---
+
+constexpr int TF_EPI = 512;               // epilogue threads
+constexpr int TF_THREADS = TF_EPI + 64;   // + producer warp + MMA warp
+constexpr int TF_MAXNS = 8;               // most x sub-tiles in flight
+constexpr int TF_SMEM = 220 * 1024;
+
+struct FwdSmem {
+    uint32_t zbytes, ubytes, opsize, ring, boxb, slot, bars, tmem, total;
+    __host__ __device__ FwdSmem(const TcMap &m, int ns) {
+        const int rb = m.SF == 32 ? 64 : 128;
+        const int nbx = m.SF == 128 ? 2 : 1;
+        boxb = up1024((uint32_t)(rb * (TC_M + m.W - 1)));
+        slot = (uint32_t)nbx * boxb;
+        zbytes = (uint32_t)(TC_M * m.RP * 2);
+        ubytes = (uint32_t)(m.RP * m.NF * 2);
+        opsize = up1024(zbytes + ubytes);
+        ring = 2 * opsize;
+        bars = ring + (uint32_t)ns * slot;  // OPF[2] OPE[2] WF[2] WE[2] XF[MAXNS] XE[MAXNS]
+        tmem = bars + (8 + 2 * TF_MAXNS) * 8;
+        total = tmem + 16 + 1024;           // + slack to align the base to 1024 bytes
+    }
+};
+
+struct FwdBars {
+    uint32_t base;
+    __device__ uint32_t opf(int b) const { return base + 8u * (uint32_t)b; }
+    __device__ uint32_t ope(int b) const { return base + 16u + 8u * (uint32_t)b; }
+    __device__ uint32_t wf(int b) const { return base + 32u + 8u * (uint32_t)b; }
+    __device__ uint32_t we(int b) const { return base + 48u + 8u * (uint32_t)b; }
+    __device__ uint32_t xf(int s) const { return base + 64u + 8u * (uint32_t)s; }
+    __device__ uint32_t xe(int s) const { return base + 64u + 8u * TF_MAXNS + 8u * (uint32_t)s; }
+};
+
+// Coordinates of consecutive items (tile-major, block-minor), advanced
+// without divisions.
+struct ItemWalk {
+    int blk, t0, b;
+    __device__ void init(const TcMap &m, int64_t item) {
+        const int64_t tile = item / m.nBlkF;
+        blk = (int)(item % m.nBlkF);
+        b = (int)(tile / m.tilesPerSeq);
+        t0 = (int)(tile % m.tilesPerSeq) * TC_M;
+    }
+    __device__ void next(const TcMap &m) {
+        if (++blk == m.nBlkF) {
+            blk = 0;
+            t0 += TC_M;
+            if (t0 >= m.T) {
+                t0 = 0;
+                ++b;
+            }
+        }
+    }
+};
+
+// Epilogue of one sub-tile: y for VPT vectors of 8 channels of token t.
+// GPV: filter groups inside one vector (8/H for H < 8, else 1).  NGT (only
+// for GPV == 1): groups among the thread's 8*VPT channels.
+template <int W, int GPV, int VPT, int NGT, int RB>
+__device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
+                                            int part, int t_loc, int ci0, bf16 *yrow, bool store, float res) {
+    constexpr int WIN = W - 1;
+    constexpr int NT = GPV * W;
+    constexpr int CPG = 8 / GPV;
+    constexpr int VBW = W >= 8 ? 1 : (W == 4 ? 2 : 4);
+    constexpr int VB = VBW < VPT ? VBW : VPT;  // vectors whose x rows are loaded together
+    const int cs0 = part * (8 * VPT);  // sub-tile channel of the thread's first vector
+    float wt[GPV == 1 ? NGT * W : 2 * NT];
+    if constexpr (GPV == 1) {
+        // one TMEM load covers the thread's NGT groups
+        tmem_ld<NGT * W>(tb + (uint32_t)((ci0 >> m.lgH) * W), *reinterpret_cast<float(*)[NGT * W]>(wt));
+        tc::tmem_wait_ld();
+#pragma unroll
+        for (int k = 0; k < NGT * W; k += W) wt[k] += res;
+    } else {
+        tmem_ld<NT>(tb + (uint32_t)((ci0 >> m.lgH) * W), *reinterpret_cast<float(*)[NT]>(wt));
+    }
+#pragma unroll
+    for (int v0 = 0; v0 < VPT; v0 += VB) {
+        uint4 xw[VB][W];
+#pragma unroll
+        for (int vv = 0; vv < VB; ++vv) {
+            const int cs = cs0 + 8 * (v0 + vv);
+            const unsigned char *bx = xs + (uint32_t)(cs / (RB / 2)) * boxb;
+            const int chunk = (cs % (RB / 2)) / 8;
+#pragma unroll
+            for (int k = 0; k < W; ++k)
+                xw[vv][k] = *reinterpret_cast<const uint4 *>(bx + tc::swz<RB>(t_loc + WIN - k, chunk));
+        }
+#pragma unroll
+        for (int vv = 0; vv < VB; ++vv) {
+            const int v = v0 + vv;
+            if constexpr (GPV == 1) {
+                const int gi = (v * NGT) / VPT;  // the vector's group among the thread's
+                u64 yp[4];
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    u64 acc2 = 0ull;
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
+                        const uint32_t word = word_of(xw[vv][k], pp);
+                        const u64 xp = mk2(bf_lo(word), bf_hi(word));
+                        const float wk = wt[gi * W + k];
+                        acc2 = k == 0 ? mul2(mk2(wk, wk), xp) : fma2(mk2(wk, wk), xp, acc2);
+                    }
+                    yp[pp] = acc2;
+                }
+                if (store)
+                    st16(yrow + ci0 + 8 * v,
+                         make_uint4(pack_bf2(lo2(yp[0]), hi2(yp[0])), pack_bf2(lo2(yp[1]), hi2(yp[1])),
+                                    pack_bf2(lo2(yp[2]), hi2(yp[2])), pack_bf2(lo2(yp[3]), hi2(yp[3]))));
+            } else {
+                // several groups per vector: per-vector loads, the next one in flight while this one computes
+                tc::tmem_wait_ld();
+                float *w = wt + (v & 1) * NT;
+                if (v + 1 < VPT)
+                    tmem_ld<NT>(tb + (uint32_t)(((ci0 + 8 * (v + 1)) >> m.lgH) * W),
+                                *reinterpret_cast<float(*)[NT]>(wt + ((v + 1) & 1) * NT));
+                float y[8];
+#pragma unroll
+                for (int pp = 0; pp < 4; ++pp) {
+                    const int g0 = (2 * pp) / CPG, g1 = (2 * pp + 1) / CPG;
+                    float a0 = 0.f, a1 = 0.f;
+#pragma unroll
+                    for (int k = 0; k < W; ++k) {
+                        const uint32_t word = word_of(xw[vv][k], pp);
+                        const float w0 = w[g0 * W + k] + (k == 0 ? res : 0.f);
+                        const float w1 = w[g1 * W + k] + (k == 0 ? res : 0.f);
+                        a0 = k == 0 ? w0 * bf_lo(word) : fmaf(w0, bf_lo(word), a0);
+                        a1 = k == 0 ? w1 * bf_hi(word) : fmaf(w1, bf_hi(word), a1);
+                    }
+                    y[2 * pp] = a0;
+                    y[2 * pp + 1] = a1;
+                }
+                if (store)
+                    st16(yrow + ci0 + 8 * v, make_uint4(pack_bf2(y[0], y[1]), pack_bf2(y[2], y[3]),
+                                                        pack_bf2(y[4], y[5]), pack_bf2(y[6], y[7])));
+            }
+        }
+    }
+}
+
+template <int W, int GPV, int VPT, int NGT>
+__global__ void __launch_bounds__(TF_THREADS, 1)
+    k_lr_tc_fwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmz,
+                const __grid_constant__ CUtensorMap tmu, const TcArgs a) {
+    constexpr int WIN = W - 1;
+    constexpr int RB = VPT == 1 ? 64 : 128;  // x box row bytes
+    constexpr int NBX = VPT == 4 ? 2 : 1;    // x boxes per sub-tile
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    const TcMap &m = a.m;
+    const int NS = m.NSF;
+    const FwdSmem S(m, NS);
+    const int64_t total = m.nItemsF * m.nSubF;
+    const int64_t per = (total + gridDim.x - 1) / gridDim.x;
+    const int64_t g_lo = (int64_t)blockIdx.x * per;
+    const int64_t g_hi = min(total, g_lo + per);
+    if (g_lo >= g_hi) return;
+    const int64_t i_lo = g_lo / m.nSubF;
+    const int nI = (int)((g_hi - 1) / m.nSubF - i_lo + 1);
+    const int nG = (int)(g_hi - g_lo);
+    const int s_first = (int)(g_lo % m.nSubF);          // first sub-tile of the first item
+    const int s_last = (int)((g_hi - 1) % m.nSubF) + 1;  // end of the last item's sub-tiles
+
+    const uint32_t sraw = tc::smem_u32(smem_raw);
+    const uint32_t sbase = (sraw + 1023u) & ~1023u;
+    unsigned char *smem = smem_raw + (sbase - sraw);
+    const FwdBars bars{sbase + S.bars};
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int kz = m.R / 8;  // z boxes loaded per item; k-chunks kz .. RP/8-1 stay zero
+
+    if (tid == 0) {
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(bars.opf(i), 1);
+            tc::mbar_init(bars.ope(i), 1);
+            tc::mbar_init(bars.wf(i), 1);
+            tc::mbar_init(bars.we(i), TF_EPI / 32);
+        }
+        for (int i = 0; i < NS; ++i) {
+            tc::mbar_init(bars.xf(i), 1);
+            tc::mbar_init(bars.xe(i), TF_EPI / 32);
+        }
+        tc::fence_mbar_init();
+    }
+    // zero the padded k-chunks of both z buffers (read by the MMA, never loaded)
+    const int zpad = (m.RP / 8 - kz) * 128;
+    for (int i = tid; i < 2 * zpad; i += TF_THREADS) {
+        const int b = i / zpad, r = i % zpad;
+        *reinterpret_cast<uint4 *>(smem + (uint32_t)b * S.opsize + (uint32_t)kz * 2048 + (uint32_t)r * 16) =
+            make_uint4(0, 0, 0, 0);
+    }
+    tc::fence_proxy_async();
+    if (warp == 17) tc::tmem_alloc(sbase + S.tmem, (uint32_t)(2 * m.NF));
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + S.tmem);
+    bool timed_out = false;
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+        if (!timed_out && !tc::mbar_wait(bar, parity, TC_WAIT_LIMIT)) timed_out = true;  // sticky: later waits skip
+    };
+
+    if (warp == 16) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            tc::tma_prefetch_desc(&tmx);
+            tc::tma_prefetch_desc(&tmz);
+            tc::tma_prefetch_desc(&tmu);
+            ItemWalk it;
+            it.init(m, i_lo);
+            int slot = 0, l = 0;
+            uint32_t xph = 0;
+            for (int li = 0; li < nI; ++li, it.next(m)) {
+                const int b = li & 1;
+                if (li >= 2) wait(bars.ope(b), (uint32_t)(((li - 2) >> 1) & 1));
+                const uint32_t zb = sbase + (uint32_t)b * S.opsize, ub = zb + S.zbytes;
+                tc::mbar_expect_tx(bars.opf(b), (uint32_t)kz * 2048u + S.ubytes);
+                for (int j = 0; j < kz; ++j)
+                    tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, it.b, bars.opf(b));
+                const int col0 = it.blk * m.NF;
+                for (int j = 0; j < m.NF / 8; ++j)
+                    tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), &tmu, col0 + 8 * j, 0, bars.opf(b));
+                const int se = li == nI - 1 ? s_last : m.nSubF;
+                for (int s = li == 0 ? s_first : 0; s < se; ++s, ++l) {
+                    if (l >= NS) wait(bars.xe(slot), xph ^ 1u);
+                    const uint32_t xb = sbase + S.ring + (uint32_t)slot * S.slot;
+                    tc::mbar_expect_tx(bars.xf(slot), (uint32_t)(NBX * RB * (TC_M + WIN)));
+                    const int c = it.blk * m.CF + s * m.SF;
+#pragma unroll
+                    for (int bx = 0; bx < NBX; ++bx)
+                        tc::tma_load_3d(xb + (uint32_t)bx * S.boxb, &tmx, c + bx * (RB / 2), it.t0 - WIN, it.b,
+                                        bars.xf(slot));
+                    if (++slot == NS) {
+                        slot = 0;
+                        xph ^= 1u;
+                    }
+                }
+            }
+        }
+    } else if (warp == 17) {
+        // ----------------------------------------------------------------- MMA
+        if (lane == 0) {
+            const uint32_t id_w = tc::idesc_bf16(TC_M, m.NF, 0, 1);
+            for (int li = 0; li < nI; ++li) {
+                const int b = li & 1;
+                wait(bars.opf(b), (uint32_t)((li >> 1) & 1));
+                if (li >= 2) wait(bars.we(b), (uint32_t)(((li - 2) >> 1) & 1));
+                tc::fence_after_sync();
+                const uint32_t zb = sbase + (uint32_t)b * S.opsize, ub = zb + S.zbytes;
+                for (int ks = 0; ks < m.RP / 16; ++ks) {
+                    const uint64_t ad = tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
+                    const uint64_t bd = tc::smem_desc(ub + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
+                    tc::mma_bf16(tmem + (uint32_t)(b * m.NF), ad, bd, id_w, ks > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(bars.wf(b));
+                tc::mma_commit(bars.ope(b));
+            }
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue
+        const int t_loc = tid & (TC_M - 1), part = tid >> 7, quarter = warp & 3;
+        const float res = m.residual ? 1.f : 0.f;
+        const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
+        ItemWalk it;
+        it.init(m, i_lo);
+        int slot = 0;
+        uint32_t xph = 0;
+        for (int li = 0; li < nI; ++li, it.next(m)) {
+            const int b = li & 1;
+            const int t = it.t0 + t_loc;
+            bf16 *yrow = a.y + ((int64_t)it.b * m.T + t) * m.D + (int64_t)it.blk * m.CF;
+            wait(bars.wf(b), (uint32_t)((li >> 1) & 1));
+            tc::fence_after_sync();
+            const uint32_t tb = tlane + (uint32_t)(b * m.NF);
+            const int se = li == nI - 1 ? s_last : m.nSubF;
+            for (int s = li == 0 ? s_first : 0; s < se; ++s) {
+                wait(bars.xf(slot), xph);
+                fwd_subtile<W, GPV, VPT, NGT, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, part, t_loc,
+                                                  s * m.SF + part * (8 * VPT), yrow, t < m.T, res);
+                __syncwarp();
+                if (lane == 0) tc::mbar_arrive(bars.xe(slot));
+                if (++slot == NS) {
+                    slot = 0;
+                    xph ^= 1u;
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bars.we(b));
+        }
+    }
+
+    // teardown: every load and MMA this CTA issued has landed before the
+    // shared memory and TMEM are given back (bounded, also after a time-out)
+    if (warp == 16 && lane == 0) {
+        for (int s = 0; s < NS && s < nG; ++s) {
+            const int lastl = s + ((nG - 1 - s) / NS) * NS;
+            tc::mbar_wait(bars.xf(s), (uint32_t)((lastl / NS) & 1), TC_WAIT_LIMIT);
+        }
+    }
+    if (warp == 17 && lane == 0) {
+        for (int b = 0; b < 2 && b < nI; ++b) {
+            const int lastli = b + ((nI - 1 - b) / 2) * 2;
+            tc::mbar_wait(bars.ope(b), (uint32_t)((lastli >> 1) & 1), TC_WAIT_LIMIT);
+        }
+    }
+    if (timed_out) atomicExch(&g_dsc_status_tcf, (int)DSC_ERR_TIMEOUT);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (warp == 17) tc::tmem_dealloc(tmem, (uint32_t)(2 * m.NF));
+}
+
+// Forward plan: the widest channel block whose filters fit half of TMEM
+// (NF <= 256 columns), narrowed while it still spans 8 or more sub-tiles of
+// 128 channels; sub-tiles of up to 128 channels (256-byte rows); as many x
+// sub-tiles in flight as shared memory holds (2 .. 8).
+bool tc_fwd_plan(TcMap &m) {
+    int mm = 1;
+    while (TC_GROUPS * 2 * mm * m.W <= 256 && m.D % (TC_GROUPS * m.H * 2 * mm) == 0) mm *= 2;
+    while (mm > 1 && (TC_GROUPS * m.H * mm / 2) / 128 >= 8) mm /= 2;
+    m.CF = (int)(TC_GROUPS * m.H * mm);
+    m.NF = TC_GROUPS * mm * m.W;
+    m.SF = m.CF < 128 ? m.CF : 128;
+    m.nSubF = m.CF / m.SF;
+    m.nBlkF = (int)(m.D / m.CF);
+    m.nItemsF = m.B * (int64_t)m.tilesPerSeq * m.nBlkF;
+    for (m.NSF = TF_MAXNS; m.NSF >= 2; --m.NSF)
+        if (FwdSmem(m, m.NSF).total <= TF_SMEM) return true;
+    return false;
+}
+
+struct FwdMaps {
+    CUtensorMap x, z, u;
+};
+
+bool fwd_maps(const TcArgs &a, FwdMaps &f) {
+    const TcMap &m = a.m;
+    const int rb = m.SF == 32 ? 64 : 128;
+    const uint64_t xd[3] = {(uint64_t)m.D, (uint64_t)m.T, (uint64_t)m.B};
+    const uint64_t xs[2] = {(uint64_t)m.D * 2, (uint64_t)(m.T * m.D * 2)};
+    const uint32_t xb[3] = {(uint32_t)(rb / 2), (uint32_t)(TC_M + m.W - 1), 1};
+    const uint64_t zd[3] = {(uint64_t)m.R, (uint64_t)m.T, (uint64_t)m.B};
+    const uint64_t zs[2] = {(uint64_t)m.R * 2, (uint64_t)(m.T * m.R * 2)};
+    const uint32_t zb[3] = {8, (uint32_t)TC_M, 1};
+    const uint64_t ud[2] = {(uint64_t)m.GW, (uint64_t)m.R};
+    const uint64_t us[1] = {(uint64_t)m.GW * 2};
+    const uint32_t ub[2] = {8, (uint32_t)m.RP};
+    return make_map(&f.x, a.x, 3, xd, xs, xb, rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
+           make_map(&f.z, a.z, 3, zd, zs, zb, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
+           make_map(&f.u, a.U, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
+}
+
+template <int W, int GPV, int VPT, int NGT>
+cudaError_t launch_fwd(const Ctx &c, const TcArgs &a) {
+    const FwdSmem S(a.m, a.m.NSF);
+    static const cudaError_t attr = cudaFuncSetAttribute(k_lr_tc_fwd<W, GPV, VPT, NGT>,
+                                                         cudaFuncAttributeMaxDynamicSharedMemorySize, TF_SMEM);
+    if (attr != cudaSuccess) return attr;
+    if (S.total > TF_SMEM) return cudaErrorInvalidValue;
+    FwdMaps f;
+    if (!fwd_maps(a, f)) return cudaErrorNotSupported;
+    const int64_t total = a.m.nItemsF * a.m.nSubF;
+    const int64_t per = (total + c.sms - 1) / c.sms;
+    const int64_t grid = (total + per - 1) / per;
+    // More than half of TMEM per CTA: enough shared memory that no second CTA shares the SM.
+    const uint32_t smem = 2 * a.m.NF > 256 && S.total < 120 * 1024 ? 120 * 1024 : S.total;
+    k_lr_tc_fwd<W, GPV, VPT, NGT><<<(unsigned)grid, TF_THREADS, smem, c.stream>>>(f.x, f.z, f.u, a);
+    count_launch();
+    return cudaGetLastError();
+}
+
+// A sub-tile's filters fit one block (4 * VPT * GPV * W <= NF <= 256); other
+// combinations never come out of the plan and are not instantiated.
+template <int W, int GPV, int VPT> cudaError_t fwd_by_ngt(const Ctx &c, const TcArgs &a) {
+    if constexpr (GPV > 1) {
+        return launch_fwd<W, GPV, VPT, 1>(c, a);
+    } else {
+        const int ngt = (8 * VPT) >> a.m.lgH;  // groups among the thread's 8*VPT channels (H >= 8)
+        if (ngt <= 1) return launch_fwd<W, 1, VPT, 1>(c, a);
+        if constexpr (VPT >= 2)
+            if (ngt == 2) return launch_fwd<W, 1, VPT, 2>(c, a);
+        if constexpr (VPT == 4)
+            if (ngt == 4) return launch_fwd<W, 1, VPT, 4>(c, a);
+        return cudaErrorNotSupported;
+    }
+}
+
+template <int W, int GPV> cudaError_t fwd_by_vpt(const Ctx &c, const TcArgs &a) {
+    switch (a.m.SF) {
+    case 32: return fwd_by_ngt<W, GPV, 1>(c, a);
+    case 64:
+        if constexpr (2 * GPV * W <= 64) return fwd_by_ngt<W, GPV, 2>(c, a);
+        break;
+    case 128:
+        if constexpr (4 * GPV * W <= 64) return fwd_by_ngt<W, GPV, 4>(c, a);
+        break;
+    }
+    return cudaErrorNotSupported;
+}
+
+template <int W> cudaError_t fwd_by_gpv(const Ctx &c, const TcArgs &a) {
+    switch (a.m.H) {
+    case 1: return fwd_by_vpt<W, 8>(c, a);
+    case 2: return fwd_by_vpt<W, 4>(c, a);
+    case 4: return fwd_by_vpt<W, 2>(c, a);
+    default: return fwd_by_vpt<W, 1>(c, a);
+    }
+}
+
+}  // namespace
+}  // namespace lrtc
+
+bool lowrank_tc_ok(const dsc_problem &p) {
+    lrtc::TcMap m;
+    return lrtc::tc_map(p, m) && lrtc::tc_fwd_plan(m);
+}
+
+cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U, void *y) {
+    lrtc::TcArgs a{};
+    if (!lrtc::tc_map(p, a.m) || !lrtc::tc_fwd_plan(a.m)) return cudaErrorNotSupported;
+    a.x = static_cast<const bf16 *>(x);
+    a.z = static_cast<const bf16 *>(z);
+    a.U = static_cast<const bf16 *>(U);
+    a.y = static_cast<bf16 *>(y);
+    switch (a.m.W) {
+    case 1: return lrtc::fwd_by_gpv<1>(c, a);
+    case 2: return lrtc::fwd_by_gpv<2>(c, a);
+    case 4: return lrtc::fwd_by_gpv<4>(c, a);
+    case 8: return lrtc::fwd_by_gpv<8>(c, a);
+    }
+    return cudaErrorNotSupported;
+}
+
+}  // namespace dsc

@@ -116,5 +116,46 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, long lo
     }
 }
 
+// One arrival on the mbarrier.
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+// One arrival that also raises the phase's expected transaction count by `bytes`.
+__device__ __forceinline__ void mbar_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes) : "memory");
+}
+
+// Tensor-memory-access (TMA) tile loads into this CTA's shared memory; the
+// mbarrier's transaction count drops by the box's bytes when they land.
+// Coordinates are element indices, innermost first; boxes that reach outside
+// the tensor are filled with zeros.  No multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int c0, int c1, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+            dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int c0, int c1, int c2, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], "
+        "[%5];" ::"r"(dst),
+        "l"(reinterpret_cast<uint64_t>(tmap)), "r"(c0), "r"(c1), "r"(c2), "r"(bar)
+        : "memory");
+}
+__device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(tmap)) : "memory");
+}
+
+// Byte offset of the 16-byte chunk `chunk` of row `row` in a tile that a TMA
+// load wrote with 64- or 128-byte swizzling (rows of RB = 64 or 128 bytes,
+// tile base aligned to 1024 bytes): address bits [4, 4+b) are XORed with bits
+// [7, 7+b), b = log2(RB / 16).
+template <int RB> __device__ __forceinline__ uint32_t swz(int row, int chunk) {
+    static_assert(RB == 64 || RB == 128, "64- or 128-byte rows");
+    const uint32_t off = (uint32_t)row * RB;
+    return off + ((((uint32_t)chunk) ^ ((off >> 7) & (RB / 16 - 1))) << 4);
+}
+
 }  // namespace tc
 }  // namespace dsc

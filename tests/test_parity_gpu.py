@@ -158,6 +158,13 @@ LOWRANK_SHAPES = [
     (1, 140, 512, 4, 16, 16),
     (2, 150, 2048, 4, 64, 32),
     (1, 260, 256, 8, 8, 24),
+    # enough tiles that each tensor-core CTA walks several items: operand and
+    # TMEM double buffers and the sub-tile ring wrap, items split between CTAs
+    (4, 1024, 4096, 4, 1, 32),
+    (2, 1000, 8192, 4, 64, 64),
+    (2, 700, 2048, 8, 2, 48),
+    (2, 600, 1024, 8, 1, 16),
+    (2, 500, 4096, 2, 1, 32),
 ]
 
 
@@ -229,6 +236,45 @@ def test_outputs_do_not_touch_neighbouring_memory():
         assert torch.all(b[:pad] == 7.0) and torch.all(b[pad + n:] == 7.0)
     ref = run_oracle(wl, t)
     assert rel_err(to_host64(buf_y[pad:pad + n_y]).reshape(ref["y"].shape), ref["y"]) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("shape", [(2, 150, 2048, 4, 64, 32), (1, 200, 256, 4, 1, 16), (2, 70, 512, 8, 8, 24)],
+                         ids=lambda s: "B{}T{}D{}W{}H{}R{}".format(*s))
+def test_lowrank_outputs_do_not_touch_neighbouring_memory(shape):
+    """Canary bands around y, dx, dz and dU of the tensor-core low-rank kernels
+    (TMA loads, ragged last tile, partial-sum workspaces)."""
+    from input_dependent_short_b200 import _lib
+
+    o = ops()
+    B, T, D, W, H, R = shape
+    wl = W_("canary-lr", LOWRANK, B, T, D, W, H, R)
+    t = wls.make_inputs(wl)
+    x, z, U, dy = (to_dev(t[k], "bf16") for k in ("x", "z", "U", "dy"))
+    pad = 4096
+    L = _lib.lib()
+
+    def band(n, dtype):
+        return torch.full((n + 2 * pad,), 7.0, device="cuda", dtype=dtype)
+
+    buf = {"y": band(x.numel(), torch.bfloat16), "dx": band(x.numel(), torch.bfloat16),
+           "dz": band(z.numel(), torch.bfloat16), "dU": band(U.numel(), torch.float32)}
+    p = o.problem(x, W, H, R)
+    s = torch.cuda.current_stream().cuda_stream
+    nf, nb = L.dsc_fwd_lowrank_workspace_bytes(p), L.dsc_bwd_lowrank_workspace_bytes(p)
+    wsf = torch.empty(max(nf, 16), dtype=torch.uint8, device="cuda")
+    wsb = torch.empty(max(nb, 16), dtype=torch.uint8, device="cuda")
+    _lib.call("dsc_fwd_lowrank", p, x.data_ptr(), z.data_ptr(), U.data_ptr(), buf["y"][pad:].data_ptr(),
+              wsf.data_ptr(), nf, s)
+    _lib.call("dsc_bwd_lowrank", p, x.data_ptr(), z.data_ptr(), U.data_ptr(), dy.data_ptr(),
+              buf["dx"][pad:].data_ptr(), buf["dz"][pad:].data_ptr(), buf["dU"][pad:].data_ptr(),
+              wsb.data_ptr(), nb, s)
+    torch.cuda.synchronize()
+    assert L.dsc_check(s) == _lib.DSC_OK
+    ref = run_oracle(wl, t)
+    for k, b in buf.items():
+        n = ref[k].size
+        assert torch.all(b[:pad] == 7.0) and torch.all(b[pad + n:] == 7.0), k
+        assert rel_err(to_host64(b[pad:pad + n]).reshape(ref[k].shape), ref[k]) <= TOL["bf16"], k
 
 
 # ------------------------------------------------- full-size workloads ---
