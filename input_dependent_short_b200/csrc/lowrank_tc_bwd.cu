@@ -60,17 +60,19 @@ constexpr int TB_ZROWS = 136;            // z rows per tile: 128 + up to 7 for t
 constexpr uint32_t TB_ZR = TB_ZROWS * 16;  // bytes per 8-wide k-chunk of the z tile
 
 struct BwdSmem {
-    uint32_t zbytes, ubytes, opsize, dw, dwsize, xch, ring, boxb, slot, bars, tmem, total;
+    uint32_t zbytes, ubytes, opsize, dw, dwsize, xch, ystage, ybox, ring, boxb, slot, bars, tmem, total;
     __host__ __device__ BwdSmem(const TcMap &m, int nop, int ns, int dwb, bool xchg) {
         const int rb = m.SB == 32 ? 64 : 128;
         boxb = up1024((uint32_t)(rb * (TC_M + m.W - 1)));
         slot = 2 * boxb;  // x box + dy box
+        ybox = (uint32_t)(rb * TC_M);
         zbytes = (uint32_t)(m.RP / 8) * TB_ZR;
         ubytes = (uint32_t)(m.RP * TB_NB * 2);
         opsize = up1024(zbytes + ubytes);
         dw = (uint32_t)nop * opsize;
         dwsize = (uint32_t)(TC_M * TB_NB * 2);
-        xch = dw + (uint32_t)dwb * dwsize;
+        ystage = dw + (uint32_t)dwb * dwsize;  // two dx staging tiles (TMA store sources)
+        xch = ystage + 2 * ybox;
         ring = up1024(xch + (xchg ? (uint32_t)(2 * 4 * TC_M * m.W * 4) : 0u));
         bars = ring + (uint32_t)ns * slot;
         tmem = bars + (17 + 2 * TB_MAXNS) * 8;
@@ -148,8 +150,8 @@ template <int N> __device__ __forceinline__ void st_dw(unsigned char *p, const f
 //   (1 when the group is wider: PPG parts then share it).
 template <int W, int VPT, int GPT, int PPG, int RB>
 __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
-                                            unsigned char *dwt, float *xch, int part, int t_loc, int s, bf16 *dxrow,
-                                            bool store, float res) {
+                                            unsigned char *dwt, float *xch, int part, int t_loc, int s,
+                                            unsigned char *ys, float res) {
     constexpr int WIN = W - 1;
     constexpr int CT = 8 * VPT;                      // the thread's channels
     constexpr int GPV = GPT >= VPT ? GPT / VPT : 1;  // groups inside one vector
@@ -205,9 +207,9 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
                 dxv[2 * pp + 1] = a1;
             }
         }
-        if (store)
-            st16(dxrow + ci0 + 8 * v, make_uint4(pack_bf2(dxv[0], dxv[1]), pack_bf2(dxv[2], dxv[3]),
-                                                 pack_bf2(dxv[4], dxv[5]), pack_bf2(dxv[6], dxv[7])));
+        *reinterpret_cast<uint4 *>(ys + tc::swz<RB>(t_loc, ((cs0 + 8 * v) % (RB / 2)) / 8)) =
+            make_uint4(pack_bf2(dxv[0], dxv[1]), pack_bf2(dxv[2], dxv[3]), pack_bf2(dxv[4], dxv[5]),
+                       pack_bf2(dxv[6], dxv[7]));
     }
     // dw[t, g, k] over the thread's channels
     float pk[W][GPT];
@@ -257,7 +259,8 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
 template <int W, int VPT, int GPT, int PPG>
 __global__ void __launch_bounds__(TB_THREADS, 1)
     k_lr_tc_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmdy,
-                const __grid_constant__ CUtensorMap tmz, const __grid_constant__ CUtensorMap tmu, const TcArgs a) {
+                const __grid_constant__ CUtensorMap tmz, const __grid_constant__ CUtensorMap tmu,
+                const __grid_constant__ CUtensorMap tmdx, const TcArgs a) {
     constexpr int WIN = W - 1;
     constexpr int RB = VPT == 1 ? 64 : 128;  // box row bytes (32 or 64 channels)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -454,24 +457,33 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         };
         BwdWalk it;
         it.init(m, tile_lo, chunk_lo);
-        int slot = 0, db = 0, pb = 0, pt0 = 0;
+        int slot = 0, db = 0, pb = 0, pt0 = 0, ybuf = 0;
         uint32_t xph = 0, dph = 0;
         for (int li = 0; li < nI; ++li) {
             const int b = li & 1;
-            const int t = it.t0 + t_loc;
             if (li >= 1 && it.cl == 0) dz_out(it.tl - 1, pb, pt0);  // previous tile done
             wait(bars.wf(b), (uint32_t)((li >> 1) & 1));
             if (li >= DWB) wait(bars.dwe(db), dph ^ 1u);
             tc::fence_after_sync();
             const uint32_t tb = tlane + (uint32_t)(b * TB_NB);
             unsigned char *dwt = smem + S.dw + (uint32_t)db * S.dwsize;
-            bf16 *dxrow = a.dx + ((int64_t)it.b * m.T + t) * m.D + (int64_t)it.blk * m.CB;
             for (int s = 0; s < m.nSubB; ++s) {
                 wait(bars.xf(slot), xph);
                 bwd_subtile<W, VPT, GPT, PPG, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, xch, part,
-                                                  t_loc, s, dxrow, t < m.T, res);
+                                                  t_loc, s, smem + S.ystage + (uint32_t)ybuf * S.ybox, res);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars.xe(slot));
+                // dx tile -> global by TMA (the staging tile the next sub-tile writes was read
+                // by the store issued one sub-tile ago, waited for before this barrier)
+                tc::fence_proxy_async();
+                if (tid == 0) tc::bulk_wait_read_all();
+                epi_bar();
+                if (tid == 0) {
+                    tc::tma_store_3d(&tmdx, sbase + S.ystage + (uint32_t)ybuf * S.ybox, it.blk * m.CB + s * m.SB, it.t0,
+                                     it.b);
+                    tc::bulk_commit();
+                }
+                ybuf ^= 1;
                 if (++slot == NS) {
                     slot = 0;
                     xph ^= 1u;
@@ -513,6 +525,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                 }
             }
         }
+        if (tid == 0) tc::bulk_wait_all();
     }
 
     // teardown: every load and MMA this CTA issued has landed before the
@@ -625,7 +638,7 @@ size_t tc_bwd_ws_bytes(const TcMap &m) {
 }
 
 struct BwdMaps {
-    CUtensorMap x, dy, z, u;
+    CUtensorMap x, dy, z, u, dx;
 };
 
 bool bwd_maps(const TcArgs &a, BwdMaps &f) {
@@ -634,6 +647,7 @@ bool bwd_maps(const TcArgs &a, BwdMaps &f) {
     const uint64_t xd[3] = {(uint64_t)m.D, (uint64_t)m.T, (uint64_t)m.B};
     const uint64_t xs[2] = {(uint64_t)m.D * 2, (uint64_t)(m.T * m.D * 2)};
     const uint32_t xb[3] = {(uint32_t)(rb / 2), (uint32_t)(TC_M + m.W - 1), 1};
+    const uint32_t yb[3] = {(uint32_t)(rb / 2), (uint32_t)TC_M, 1};
     const uint64_t zd[3] = {(uint64_t)m.R, (uint64_t)m.T, (uint64_t)m.B};
     const uint64_t zs[2] = {(uint64_t)m.R * 2, (uint64_t)(m.T * m.R * 2)};
     const uint32_t zb[3] = {8, (uint32_t)TB_ZROWS, 1};
@@ -643,6 +657,7 @@ bool bwd_maps(const TcArgs &a, BwdMaps &f) {
     const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     return make_map(&f.x, a.x, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
            make_map(&f.dy, a.dy, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
+           make_map(&f.dx, a.dx, 3, xd, xs, yb, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE) &&
            make_map(&f.z, a.z, 3, zd, zs, zb, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
            make_map(&f.u, a.Up, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
 }
@@ -659,7 +674,7 @@ cudaError_t launch_bwd(const Ctx &c, const TcArgs &a) {
     // the whole of TMEM per CTA: enough shared memory that no second CTA shares the SM
     const uint32_t smem = S.total < 120 * 1024 ? 120 * 1024 : S.total;
     k_lr_tc_bwd<W, VPT, GPT, PPG><<<(unsigned)(a.m.nGroups * a.m.nRanges), TB_THREADS, smem, c.stream>>>(f.x, f.dy, f.z,
-                                                                                                       f.u, a);
+                                                                                                       f.u, f.dx, a);
     count_launch();
     return cudaGetLastError();
 }

@@ -129,19 +129,21 @@ constexpr int TF_MAXNS = 8;               // most x sub-tiles in flight
 constexpr int TF_SMEM = 220 * 1024;
 
 struct FwdSmem {
-    uint32_t zbytes, ubytes, opsize, ring, boxb, slot, bars, tmem, total;
+    uint32_t zbytes, ubytes, opsize, ring, boxb, slot, ystage, ybox, bars, tmem, total;
     __host__ __device__ FwdSmem(const TcMap &m, int ns) {
         const int rb = m.SF == 32 ? 64 : 128;
         const int nbx = m.SF == 128 ? 2 : 1;
         boxb = up1024((uint32_t)(rb * (TC_M + m.W - 1)));
         slot = (uint32_t)nbx * boxb;
+        ybox = (uint32_t)(rb * TC_M);
         zbytes = (uint32_t)(TC_M * m.RP * 2);
         ubytes = (uint32_t)(m.RP * m.NF * 2);
         opsize = up1024(zbytes + ubytes);
-        ring = 2 * opsize;
-        bars = ring + (uint32_t)ns * slot;  // OPF[2] OPE[2] WF[2] WE[2] XF[MAXNS] XE[MAXNS]
+        ystage = 2 * opsize;                      // two y staging tiles (TMA store sources)
+        ring = ystage + 2 * (uint32_t)nbx * ybox;
+        bars = ring + (uint32_t)ns * slot;        // OPF[2] OPE[2] WF[2] WE[2] XF[MAXNS] XE[MAXNS]
         tmem = bars + (8 + 2 * TF_MAXNS) * 8;
-        total = tmem + 16 + 1024;           // + slack to align the base to 1024 bytes
+        total = tmem + 16 + 1024;                 // + slack to align the base to 1024 bytes
     }
 };
 
@@ -155,23 +157,24 @@ struct FwdBars {
     __device__ uint32_t xe(int s) const { return base + 64u + 8u * TF_MAXNS + 8u * (uint32_t)s; }
 };
 
-// Coordinates of consecutive items (tile-major, block-minor), advanced
-// without divisions.
+// Coordinates of consecutive items (block-major, tile-minor: a CTA keeps one
+// U block for many items), advanced without divisions.
 struct ItemWalk {
     int blk, t0, b;
     __device__ void init(const TcMap &m, int64_t item) {
-        const int64_t tile = item / m.nBlkF;
-        blk = (int)(item % m.nBlkF);
+        const int64_t ntiles = m.B * (int64_t)m.tilesPerSeq;
+        blk = (int)(item / ntiles);
+        const int64_t tile = item % ntiles;
         b = (int)(tile / m.tilesPerSeq);
         t0 = (int)(tile % m.tilesPerSeq) * TC_M;
     }
     __device__ void next(const TcMap &m) {
-        if (++blk == m.nBlkF) {
-            blk = 0;
-            t0 += TC_M;
-            if (t0 >= m.T) {
-                t0 = 0;
-                ++b;
+        t0 += TC_M;
+        if (t0 >= m.T) {
+            t0 = 0;
+            if (++b == m.B) {
+                b = 0;
+                ++blk;
             }
         }
     }
@@ -182,7 +185,7 @@ struct ItemWalk {
 // for GPV == 1): groups among the thread's 8*VPT channels.
 template <int W, int GPV, int VPT, int NGT, int RB>
 __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
-                                            int part, int t_loc, int ci0, bf16 *yrow, bool store, float res) {
+                                            int part, int t_loc, int ci0, unsigned char *ys, uint32_t ybox, float res) {
     constexpr int WIN = W - 1;
     constexpr int NT = GPV * W;
     constexpr int CPG = 8 / GPV;
@@ -229,10 +232,10 @@ __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char 
                     }
                     yp[pp] = acc2;
                 }
-                if (store)
-                    st16(yrow + ci0 + 8 * v,
-                         make_uint4(pack_bf2(lo2(yp[0]), hi2(yp[0])), pack_bf2(lo2(yp[1]), hi2(yp[1])),
-                                    pack_bf2(lo2(yp[2]), hi2(yp[2])), pack_bf2(lo2(yp[3]), hi2(yp[3]))));
+                const int cs = cs0 + 8 * v;
+                *reinterpret_cast<uint4 *>(ys + (uint32_t)(cs / (RB / 2)) * ybox + tc::swz<RB>(t_loc, (cs % (RB / 2)) / 8)) =
+                    make_uint4(pack_bf2(lo2(yp[0]), hi2(yp[0])), pack_bf2(lo2(yp[1]), hi2(yp[1])),
+                               pack_bf2(lo2(yp[2]), hi2(yp[2])), pack_bf2(lo2(yp[3]), hi2(yp[3])));
             } else {
                 // several groups per vector: per-vector loads, the next one in flight while this one computes
                 tc::tmem_wait_ld();
@@ -256,9 +259,9 @@ __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char 
                     y[2 * pp] = a0;
                     y[2 * pp + 1] = a1;
                 }
-                if (store)
-                    st16(yrow + ci0 + 8 * v, make_uint4(pack_bf2(y[0], y[1]), pack_bf2(y[2], y[3]),
-                                                        pack_bf2(y[4], y[5]), pack_bf2(y[6], y[7])));
+                const int cs = cs0 + 8 * v;
+                *reinterpret_cast<uint4 *>(ys + (uint32_t)(cs / (RB / 2)) * ybox + tc::swz<RB>(t_loc, (cs % (RB / 2)) / 8)) =
+                    make_uint4(pack_bf2(y[0], y[1]), pack_bf2(y[2], y[3]), pack_bf2(y[4], y[5]), pack_bf2(y[6], y[7]));
             }
         }
     }
@@ -267,7 +270,7 @@ __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char 
 template <int W, int GPV, int VPT, int NGT>
 __global__ void __launch_bounds__(TF_THREADS, 1)
     k_lr_tc_fwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmz,
-                const __grid_constant__ CUtensorMap tmu, const TcArgs a) {
+                const __grid_constant__ CUtensorMap tmu, const __grid_constant__ CUtensorMap tmy, const TcArgs a) {
     constexpr int WIN = W - 1;
     constexpr int RB = VPT == 1 ? 64 : 128;  // x box row bytes
     constexpr int NBX = VPT == 4 ? 2 : 1;    // x boxes per sub-tile
@@ -333,17 +336,23 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
             ItemWalk it;
             it.init(m, i_lo);
             int slot = 0, l = 0;
+            int ublk0 = -1, ublk1 = -1;  // U block held by each operand buffer
             uint32_t xph = 0;
             for (int li = 0; li < nI; ++li, it.next(m)) {
                 const int b = li & 1;
                 if (li >= 2) wait(bars.ope(b), (uint32_t)(((li - 2) >> 1) & 1));
                 const uint32_t zb = sbase + (uint32_t)b * S.opsize, ub = zb + S.zbytes;
-                tc::mbar_expect_tx(bars.opf(b), (uint32_t)kz * 2048u + S.ubytes);
+                const bool newu = (b ? ublk1 : ublk0) != it.blk;
+                tc::mbar_expect_tx(bars.opf(b), (uint32_t)kz * 2048u + (newu ? S.ubytes : 0u));
                 for (int j = 0; j < kz; ++j)
                     tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, it.b, bars.opf(b));
-                const int col0 = it.blk * m.NF;
-                for (int j = 0; j < m.NF / 8; ++j)
-                    tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), &tmu, col0 + 8 * j, 0, bars.opf(b));
+                if (newu) {
+                    if (b) ublk1 = it.blk;
+                    else ublk0 = it.blk;
+                    const int col0 = it.blk * m.NF;
+                    for (int j = 0; j < m.NF / 8; ++j)
+                        tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), &tmu, col0 + 8 * j, 0, bars.opf(b));
+                }
                 const int se = li == nI - 1 ? s_last : m.nSubF;
                 for (int s = li == 0 ? s_first : 0; s < se; ++s, ++l) {
                     if (l >= NS) wait(bars.xe(slot), xph ^ 1u);
@@ -387,22 +396,35 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
         const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
         ItemWalk it;
         it.init(m, i_lo);
-        int slot = 0;
+        int slot = 0, ybuf = 0;
         uint32_t xph = 0;
         for (int li = 0; li < nI; ++li, it.next(m)) {
             const int b = li & 1;
-            const int t = it.t0 + t_loc;
-            bf16 *yrow = a.y + ((int64_t)it.b * m.T + t) * m.D + (int64_t)it.blk * m.CF;
             wait(bars.wf(b), (uint32_t)((li >> 1) & 1));
             tc::fence_after_sync();
             const uint32_t tb = tlane + (uint32_t)(b * m.NF);
             const int se = li == nI - 1 ? s_last : m.nSubF;
             for (int s = li == 0 ? s_first : 0; s < se; ++s) {
                 wait(bars.xf(slot), xph);
+                unsigned char *ys = smem + S.ystage + (uint32_t)ybuf * NBX * S.ybox;
                 fwd_subtile<W, GPV, VPT, NGT, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, part, t_loc,
-                                                  s * m.SF + part * (8 * VPT), yrow, t < m.T, res);
+                                                  s * m.SF + part * (8 * VPT), ys, S.ybox, res);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars.xe(slot));
+                // y tile -> global by TMA: the staging tile the next sub-tile writes was
+                // read by the store issued one sub-tile ago, waited for before the barrier
+                tc::fence_proxy_async();
+                if (tid == 0) tc::bulk_wait_read_all();
+                asm volatile("bar.sync 1, %0;" ::"n"(TF_EPI) : "memory");
+                if (tid == 0) {
+                    const int c = it.blk * m.CF + s * m.SF;
+#pragma unroll
+                    for (int bx = 0; bx < NBX; ++bx)
+                        tc::tma_store_3d(&tmy, sbase + S.ystage + (uint32_t)(ybuf * NBX + bx) * S.ybox, c + bx * (RB / 2),
+                                         it.t0, it.b);
+                    tc::bulk_commit();
+                }
+                ybuf ^= 1;
                 if (++slot == NS) {
                     slot = 0;
                     xph ^= 1u;
@@ -412,6 +434,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(bars.we(b));
         }
+        if (tid == 0) tc::bulk_wait_all();
     }
 
     // teardown: every load and MMA this CTA issued has landed before the
@@ -437,15 +460,15 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
 
 // Forward plan: the widest channel block whose filters fit half of TMEM
 // (NF <= 256 columns), narrowed while it still spans 8 or more sub-tiles of
-// 128 channels; sub-tiles of up to 128 channels (256-byte rows); as many x
-// sub-tiles in flight as shared memory holds (2 .. 8).
+// 128 channels; sub-tiles of up to 64 channels (128-byte rows, one TMA box);
+// as many x sub-tiles in flight as shared memory holds (2 .. 8).
 bool tc_fwd_plan(TcMap &m) {
     int mm = 1;
     while (TC_GROUPS * 2 * mm * m.W <= 256 && m.D % (TC_GROUPS * m.H * 2 * mm) == 0) mm *= 2;
     while (mm > 1 && (TC_GROUPS * m.H * mm / 2) / 128 >= 8) mm /= 2;
     m.CF = (int)(TC_GROUPS * m.H * mm);
     m.NF = TC_GROUPS * mm * m.W;
-    m.SF = m.CF < 128 ? m.CF : 128;
+    m.SF = m.CF < 64 ? m.CF : 64;
     m.nSubF = m.CF / m.SF;
     m.nBlkF = (int)(m.D / m.CF);
     m.nItemsF = m.B * (int64_t)m.tilesPerSeq * m.nBlkF;
@@ -455,7 +478,7 @@ bool tc_fwd_plan(TcMap &m) {
 }
 
 struct FwdMaps {
-    CUtensorMap x, z, u;
+    CUtensorMap x, z, u, y;
 };
 
 bool fwd_maps(const TcArgs &a, FwdMaps &f) {
@@ -464,14 +487,16 @@ bool fwd_maps(const TcArgs &a, FwdMaps &f) {
     const uint64_t xd[3] = {(uint64_t)m.D, (uint64_t)m.T, (uint64_t)m.B};
     const uint64_t xs[2] = {(uint64_t)m.D * 2, (uint64_t)(m.T * m.D * 2)};
     const uint32_t xb[3] = {(uint32_t)(rb / 2), (uint32_t)(TC_M + m.W - 1), 1};
+    const uint32_t yb[3] = {(uint32_t)(rb / 2), (uint32_t)TC_M, 1};
     const uint64_t zd[3] = {(uint64_t)m.R, (uint64_t)m.T, (uint64_t)m.B};
     const uint64_t zs[2] = {(uint64_t)m.R * 2, (uint64_t)(m.T * m.R * 2)};
     const uint32_t zb[3] = {8, (uint32_t)TC_M, 1};
     const uint64_t ud[2] = {(uint64_t)m.GW, (uint64_t)m.R};
     const uint64_t us[1] = {(uint64_t)m.GW * 2};
     const uint32_t ub[2] = {8, (uint32_t)m.RP};
-    return make_map(&f.x, a.x, 3, xd, xs, xb, rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
+    const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    return make_map(&f.x, a.x, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
+           make_map(&f.y, a.y, 3, xd, xs, yb, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE) &&
            make_map(&f.z, a.z, 3, zd, zs, zb, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
            make_map(&f.u, a.U, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
 }
@@ -490,7 +515,7 @@ cudaError_t launch_fwd(const Ctx &c, const TcArgs &a) {
     const int64_t grid = (total + per - 1) / per;
     // More than half of TMEM per CTA: enough shared memory that no second CTA shares the SM.
     const uint32_t smem = 2 * a.m.NF > 256 && S.total < 120 * 1024 ? 120 * 1024 : S.total;
-    k_lr_tc_fwd<W, GPV, VPT, NGT><<<(unsigned)grid, TF_THREADS, smem, c.stream>>>(f.x, f.z, f.u, a);
+    k_lr_tc_fwd<W, GPV, VPT, NGT><<<(unsigned)grid, TF_THREADS, smem, c.stream>>>(f.x, f.z, f.u, f.y, a);
     count_launch();
     return cudaGetLastError();
 }
@@ -516,9 +541,6 @@ template <int W, int GPV> cudaError_t fwd_by_vpt(const Ctx &c, const TcArgs &a) 
     case 32: return fwd_by_ngt<W, GPV, 1>(c, a);
     case 64:
         if constexpr (2 * GPV * W <= 64) return fwd_by_ngt<W, GPV, 2>(c, a);
-        break;
-    case 128:
-        if constexpr (4 * GPV * W <= 64) return fwd_by_ngt<W, GPV, 4>(c, a);
         break;
     }
     return cudaErrorNotSupported;
