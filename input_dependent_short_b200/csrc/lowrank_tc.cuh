@@ -47,7 +47,8 @@ struct TcArgs {
     const bf16 *x, *z, *U, *dy;
     bf16 *y, *dx, *dz;
     float *dU, *dz_acc, *dU_part;
-    bf16 *Up;  // backward: U with the columns of each block in tap-major order
+    bf16 *Up;    // backward: U blocks as shared-memory images (columns tap-major, rows padded to RP)
+    bf16 *zimg;  // backward: z tiles (136 rows) as shared-memory images
 };
 
 // Fills the common part of the map; false when the tensor-core kernels do not take the shape.

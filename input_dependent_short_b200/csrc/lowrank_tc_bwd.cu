@@ -58,6 +58,8 @@ constexpr int TB_SMEM = 220 * 1024;
 constexpr int TB_NB = 128;               // filter columns per block (W * GB)
 constexpr int TB_ZROWS = 136;            // z rows per tile: 128 + up to 7 for the shifted filters
 constexpr uint32_t TB_ZR = TB_ZROWS * 16;  // bytes per 8-wide k-chunk of the z tile
+constexpr int TB_MAXOP = 4;              // most operand (z, U) buffers
+constexpr int TB_NBARS = 2 * TB_MAXOP + 13 + 2 * TB_MAXNS;
 
 struct BwdSmem {
     uint32_t zbytes, ubytes, opsize, dw, dwsize, xch, ystage, ybox, ring, boxb, slot, bars, tmem, total;
@@ -75,25 +77,25 @@ struct BwdSmem {
         xch = ystage + 2 * ybox;
         ring = up1024(xch + (xchg ? (uint32_t)(2 * 4 * TC_M * m.W * 4) : 0u));
         bars = ring + (uint32_t)ns * slot;
-        tmem = bars + (17 + 2 * TB_MAXNS) * 8;
+        tmem = bars + TB_NBARS * 8;
         total = tmem + 16 + 1024;  // + slack to align the base to 1024 bytes
     }
 };
 
-// OPF[3] OPE[3] WF[2] WE[2] DWF[2] DWE[2] DZF[2] DZE[2] DUF XF[MAXNS] XE[MAXNS]
+// OPF[4] OPE[4] WF[2] WE[2] DWF[2] DWE[2] DZF[2] DZE[2] DUF XF[MAXNS] XE[MAXNS]
 struct BwdBars {
     uint32_t base;
     __device__ uint32_t opf(int b) const { return base + 8u * (uint32_t)b; }
-    __device__ uint32_t ope(int b) const { return base + 24u + 8u * (uint32_t)b; }
-    __device__ uint32_t wf(int b) const { return base + 48u + 8u * (uint32_t)b; }
-    __device__ uint32_t we(int b) const { return base + 64u + 8u * (uint32_t)b; }
-    __device__ uint32_t dwf(int b) const { return base + 80u + 8u * (uint32_t)b; }
-    __device__ uint32_t dwe(int b) const { return base + 96u + 8u * (uint32_t)b; }
-    __device__ uint32_t dzf(int b) const { return base + 112u + 8u * (uint32_t)b; }
-    __device__ uint32_t dze(int b) const { return base + 128u + 8u * (uint32_t)b; }
-    __device__ uint32_t duf() const { return base + 144u; }
-    __device__ uint32_t xf(int s) const { return base + 152u + 8u * (uint32_t)s; }
-    __device__ uint32_t xe(int s) const { return base + 152u + 8u * TB_MAXNS + 8u * (uint32_t)s; }
+    __device__ uint32_t ope(int b) const { return base + 32u + 8u * (uint32_t)b; }
+    __device__ uint32_t wf(int b) const { return base + 64u + 8u * (uint32_t)b; }
+    __device__ uint32_t we(int b) const { return base + 80u + 8u * (uint32_t)b; }
+    __device__ uint32_t dwf(int b) const { return base + 96u + 8u * (uint32_t)b; }
+    __device__ uint32_t dwe(int b) const { return base + 112u + 8u * (uint32_t)b; }
+    __device__ uint32_t dzf(int b) const { return base + 128u + 8u * (uint32_t)b; }
+    __device__ uint32_t dze(int b) const { return base + 144u + 8u * (uint32_t)b; }
+    __device__ uint32_t duf() const { return base + 160u; }
+    __device__ uint32_t xf(int s) const { return base + 168u + 8u * (uint32_t)s; }
+    __device__ uint32_t xe(int s) const { return base + 168u + 8u * TB_MAXNS + 8u * (uint32_t)s; }
 };
 
 // Items of a CTA in order (tile-major, block-minor), advanced without divisions.
@@ -259,7 +261,6 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
 template <int W, int VPT, int GPT, int PPG>
 __global__ void __launch_bounds__(TB_THREADS, 1)
     k_lr_tc_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmdy,
-                const __grid_constant__ CUtensorMap tmz, const __grid_constant__ CUtensorMap tmu,
                 const __grid_constant__ CUtensorMap tmdx, const TcArgs a) {
     constexpr int WIN = W - 1;
     constexpr int RB = VPT == 1 ? 64 : 128;  // box row bytes (32 or 64 channels)
@@ -282,11 +283,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
     unsigned char *smem = smem_raw + (sbase - sraw);
     const BwdBars bars{sbase + S.bars};
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int kz = m.R / 8;  // z k-chunks loaded per item; kz .. RP/8-1 stay zero
     const uint32_t col_dz = 2 * TB_NB, col_dU = 2 * TB_NB + 2 * m.RP;
 
     if (tid == 0) {
-        for (int i = 0; i < 3; ++i) {
+        for (int i = 0; i < TB_MAXOP; ++i) {
             tc::mbar_init(bars.opf(i), 1);
             tc::mbar_init(bars.ope(i), 1);
         }
@@ -305,14 +305,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         }
         tc::fence_mbar_init();
     }
-    // zero the padded k-chunks of every z buffer (read by the MMAs, never loaded)
-    const int zpad = (m.RP / 8 - kz) * TB_ZROWS;
-    for (int i = tid; i < NOP * zpad; i += TB_THREADS) {
-        const int b = i / zpad, r = i % zpad;
-        *reinterpret_cast<uint4 *>(smem + (uint32_t)b * S.opsize + (uint32_t)kz * TB_ZR + (uint32_t)r * 16) =
-            make_uint4(0, 0, 0, 0);
-    }
-    tc::fence_proxy_async();
     if (warp == 17) tc::tmem_alloc(sbase + S.tmem, 512);
     tc::fence_before_sync();
     __syncthreads();
@@ -324,27 +316,36 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
     };
 
     if (warp == 16) {
-        // ------------------------------------------------------------ producer
+        // ----------------------------------------------------- producers
         if (lane == 0) {
-            tc::tma_prefetch_desc(&tmx);
-            tc::tma_prefetch_desc(&tmdy);
-            tc::tma_prefetch_desc(&tmz);
-            tc::tma_prefetch_desc(&tmu);
+            // operands: the tile's z image and the block's U image, one bulk copy each
             BwdWalk it;
             it.init(m, tile_lo, chunk_lo);
-            int ob = 0, slot = 0, l = 0;
-            uint32_t oph = 0, xph = 0;
+            int ob = 0;
+            uint32_t oph = 0;
             for (int li = 0; li < nI; ++li, it.next(m, chunk_lo, ncl)) {
                 if (li >= NOP) wait(bars.ope(ob), oph ^ 1u);
                 const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
-                tc::mbar_expect_tx(bars.opf(ob), (uint32_t)kz * TB_ZR + S.ubytes);
-                for (int j = 0; j < kz; ++j) tc::tma_load_3d(zb + (uint32_t)j * TB_ZR, &tmz, 8 * j, it.t0, it.b, bars.opf(ob));
-                for (int j = 0; j < TB_NB / 8; ++j)
-                    tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), &tmu, it.blk * TB_NB + 8 * j, 0, bars.opf(ob));
+                tc::mbar_expect_tx(bars.opf(ob), S.zbytes + S.ubytes);
+                tc::bulk_load(zb, a.zimg + (size_t)(tile_lo + it.tl) * (S.zbytes / 2), S.zbytes, bars.opf(ob));
+                tc::bulk_load(ub, a.Up + (size_t)it.blk * (S.ubytes / 2), S.ubytes, bars.opf(ob));
                 if (++ob == NOP) {
                     ob = 0;
                     oph ^= 1u;
                 }
+            }
+            for (int b = 0; b < NOP && b < nI; ++b) {  // the last loads have landed
+                const int last = b + ((nI - 1 - b) / NOP) * NOP;
+                tc::mbar_wait(bars.opf(b), (uint32_t)((last / NOP) & 1), TC_WAIT_LIMIT);
+            }
+        } else if (lane == 1) {
+            tc::tma_prefetch_desc(&tmx);
+            tc::tma_prefetch_desc(&tmdy);
+            BwdWalk it;
+            it.init(m, tile_lo, chunk_lo);
+            int slot = 0, l = 0;
+            uint32_t xph = 0;
+            for (int li = 0; li < nI; ++li, it.next(m, chunk_lo, ncl)) {
                 for (int s = 0; s < m.nSubB; ++s, ++l) {
                     if (l >= NS) wait(bars.xe(slot), xph ^ 1u);
                     const uint32_t xb = sbase + S.ring + (uint32_t)slot * S.slot;
@@ -358,6 +359,10 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                     }
                 }
             }
+            for (int s = 0; s < NS && s < nG; ++s) {  // the last loads have landed
+                const int lastl = s + ((nG - 1 - s) / NS) * NS;
+                tc::mbar_wait(bars.xf(s), (uint32_t)((lastl / NS) & 1), TC_WAIT_LIMIT);
+            }
         }
     } else if (warp == 17) {
         // ----------------------------------------------------------------- MMA
@@ -365,63 +370,83 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             const uint32_t id_w = tc::idesc_bf16(TC_M, m.GB, 0, 1);
             const uint32_t id_dz = tc::idesc_bf16(TC_M, m.RP, 0, 0);
             const uint32_t id_dU = tc::idesc_bf16(TC_M, m.RP, 1, 1);
-            // dz / dU of item j (its dw tile is complete), then release its buffers
-            int fob = 0, fdb = 0, ftl = 0, fcl = 0;
-            uint32_t fdph = 0;
-            auto finish = [&](void) {
-                wait(bars.dwf(fdb), fdph);
-                tc::fence_after_sync();
-                const int tp = ftl & 1;
-                if (fcl == 0 && ftl >= 2) wait(bars.dze(tp), (uint32_t)(((ftl - 2) >> 1) & 1));
-                tc::fence_after_sync();
-                const uint32_t zb = sbase + (uint32_t)fob * S.opsize, ub = zb + S.zbytes;
-                const uint32_t dwb = sbase + S.dw + (uint32_t)fdb * S.dwsize;
-                for (int ks = 0; ks < TB_NB / 16; ++ks) {
-                    const uint64_t ad = tc::smem_desc(dwb + (uint32_t)ks * 256u, 128, (TB_NB / 8) * 128);
-                    const uint64_t bd = tc::smem_desc(ub + (uint32_t)(ks * 2 * m.RP * 16), (uint32_t)(m.RP * 16), 128);
-                    tc::mma_bf16(tmem + col_dz + (uint32_t)(tp * m.RP), ad, bd, id_dz, (fcl > 0 || ks > 0) ? 1u : 0u);
-                }
-                for (int ks = 0; ks < TC_M / 16; ++ks) {
-                    const uint64_t ad = tc::smem_desc(dwb + (uint32_t)ks * 2u * ((TB_NB / 8) * 128), (TB_NB / 8) * 128, 128);
-                    const uint64_t bd = tc::smem_desc(zb + (uint32_t)ks * 256u, 128, TB_ZR);
-                    tc::mma_bf16(tmem + col_dU + (uint32_t)(fcl * m.RP), ad, bd, id_dU, (ftl > 0 || ks > 0) ? 1u : 0u);
-                }
-                tc::mma_commit(bars.dwe(fdb));
-                tc::mma_commit(bars.ope(fob));
-                if (fcl == ncl - 1) tc::mma_commit(bars.dzf(tp));
-                if (++fob == NOP) fob = 0;
-                if (++fdb == DWB) {
-                    fdb = 0;
-                    fdph ^= 1u;
-                }
-                if (++fcl == ncl) {
-                    fcl = 0;
-                    ++ftl;
-                }
-            };
-            int ob = 0;
-            uint32_t oph = 0;
-            for (int li = 0; li < nI; ++li) {
-                const int b = li & 1;
-                wait(bars.opf(ob), oph);
-                if (li >= 2) wait(bars.we(b), (uint32_t)(((li - 2) >> 1) & 1));
-                tc::fence_after_sync();
-                const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
-                for (int k = 0; k < W; ++k)
-                    for (int ks = 0; ks < m.RP / 16; ++ks) {
-                        const uint64_t ad = tc::smem_desc(zb + (uint32_t)(k * 16) + (uint32_t)ks * 2u * TB_ZR, TB_ZR, 128);
-                        const uint64_t bd = tc::smem_desc(ub + (uint32_t)((k * m.GB / 8) * m.RP * 16) + (uint32_t)ks * 256u,
-                                                          128, (uint32_t)(m.RP * 16));
-                        tc::mma_bf16(tmem + (uint32_t)(b * TB_NB + k * m.GB), ad, bd, id_w, ks > 0 ? 1u : 0u);
+            // w(li_w): filters of the next item; fin(li_f): dz / dU of the oldest item whose dw
+            // tile is complete.  Each is issued as soon as its inputs are ready.
+            int li_w = 0, wob = 0, li_f = 0, fob = 0, fdb = 0, ftl = 0, fcl = 0;
+            uint32_t woph = 0, fdph = 0;
+            long long last = clock64();
+            while (li_f < nI) {
+                bool prog = false;
+                if (li_w < nI) {
+                    const int b = li_w & 1;
+                    if (tc::mbar_test(bars.opf(wob), woph) &&
+                        (li_w < 2 || tc::mbar_test(bars.we(b), (uint32_t)(((li_w - 2) >> 1) & 1)))) {
+                        tc::fence_after_sync();
+                        const uint32_t zb = sbase + (uint32_t)wob * S.opsize, ub = zb + S.zbytes;
+                        for (int k = 0; k < W; ++k)
+                            for (int ks = 0; ks < m.RP / 16; ++ks) {
+                                const uint64_t ad =
+                                    tc::smem_desc(zb + (uint32_t)(k * 16) + (uint32_t)ks * 2u * TB_ZR, TB_ZR, 128);
+                                const uint64_t bd = tc::smem_desc(
+                                    ub + (uint32_t)((k * m.GB / 8) * m.RP * 16) + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
+                                tc::mma_bf16(tmem + (uint32_t)(b * TB_NB + k * m.GB), ad, bd, id_w, ks > 0 ? 1u : 0u);
+                            }
+                        tc::mma_commit(bars.wf(b));
+                        if (++wob == NOP) {
+                            wob = 0;
+                            woph ^= 1u;
+                        }
+                        ++li_w;
+                        prog = true;
                     }
-                tc::mma_commit(bars.wf(b));
-                if (++ob == NOP) {
-                    ob = 0;
-                    oph ^= 1u;
                 }
-                if (li >= 1) finish();
+                if (li_f < li_w) {
+                    const int tp = ftl & 1;
+                    if (tc::mbar_test(bars.dwf(fdb), fdph) &&
+                        (fcl != 0 || ftl < 2 || tc::mbar_test(bars.dze(tp), (uint32_t)(((ftl - 2) >> 1) & 1)))) {
+                        tc::fence_after_sync();
+                        const uint32_t zb = sbase + (uint32_t)fob * S.opsize, ub = zb + S.zbytes;
+                        const uint32_t dwb = sbase + S.dw + (uint32_t)fdb * S.dwsize;
+                        for (int ks = 0; ks < TB_NB / 16; ++ks) {
+                            const uint64_t ad = tc::smem_desc(dwb + (uint32_t)ks * 256u, 128, (TB_NB / 8) * 128);
+                            const uint64_t bd =
+                                tc::smem_desc(ub + (uint32_t)(ks * 2 * m.RP * 16), (uint32_t)(m.RP * 16), 128);
+                            tc::mma_bf16(tmem + col_dz + (uint32_t)(tp * m.RP), ad, bd, id_dz,
+                                         (fcl > 0 || ks > 0) ? 1u : 0u);
+                        }
+                        for (int ks = 0; ks < TC_M / 16; ++ks) {
+                            const uint64_t ad =
+                                tc::smem_desc(dwb + (uint32_t)ks * 2u * ((TB_NB / 8) * 128), (TB_NB / 8) * 128, 128);
+                            const uint64_t bd = tc::smem_desc(zb + (uint32_t)ks * 256u, 128, TB_ZR);
+                            tc::mma_bf16(tmem + col_dU + (uint32_t)(fcl * m.RP), ad, bd, id_dU,
+                                         (ftl > 0 || ks > 0) ? 1u : 0u);
+                        }
+                        tc::mma_commit(bars.dwe(fdb));
+                        tc::mma_commit(bars.ope(fob));
+                        if (fcl == ncl - 1) tc::mma_commit(bars.dzf(tp));
+                        if (++fob == NOP) fob = 0;
+                        if (++fdb == DWB) {
+                            fdb = 0;
+                            fdph ^= 1u;
+                        }
+                        if (++fcl == ncl) {
+                            fcl = 0;
+                            ++ftl;
+                        }
+                        ++li_f;
+                        prog = true;
+                    }
+                }
+                if (prog) {
+                    last = clock64();
+                } else {
+                    if (clock64() - last > TC_WAIT_LIMIT) {
+                        timed_out = true;
+                        break;
+                    }
+                    __nanosleep(32);
+                }
             }
-            finish();
             tc::mma_commit(bars.duf());
         }
     } else {
@@ -530,12 +555,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 
     // teardown: every load and MMA this CTA issued has landed before the
     // shared memory and TMEM are given back (bounded, also after a time-out)
-    if (warp == 16 && lane == 0) {
-        for (int s = 0; s < NS && s < nG; ++s) {
-            const int lastl = s + ((nG - 1 - s) / NS) * NS;
-            tc::mbar_wait(bars.xf(s), (uint32_t)((lastl / NS) & 1), TC_WAIT_LIMIT);
-        }
-    }
     if (warp == 17 && lane == 0) tc::mbar_wait(bars.duf(), 0, TC_WAIT_LIMIT);
     if (timed_out) atomicExch(&g_dsc_status_tcb, (int)DSC_ERR_TIMEOUT);
     tc::fence_before_sync();
@@ -544,15 +563,34 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
     if (warp == 17) tc::tmem_dealloc(tmem, 512);
 }
 
-// U_perm[r][blk*128 + k*GB + g] = U[r][(blk*GB + g)*W + k]
-__global__ void k_uperm(const bf16 *U, bf16 *Up, int64_t R, int64_t GW, int W, int GB) {
-    const int64_t n = R * GW;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / GW, j = i % GW;
-        const int64_t blk = j / TB_NB;
-        const int rem = (int)(j % TB_NB);
-        const int k = rem / GB, g = rem % GB;
-        Up[i] = U[r * GW + (blk * GB + g) * W + k];
+// Operand images the backward loads with one bulk copy each:
+//   U image of block blk: element (j, r) at (j/8)*(RP*8) + r*8 + j%8, column
+//     j = k*GB + g holding U[r][(blk*GB + g)*W + k] (tap-major), rows r >= R zero;
+//   z image of tile i (sequence b, first token t0): element (t, r) at
+//     (r/8)*(136*8) + t*8 + r%8 holding z[b][t0+t][r], zero for r >= R or t0+t >= T.
+__global__ void k_bwd_prep(const TcArgs a) {
+    const TcMap &m = a.m;
+    const int64_t ublk = (int64_t)m.RP * TB_NB;
+    const int64_t nU = (int64_t)m.nBlkB * ublk;
+    const int64_t ztile = (int64_t)(m.RP / 8) * TB_ZROWS * 8;
+    const int64_t nZ = m.totalTiles * ztile;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nU + nZ; i += (int64_t)gridDim.x * blockDim.x) {
+        if (i < nU) {
+            const int64_t blk = i / ublk;
+            const int rem = (int)(i % ublk);
+            const int jc = rem / (m.RP * 8), r = (rem % (m.RP * 8)) / 8, e = rem % 8;
+            const int j = jc * 8 + e, k = j / m.GB, g = j % m.GB;
+            a.Up[i] = r < m.R ? a.U[(int64_t)r * m.GW + (blk * m.GB + g) * m.W + k] : __float2bfloat16_rn(0.f);
+        } else {
+            const int64_t i2 = i - nU;
+            const int64_t tile = i2 / ztile;
+            const int rem = (int)(i2 % ztile);
+            const int rc = rem / (TB_ZROWS * 8), t = (rem % (TB_ZROWS * 8)) / 8, e = rem % 8;
+            const int r = rc * 8 + e;
+            const int64_t b = tile / m.tilesPerSeq;
+            const int64_t tt = (tile % m.tilesPerSeq) * TC_M + t;
+            a.zimg[i2] = (r < m.R && tt < m.T) ? a.z[(b * m.T + tt) * m.R + r] : __float2bfloat16_rn(0.f);
+        }
     }
 }
 
@@ -619,26 +657,28 @@ bool tc_bwd_plan(TcMap &m, int sms) {
     const int vpt = m.SB / 32, ct = 8 * vpt;
     const bool xchg = m.H > ct;
     const bool short_items = m.nSubB < 4;
-    const int nop = short_items ? 3 : 2, dwb = short_items ? 2 : 1;
-    for (m.NSB = TB_MAXNS; m.NSB >= 2; --m.NSB) {
-        m.NOP = nop;
-        m.DWB = dwb;
-        if (BwdSmem(m, nop, m.NSB, dwb, xchg).total <= TB_SMEM) return true;
-    }
+    const int dwb = short_items ? 2 : 1;
+    m.DWB = dwb;
+    for (int nop = short_items ? TB_MAXOP : 2; nop >= 2; --nop)
+        for (m.NSB = TB_MAXNS; m.NSB >= (nop > 2 ? 4 : 2); --m.NSB) {
+            m.NOP = nop;
+            if (BwdSmem(m, nop, m.NSB, dwb, xchg).total <= TB_SMEM) return true;
+        }
     return false;
 }
 
-size_t up_bytes(const TcMap &m) { return ((size_t)m.R * m.GW * 2 + 255) & ~(size_t)255; }
+size_t up_bytes(const TcMap &m) { return ((size_t)m.nBlkB * m.RP * TB_NB * 2 + 255) & ~(size_t)255; }
+size_t zimg_bytes(const TcMap &m) { return ((size_t)m.totalTiles * (m.RP / 8) * TB_ZR + 255) & ~(size_t)255; }
 
 size_t tc_bwd_ws_bytes(const TcMap &m) {
-    size_t n = up_bytes(m);
+    size_t n = up_bytes(m) + zimg_bytes(m);
     if (m.nRanges > 1) n += (size_t)m.nRanges * m.R * m.GW * 4;
     if (m.nGroups > 1) n += (size_t)m.B * m.T * m.R * 4;
     return n;
 }
 
 struct BwdMaps {
-    CUtensorMap x, dy, z, u, dx;
+    CUtensorMap x, dy, dx;
 };
 
 bool bwd_maps(const TcArgs &a, BwdMaps &f) {
@@ -648,18 +688,10 @@ bool bwd_maps(const TcArgs &a, BwdMaps &f) {
     const uint64_t xs[2] = {(uint64_t)m.D * 2, (uint64_t)(m.T * m.D * 2)};
     const uint32_t xb[3] = {(uint32_t)(rb / 2), (uint32_t)(TC_M + m.W - 1), 1};
     const uint32_t yb[3] = {(uint32_t)(rb / 2), (uint32_t)TC_M, 1};
-    const uint64_t zd[3] = {(uint64_t)m.R, (uint64_t)m.T, (uint64_t)m.B};
-    const uint64_t zs[2] = {(uint64_t)m.R * 2, (uint64_t)(m.T * m.R * 2)};
-    const uint32_t zb[3] = {8, (uint32_t)TB_ZROWS, 1};
-    const uint64_t ud[2] = {(uint64_t)m.GW, (uint64_t)m.R};
-    const uint64_t us[1] = {(uint64_t)m.GW * 2};
-    const uint32_t ub[2] = {8, (uint32_t)m.RP};
     const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     return make_map(&f.x, a.x, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
            make_map(&f.dy, a.dy, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
-           make_map(&f.dx, a.dx, 3, xd, xs, yb, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE) &&
-           make_map(&f.z, a.z, 3, zd, zs, zb, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
-           make_map(&f.u, a.Up, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
+           make_map(&f.dx, a.dx, 3, xd, xs, yb, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE);
 }
 
 template <int W, int VPT, int GPT, int PPG>
@@ -673,8 +705,8 @@ cudaError_t launch_bwd(const Ctx &c, const TcArgs &a) {
     if (!bwd_maps(a, f)) return cudaErrorNotSupported;
     // the whole of TMEM per CTA: enough shared memory that no second CTA shares the SM
     const uint32_t smem = S.total < 120 * 1024 ? 120 * 1024 : S.total;
-    k_lr_tc_bwd<W, VPT, GPT, PPG><<<(unsigned)(a.m.nGroups * a.m.nRanges), TB_THREADS, smem, c.stream>>>(f.x, f.dy, f.z,
-                                                                                                       f.u, f.dx, a);
+    k_lr_tc_bwd<W, VPT, GPT, PPG><<<(unsigned)(a.m.nGroups * a.m.nRanges), TB_THREADS, smem, c.stream>>>(f.x, f.dy, f.dx,
+                                                                                                       a);
     count_launch();
     return cudaGetLastError();
 }
@@ -728,13 +760,14 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     unsigned char *w = static_cast<unsigned char *>(ws);
     a.Up = reinterpret_cast<bf16 *>(w);
     w += up_bytes(a.m);
+    a.zimg = reinterpret_cast<bf16 *>(w);
+    w += zimg_bytes(a.m);
     if (a.m.nRanges > 1) {
         a.dU_part = reinterpret_cast<float *>(w);
         w += (size_t)a.m.nRanges * a.m.R * a.m.GW * 4;
     }
-    const int64_t nUp = a.m.R * a.m.GW;
-    k_uperm<<<(unsigned)min((int64_t)1024, (nUp + 255) / 256), 256, 0, c.stream>>>(a.U, a.Up, a.m.R, a.m.GW, a.m.W,
-                                                                                   a.m.GB);
+    const int64_t nprep = (int64_t)a.m.nBlkB * a.m.RP * TB_NB + a.m.totalTiles * (a.m.RP / 8) * TB_ZROWS * 8;
+    k_bwd_prep<<<(unsigned)min((int64_t)2048, (nprep + 255) / 256), 256, 0, c.stream>>>(a);
     count_launch();
     if (a.m.nGroups > 1) {
         a.dz_acc = reinterpret_cast<float *>(w);
