@@ -444,7 +444,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                         timed_out = true;
                         break;
                     }
-                    __nanosleep(32);
+                    // sleep on the barrier the oldest pending step needs; it wakes the lane at once
+                    if (li_f < li_w) tc::mbar_try(bars.dwf(fdb), fdph, 1000);
+                    else tc::mbar_try(bars.opf(wob), woph, 1000);
                 }
             }
             tc::mma_commit(bars.duf());
@@ -486,7 +488,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         uint32_t xph = 0, dph = 0;
         for (int li = 0; li < nI; ++li) {
             const int b = li & 1;
-            if (li >= 1 && it.cl == 0) dz_out(it.tl - 1, pb, pt0);  // previous tile done
             wait(bars.wf(b), (uint32_t)((li >> 1) & 1));
             if (li >= DWB) wait(bars.dwe(db), dph ^ 1u);
             tc::fence_after_sync();
@@ -525,6 +526,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                 db = 0;
                 dph ^= 1u;
             }
+            // the previous tile's dz (its last MMAs have had this whole item to finish)
+            if (li >= 1 && it.cl == 0) dz_out(it.tl - 1, pb, pt0);
             pb = it.b;
             pt0 = it.t0;
             it.next(m, chunk_lo, ncl);
