@@ -335,7 +335,8 @@ def run_dsc(args, wl0):
     bwd_gbs = bb / (bwd_ms / 1e3) / 1e9
     fwd_gbs = fb / (fwd_ms / 1e3) / 1e9
     step_gbs = (fb + bb) / (ms / K / 1e3) / 1e9
-    kname = {"headwise": "k_stream_bwd", "static": "k_stream_bwd", "lowrank": "k_lr_bwd"}[wl.variant]
+    kname = {"headwise": "k_stream_bwd", "static": "k_stream_bwd",
+             "lowrank": "k_lr_tc_bwd" if wl.dtype == "bf16" else "k_lr_bwd"}[wl.variant]
     traffic = ncu_traffic(kname, wl0.name, digest)
 
     result = None

@@ -173,11 +173,20 @@ template <bool B> struct BoolC { static constexpr bool value = B; };
 // Tap k of the filters of channel pair p (channels 2p, 2p+1 of the thread's
 // vector) as an fp32 pair; `add` is added to both (the residual on tap 0).
 template <typename F, int W, int CPG>
-__device__ __forceinline__ u64 tap2(const uint32_t (&wv)[F::WORDS], int p, int k, float add = 0.f) {
+__device__ __forceinline__ u64 tap2(const uint32_t (&wv)[F::WORDS], int p, int k, float add) {
     const int g0 = (2 * p) / CPG, g1 = (2 * p + 1) / CPG;
     const float a = F::get(wv, g0 * W + k) + add;
     if (g0 == g1) return mk2(a, a);
     return mk2(a, F::get(wv, g1 * W + k) + add);
+}
+// The same pair without an added constant (x + 0.f is not x for x = -0, so a
+// default of 0 would cost an add per tap).
+template <typename F, int W, int CPG>
+__device__ __forceinline__ u64 tap2(const uint32_t (&wv)[F::WORDS], int p, int k) {
+    const int g0 = (2 * p) / CPG, g1 = (2 * p + 1) / CPG;
+    const float a = F::get(wv, g0 * W + k);
+    if (g0 == g1) return mk2(a, a);
+    return mk2(a, F::get(wv, g1 * W + k));
 }
 
 // Sum part[k] (k < N) over the L lanes of a filter group; afterwards the
@@ -234,7 +243,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
 #pragma unroll
         for (int pp = 0; pp < P; ++pp)
 #pragma unroll
-            for (int k = 0; k < W; ++k) wsp[pp][k] = tap2<F, W, CPG>(wst, pp, k, k == 0 ? res : 0.f);
+            for (int k = 0; k < W; ++k) wsp[pp][k] = k == 0 ? tap2<F, W, CPG>(wst, pp, 0, res) : tap2<F, W, CPG>(wst, pp, k);
     }
     uint32_t wreg[C::WREG ? NS : 1][F::WORDS];
 
@@ -343,7 +352,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
         for (int pp = 0; pp < P; ++pp)
 #pragma unroll
             for (int k = 0; k < W; ++k) {
-                wsp[pp][k] = tap2<F, W, CPG>(wst, pp, k, k == 0 ? res : 0.f);
+                wsp[pp][k] = k == 0 ? tap2<F, W, CPG>(wst, pp, 0, res) : tap2<F, W, CPG>(wst, pp, k);
                 dws[pp][k] = 0ull;
             }
     }

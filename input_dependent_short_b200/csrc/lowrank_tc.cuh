@@ -32,7 +32,7 @@ struct TcMap {
     int lgH;             // log2 H
     int residual;
     // forward: item = (tile, block of CF channels) -> NF TMEM columns; sub-tiles of SF channels
-    int CF, NF, SF, nSubF, nBlkF, NSF;
+    int CF, NF, SF, nSubF, nBlkF, NSF, NOPF;
     int64_t nItemsF;
     // backward: block of CB channels = GB groups -> W*GB = 128 filter columns;
     // sub-tiles of SB channels; CTA = (range of tiles) x (group of CPC blocks)

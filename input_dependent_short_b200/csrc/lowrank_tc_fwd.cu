@@ -126,11 +126,12 @@ namespace {
 constexpr int TF_EPI = 512;               // epilogue threads
 constexpr int TF_THREADS = TF_EPI + 64;   // + producer warp + MMA warp
 constexpr int TF_MAXNS = 8;               // most x sub-tiles in flight
+constexpr int TF_MAXOP = 4;               // most operand (z, U) buffers
 constexpr int TF_SMEM = 220 * 1024;
 
 struct FwdSmem {
     uint32_t zbytes, ubytes, opsize, ring, boxb, slot, ystage, ybox, bars, tmem, total;
-    __host__ __device__ FwdSmem(const TcMap &m, int ns) {
+    __host__ __device__ FwdSmem(const TcMap &m, int nop, int ns) {
         const int rb = m.SF == 32 ? 64 : 128;
         const int nbx = m.SF == 128 ? 2 : 1;
         boxb = up1024((uint32_t)(rb * (TC_M + m.W - 1)));
@@ -139,10 +140,10 @@ struct FwdSmem {
         zbytes = (uint32_t)(TC_M * m.RP * 2);
         ubytes = (uint32_t)(m.RP * m.NF * 2);
         opsize = up1024(zbytes + ubytes);
-        ystage = 2 * opsize;                      // two y staging tiles (TMA store sources)
+        ystage = (uint32_t)nop * opsize;          // two y staging tiles (TMA store sources)
         ring = ystage + 2 * (uint32_t)nbx * ybox;
-        bars = ring + (uint32_t)ns * slot;        // OPF[2] OPE[2] WF[2] WE[2] XF[MAXNS] XE[MAXNS]
-        tmem = bars + (8 + 2 * TF_MAXNS) * 8;
+        bars = ring + (uint32_t)ns * slot;        // OPF[MAXOP] OPE[MAXOP] WF[2] WE[2] XF[MAXNS] XE[MAXNS]
+        tmem = bars + (2 * TF_MAXOP + 4 + 2 * TF_MAXNS) * 8;
         total = tmem + 16 + 1024;                 // + slack to align the base to 1024 bytes
     }
 };
@@ -150,11 +151,11 @@ struct FwdSmem {
 struct FwdBars {
     uint32_t base;
     __device__ uint32_t opf(int b) const { return base + 8u * (uint32_t)b; }
-    __device__ uint32_t ope(int b) const { return base + 16u + 8u * (uint32_t)b; }
-    __device__ uint32_t wf(int b) const { return base + 32u + 8u * (uint32_t)b; }
-    __device__ uint32_t we(int b) const { return base + 48u + 8u * (uint32_t)b; }
-    __device__ uint32_t xf(int s) const { return base + 64u + 8u * (uint32_t)s; }
-    __device__ uint32_t xe(int s) const { return base + 64u + 8u * TF_MAXNS + 8u * (uint32_t)s; }
+    __device__ uint32_t ope(int b) const { return base + 8u * TF_MAXOP + 8u * (uint32_t)b; }
+    __device__ uint32_t wf(int b) const { return base + 16u * TF_MAXOP + 8u * (uint32_t)b; }
+    __device__ uint32_t we(int b) const { return base + 16u * TF_MAXOP + 16u + 8u * (uint32_t)b; }
+    __device__ uint32_t xf(int s) const { return base + 16u * TF_MAXOP + 32u + 8u * (uint32_t)s; }
+    __device__ uint32_t xe(int s) const { return base + 16u * TF_MAXOP + 32u + 8u * TF_MAXNS + 8u * (uint32_t)s; }
 };
 
 // Coordinates of consecutive items (block-major, tile-minor: a CTA keeps one
@@ -251,10 +252,13 @@ __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char 
 #pragma unroll
                     for (int k = 0; k < W; ++k) {
                         const uint32_t word = word_of(xw[vv][k], pp);
-                        const float w0 = w[g0 * W + k] + (k == 0 ? res : 0.f);
-                        const float w1 = w[g1 * W + k] + (k == 0 ? res : 0.f);
-                        a0 = k == 0 ? w0 * bf_lo(word) : fmaf(w0, bf_lo(word), a0);
-                        a1 = k == 0 ? w1 * bf_hi(word) : fmaf(w1, bf_hi(word), a1);
+                        if (k == 0) {  // tap 0 carries the residual
+                            a0 = (w[g0 * W] + res) * bf_lo(word);
+                            a1 = (w[g1 * W] + res) * bf_hi(word);
+                        } else {
+                            a0 = fmaf(w[g0 * W + k], bf_lo(word), a0);
+                            a1 = fmaf(w[g1 * W + k], bf_hi(word), a1);
+                        }
                     }
                     y[2 * pp] = a0;
                     y[2 * pp + 1] = a1;
@@ -276,8 +280,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
     constexpr int NBX = VPT == 4 ? 2 : 1;    // x boxes per sub-tile
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const TcMap &m = a.m;
-    const int NS = m.NSF;
-    const FwdSmem S(m, NS);
+    const int NS = m.NSF, NOP = m.NOPF;
+    const FwdSmem S(m, NOP, NS);
     const int64_t total = m.nItemsF * m.nSubF;
     const int64_t per = (total + gridDim.x - 1) / gridDim.x;
     const int64_t g_lo = (int64_t)blockIdx.x * per;
@@ -297,9 +301,11 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
     const int kz = m.R / 8;  // z boxes loaded per item; k-chunks kz .. RP/8-1 stay zero
 
     if (tid == 0) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < TF_MAXOP; ++i) {
             tc::mbar_init(bars.opf(i), 1);
             tc::mbar_init(bars.ope(i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
             tc::mbar_init(bars.wf(i), 1);
             tc::mbar_init(bars.we(i), TF_EPI / 32);
         }
@@ -309,9 +315,9 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
         }
         tc::fence_mbar_init();
     }
-    // zero the padded k-chunks of both z buffers (read by the MMA, never loaded)
+    // zero the padded k-chunks of every z buffer (read by the MMA, never loaded)
     const int zpad = (m.RP / 8 - kz) * 128;
-    for (int i = tid; i < 2 * zpad; i += TF_THREADS) {
+    for (int i = tid; i < NOP * zpad; i += TF_THREADS) {
         const int b = i / zpad, r = i % zpad;
         *reinterpret_cast<uint4 *>(smem + (uint32_t)b * S.opsize + (uint32_t)kz * 2048 + (uint32_t)r * 16) =
             make_uint4(0, 0, 0, 0);
@@ -336,22 +342,34 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
             ItemWalk it;
             it.init(m, i_lo);
             int slot = 0, l = 0;
-            int ublk0 = -1, ublk1 = -1;  // U block held by each operand buffer
             uint32_t xph = 0;
+            int ublk[TF_MAXOP];  // U block held by each operand buffer
+#pragma unroll
+            for (int i = 0; i < TF_MAXOP; ++i) ublk[i] = -1;
+            int ob = 0;
+            uint32_t oph = 0;
             for (int li = 0; li < nI; ++li, it.next(m)) {
-                const int b = li & 1;
-                if (li >= 2) wait(bars.ope(b), (uint32_t)(((li - 2) >> 1) & 1));
-                const uint32_t zb = sbase + (uint32_t)b * S.opsize, ub = zb + S.zbytes;
-                const bool newu = (b ? ublk1 : ublk0) != it.blk;
-                tc::mbar_expect_tx(bars.opf(b), (uint32_t)kz * 2048u + (newu ? S.ubytes : 0u));
+                if (li >= NOP) wait(bars.ope(ob), oph ^ 1u);
+                const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
+                int held = -1;
+#pragma unroll
+                for (int i = 0; i < TF_MAXOP; ++i)
+                    if (i == ob) held = ublk[i];
+                const bool newu = held != it.blk;
+                tc::mbar_expect_tx(bars.opf(ob), (uint32_t)kz * 2048u + (newu ? S.ubytes : 0u));
                 for (int j = 0; j < kz; ++j)
-                    tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, it.b, bars.opf(b));
+                    tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, it.b, bars.opf(ob));
                 if (newu) {
-                    if (b) ublk1 = it.blk;
-                    else ublk0 = it.blk;
+#pragma unroll
+                    for (int i = 0; i < TF_MAXOP; ++i)
+                        if (i == ob) ublk[i] = it.blk;
                     const int col0 = it.blk * m.NF;
                     for (int j = 0; j < m.NF / 8; ++j)
-                        tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), &tmu, col0 + 8 * j, 0, bars.opf(b));
+                        tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), &tmu, col0 + 8 * j, 0, bars.opf(ob));
+                }
+                if (++ob == NOP) {
+                    ob = 0;
+                    oph ^= 1u;
                 }
                 const int se = li == nI - 1 ? s_last : m.nSubF;
                 for (int s = li == 0 ? s_first : 0; s < se; ++s, ++l) {
@@ -374,19 +392,25 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
         // ----------------------------------------------------------------- MMA
         if (lane == 0) {
             const uint32_t id_w = tc::idesc_bf16(TC_M, m.NF, 0, 1);
+            int ob = 0;
+            uint32_t oph = 0;
             for (int li = 0; li < nI; ++li) {
                 const int b = li & 1;
-                wait(bars.opf(b), (uint32_t)((li >> 1) & 1));
+                wait(bars.opf(ob), oph);
                 if (li >= 2) wait(bars.we(b), (uint32_t)(((li - 2) >> 1) & 1));
                 tc::fence_after_sync();
-                const uint32_t zb = sbase + (uint32_t)b * S.opsize, ub = zb + S.zbytes;
+                const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
                 for (int ks = 0; ks < m.RP / 16; ++ks) {
                     const uint64_t ad = tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
                     const uint64_t bd = tc::smem_desc(ub + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
                     tc::mma_bf16(tmem + (uint32_t)(b * m.NF), ad, bd, id_w, ks > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(bars.wf(b));
-                tc::mma_commit(bars.ope(b));
+                tc::mma_commit(bars.ope(ob));
+                if (++ob == NOP) {
+                    ob = 0;
+                    oph ^= 1u;
+                }
             }
         }
     } else {
@@ -446,9 +470,9 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
         }
     }
     if (warp == 17 && lane == 0) {
-        for (int b = 0; b < 2 && b < nI; ++b) {
-            const int lastli = b + ((nI - 1 - b) / 2) * 2;
-            tc::mbar_wait(bars.ope(b), (uint32_t)((lastli >> 1) & 1), TC_WAIT_LIMIT);
+        for (int b = 0; b < NOP && b < nI; ++b) {
+            const int lastli = b + ((nI - 1 - b) / NOP) * NOP;
+            tc::mbar_wait(bars.ope(b), (uint32_t)((lastli / NOP) & 1), TC_WAIT_LIMIT);
         }
     }
     if (timed_out) atomicExch(&g_dsc_status_tcf, (int)DSC_ERR_TIMEOUT);
@@ -472,8 +496,10 @@ bool tc_fwd_plan(TcMap &m) {
     m.nSubF = m.CF / m.SF;
     m.nBlkF = (int)(m.D / m.CF);
     m.nItemsF = m.B * (int64_t)m.tilesPerSeq * m.nBlkF;
-    for (m.NSF = TF_MAXNS; m.NSF >= 2; --m.NSF)
-        if (FwdSmem(m, m.NSF).total <= TF_SMEM) return true;
+    // short items (few sub-tiles each) keep more operand loads in flight
+    for (m.NOPF = m.nSubF <= 2 ? TF_MAXOP : 2; m.NOPF >= 2; --m.NOPF)
+        for (m.NSF = TF_MAXNS; m.NSF >= (m.NOPF > 2 ? 4 : 2); --m.NSF)
+            if (FwdSmem(m, m.NOPF, m.NSF).total <= TF_SMEM) return true;
     return false;
 }
 
@@ -503,7 +529,7 @@ bool fwd_maps(const TcArgs &a, FwdMaps &f) {
 
 template <int W, int GPV, int VPT, int NGT>
 cudaError_t launch_fwd(const Ctx &c, const TcArgs &a) {
-    const FwdSmem S(a.m, a.m.NSF);
+    const FwdSmem S(a.m, a.m.NOPF, a.m.NSF);
     static const cudaError_t attr = cudaFuncSetAttribute(k_lr_tc_fwd<W, GPV, VPT, NGT>,
                                                          cudaFuncAttributeMaxDynamicSharedMemorySize, TF_SMEM);
     if (attr != cudaSuccess) return attr;
