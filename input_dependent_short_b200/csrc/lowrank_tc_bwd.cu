@@ -153,7 +153,7 @@ template <int N> __device__ __forceinline__ void st_dw(unsigned char *p, const f
 template <int W, int VPT, int GPT, int PPG, int RB>
 __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
                                             unsigned char *dwt, float *xch, int part, int t_loc, int s,
-                                            unsigned char *ys, float res) {
+                                            unsigned char *ys, float res, uint32_t release_w) {
     constexpr int WIN = W - 1;
     constexpr int CT = 8 * VPT;                      // the thread's channels
     constexpr int GPV = GPT >= VPT ? GPT / VPT : 1;  // groups inside one vector
@@ -176,6 +176,11 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
         for (int k = 0; k < W; ++k) dyv[v][k] = *reinterpret_cast<const uint4 *>(yb + tc::swz<RB>(t_loc + k, bo));
     }
     tc::tmem_wait_ld();
+    if (release_w) {  // the item's last filter read: its TMEM buffer is free for the next MMA
+        tc::fence_before_sync();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) tc::mbar_arrive(release_w);
+    }
 #pragma unroll
     for (int g = 0; g < GPT; ++g) wt[0][g] += res;
     // dx
@@ -319,11 +324,22 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         // ----------------------------------------------------- producers
         if (lane == 0) {
             // operands: the tile's z image and the block's U image, one bulk copy each
-            BwdWalk it;
+            BwdWalk it, pf;
             it.init(m, tile_lo, chunk_lo);
+            pf.init(m, tile_lo, chunk_lo);
+            constexpr int PF = 6;  // operand images are prefetched into L2 this many items ahead
+            for (int li = 0; li < PF && li < nI; ++li, pf.next(m, chunk_lo, ncl)) {
+                tc::bulk_prefetch_l2(a.zimg + (size_t)(tile_lo + pf.tl) * (S.zbytes / 2), S.zbytes);
+                tc::bulk_prefetch_l2(a.Up + (size_t)pf.blk * (S.ubytes / 2), S.ubytes);
+            }
             int ob = 0;
             uint32_t oph = 0;
             for (int li = 0; li < nI; ++li, it.next(m, chunk_lo, ncl)) {
+                if (li + PF < nI) {
+                    tc::bulk_prefetch_l2(a.zimg + (size_t)(tile_lo + pf.tl) * (S.zbytes / 2), S.zbytes);
+                    tc::bulk_prefetch_l2(a.Up + (size_t)pf.blk * (S.ubytes / 2), S.ubytes);
+                    pf.next(m, chunk_lo, ncl);
+                }
                 if (li >= NOP) wait(bars.ope(ob), oph ^ 1u);
                 const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
                 tc::mbar_expect_tx(bars.opf(ob), S.zbytes + S.ubytes);
@@ -496,7 +512,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             for (int s = 0; s < m.nSubB; ++s) {
                 wait(bars.xf(slot), xph);
                 bwd_subtile<W, VPT, GPT, PPG, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, xch, part,
-                                                  t_loc, s, smem + S.ystage + (uint32_t)ybuf * S.ybox, res);
+                                                  t_loc, s, smem + S.ystage + (uint32_t)ybuf * S.ybox, res,
+                                                  s == m.nSubB - 1 ? bars.we(b) : 0u);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars.xe(slot));
                 // dx tile -> global by TMA (the staging tile the next sub-tile writes was read
@@ -518,10 +535,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             tc::fence_proxy_async();  // dw tile (generic stores) -> MMA operand
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(bars.dwf(db));
-                tc::mbar_arrive(bars.we(b));
-            }
+            if (lane == 0) tc::mbar_arrive(bars.dwf(db));
             if (++db == DWB) {
                 db = 0;
                 dph ^= 1u;
