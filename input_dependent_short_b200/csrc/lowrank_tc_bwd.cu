@@ -24,10 +24,11 @@
 // block groups exist), dU after the range (directly, or as a per-range
 // partial summed by a finalize kernel).
 //
-// Warp roles (576 threads): warp 16 TMA producer, warp 17 TMEM owner and MMA
-// issuer, warps 0-15 epilogue (thread part p of token t: VPT 8-channel
-// vectors of each sub-tile).  Groups wider than a part's channels (PPG parts
-// per group) add their dw partial sums through a small exchange buffer.
+// Warp roles (640 threads): warp 16 x/dy TMA producer, warp 17 TMEM owner and
+// filter-MMA issuer, warp 18 operand loader, warp 19 dz/dU-MMA issuer, warps
+// 0-15 epilogue (thread part p of token t: VPT 8-channel vectors of each
+// sub-tile).  Groups wider than a part's channels (PPG parts per group) add
+// their dw partial sums through a small exchange buffer.
 #include "lowrank_tc.cuh"
 
 namespace dsc {
@@ -52,7 +53,7 @@ int take_tc_bwd_status(cudaStream_t stream) {
 namespace {
 
 constexpr int TB_EPI = 512;              // epilogue threads
-constexpr int TB_THREADS = TB_EPI + 64;  // + producer warp + MMA warp
+constexpr int TB_THREADS = TB_EPI + 128;  // + x/dy producer, filter-MMA, operand-loader and dz/dU-MMA warps
 constexpr int TB_MAXNS = 8;              // most sub-tiles in flight
 constexpr int TB_SMEM = 220 * 1024;
 constexpr int TB_NB = 128;               // filter columns per block (W * GB)
@@ -121,6 +122,15 @@ struct BwdWalk {
         blk = chunk_lo + cl;
     }
 };
+
+// 16-byte cp.async global -> shared (L2 only) and its mbarrier arrival (no count increment).
+__device__ __forceinline__ void tc_cp16(uint32_t dst, const void *src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void tc_cp_arrive(uint32_t bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
+}
+__device__ __forceinline__ void tc_cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(TB_EPI) : "memory"); }
 
@@ -292,7 +302,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 
     if (tid == 0) {
         for (int i = 0; i < TB_MAXOP; ++i) {
-            tc::mbar_init(bars.opf(i), 1);
+            tc::mbar_init(bars.opf(i), 32);  // one cp.async arrival per loader lane
             tc::mbar_init(bars.ope(i), 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -320,43 +330,46 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         if (!timed_out && !tc::mbar_wait(bar, parity, TC_WAIT_LIMIT)) timed_out = true;  // sticky: later waits skip
     };
 
-    if (warp == 16) {
-        // ----------------------------------------------------- producers
-        if (lane == 0) {
-            // operands: the tile's z image and the block's U image, one bulk copy each
-            BwdWalk it, pf;
-            it.init(m, tile_lo, chunk_lo);
-            pf.init(m, tile_lo, chunk_lo);
-            constexpr int PF = 6;  // operand images are prefetched into L2 this many items ahead
+    if (warp == 18) {
+        // ----------------------------------------------- operand loader warp
+        // The tile's z image and the block's U image, copied by the 32 lanes with
+        // cp.async (16 bytes each, the load/store path), so they never queue behind
+        // the x/dy tensor loads; each lane's arrival completes when its copies land.
+        BwdWalk it, pf;
+        it.init(m, tile_lo, chunk_lo);
+        pf.init(m, tile_lo, chunk_lo);
+        constexpr int PF = 6;  // operand images are prefetched into L2 this many items ahead
+        if (lane == 0)
             for (int li = 0; li < PF && li < nI; ++li, pf.next(m, chunk_lo, ncl)) {
                 tc::bulk_prefetch_l2(a.zimg + (size_t)(tile_lo + pf.tl) * (S.zbytes / 2), S.zbytes);
                 tc::bulk_prefetch_l2(a.Up + (size_t)pf.blk * (S.ubytes / 2), S.ubytes);
             }
-            int ob = 0;
-            uint32_t oph = 0;
-            for (int li = 0; li < nI; ++li, it.next(m, chunk_lo, ncl)) {
-                if (li + PF < nI) {
-                    tc::bulk_prefetch_l2(a.zimg + (size_t)(tile_lo + pf.tl) * (S.zbytes / 2), S.zbytes);
-                    tc::bulk_prefetch_l2(a.Up + (size_t)pf.blk * (S.ubytes / 2), S.ubytes);
-                    pf.next(m, chunk_lo, ncl);
-                }
-                if (li >= NOP) wait(bars.ope(ob), oph ^ 1u);
-                const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
-                tc::mbar_expect_tx(bars.opf(ob), S.zbytes + S.ubytes);
-                tc::bulk_load(zb, a.zimg + (size_t)(tile_lo + it.tl) * (S.zbytes / 2), S.zbytes, bars.opf(ob));
-                tc::bulk_load(ub, a.Up + (size_t)it.blk * (S.ubytes / 2), S.ubytes, bars.opf(ob));
-                if (++ob == NOP) {
-                    ob = 0;
-                    oph ^= 1u;
-                }
+        int ob = 0;
+        uint32_t oph = 0;
+        const uint32_t zch = S.zbytes / 16, uch = S.ubytes / 16;
+        for (int li = 0; li < nI; ++li, it.next(m, chunk_lo, ncl)) {
+            if (lane == 0 && li + PF < nI) {
+                tc::bulk_prefetch_l2(a.zimg + (size_t)(tile_lo + pf.tl) * (S.zbytes / 2), S.zbytes);
+                tc::bulk_prefetch_l2(a.Up + (size_t)pf.blk * (S.ubytes / 2), S.ubytes);
+                pf.next(m, chunk_lo, ncl);
             }
-            for (int b = 0; b < NOP && b < nI; ++b) {  // the last loads have landed
-                const int last = b + ((nI - 1 - b) / NOP) * NOP;
-                tc::mbar_wait(bars.opf(b), (uint32_t)((last / NOP) & 1), TC_WAIT_LIMIT);
+            if (li >= NOP) wait(bars.ope(ob), oph ^ 1u);
+            const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
+            const unsigned char *zs = reinterpret_cast<const unsigned char *>(a.zimg + (size_t)(tile_lo + it.tl) * (S.zbytes / 2));
+            const unsigned char *us = reinterpret_cast<const unsigned char *>(a.Up + (size_t)it.blk * (S.ubytes / 2));
+            for (uint32_t c = lane; c < zch; c += 32) tc_cp16(zb + 16u * c, zs + 16u * c);
+            for (uint32_t c = lane; c < uch; c += 32) tc_cp16(ub + 16u * c, us + 16u * c);
+            tc_cp_arrive(bars.opf(ob));
+            if (++ob == NOP) {
+                ob = 0;
+                oph ^= 1u;
             }
-        } else if (lane == 1) {
-            tc::tma_prefetch_desc(&tmx);
-            tc::tma_prefetch_desc(&tmdy);
+        }
+        tc_cp_wait_all();
+    } else if (warp == 16) {
+        // ------------------------------------------------- x / dy producer
+        if (lane == 0) {
+            tc::tma_prefetch_desc(&tmx);            tc::tma_prefetch_desc(&tmdy);
             BwdWalk it;
             it.init(m, tile_lo, chunk_lo);
             int slot = 0, l = 0;
@@ -381,88 +394,70 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             }
         }
     } else if (warp == 17) {
-        // ----------------------------------------------------------------- MMA
+        // ------------------------------------------------- filter MMAs (w)
+        // One lane issues each item's per-tap MMAs; the dz / dU MMAs come from
+        // warp 19, so the two streams of instructions overlap (a commit tracks
+        // only the MMAs of the thread that issues it).
         if (lane == 0) {
             const uint32_t id_w = tc::idesc_bf16(TC_M, m.GB, 0, 1);
+            int ob = 0;
+            uint32_t oph = 0;
+            for (int li = 0; li < nI; ++li) {
+                const int b = li & 1;
+                wait(bars.opf(ob), oph);
+                if (li >= 2) wait(bars.we(b), (uint32_t)(((li - 2) >> 1) & 1));
+                tc::fence_after_sync();
+                const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
+                for (int k = 0; k < W; ++k)
+                    for (int ks = 0; ks < m.RP / 16; ++ks) {
+                        const uint64_t ad = tc::smem_desc(zb + (uint32_t)(k * 16) + (uint32_t)ks * 2u * TB_ZR, TB_ZR, 128);
+                        const uint64_t bd = tc::smem_desc(ub + (uint32_t)((k * m.GB / 8) * m.RP * 16) + (uint32_t)ks * 256u,
+                                                          128, (uint32_t)(m.RP * 16));
+                        tc::mma_bf16(tmem + (uint32_t)(b * TB_NB + k * m.GB), ad, bd, id_w, ks > 0 ? 1u : 0u);
+                    }
+                tc::mma_commit(bars.wf(b));
+                if (++ob == NOP) {
+                    ob = 0;
+                    oph ^= 1u;
+                }
+            }
+        }
+    } else if (warp == 19) {
+        // ------------------------------------------------ dz / dU MMAs
+        if (lane == 0) {
             const uint32_t id_dz = tc::idesc_bf16(TC_M, m.RP, 0, 0);
             const uint32_t id_dU = tc::idesc_bf16(TC_M, m.RP, 1, 1);
-            // w(li_w): filters of the next item; fin(li_f): dz / dU of the oldest item whose dw
-            // tile is complete.  Each is issued as soon as its inputs are ready.
-            int li_w = 0, wob = 0, li_f = 0, fob = 0, fdb = 0, ftl = 0, fcl = 0;
-            uint32_t woph = 0, fdph = 0;
-            long long last = clock64();
-            while (li_f < nI) {
-                bool prog = false;
-                if (li_w < nI) {
-                    const int b = li_w & 1;
-                    if (tc::mbar_test(bars.opf(wob), woph) &&
-                        (li_w < 2 || tc::mbar_test(bars.we(b), (uint32_t)(((li_w - 2) >> 1) & 1)))) {
-                        tc::fence_after_sync();
-                        const uint32_t zb = sbase + (uint32_t)wob * S.opsize, ub = zb + S.zbytes;
-                        for (int k = 0; k < W; ++k)
-                            for (int ks = 0; ks < m.RP / 16; ++ks) {
-                                const uint64_t ad =
-                                    tc::smem_desc(zb + (uint32_t)(k * 16) + (uint32_t)ks * 2u * TB_ZR, TB_ZR, 128);
-                                const uint64_t bd = tc::smem_desc(
-                                    ub + (uint32_t)((k * m.GB / 8) * m.RP * 16) + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
-                                tc::mma_bf16(tmem + (uint32_t)(b * TB_NB + k * m.GB), ad, bd, id_w, ks > 0 ? 1u : 0u);
-                            }
-                        tc::mma_commit(bars.wf(b));
-                        if (++wob == NOP) {
-                            wob = 0;
-                            woph ^= 1u;
-                        }
-                        ++li_w;
-                        prog = true;
-                    }
+            int fob = 0, fdb = 0, ftl = 0, fcl = 0;
+            uint32_t fdph = 0;
+            for (int li = 0; li < nI; ++li) {
+                const int tp = ftl & 1;
+                wait(bars.dwf(fdb), fdph);  // item li's dw tile is complete (so are its filter MMAs)
+                if (fcl == 0 && ftl >= 2) wait(bars.dze(tp), (uint32_t)(((ftl - 2) >> 1) & 1));
+                tc::fence_after_sync();
+                const uint32_t zb = sbase + (uint32_t)fob * S.opsize, ub = zb + S.zbytes;
+                const uint32_t dwb = sbase + S.dw + (uint32_t)fdb * S.dwsize;
+                for (int ks = 0; ks < TB_NB / 16; ++ks) {
+                    const uint64_t ad = tc::smem_desc(dwb + (uint32_t)ks * 256u, 128, (TB_NB / 8) * 128);
+                    const uint64_t bd = tc::smem_desc(ub + (uint32_t)(ks * 2 * m.RP * 16), (uint32_t)(m.RP * 16), 128);
+                    tc::mma_bf16(tmem + col_dz + (uint32_t)(tp * m.RP), ad, bd, id_dz, (fcl > 0 || ks > 0) ? 1u : 0u);
                 }
-                if (li_f < li_w) {
-                    const int tp = ftl & 1;
-                    if (tc::mbar_test(bars.dwf(fdb), fdph) &&
-                        (fcl != 0 || ftl < 2 || tc::mbar_test(bars.dze(tp), (uint32_t)(((ftl - 2) >> 1) & 1)))) {
-                        tc::fence_after_sync();
-                        const uint32_t zb = sbase + (uint32_t)fob * S.opsize, ub = zb + S.zbytes;
-                        const uint32_t dwb = sbase + S.dw + (uint32_t)fdb * S.dwsize;
-                        for (int ks = 0; ks < TB_NB / 16; ++ks) {
-                            const uint64_t ad = tc::smem_desc(dwb + (uint32_t)ks * 256u, 128, (TB_NB / 8) * 128);
-                            const uint64_t bd =
-                                tc::smem_desc(ub + (uint32_t)(ks * 2 * m.RP * 16), (uint32_t)(m.RP * 16), 128);
-                            tc::mma_bf16(tmem + col_dz + (uint32_t)(tp * m.RP), ad, bd, id_dz,
-                                         (fcl > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        for (int ks = 0; ks < TC_M / 16; ++ks) {
-                            const uint64_t ad =
-                                tc::smem_desc(dwb + (uint32_t)ks * 2u * ((TB_NB / 8) * 128), (TB_NB / 8) * 128, 128);
-                            const uint64_t bd = tc::smem_desc(zb + (uint32_t)ks * 256u, 128, TB_ZR);
-                            tc::mma_bf16(tmem + col_dU + (uint32_t)(fcl * m.RP), ad, bd, id_dU,
-                                         (ftl > 0 || ks > 0) ? 1u : 0u);
-                        }
-                        tc::mma_commit(bars.dwe(fdb));
-                        tc::mma_commit(bars.ope(fob));
-                        if (fcl == ncl - 1) tc::mma_commit(bars.dzf(tp));
-                        if (++fob == NOP) fob = 0;
-                        if (++fdb == DWB) {
-                            fdb = 0;
-                            fdph ^= 1u;
-                        }
-                        if (++fcl == ncl) {
-                            fcl = 0;
-                            ++ftl;
-                        }
-                        ++li_f;
-                        prog = true;
-                    }
+                for (int ks = 0; ks < TC_M / 16; ++ks) {
+                    const uint64_t ad =
+                        tc::smem_desc(dwb + (uint32_t)ks * 2u * ((TB_NB / 8) * 128), (TB_NB / 8) * 128, 128);
+                    const uint64_t bd = tc::smem_desc(zb + (uint32_t)ks * 256u, 128, TB_ZR);
+                    tc::mma_bf16(tmem + col_dU + (uint32_t)(fcl * m.RP), ad, bd, id_dU, (ftl > 0 || ks > 0) ? 1u : 0u);
                 }
-                if (prog) {
-                    last = clock64();
-                } else {
-                    if (clock64() - last > TC_WAIT_LIMIT) {
-                        timed_out = true;
-                        break;
-                    }
-                    // sleep on the barrier the oldest pending step needs; it wakes the lane at once
-                    if (li_f < li_w) tc::mbar_try(bars.dwf(fdb), fdph, 1000);
-                    else tc::mbar_try(bars.opf(wob), woph, 1000);
+                tc::mma_commit(bars.dwe(fdb));
+                tc::mma_commit(bars.ope(fob));
+                if (fcl == ncl - 1) tc::mma_commit(bars.dzf(tp));
+                if (++fob == NOP) fob = 0;
+                if (++fdb == DWB) {
+                    fdb = 0;
+                    fdph ^= 1u;
+                }
+                if (++fcl == ncl) {
+                    fcl = 0;
+                    ++ftl;
                 }
             }
             tc::mma_commit(bars.duf());
@@ -572,7 +567,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 
     // teardown: every load and MMA this CTA issued has landed before the
     // shared memory and TMEM are given back (bounded, also after a time-out)
-    if (warp == 17 && lane == 0) tc::mbar_wait(bars.duf(), 0, TC_WAIT_LIMIT);
+    if (warp == 19 && lane == 0) tc::mbar_wait(bars.duf(), 0, TC_WAIT_LIMIT);
     if (timed_out) atomicExch(&g_dsc_status_tcb, (int)DSC_ERR_TIMEOUT);
     tc::fence_before_sync();
     __syncthreads();
