@@ -25,7 +25,7 @@
 // partial summed by a finalize kernel).
 //
 // Warp roles (640 threads): warp 16 x/dy TMA producer, warp 17 TMEM owner and
-// filter-MMA issuer, warp 18 operand loader, warp 19 dz/dU-MMA issuer, warps
+// filter-MMA issuer, warp 18 operand loads and dU MMAs, warp 19 dz MMAs, warps
 // 0-15 epilogue (thread part p of token t: VPT 8-channel vectors of each
 // sub-tile).  Groups wider than a part's channels (PPG parts per group) add
 // their dw partial sums through a small exchange buffer.
@@ -122,15 +122,6 @@ struct BwdWalk {
         blk = chunk_lo + cl;
     }
 };
-
-// 16-byte cp.async global -> shared (L2 only) and its mbarrier arrival (no count increment).
-__device__ __forceinline__ void tc_cp16(uint32_t dst, const void *src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void tc_cp_arrive(uint32_t bar) {
-    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
-}
-__device__ __forceinline__ void tc_cp_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, %0;" ::"n"(TB_EPI) : "memory"); }
 
@@ -302,14 +293,14 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 
     if (tid == 0) {
         for (int i = 0; i < TB_MAXOP; ++i) {
-            tc::mbar_init(bars.opf(i), 32);  // one cp.async arrival per loader lane
-            tc::mbar_init(bars.ope(i), 1);
+            tc::mbar_init(bars.opf(i), 1);
+            tc::mbar_init(bars.ope(i), 2);  // dz and dU MMAs of the item, from two threads
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(bars.wf(i), 1);
             tc::mbar_init(bars.we(i), TB_EPI / 32);
             tc::mbar_init(bars.dwf(i), TB_EPI / 32);
-            tc::mbar_init(bars.dwe(i), 1);
+            tc::mbar_init(bars.dwe(i), 2);
             tc::mbar_init(bars.dzf(i), 1);
             tc::mbar_init(bars.dze(i), TB_EPI / 32);
         }
@@ -331,41 +322,72 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
     };
 
     if (warp == 18) {
-        // ----------------------------------------------- operand loader warp
-        // The tile's z image and the block's U image, copied by the 32 lanes with
-        // cp.async (16 bytes each, the load/store path), so they never queue behind
-        // the x/dy tensor loads; each lane's arrival completes when its copies land.
-        BwdWalk it, pf;
-        it.init(m, tile_lo, chunk_lo);
-        pf.init(m, tile_lo, chunk_lo);
-        constexpr int PF = 6;  // operand images are prefetched into L2 this many items ahead
-        if (lane == 0)
+        // --------------------------- operand loads and dU MMAs (one lane)
+        // The tile's z image and the block's U image arrive by one bulk copy each;
+        // a buffer is refilled once the dz and dU MMAs of its previous item are done.
+        if (lane == 0) {
+            const uint32_t id_dU = tc::idesc_bf16(TC_M, m.RP, 1, 1);
+            BwdWalk it, pf;
+            it.init(m, tile_lo, chunk_lo);
+            pf.init(m, tile_lo, chunk_lo);
+            constexpr int PF = 6;  // operand images are prefetched into L2 this many items ahead
             for (int li = 0; li < PF && li < nI; ++li, pf.next(m, chunk_lo, ncl)) {
                 tc::bulk_prefetch_l2(a.zimg + (size_t)(tile_lo + pf.tl) * (S.zbytes / 2), S.zbytes);
                 tc::bulk_prefetch_l2(a.Up + (size_t)pf.blk * (S.ubytes / 2), S.ubytes);
             }
-        int ob = 0;
-        uint32_t oph = 0;
-        const uint32_t zch = S.zbytes / 16, uch = S.ubytes / 16;
-        for (int li = 0; li < nI; ++li, it.next(m, chunk_lo, ncl)) {
-            if (lane == 0 && li + PF < nI) {
-                tc::bulk_prefetch_l2(a.zimg + (size_t)(tile_lo + pf.tl) * (S.zbytes / 2), S.zbytes);
-                tc::bulk_prefetch_l2(a.Up + (size_t)pf.blk * (S.ubytes / 2), S.ubytes);
-                pf.next(m, chunk_lo, ncl);
+            auto load_op = [&](int ob) {
+                const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
+                tc::mbar_expect_tx(bars.opf(ob), S.zbytes + S.ubytes);
+                tc::bulk_load(zb, a.zimg + (size_t)(tile_lo + it.tl) * (S.zbytes / 2), S.zbytes, bars.opf(ob));
+                tc::bulk_load(ub, a.Up + (size_t)it.blk * (S.ubytes / 2), S.ubytes, bars.opf(ob));
+                if (pf.tl < ntl) {
+                    tc::bulk_prefetch_l2(a.zimg + (size_t)(tile_lo + pf.tl) * (S.zbytes / 2), S.zbytes);
+                    tc::bulk_prefetch_l2(a.Up + (size_t)pf.blk * (S.ubytes / 2), S.ubytes);
+                    pf.next(m, chunk_lo, ncl);
+                }
+                it.next(m, chunk_lo, ncl);
+            };
+            int nload = 0;
+            for (; nload < NOP && nload < nI; ++nload) load_op(nload);
+            int fob = 0, fdb = 0, ftl = 0, fcl = 0;
+            uint32_t fdph = 0, foph = 0;
+            for (int li = 0; li < nI; ++li) {
+                wait(bars.dwf(fdb), fdph);  // item li's dw tile is complete
+                tc::fence_after_sync();
+                const uint32_t zb = sbase + (uint32_t)fob * S.opsize;
+                const uint32_t dwb = sbase + S.dw + (uint32_t)fdb * S.dwsize;
+                for (int ks = 0; ks < TC_M / 16; ++ks) {
+                    const uint64_t ad =
+                        tc::smem_desc(dwb + (uint32_t)ks * 2u * ((TB_NB / 8) * 128), (TB_NB / 8) * 128, 128);
+                    const uint64_t bd = tc::smem_desc(zb + (uint32_t)ks * 256u, 128, TB_ZR);
+                    tc::mma_bf16(tmem + col_dU + (uint32_t)(fcl * m.RP), ad, bd, id_dU, (ftl > 0 || ks > 0) ? 1u : 0u);
+                }
+                tc::mma_commit(bars.dwe(fdb));
+                tc::mma_commit(bars.ope(fob));
+                if (nload < nI) {  // refill this buffer for item li + NOP
+                    wait(bars.ope(fob), foph);
+                    load_op(fob);
+                    ++nload;
+                }
+                if (++fob == NOP) {
+                    fob = 0;
+                    foph ^= 1u;
+                }
+                if (++fdb == DWB) {
+                    fdb = 0;
+                    fdph ^= 1u;
+                }
+                if (++fcl == ncl) {
+                    fcl = 0;
+                    ++ftl;
+                }
             }
-            if (li >= NOP) wait(bars.ope(ob), oph ^ 1u);
-            const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
-            const unsigned char *zs = reinterpret_cast<const unsigned char *>(a.zimg + (size_t)(tile_lo + it.tl) * (S.zbytes / 2));
-            const unsigned char *us = reinterpret_cast<const unsigned char *>(a.Up + (size_t)it.blk * (S.ubytes / 2));
-            for (uint32_t c = lane; c < zch; c += 32) tc_cp16(zb + 16u * c, zs + 16u * c);
-            for (uint32_t c = lane; c < uch; c += 32) tc_cp16(ub + 16u * c, us + 16u * c);
-            tc_cp_arrive(bars.opf(ob));
-            if (++ob == NOP) {
-                ob = 0;
-                oph ^= 1u;
+            tc::mma_commit(bars.duf());
+            for (int b = 0; b < NOP && b < nI; ++b) {  // the last loads have landed
+                const int last = b + ((nI - 1 - b) / NOP) * NOP;
+                tc::mbar_wait(bars.opf(b), (uint32_t)((last / NOP) & 1), TC_WAIT_LIMIT);
             }
         }
-        tc_cp_wait_all();
     } else if (warp == 16) {
         // ------------------------------------------------- x / dy producer
         if (lane == 0) {
@@ -423,10 +445,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             }
         }
     } else if (warp == 19) {
-        // ------------------------------------------------ dz / dU MMAs
+        // ---------------------------------------------------- dz MMAs
         if (lane == 0) {
             const uint32_t id_dz = tc::idesc_bf16(TC_M, m.RP, 0, 0);
-            const uint32_t id_dU = tc::idesc_bf16(TC_M, m.RP, 1, 1);
             int fob = 0, fdb = 0, ftl = 0, fcl = 0;
             uint32_t fdph = 0;
             for (int li = 0; li < nI; ++li) {
@@ -434,18 +455,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                 wait(bars.dwf(fdb), fdph);  // item li's dw tile is complete (so are its filter MMAs)
                 if (fcl == 0 && ftl >= 2) wait(bars.dze(tp), (uint32_t)(((ftl - 2) >> 1) & 1));
                 tc::fence_after_sync();
-                const uint32_t zb = sbase + (uint32_t)fob * S.opsize, ub = zb + S.zbytes;
+                const uint32_t ub = sbase + (uint32_t)fob * S.opsize + S.zbytes;
                 const uint32_t dwb = sbase + S.dw + (uint32_t)fdb * S.dwsize;
                 for (int ks = 0; ks < TB_NB / 16; ++ks) {
                     const uint64_t ad = tc::smem_desc(dwb + (uint32_t)ks * 256u, 128, (TB_NB / 8) * 128);
                     const uint64_t bd = tc::smem_desc(ub + (uint32_t)(ks * 2 * m.RP * 16), (uint32_t)(m.RP * 16), 128);
                     tc::mma_bf16(tmem + col_dz + (uint32_t)(tp * m.RP), ad, bd, id_dz, (fcl > 0 || ks > 0) ? 1u : 0u);
-                }
-                for (int ks = 0; ks < TC_M / 16; ++ks) {
-                    const uint64_t ad =
-                        tc::smem_desc(dwb + (uint32_t)ks * 2u * ((TB_NB / 8) * 128), (TB_NB / 8) * 128, 128);
-                    const uint64_t bd = tc::smem_desc(zb + (uint32_t)ks * 256u, 128, TB_ZR);
-                    tc::mma_bf16(tmem + col_dU + (uint32_t)(fcl * m.RP), ad, bd, id_dU, (ftl > 0 || ks > 0) ? 1u : 0u);
                 }
                 tc::mma_commit(bars.dwe(fdb));
                 tc::mma_commit(bars.ope(fob));
@@ -460,7 +475,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                     ++ftl;
                 }
             }
-            tc::mma_commit(bars.duf());
         }
     } else {
         // ------------------------------------------------------------ epilogue
@@ -567,7 +581,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 
     // teardown: every load and MMA this CTA issued has landed before the
     // shared memory and TMEM are given back (bounded, also after a time-out)
-    if (warp == 19 && lane == 0) tc::mbar_wait(bars.duf(), 0, TC_WAIT_LIMIT);
+    if (warp == 18 && lane == 0) tc::mbar_wait(bars.duf(), 0, TC_WAIT_LIMIT);
     if (timed_out) atomicExch(&g_dsc_status_tcb, (int)DSC_ERR_TIMEOUT);
     tc::fence_before_sync();
     __syncthreads();
