@@ -221,6 +221,8 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
     const StreamMap &m = a.m;
     Pos q;
     if (!locate<VecOf<T>::V>(m, q) || !q.active) return;
+    pdl_wait();  // inputs may come from the previous kernel of the stream
+    pdl_trigger();
 
     const int n = q.t_end - q.t_start;
     const int64_t xstep = m.D * (int64_t)sizeof(T);
@@ -318,6 +320,8 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
     const StreamMap &m = a.m;
     Pos q;
     if (!locate<VecOf<T>::V>(m, q)) return;  // whole warp out of range; partial warps stay for the shuffles
+    pdl_wait();  // inputs may come from the previous kernel of the stream
+    pdl_trigger();
     // Inactive lanes (no channels of their own) stream channel 0 of the same rows: in bounds, never
     // stored, and never in a filter group with an active lane.
     const bool act = q.active;
@@ -577,9 +581,10 @@ static cudaError_t run_stream(const Ctx &c, HwArgs a) {
     const size_t smem = stream_setup<T, W, GPT, WS, BWD>(per_sm);
     finish_map(a.m, (int64_t)per_sm * c.sms);
     const int64_t blocks = (a.m.n_warps + STREAM_THREADS / 32 - 1) / (STREAM_THREADS / 32);
-    if constexpr (BWD) { k_stream_bwd<T, W, GPT, WS><<<(unsigned)blocks, STREAM_THREADS, smem, c.stream>>>(a); count_launch(); }
-    else { k_stream_fwd<T, W, GPT, WS><<<(unsigned)blocks, STREAM_THREADS, smem, c.stream>>>(a); count_launch(); }
-    return cudaGetLastError();
+    cudaError_t e;
+    if constexpr (BWD) e = launch_pdl(k_stream_bwd<T, W, GPT, WS>, dim3((unsigned)blocks), dim3(STREAM_THREADS), smem, c.stream, a);
+    else e = launch_pdl(k_stream_fwd<T, W, GPT, WS>, dim3((unsigned)blocks), dim3(STREAM_THREADS), smem, c.stream, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 template <typename T, bool WS, bool BWD, int GPT>

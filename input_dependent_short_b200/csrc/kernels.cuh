@@ -1,6 +1,8 @@
 // Launch interface between the C entry points (api.cu) and the kernels.
 #pragma once
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace dsc {
@@ -86,6 +88,33 @@ int resident_blocks(const void *kernel, int threads, size_t smem);
 
 // Records one kernel launch (api.cu keeps the process-wide count).
 void count_launch();
+
+// Programmatic dependent launch.  A kernel launched with launch_pdl may be
+// scheduled while the previous kernel of the stream is still finishing; it
+// runs its prologue, then pdl_wait() blocks until that kernel has completed
+// and its writes are visible, so it must come before the first access to
+// global memory.  pdl_trigger() lets the next kernel of the stream be
+// scheduled the same way (it still waits for this one to complete).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args &&...args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+    count_launch();
+    return e;
+}
 
 // Status word of kernels with bounded waits (lowrank.cu): returns the
 // recorded dsc_status of the current device and clears it.

@@ -320,6 +320,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
     auto wait = [&](uint32_t bar, uint32_t parity) {
         if (!timed_out && !tc::mbar_wait(bar, parity, TC_WAIT_LIMIT)) timed_out = true;  // sticky: later waits skip
     };
+    pdl_wait();  // inputs and operand images come from earlier kernels of the stream
+    pdl_trigger();
 
     if (warp == 18) {
         // --------------------------- operand loads and dU MMAs (one lane)
@@ -595,6 +597,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 //   z image of tile i (sequence b, first token t0): element (t, r) at
 //     (r/8)*(136*8) + t*8 + r%8 holding z[b][t0+t][r], zero for r >= R or t0+t >= T.
 __global__ void k_bwd_prep(const TcArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const TcMap &m = a.m;
     const int64_t ublk = (int64_t)m.RP * TB_NB;
     const int64_t nU = (int64_t)m.nBlkB * ublk;
@@ -621,11 +625,15 @@ __global__ void k_bwd_prep(const TcArgs a) {
 }
 
 __global__ void k_tc_zero(float *p, int64_t n) {
+    pdl_wait();
+    pdl_trigger();
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) p[i] = 0.f;
 }
 
 // dU = sum of the per-range partials (fixed order); dz = the fp32 accumulator in bf16.
 __global__ void k_tc_finalize(const TcArgs a) {
+    pdl_wait();
+    pdl_trigger();
     const TcMap &m = a.m;
     const int64_t nU = m.nRanges > 1 ? m.R * m.GW : 0;
     const int64_t nz = m.nGroups > 1 ? m.B * m.T * m.R : 0;
@@ -731,10 +739,9 @@ cudaError_t launch_bwd(const Ctx &c, const TcArgs &a) {
     if (!bwd_maps(a, f)) return cudaErrorNotSupported;
     // the whole of TMEM per CTA: enough shared memory that no second CTA shares the SM
     const uint32_t smem = S.total < 120 * 1024 ? 120 * 1024 : S.total;
-    k_lr_tc_bwd<W, VPT, GPT, PPG><<<(unsigned)(a.m.nGroups * a.m.nRanges), TB_THREADS, smem, c.stream>>>(f.x, f.dy, f.dx,
-                                                                                                       a);
-    count_launch();
-    return cudaGetLastError();
+    const cudaError_t e = launch_pdl(k_lr_tc_bwd<W, VPT, GPT, PPG>, dim3((unsigned)(a.m.nGroups * a.m.nRanges)),
+                                     dim3(TB_THREADS), smem, c.stream, f.x, f.dy, f.dx, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // Thread channels per sub-tile: CT = 8*VPT (SB = 32 or 64, four parts).
@@ -793,15 +800,16 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
         w += (size_t)a.m.nRanges * a.m.R * a.m.GW * 4;
     }
     const int64_t nprep = (int64_t)a.m.nBlkB * a.m.RP * TB_NB + a.m.totalTiles * (a.m.RP / 8) * TB_ZROWS * 8;
-    k_bwd_prep<<<(unsigned)min((int64_t)2048, (nprep + 255) / 256), 256, 0, c.stream>>>(a);
-    count_launch();
+    cudaError_t e = launch_pdl(k_bwd_prep, dim3((unsigned)min((int64_t)2048, (nprep + 255) / 256)), dim3(256), 0,
+                               c.stream, a);
+    if (e != cudaSuccess) return e;
     if (a.m.nGroups > 1) {
         a.dz_acc = reinterpret_cast<float *>(w);
         const int64_t n = a.m.B * a.m.T * a.m.R;
-        k_tc_zero<<<(unsigned)min((int64_t)1024, (n + 255) / 256), 256, 0, c.stream>>>(a.dz_acc, n);
-        count_launch();
+        e = launch_pdl(k_tc_zero, dim3((unsigned)min((int64_t)1024, (n + 255) / 256)), dim3(256), 0, c.stream, a.dz_acc, n);
+        if (e != cudaSuccess) return e;
     }
-    cudaError_t e = cudaErrorNotSupported;
+    e = cudaErrorNotSupported;
     switch (a.m.W) {
     case 1: e = bwd_by_vpt<1>(c, a); break;
     case 2: e = bwd_by_vpt<2>(c, a); break;
@@ -811,8 +819,8 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     if (e != cudaSuccess) return e;
     if (a.m.nRanges > 1 || a.m.nGroups > 1) {
         const int64_t n = (a.m.nRanges > 1 ? a.m.R * a.m.GW : 0) + (a.m.nGroups > 1 ? a.m.B * a.m.T * a.m.R : 0);
-        k_tc_finalize<<<(unsigned)min((int64_t)2048, (n + 255) / 256), 256, 0, c.stream>>>(a);
-        count_launch();
+        e = launch_pdl(k_tc_finalize, dim3((unsigned)min((int64_t)2048, (n + 255) / 256)), dim3(256), 0, c.stream, a);
+        if (e != cudaSuccess) return e;
     }
     return cudaGetLastError();
 }

@@ -332,6 +332,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
     auto wait = [&](uint32_t bar, uint32_t parity) {
         if (!timed_out && !tc::mbar_wait(bar, parity, TC_WAIT_LIMIT)) timed_out = true;  // sticky: later waits skip
     };
+    pdl_wait();  // inputs may come from the previous kernel of the stream
+    pdl_trigger();
 
     if (warp == 16) {
         // ------------------------------------------------------------ producer
@@ -541,9 +543,9 @@ cudaError_t launch_fwd(const Ctx &c, const TcArgs &a) {
     const int64_t grid = (total + per - 1) / per;
     // More than half of TMEM per CTA: enough shared memory that no second CTA shares the SM.
     const uint32_t smem = 2 * a.m.NF > 256 && S.total < 120 * 1024 ? 120 * 1024 : S.total;
-    k_lr_tc_fwd<W, GPV, VPT, NGT><<<(unsigned)grid, TF_THREADS, smem, c.stream>>>(f.x, f.z, f.u, f.y, a);
-    count_launch();
-    return cudaGetLastError();
+    const cudaError_t e =
+        launch_pdl(k_lr_tc_fwd<W, GPV, VPT, NGT>, dim3((unsigned)grid), dim3(TF_THREADS), smem, c.stream, f.x, f.z, f.u, f.y, a);
+    return e != cudaSuccess ? e : cudaGetLastError();
 }
 
 // A sub-tile's filters fit one block (4 * VPT * GPV * W <= NF <= 256); other
