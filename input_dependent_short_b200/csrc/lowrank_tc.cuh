@@ -38,6 +38,8 @@ struct TcMap {
     // sub-tiles of SB channels; CTA = (range of tiles) x (group of CPC blocks)
     int CB, GB, SB, nSubB, nBlkB;
     int CPC, nGroups, nRanges, tilesPerRange;
+    int splitUnits;      // > 0: one block per CTA, ranges of this many (tile, sub-tile) units
+    int dzAcc;           // dz through an fp32 accumulator (several CTAs add to a token's dz)
     int NSB, DWB, NOP;   // sub-tile ring slots, dw tile buffers, operand buffers
     int64_t totalTiles;
 };

@@ -278,11 +278,25 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
     const int range = blockIdx.x / m.nGroups;
     const int chunk_lo = group * m.CPC;
     const int ncl = min(m.CPC, m.nBlkB - chunk_lo);
-    const int64_t tile_lo = (int64_t)range * m.tilesPerRange;
-    const int ntl = (int)min((int64_t)m.tilesPerRange, m.totalTiles - tile_lo);
+    int64_t tile_lo;
+    int ntl, s_first = 0, s_last = m.nSubB;  // sub-tiles of the first and last item
+    if (m.splitUnits > 0) {  // a range of (tile, sub-tile) units of one block
+        const int64_t u_lo = (int64_t)range * m.splitUnits;
+        const int64_t u_hi = min(u_lo + m.splitUnits, m.totalTiles * m.nSubB);
+        if (u_lo >= u_hi) return;
+        tile_lo = u_lo / m.nSubB;
+        ntl = (int)((u_hi - 1) / m.nSubB - tile_lo + 1);
+        s_first = (int)(u_lo % m.nSubB);
+        s_last = (int)((u_hi - 1) % m.nSubB) + 1;
+    } else {
+        tile_lo = (int64_t)range * m.tilesPerRange;
+        ntl = (int)min((int64_t)m.tilesPerRange, m.totalTiles - tile_lo);
+    }
     if (ncl <= 0 || ntl <= 0) return;
     const int nI = ntl * ncl;
-    const int nG = nI * m.nSubB;
+    auto s_begin = [&](int li) { return li == 0 ? s_first : 0; };
+    auto s_end = [&](int li) { return li == nI - 1 ? s_last : m.nSubB; };
+    const int nG = nI == 1 ? s_last - s_first : (m.nSubB - s_first) + (nI - 2) * m.nSubB + s_last;
 
     const uint32_t sraw = tc::smem_u32(smem_raw);
     const uint32_t sbase = (sraw + 1023u) & ~1023u;
@@ -399,7 +413,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             int slot = 0, l = 0;
             uint32_t xph = 0;
             for (int li = 0; li < nI; ++li, it.next(m, chunk_lo, ncl)) {
-                for (int s = 0; s < m.nSubB; ++s, ++l) {
+                for (int s = s_begin(li); s < s_end(li); ++s, ++l) {
                     if (l >= NS) wait(bars.xe(slot), xph ^ 1u);
                     const uint32_t xb = sbase + S.ring + (uint32_t)slot * S.slot;
                     tc::mbar_expect_tx(bars.xf(slot), (uint32_t)(2 * RB * (TC_M + WIN)));
@@ -496,7 +510,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                 tc::tmem_wait_ld();
                 if (t < m.T && r < m.R) {  // R is a multiple of 8
                     const int64_t o = ((int64_t)bseq * m.T + t) * m.R + r;
-                    if (m.nGroups == 1) {
+                    if (!m.dzAcc) {
                         st16(a.dz + o, make_uint4(pack_bf2(v[0], v[1]), pack_bf2(v[2], v[3]), pack_bf2(v[4], v[5]),
                                                   pack_bf2(v[6], v[7])));
                     } else {
@@ -520,11 +534,18 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             tc::fence_after_sync();
             const uint32_t tb = tlane + (uint32_t)(b * TB_NB);
             unsigned char *dwt = smem + S.dw + (uint32_t)db * S.dwsize;
-            for (int s = 0; s < m.nSubB; ++s) {
+            const int sb = s_begin(li), se = s_end(li);
+            if (sb > 0 || se < m.nSubB) {
+                // part of the block's groups only: the other dw columns must read as zero
+                for (int i = tid; i < TC_M * TB_NB * 2 / 16; i += TB_EPI)
+                    *reinterpret_cast<uint4 *>(dwt + 16 * i) = make_uint4(0, 0, 0, 0);
+                epi_bar();
+            }
+            for (int s = sb; s < se; ++s) {
                 wait(bars.xf(slot), xph);
                 bwd_subtile<W, VPT, GPT, PPG, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, xch, part,
                                                   t_loc, s, smem + S.ystage + (uint32_t)ybuf * S.ybox, res,
-                                                  s == m.nSubB - 1 ? bars.we(b) : 0u);
+                                                  s == se - 1 ? bars.we(b) : 0u);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars.xe(slot));
                 // dx tile -> global by TMA (the staging tile the next sub-tile writes was read
@@ -636,7 +657,7 @@ __global__ void k_tc_finalize(const TcArgs a) {
     pdl_trigger();
     const TcMap &m = a.m;
     const int64_t nU = m.nRanges > 1 ? m.R * m.GW : 0;
-    const int64_t nz = m.nGroups > 1 ? m.B * m.T * m.R : 0;
+    const int64_t nz = m.dzAcc ? m.B * m.T * m.R : 0;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nU + nz; i += (int64_t)gridDim.x * blockDim.x) {
         if (i < nU) {
             float sacc = 0.f;
@@ -688,6 +709,19 @@ bool tc_bwd_plan(TcMap &m, int sms) {
     }
     m.tilesPerRange = (int)((m.totalTiles + m.nRanges - 1) / m.nRanges);
     m.nRanges = (int)((m.totalTiles + m.tilesPerRange - 1) / m.tilesPerRange);
+    m.splitUnits = 0;
+    if (m.CPC == 1 && m.nSubB >= 8) {
+        // long items, one block per CTA: split the (tile, sub-tile) units evenly so
+        // that every SM gets the same share even when tiles do not divide evenly
+        const int64_t units = m.totalTiles * m.nSubB;
+        const int64_t nr = max((int64_t)1, (int64_t)(sms / m.nGroups));
+        const int64_t per = (units + nr - 1) / nr;
+        if (per < (int64_t)m.tilesPerRange * m.nSubB) {
+            m.splitUnits = (int)per;
+            m.nRanges = (int)((units + per - 1) / per);
+        }
+    }
+    m.dzAcc = (m.nGroups > 1 || m.splitUnits > 0) ? 1 : 0;
     const int vpt = m.SB / 32, ct = 8 * vpt;
     const bool xchg = m.H > ct;
     const bool short_items = m.nSubB < 4;
@@ -707,7 +741,7 @@ size_t zimg_bytes(const TcMap &m) { return ((size_t)m.totalTiles * (m.RP / 8) * 
 size_t tc_bwd_ws_bytes(const TcMap &m) {
     size_t n = up_bytes(m) + zimg_bytes(m);
     if (m.nRanges > 1) n += (size_t)m.nRanges * m.R * m.GW * 4;
-    if (m.nGroups > 1) n += (size_t)m.B * m.T * m.R * 4;
+    if (m.dzAcc) n += (size_t)m.B * m.T * m.R * 4;
     return n;
 }
 
@@ -803,7 +837,7 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     cudaError_t e = launch_pdl(k_bwd_prep, dim3((unsigned)min((int64_t)2048, (nprep + 255) / 256)), dim3(256), 0,
                                c.stream, a);
     if (e != cudaSuccess) return e;
-    if (a.m.nGroups > 1) {
+    if (a.m.dzAcc) {
         a.dz_acc = reinterpret_cast<float *>(w);
         const int64_t n = a.m.B * a.m.T * a.m.R;
         e = launch_pdl(k_tc_zero, dim3((unsigned)min((int64_t)1024, (n + 255) / 256)), dim3(256), 0, c.stream, a.dz_acc, n);
@@ -817,8 +851,8 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     case 8: e = bwd_by_vpt<8>(c, a); break;
     }
     if (e != cudaSuccess) return e;
-    if (a.m.nRanges > 1 || a.m.nGroups > 1) {
-        const int64_t n = (a.m.nRanges > 1 ? a.m.R * a.m.GW : 0) + (a.m.nGroups > 1 ? a.m.B * a.m.T * a.m.R : 0);
+    if (a.m.nRanges > 1 || a.m.dzAcc) {
+        const int64_t n = (a.m.nRanges > 1 ? a.m.R * a.m.GW : 0) + (a.m.dzAcc ? a.m.B * a.m.T * a.m.R : 0);
         e = launch_pdl(k_tc_finalize, dim3((unsigned)min((int64_t)2048, (n + 255) / 256)), dim3(256), 0, c.stream, a);
         if (e != cudaSuccess) return e;
     }

@@ -354,9 +354,13 @@ def test_sweep_workloads_sampled(wl):
                          ids=["all-linear-shape", "qkv-shape"])
 def test_lowrank_fused_materialises_no_filters(shape):
     """The fused low-rank kernels never hold w = zU or dw in device memory: the
-    forward needs no workspace, the backward's workspace (per-range dU partials
-    and an fp32 dz accumulator) is far smaller than the filter tensor, and the
-    peak allocation grows by the outputs and that workspace only."""
+    forward needs no workspace, the backward's workspace (operand images of z
+    and U, per-range dU partials and an fp32 dz accumulator: O(B*T*R +
+    ranges*R*G*W), not O(B*T*G*W)) stays well below the fp32 filter tensor,
+    and the peak allocation grows by the outputs and that workspace only.  On
+    the all-linear shape G*W = 512 is small, so the bound there is half the
+    filter tensor; on the Q/K/V-like shape (G*W = 24576) it is about 12 MB
+    against a 400 MB filter tensor."""
     import ctypes as C
 
     from input_dependent_short_b200 import _lib
@@ -371,7 +375,9 @@ def test_lowrank_fused_materialises_no_filters(shape):
     filters = B * T * (D // H) * W * 4
     ws = L.dsc_bwd_lowrank_workspace_bytes(C.byref(p))
     assert L.dsc_fwd_lowrank_workspace_bytes(C.byref(p)) == 0
-    assert ws < filters / 3
+    assert ws < filters / 2
+    if (D // H) * W > 4096:
+        assert ws < filters / 20
     torch.cuda.synchronize()
     base = torch.cuda.memory_allocated()
     torch.cuda.reset_peak_memory_stats()
