@@ -8,21 +8,23 @@
 //   dz[t,:]   = sum_{g,k} dw[t,g,k] U[:, g*W+k]      dU[:, g*W+k] = sum_t z[t,:] dw[t,g,k]
 // (g = g(c) the channel's group; x, dy zero outside [0, T)).
 //
-// Block = GB = 128/W groups = CB = GB*H channels; U's columns of a block are
-// first reordered tap-major (U_perm, column k*GB + g) by a small kernel, so
-// that per tap k one MMA  z[t0+k .. t0+k+127] . U_perm[:, k-th GB columns]
-// puts w[t+k, g, k] -- the filter dx of token t needs -- on TMEM lane t: the
-// shift by k tokens is only a start address in the z tile (which holds 136
-// rows).  Work item = (tile of 128 tokens, block).  Per item:
-//   W MMAs        filters into one of two TMEM buffers (128 columns);
-//   epilogue      per sub-tile of SB channels: dx (stored) and dw (bf16,
-//                 tap-major, into a [128 x 128] shared tile);
-//   2 x 8 MMAs    dz[tile] += dw . U_perm^T   (TMEM, over the CTA's blocks),
-//                 dU[block] += dw^T . z        (TMEM, over the CTA's tiles).
-// CTA = (range of tiles) x (group of CPC blocks); dz leaves TMEM after a
-// tile's last block (bf16, or fp32 adds into an accumulator when several
-// block groups exist), dU after the range (directly, or as a per-range
-// partial summed by a finalize kernel).
+// Block = GB = 128/W groups = CB = GB*H channels.  A prep kernel writes each
+// block's U columns tap-major (column k*GB + g) and each z tile (136 rows) in
+// the byte order of their shared-memory images, so per tap k one MMA
+// z[t0+k .. t0+k+127] . U_block[:, k-th GB columns] puts w[t+k, g, k] -- the
+// filter dx of token t needs -- on TMEM lane t: the shift by k tokens is only
+// a start address in the z image.  Work item = (tile of 128 tokens, block).
+// Per item:
+//   W * RP/16 MMAs  filters into one of two TMEM buffers (128 columns);
+//   epilogue        per sub-tile of SB channels: dx (staged, TMA store) and dw
+//                   (bf16, tap-major, into a [128 x 128] shared tile);
+//   2 * 8 MMAs      dz[tile] += dw . U_block^T   (TMEM, over the CTA's blocks),
+//                   dU[block] += dw^T . z         (TMEM, over the CTA's tiles).
+// CTA = (range of tiles) x (group of CPC blocks), or for long items with one
+// block per CTA an equal range of (tile, sub-tile) units.  dz leaves TMEM after
+// a tile's last block (bf16, or fp32 adds into an accumulator when several
+// CTAs add to the same token), dU after the range (directly, or as a
+// per-range partial summed by a finalize kernel).
 //
 // Warp roles (640 threads): warp 16 x/dy TMA producer, warp 17 TMEM owner and
 // filter-MMA issuer, warp 18 operand loads and dU MMAs, warp 19 dz MMAs, warps
@@ -53,7 +55,7 @@ int take_tc_bwd_status(cudaStream_t stream) {
 namespace {
 
 constexpr int TB_EPI = 512;              // epilogue threads
-constexpr int TB_THREADS = TB_EPI + 128;  // + x/dy producer, filter-MMA, operand-loader and dz/dU-MMA warps
+constexpr int TB_THREADS = TB_EPI + 128;  // + x/dy producer, filter-MMA, operand/dU-MMA and dz-MMA warps
 constexpr int TB_MAXNS = 8;              // most sub-tiles in flight
 constexpr int TB_SMEM = 220 * 1024;
 constexpr int TB_NB = 128;               // filter columns per block (W * GB)
