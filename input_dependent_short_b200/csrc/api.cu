@@ -178,6 +178,13 @@ dsc_status dsc_bwd_static(const dsc_problem *p, const void *x, const void *ws, c
     return done(e);
 }
 
+int dsc_lowrank_kernels(const dsc_problem *p, int backward) {
+    if (validate(p, true) != DSC_OK) return -1;
+    if (backward ? lowrank_tc_bwd_ok(*p, sm_count()) : lowrank_tc_ok(*p)) return DSC_LR_TENSOR_CORE;
+    if (lowrank_fused_ok(*p)) return DSC_LR_FUSED;
+    return DSC_LR_UNFUSED;
+}
+
 size_t dsc_fwd_lowrank_workspace_bytes(const dsc_problem *p) {
     if (validate(p, true) != DSC_OK) return 0;
     if (lowrank_tc_ok(*p) || lowrank_fused_ok(*p)) return 0;

@@ -8,7 +8,7 @@
 // training implementation" (the fused kernels form zU on chip and convolve at
 // once; the filter tensor never reaches HBM).
 //
-// Used for bf16 with R a multiple of 8 up to 64, W in {1, 2, 4, 8}, H a
+// Used for bf16 with R a multiple of 8 up to 64, W in {1, 2, 3, 4, 8}, H a
 // divisor of 64 and D a multiple of 32*H; the CUDA-core kernels cover every
 // other shape.
 #pragma once
@@ -33,10 +33,11 @@ struct TcMap {
     int residual;
     // forward: item = (tile, block of CF channels) -> NF TMEM columns; sub-tiles of SF channels
     int CF, NF, SF, nSubF, nBlkF, NSF, NOPF;
+    int NFS;             // TMEM columns per filter buffer: NF rounded up to a power of two
     int64_t nItemsF;
-    // backward: block of CB channels = GB groups -> W*GB = 128 filter columns;
+    // backward: block of CB channels = GB groups -> NBW = W*GB <= 128 filter columns;
     // sub-tiles of SB channels; CTA = (range of tiles) x (group of CPC blocks)
-    int CB, GB, SB, nSubB, nBlkB;
+    int CB, GB, NBW, SB, nSubB, nBlkB;
     int CPC, nGroups, nRanges, tilesPerRange;
     int splitUnits;      // > 0: one block per CTA, ranges of this many (tile, sub-tile) units
     int dzAcc;           // dz through an fp32 accumulator (several CTAs add to a token's dz)
@@ -66,26 +67,24 @@ int take_tc_bwd_status(cudaStream_t stream);
 
 __host__ __device__ constexpr uint32_t up1024(uint32_t v) { return (v + 1023u) & ~1023u; }
 
-// 32 lanes x N consecutive fp32 TMEM columns (N = 1, 2, 4 or a multiple of 8).
+// 32 lanes x N consecutive fp32 TMEM columns (any N: loads of 8, then 4, 2, 1).
 template <int N> __device__ __forceinline__ void tmem_ld(uint32_t taddr, float (&v)[N]) {
     uint32_t r[N];
-    if constexpr (N == 1) {
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[0]) : "r"(taddr));
-    } else if constexpr (N == 2) {
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[0]), "=r"(r[1]) : "r"(taddr));
-    } else if constexpr (N == 4) {
-        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
-                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-                     : "r"(taddr));
-    } else {
-        static_assert(N % 8 == 0, "TMEM loads of 8 columns at a time");
 #pragma unroll
-        for (int i = 0; i < N / 8; ++i)
-            asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                         : "=r"(r[8 * i]), "=r"(r[8 * i + 1]), "=r"(r[8 * i + 2]), "=r"(r[8 * i + 3]),
-                           "=r"(r[8 * i + 4]), "=r"(r[8 * i + 5]), "=r"(r[8 * i + 6]), "=r"(r[8 * i + 7])
-                         : "r"(taddr + 8 * i));
-    }
+    for (int i = 0; i < N / 8; ++i)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[8 * i]), "=r"(r[8 * i + 1]), "=r"(r[8 * i + 2]), "=r"(r[8 * i + 3]),
+                       "=r"(r[8 * i + 4]), "=r"(r[8 * i + 5]), "=r"(r[8 * i + 6]), "=r"(r[8 * i + 7])
+                     : "r"(taddr + 8 * i));
+    constexpr int o4 = N / 8 * 8, o2 = o4 + (N & 4), o1 = o2 + (N & 2);
+    if constexpr ((N & 4) != 0)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x4.b32 {%0,%1,%2,%3}, [%4];"
+                     : "=r"(r[o4]), "=r"(r[o4 + 1]), "=r"(r[o4 + 2]), "=r"(r[o4 + 3])
+                     : "r"(taddr + o4));
+    if constexpr ((N & 2) != 0)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x2.b32 {%0,%1}, [%2];" : "=r"(r[o2]), "=r"(r[o2 + 1]) : "r"(taddr + o2));
+    if constexpr ((N & 1) != 0)
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r[o1]) : "r"(taddr + o1));
 #pragma unroll
     for (int i = 0; i < N; ++i) v[i] = __uint_as_float(r[i]);
 }

@@ -8,9 +8,12 @@
 //   dz[t,:]   = sum_{g,k} dw[t,g,k] U[:, g*W+k]      dU[:, g*W+k] = sum_t z[t,:] dw[t,g,k]
 // (g = g(c) the channel's group; x, dy zero outside [0, T)).
 //
-// Block = GB = 128/W groups = CB = GB*H channels.  A prep kernel writes each
-// block's U columns tap-major (column k*GB + g) and each z tile (136 rows) in
-// the byte order of their shared-memory images, so per tap k one MMA
+// Block = GB groups = CB = GB*H channels, GB the largest power of two with
+// NBW = W*GB <= 128 filter columns whose block divides D (128/W for W = 1, 2,
+// 4, 8 and 32 for W = 3 unless D is too narrow for that; columns NBW .. 127
+// of the filter and dw tiles stay unused).  A prep kernel
+// writes each block's U columns tap-major (column k*GB + g) and each z tile
+// (136 rows) in the byte order of their shared-memory images, so per tap k one MMA
 // z[t0+k .. t0+k+127] . U_block[:, k-th GB columns] puts w[t+k, g, k] -- the
 // filter dx of token t needs -- on TMEM lane t: the shift by k tokens is only
 // a start address in the z image.  Work item = (tile of 128 tokens, block).
@@ -18,7 +21,7 @@
 //   W * RP/16 MMAs  filters into one of two TMEM buffers (128 columns);
 //   epilogue        per sub-tile of SB channels: dx (staged, TMA store) and dw
 //                   (bf16, tap-major, into a [128 x 128] shared tile);
-//   2 * 8 MMAs      dz[tile] += dw . U_block^T   (TMEM, over the CTA's blocks),
+//   NBW/16 + 8 MMAs dz[tile] += dw . U_block^T   (TMEM, over the CTA's blocks),
 //                   dU[block] += dw^T . z         (TMEM, over the CTA's tiles).
 // CTA = (range of tiles) x (group of CPC blocks), or for long items with one
 // block per CTA an equal range of (tile, sub-tile) units.  dz leaves TMEM after
@@ -58,7 +61,7 @@ constexpr int TB_EPI = 512;              // epilogue threads
 constexpr int TB_THREADS = TB_EPI + 128;  // + x/dy producer, filter-MMA, operand/dU-MMA and dz-MMA warps
 constexpr int TB_MAXNS = 8;              // most sub-tiles in flight
 constexpr int TB_SMEM = 220 * 1024;
-constexpr int TB_NB = 128;               // filter columns per block (W * GB)
+constexpr int TB_NB = 128;               // columns of a filter buffer and a dw tile (W * GB of them in use)
 constexpr int TB_ZROWS = 136;            // z rows per tile: 128 + up to 7 for the shifted filters
 constexpr uint32_t TB_ZR = TB_ZROWS * 16;  // bytes per 8-wide k-chunk of the z tile
 constexpr int TB_MAXOP = 4;              // most operand (z, U) buffers
@@ -475,7 +478,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                 tc::fence_after_sync();
                 const uint32_t ub = sbase + (uint32_t)fob * S.opsize + S.zbytes;
                 const uint32_t dwb = sbase + S.dw + (uint32_t)fdb * S.dwsize;
-                for (int ks = 0; ks < TB_NB / 16; ++ks) {
+                for (int ks = 0; ks < m.NBW / 16; ++ks) {  // dw columns NBW .. 127 are never written
                     const uint64_t ad = tc::smem_desc(dwb + (uint32_t)ks * 256u, 128, (TB_NB / 8) * 128);
                     const uint64_t bd = tc::smem_desc(ub + (uint32_t)(ks * 2 * m.RP * 16), (uint32_t)(m.RP * 16), 128);
                     tc::mma_bf16(tmem + col_dz + (uint32_t)(tp * m.RP), ad, bd, id_dz, (fcl > 0 || ks > 0) ? 1u : 0u);
@@ -582,11 +585,12 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         }
         dz_out(ntl - 1, pb, pt0);
         // dU of the CTA's blocks over its tile range: TMEM lane = block column k*GB + g
+        // (lanes NBW .. 127 hold no filter column)
         wait(bars.duf(), 0);
         tc::fence_after_sync();
         const int k = t_loc / m.GB, gl = t_loc % m.GB;
         for (int cl = 0; cl < ncl; ++cl) {
-            const int64_t col = (int64_t)(chunk_lo + cl) * TB_NB + gl * W + k;
+            const int64_t col = (int64_t)(chunk_lo + cl) * m.NBW + gl * W + k;
             for (int r8 = 8 * part; r8 < m.RP; r8 += 32) {  // 8-column chunks, dealt round the parts
                 float v[8];
                 tmem_ld<8>(tlane + col_dU + (uint32_t)(cl * m.RP + r8), v);
@@ -594,7 +598,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const int r = r8 + j;
-                    if (r < m.R) {
+                    if (r < m.R && k < W) {
                         if (m.nRanges == 1) a.dU[(int64_t)r * m.GW + col] = v[j];
                         else a.dU_part[((int64_t)range * m.R + r) * m.GW + col] = v[j];
                     }
@@ -616,7 +620,8 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 
 // Operand images the backward loads with one bulk copy each:
 //   U image of block blk: element (j, r) at (j/8)*(RP*8) + r*8 + j%8, column
-//     j = k*GB + g holding U[r][(blk*GB + g)*W + k] (tap-major), rows r >= R zero;
+//     j = k*GB + g holding U[r][(blk*GB + g)*W + k] (tap-major), rows r >= R and
+//     columns j >= NBW zero;
 //   z image of tile i (sequence b, first token t0): element (t, r) at
 //     (r/8)*(136*8) + t*8 + r%8 holding z[b][t0+t][r], zero for r >= R or t0+t >= T.
 __global__ void k_bwd_prep(const TcArgs a) {
@@ -633,7 +638,7 @@ __global__ void k_bwd_prep(const TcArgs a) {
             const int rem = (int)(i % ublk);
             const int jc = rem / (m.RP * 8), r = (rem % (m.RP * 8)) / 8, e = rem % 8;
             const int j = jc * 8 + e, k = j / m.GB, g = j % m.GB;
-            a.Up[i] = r < m.R ? a.U[(int64_t)r * m.GW + (blk * m.GB + g) * m.W + k] : __float2bfloat16_rn(0.f);
+            a.Up[i] = (r < m.R && k < m.W) ? a.U[(int64_t)r * m.GW + (blk * m.GB + g) * m.W + k] : __float2bfloat16_rn(0.f);
         } else {
             const int64_t i2 = i - nU;
             const int64_t tile = i2 / ztile;
@@ -671,23 +676,16 @@ __global__ void k_tc_finalize(const TcArgs a) {
     }
 }
 
-// Backward plan.  Blocks of GB = 128/W groups; TMEM holds two filter buffers
-// (2 x 128 columns), two dz accumulators (2 x RP) and one dU accumulator per
-// block of the CTA (RP each).  Among the block-group sizes that fit, take the
-// one with the fewest items on the busiest SM, then the least partial-sum
-// traffic (dU partials of the token ranges, dz contributions of the block
-// groups).  Shared memory: operand buffers (3 when items are short), dw tiles
-// (2 when items are short), the exchange buffer, and as deep a sub-tile ring
-// as fits.
-bool tc_bwd_plan(TcMap &m, int sms) {
-    m.GB = TB_NB / m.W;
-    m.CB = (int)(m.GB * m.H);
-    if (m.D % m.CB) return false;
-    m.SB = m.CB < 64 ? m.CB : 64;
-    if (m.SB < 32) return false;
+// CTA split and shared-memory layout for a chosen sub-tile width m.SB.  TMEM
+// holds two filter buffers (2 x 128 columns), two dz accumulators (2 x RP) and
+// one dU accumulator per block of the CTA (RP each).  Among the block-group
+// sizes that fit, take the one with the fewest items on the busiest SM, then
+// the least partial-sum traffic (dU partials of the token ranges, dz
+// contributions of the block groups).  Shared memory: operand buffers (up to
+// 4 when items are short), dw tiles (2 when items are short and they fit),
+// the exchange buffer, and as deep a sub-tile ring as fits.
+static bool bwd_layout(TcMap &m, int sms) {
     m.nSubB = m.CB / m.SB;
-    m.nBlkB = (int)(m.D / m.CB);
-    m.totalTiles = m.B * (int64_t)m.tilesPerSeq;
     const int cpc_max = (512 - 2 * TB_NB - 2 * m.RP) / m.RP;
     if (cpc_max < 1) return false;
     double best_work = -1, best_cost = 0;
@@ -727,13 +725,31 @@ bool tc_bwd_plan(TcMap &m, int sms) {
     const int vpt = m.SB / 32, ct = 8 * vpt;
     const bool xchg = m.H > ct;
     const bool short_items = m.nSubB < 4;
-    const int dwb = short_items ? 2 : 1;
-    m.DWB = dwb;
-    for (int nop = short_items ? TB_MAXOP : 2; nop >= 2; --nop)
-        for (m.NSB = TB_MAXNS; m.NSB >= (nop > 2 ? 4 : 2); --m.NSB) {
-            m.NOP = nop;
-            if (BwdSmem(m, nop, m.NSB, dwb, xchg).total <= TB_SMEM) return true;
-        }
+    // short items: two dw tiles when they fit, else one
+    for (m.DWB = short_items ? 2 : 1; m.DWB >= 1; --m.DWB)
+        for (int nop = short_items ? TB_MAXOP : 2; nop >= 2; --nop)
+            for (m.NSB = TB_MAXNS; m.NSB >= (nop > 2 ? 4 : 2); --m.NSB) {
+                m.NOP = nop;
+                if (BwdSmem(m, nop, m.NSB, m.DWB, xchg).total <= TB_SMEM) return true;
+            }
+    return false;
+}
+
+// Backward plan: blocks of GB groups, the largest power of two with W*GB <= 128
+// whose CB = GB*H channels divide D (GB >= 16: the filter MMAs are GB wide).
+bool tc_bwd_plan(TcMap &m, int sms) {
+    m.totalTiles = m.B * (int64_t)m.tilesPerSeq;
+    for (m.GB = TB_NB; m.GB * m.W > TB_NB;) m.GB /= 2;
+    for (; m.GB >= 16; m.GB /= 2) {
+        m.NBW = m.GB * m.W;
+        m.CB = (int)(m.GB * m.H);
+        if (m.D % m.CB) continue;
+        m.nBlkB = (int)(m.D / m.CB);
+        // sub-tiles of 64 channels, or of 32 where the wider ring does not fit
+        // (a group never spans two sub-tiles)
+        for (m.SB = m.CB < 64 ? m.CB : 64; m.SB >= 32 && m.SB >= m.H; m.SB /= 2)
+            if (bwd_layout(m, sms)) return true;
+    }
     return false;
 }
 
@@ -849,6 +865,7 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     switch (a.m.W) {
     case 1: e = bwd_by_vpt<1>(c, a); break;
     case 2: e = bwd_by_vpt<2>(c, a); break;
+    case 3: e = bwd_by_vpt<3>(c, a); break;
     case 4: e = bwd_by_vpt<4>(c, a); break;
     case 8: e = bwd_by_vpt<8>(c, a); break;
     }

@@ -9,7 +9,7 @@
 //
 // Item = (tile of 128 tokens, block of CF channels); the block's filters are
 // NF = CF/H*W TMEM columns (NF <= 256) formed by one zU MMA.  TMEM holds two
-// such buffers, so the MMA of item i+1 runs while item i's outputs are formed.
+// such buffers (NFS columns apart, NF rounded up to a power of two), so the MMA of item i+1 runs while item i's outputs are formed.
 // A CTA takes a contiguous range of (item, sub-tile) pairs, so every CTA gets
 // the same number of sub-tiles; an item split between two CTAs has its MMA
 // issued by both.  Warp roles (576 threads):
@@ -71,7 +71,7 @@ namespace lrtc {
 bool tc_map(const dsc_problem &p, TcMap &m) {
     if (p.dtype != DSC_BF16) return false;
     if (p.R < 8 || p.R > 64 || p.R % 8) return false;  // 16-byte z rows
-    if (!(p.W == 1 || p.W == 2 || p.W == 4 || p.W == 8)) return false;
+    if (!(p.W == 1 || p.W == 2 || p.W == 3 || p.W == 4 || p.W == 8)) return false;
     if (p.H > 64 || (64 % p.H) != 0) return false;
     if (p.D % (TC_GROUPS * p.H)) return false;
     m = TcMap{};
@@ -323,7 +323,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
             make_uint4(0, 0, 0, 0);
     }
     tc::fence_proxy_async();
-    if (warp == 17) tc::tmem_alloc(sbase + S.tmem, (uint32_t)(2 * m.NF));
+    if (warp == 17) tc::tmem_alloc(sbase + S.tmem, (uint32_t)(2 * m.NFS));
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
@@ -405,7 +405,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
                 for (int ks = 0; ks < m.RP / 16; ++ks) {
                     const uint64_t ad = tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
                     const uint64_t bd = tc::smem_desc(ub + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
-                    tc::mma_bf16(tmem + (uint32_t)(b * m.NF), ad, bd, id_w, ks > 0 ? 1u : 0u);
+                    tc::mma_bf16(tmem + (uint32_t)(b * m.NFS), ad, bd, id_w, ks > 0 ? 1u : 0u);
                 }
                 tc::mma_commit(bars.wf(b));
                 tc::mma_commit(bars.ope(ob));
@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
             const int b = li & 1;
             wait(bars.wf(b), (uint32_t)((li >> 1) & 1));
             tc::fence_after_sync();
-            const uint32_t tb = tlane + (uint32_t)(b * m.NF);
+            const uint32_t tb = tlane + (uint32_t)(b * m.NFS);
             const int se = li == nI - 1 ? s_last : m.nSubF;
             for (int s = li == 0 ? s_first : 0; s < se; ++s) {
                 wait(bars.xf(slot), xph);
@@ -481,19 +481,21 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    if (warp == 17) tc::tmem_dealloc(tmem, (uint32_t)(2 * m.NF));
+    if (warp == 17) tc::tmem_dealloc(tmem, (uint32_t)(2 * m.NFS));
 }
 
 // Forward plan: the widest channel block whose filters fit half of TMEM
-// (NF <= 256 columns), narrowed while it still spans 8 or more sub-tiles of
-// 128 channels; sub-tiles of up to 64 channels (128-byte rows, one TMA box);
-// as many x sub-tiles in flight as shared memory holds (2 .. 8).
+// (NF <= 256 columns; a buffer takes NFS = NF rounded up to a power of two),
+// narrowed while it still spans 8 or more sub-tiles of 128 channels;
+// sub-tiles of up to 64 channels (128-byte rows, one TMA box); as many x
+// sub-tiles in flight as shared memory holds (2 .. 8).
 bool tc_fwd_plan(TcMap &m) {
     int mm = 1;
     while (TC_GROUPS * 2 * mm * m.W <= 256 && m.D % (TC_GROUPS * m.H * 2 * mm) == 0) mm *= 2;
     while (mm > 1 && (TC_GROUPS * m.H * mm / 2) / 128 >= 8) mm /= 2;
     m.CF = (int)(TC_GROUPS * m.H * mm);
     m.NF = TC_GROUPS * mm * m.W;
+    for (m.NFS = 32; m.NFS < m.NF;) m.NFS *= 2;  // TMEM is allocated in powers of two
     m.SF = m.CF < 64 ? m.CF : 64;
     m.nSubF = m.CF / m.SF;
     m.nBlkF = (int)(m.D / m.CF);
@@ -542,7 +544,7 @@ cudaError_t launch_fwd(const Ctx &c, const TcArgs &a) {
     const int64_t per = (total + c.sms - 1) / c.sms;
     const int64_t grid = (total + per - 1) / per;
     // More than half of TMEM per CTA: enough shared memory that no second CTA shares the SM.
-    const uint32_t smem = 2 * a.m.NF > 256 && S.total < 120 * 1024 ? 120 * 1024 : S.total;
+    const uint32_t smem = 2 * a.m.NFS > 256 && S.total < 120 * 1024 ? 120 * 1024 : S.total;
     const cudaError_t e =
         launch_pdl(k_lr_tc_fwd<W, GPV, VPT, NGT>, dim3((unsigned)grid), dim3(TF_THREADS), smem, c.stream, f.x, f.z, f.u, f.y, a);
     return e != cudaSuccess ? e : cudaGetLastError();
@@ -601,6 +603,7 @@ cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     switch (a.m.W) {
     case 1: return lrtc::fwd_by_gpv<1>(c, a);
     case 2: return lrtc::fwd_by_gpv<2>(c, a);
+    case 3: return lrtc::fwd_by_gpv<3>(c, a);
     case 4: return lrtc::fwd_by_gpv<4>(c, a);
     case 8: return lrtc::fwd_by_gpv<8>(c, a);
     }

@@ -107,3 +107,33 @@ def test_binding_rejects_cpu_tensors():
     w = torch.zeros(1, 4, 8, 4, dtype=torch.bfloat16)
     with pytest.raises(ValueError):
         ops.dsc_fwd_headwise(x, w)
+
+
+# (B, T, D, W, H, R) -> kernel family of the bf16 forward and backward
+# (0 tensor cores, 1 fused on CUDA cores); the plan runs on the host.
+KERNEL_CHOICE = [
+    ((8, 2048, 6144, 4, 1, 32), 0, 0),      # Q/K/V low-rank workload
+    ((4, 4096, 8192, 4, 64, 64), 0, 0),     # all-linear low-rank workload
+    ((1, 16384, 4096, 3, 1, 16), 0, 0),     # W = 3: 32-group blocks, 96 filter columns
+    ((1, 16384, 4096, 3, 1, 64), 0, 0),
+    ((2, 500, 4096, 3, 64, 64), 0, 0),
+    ((1, 200, 2048, 2, 64, 32), 0, 0),      # block narrowed to 32 groups so that it divides D
+    ((1, 16384, 4096, 2, 1, 64), 0, 0),     # backward with one dw tile
+    ((1, 16384, 4096, 8, 1, 16), 0, 1),     # W = 8, H = 1: 16-channel blocks, CUDA-core backward
+    ((2, 100, 4096, 5, 2, 16), 1, 1),       # W = 5
+    ((2, 100, 4096, 4, 1, 5), 1, 1),        # R not a multiple of 8
+    ((2, 100, 4096, 4, 1, 72), 1, 1),       # R above 64
+]
+
+
+@pytest.mark.parametrize("shape,fwd,bwd", KERNEL_CHOICE, ids=lambda v: str(v))
+def test_lowrank_kernel_choice(shape, fwd, bwd):
+    L = _lib.lib()
+    p = P(*shape, dtype=1)
+    assert L.dsc_lowrank_kernels(C.byref(p), 0) == fwd
+    assert L.dsc_lowrank_kernels(C.byref(p), 1) == bwd
+    p32 = P(*shape, dtype=0)
+    assert L.dsc_lowrank_kernels(C.byref(p32), 0) == 1
+    assert L.dsc_lowrank_kernels(C.byref(p32), 1) == 1
+    bad = P(*shape[:5], R=0)
+    assert L.dsc_lowrank_kernels(C.byref(bad), 0) == -1

@@ -149,7 +149,7 @@ LOWRANK_SHAPES = [
     (1, 40, 48, 8, 1, 3),
     (2, 3, 64, 4, 8, 1),
     (1, 70, 40, 5, 5, 7),
-    # shapes the tensor-core kernels take in bf16 (W in {1,2,4,8}, H | 64, D % 32H == 0)
+    # shapes the tensor-core kernels take in bf16 (W in {1,2,3,4,8}, H | 64, D % 32H == 0)
     (2, 300, 256, 4, 8, 16),
     (1, 200, 2048, 2, 64, 32),
     (2, 129, 64, 8, 2, 48),
@@ -165,13 +165,33 @@ LOWRANK_SHAPES = [
     (2, 700, 2048, 8, 2, 48),
     (2, 600, 1024, 8, 1, 16),
     (2, 500, 4096, 2, 1, 32),
+    # W = 3 (blocks of 32 groups: 96 of the 128 filter columns in use)
+    (2, 300, 256, 3, 8, 16),
+    (1, 200, 2048, 3, 1, 32),
+    (2, 700, 2048, 3, 2, 48),
+    (2, 500, 4096, 3, 64, 64),
+    (1, 130, 512, 3, 16, 8),
+    # W = 2, R = 64, H = 1: the backward plan that falls back to one dw tile
+    (2, 600, 1024, 2, 1, 64),
 ]
+
+
+LOWRANK_TC = LOWRANK_SHAPES[7:]  # the shapes from the tensor-core comment on
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("shape", LOWRANK_SHAPES, ids=lambda s: "B{}T{}D{}W{}H{}R{}".format(*s))
 def test_lowrank_small(shape, dtype):
     B, T, D, W, H, R = shape
+    if dtype == "bf16" and shape in LOWRANK_TC and R % 8 == 0:
+        # these run on the tensor-core kernels (the W = 8, H = 1 backward on CUDA cores)
+        import ctypes as C
+
+        from input_dependent_short_b200 import _lib
+
+        p = _lib.DscProblem(B, T, D, W, H, R, 1, 1)
+        assert _lib.lib().dsc_lowrank_kernels(C.byref(p), 0) == 0
+        assert _lib.lib().dsc_lowrank_kernels(C.byref(p), 1) == (1 if (W, H) == (8, 1) else 0)
     check_full(W_("lr", LOWRANK, B, T, D, W, H, R, dtype=dtype))
 
 
@@ -342,7 +362,8 @@ def test_full_size_workloads_sampled(name):
 
 SWEEP = [w for w in wls.sweep_workloads() if (w.variant, w.W, w.H, w.R) in {
     (HEADWISE, 2, 1, 0), (HEADWISE, 3, 16, 0), (HEADWISE, 8, 128, 0), (HEADWISE, 4, 128, 0),
-    (LOWRANK, 3, 1, 16), (LOWRANK, 8, 1, 64), (STATIC, 3, 1, 0), (STATIC, 8, 1, 0)}]
+    (LOWRANK, 3, 1, 16), (LOWRANK, 3, 1, 64), (LOWRANK, 2, 1, 64), (LOWRANK, 8, 1, 64), (STATIC, 3, 1, 0),
+    (STATIC, 8, 1, 0)}]
 
 
 @pytest.mark.parametrize("wl", SWEEP, ids=lambda w: w.name.replace(" ", "-"))
