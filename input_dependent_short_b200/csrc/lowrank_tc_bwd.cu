@@ -19,7 +19,7 @@
 // a start address in the z image.  Work item = (tile of 128 tokens, block).
 // Per item:
 //   W * RP/16 MMAs  filters into one of two TMEM buffers (128 columns);
-//   epilogue        per sub-tile of SB channels: dx (staged, TMA store) and dw
+//   epilogue        per sub-tile of SB = 16, 32 or 64 channels: dx (staged, TMA store) and dw
 //                   (bf16, tap-major, into a [128 x 128] shared tile);
 //   NBW/16 + 8 MMAs dz[tile] += dw . U_block^T   (TMEM, over the CTA's blocks),
 //                   dU[block] += dw^T . z         (TMEM, over the CTA's tiles).
@@ -32,8 +32,9 @@
 // Warp roles (640 threads): warp 16 x/dy TMA producer, warp 17 TMEM owner and
 // filter-MMA issuer, warp 18 operand loads and dU MMAs, warp 19 dz MMAs, warps
 // 0-15 epilogue (thread part p of token t: VPT 8-channel vectors of each
-// sub-tile).  Groups wider than a part's channels (PPG parts per group) add
-// their dw partial sums through a small exchange buffer.
+// sub-tile, or 4 channels of a 16-channel sub-tile).  Groups wider than a
+// part's channels (PPG parts per group) add their dw partial sums through a
+// small exchange buffer.
 #include "lowrank_tc.cuh"
 
 namespace dsc {
@@ -70,7 +71,7 @@ constexpr int TB_NBARS = 2 * TB_MAXOP + 13 + 2 * TB_MAXNS;
 struct BwdSmem {
     uint32_t zbytes, ubytes, opsize, dw, dwsize, xch, ystage, ybox, ring, boxb, slot, bars, tmem, total;
     __host__ __device__ BwdSmem(const TcMap &m, int nop, int ns, int dwb, bool xchg) {
-        const int rb = m.SB == 32 ? 64 : 128;
+        const int rb = 2 * m.SB;  // box row bytes
         boxb = up1024((uint32_t)(rb * (TC_M + m.W - 1)));
         slot = 2 * boxb;  // x box + dy box
         ybox = (uint32_t)(rb * TC_M);
@@ -269,12 +270,66 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
     }
 }
 
+// The same for sub-tiles of 16 channels (blocks of 16 groups, H = 1): the
+// thread's 4 channels are the 8 bytes at `off` in 16-byte chunk `chunk` of
+// each 32-byte row; channel i of the thread is its group g0 + i.
+template <int W>
+__device__ __forceinline__ void bwd_subtile_q(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
+                                              unsigned char *dwt, int part, int t_loc, int s, unsigned char *ys,
+                                              float res, uint32_t release_w) {
+    constexpr int WIN = W - 1;
+    const int g0 = s * m.SB + part * 4;  // block group = block channel of the thread's first channel
+    const int chunk = part >> 1;
+    const uint32_t off = (uint32_t)(part & 1) * 8u;
+    float wt[W][4];
+#pragma unroll
+    for (int k = 0; k < W; ++k) tmem_ld<4>(tb + (uint32_t)(k * m.GB + g0), wt[k]);
+    const unsigned char *xb = xs;         // x rows t0-WIN .. t0+127
+    const unsigned char *yb = xs + boxb;  // dy rows t0 .. t0+127+WIN
+    uint2 dyv[W];
+#pragma unroll
+    for (int k = 0; k < W; ++k) dyv[k] = *reinterpret_cast<const uint2 *>(yb + tc::swz<32>(t_loc + k, chunk) + off);
+    tc::tmem_wait_ld();
+    if (release_w) {  // the item's last filter read: its TMEM buffer is free for the next MMA
+        tc::fence_before_sync();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) tc::mbar_arrive(release_w);
+    }
+#pragma unroll
+    for (int g = 0; g < 4; ++g) wt[0][g] += res;
+    // dx
+    uint32_t dxw[2];
+#pragma unroll
+    for (int pp = 0; pp < 2; ++pp) {
+        u64 acc2 = 0ull;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            const uint32_t word = pp ? dyv[k].y : dyv[k].x;
+            const u64 wp = mk2(wt[k][2 * pp], wt[k][2 * pp + 1]), dp = mk2(bf_lo(word), bf_hi(word));
+            acc2 = k == 0 ? mul2(wp, dp) : fma2(wp, dp, acc2);
+        }
+        dxw[pp] = pack_bf2(lo2(acc2), hi2(acc2));
+    }
+    *reinterpret_cast<uint2 *>(ys + tc::swz<32>(t_loc, chunk) + off) = make_uint2(dxw[0], dxw[1]);
+    // dw[t, g0+i, k] = dy[t, c] x[t-k, c] (one channel per group)
+#pragma unroll
+    for (int k = 0; k < W; ++k) {
+        const uint2 xv = *reinterpret_cast<const uint2 *>(xb + tc::swz<32>(t_loc + WIN - k, chunk) + off);
+        float pk[4];
+        pk[0] = fma_bf16_lo(dyv[0].x, xv.x, 0.f);
+        pk[1] = fma_bf16_hi(dyv[0].x, xv.x, 0.f);
+        pk[2] = fma_bf16_lo(dyv[0].y, xv.y, 0.f);
+        pk[3] = fma_bf16_hi(dyv[0].y, xv.y, 0.f);
+        st_dw<4>(dwt + tc::core_off(t_loc, k * m.GB + g0, TB_NB), pk);
+    }
+}
+
 template <int W, int VPT, int GPT, int PPG>
 __global__ void __launch_bounds__(TB_THREADS, 1)
     k_lr_tc_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmdy,
                 const __grid_constant__ CUtensorMap tmdx, const TcArgs a) {
     constexpr int WIN = W - 1;
-    constexpr int RB = VPT == 1 ? 64 : 128;  // box row bytes (32 or 64 channels)
+    constexpr int RB = VPT == 0 ? 32 : (VPT == 1 ? 64 : 128);  // box row bytes (16, 32 or 64 channels)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const TcMap &m = a.m;
     const int NS = m.NSB, NOP = m.NOP, DWB = m.DWB;
@@ -548,9 +603,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             }
             for (int s = sb; s < se; ++s) {
                 wait(bars.xf(slot), xph);
-                bwd_subtile<W, VPT, GPT, PPG, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, xch, part,
-                                                  t_loc, s, smem + S.ystage + (uint32_t)ybuf * S.ybox, res,
-                                                  s == se - 1 ? bars.we(b) : 0u);
+                if constexpr (VPT == 0)
+                    bwd_subtile_q<W>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, part, t_loc, s,
+                                     smem + S.ystage + (uint32_t)ybuf * S.ybox, res, s == se - 1 ? bars.we(b) : 0u);
+                else
+                    bwd_subtile<W, VPT, GPT, PPG, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, xch,
+                                                      part, t_loc, s, smem + S.ystage + (uint32_t)ybuf * S.ybox, res,
+                                                      s == se - 1 ? bars.we(b) : 0u);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars.xe(slot));
                 // dx tile -> global by TMA (the staging tile the next sub-tile writes was read
@@ -722,7 +781,7 @@ static bool bwd_layout(TcMap &m, int sms) {
         }
     }
     m.dzAcc = (m.nGroups > 1 || m.splitUnits > 0) ? 1 : 0;
-    const int vpt = m.SB / 32, ct = 8 * vpt;
+    const int ct = m.SB / 4;  // a thread's channels per sub-tile
     const bool xchg = m.H > ct;
     const bool short_items = m.nSubB < 4;
     // short items: two dw tiles when they fit, else one
@@ -746,7 +805,13 @@ bool tc_bwd_plan(TcMap &m, int sms) {
         if (m.D % m.CB) continue;
         m.nBlkB = (int)(m.D / m.CB);
         // sub-tiles of 64 channels, or of 32 where the wider ring does not fit
-        // (a group never spans two sub-tiles)
+        // (a group never spans two sub-tiles); 16 for blocks of 16 channels
+        // (W = 8, H = 1)
+        if (m.CB == 16) {
+            m.SB = 16;
+            if (m.W == 8 && m.H == 1 && bwd_layout(m, sms)) return true;
+            continue;
+        }
         for (m.SB = m.CB < 64 ? m.CB : 64; m.SB >= 32 && m.SB >= m.H; m.SB /= 2)
             if (bwd_layout(m, sms)) return true;
     }
@@ -769,12 +834,13 @@ struct BwdMaps {
 
 bool bwd_maps(const TcArgs &a, BwdMaps &f) {
     const TcMap &m = a.m;
-    const int rb = m.SB == 32 ? 64 : 128;
+    const int rb = 2 * m.SB;
     const uint64_t xd[3] = {(uint64_t)m.D, (uint64_t)m.T, (uint64_t)m.B};
     const uint64_t xs[2] = {(uint64_t)m.D * 2, (uint64_t)(m.T * m.D * 2)};
     const uint32_t xb[3] = {(uint32_t)(rb / 2), (uint32_t)(TC_M + m.W - 1), 1};
     const uint32_t yb[3] = {(uint32_t)(rb / 2), (uint32_t)TC_M, 1};
-    const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+    const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                  : (rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
     return make_map(&f.x, a.x, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
            make_map(&f.dy, a.dy, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
            make_map(&f.dx, a.dx, 3, xd, xs, yb, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE);
@@ -812,6 +878,10 @@ template <int W, int VPT> cudaError_t bwd_by_h(const Ctx &c, const TcArgs &a) {
 }
 
 template <int W> cudaError_t bwd_by_vpt(const Ctx &c, const TcArgs &a) {
+    if (a.m.SB == 16) {  // blocks of 16 single-channel groups (W = 8, H = 1)
+        if constexpr (W == 8) return launch_bwd<W, 0, 4, 1>(c, a);
+        return cudaErrorNotSupported;
+    }
     return a.m.SB == 32 ? bwd_by_h<W, 1>(c, a) : bwd_by_h<W, 2>(c, a);
 }
 

@@ -204,11 +204,11 @@ __device__ __forceinline__ void tma_prefetch_desc(const void *tmap) {
 }
 
 // Byte offset of the 16-byte chunk `chunk` of row `row` in a tile that a TMA
-// load wrote with 64- or 128-byte swizzling (rows of RB = 64 or 128 bytes,
-// tile base aligned to 1024 bytes): address bits [4, 4+b) are XORed with bits
-// [7, 7+b), b = log2(RB / 16).
+// load wrote with 32-, 64- or 128-byte swizzling (rows of RB = 32, 64 or 128
+// bytes, tile base aligned to 1024 bytes): address bits [4, 4+b) are XORed
+// with bits [7, 7+b), b = log2(RB / 16).
 template <int RB> __device__ __forceinline__ uint32_t swz(int row, int chunk) {
-    static_assert(RB == 64 || RB == 128, "64- or 128-byte rows");
+    static_assert(RB == 32 || RB == 64 || RB == 128, "32-, 64- or 128-byte rows");
     const uint32_t off = (uint32_t)row * RB;
     return off + ((((uint32_t)chunk) ^ ((off >> 7) & (RB / 16 - 1))) << 4);
 }

@@ -119,7 +119,8 @@ KERNEL_CHOICE = [
     ((2, 500, 4096, 3, 64, 64), 0, 0),
     ((1, 200, 2048, 2, 64, 32), 0, 0),      # block narrowed to 32 groups so that it divides D
     ((1, 16384, 4096, 2, 1, 64), 0, 0),     # backward with one dw tile
-    ((1, 16384, 4096, 8, 1, 16), 0, 1),     # W = 8, H = 1: 16-channel blocks, CUDA-core backward
+    ((1, 16384, 4096, 8, 1, 16), 0, 0),     # W = 8, H = 1: 16-channel blocks and sub-tiles
+    ((1, 16384, 4096, 8, 1, 64), 0, 0),
     ((2, 100, 4096, 5, 2, 16), 1, 1),       # W = 5
     ((2, 100, 4096, 4, 1, 5), 1, 1),        # R not a multiple of 8
     ((2, 100, 4096, 4, 1, 72), 1, 1),       # R above 64

@@ -173,6 +173,9 @@ LOWRANK_SHAPES = [
     (1, 130, 512, 3, 16, 8),
     # W = 2, R = 64, H = 1: the backward plan that falls back to one dw tile
     (2, 600, 1024, 2, 1, 64),
+    # W = 8, H = 1: blocks of 16 channels, sub-tiles of 16 (4 channels a thread)
+    (2, 300, 512, 8, 1, 64),
+    (1, 200, 2048, 8, 1, 8),
 ]
 
 
@@ -184,14 +187,14 @@ LOWRANK_TC = LOWRANK_SHAPES[7:]  # the shapes from the tensor-core comment on
 def test_lowrank_small(shape, dtype):
     B, T, D, W, H, R = shape
     if dtype == "bf16" and shape in LOWRANK_TC and R % 8 == 0:
-        # these run on the tensor-core kernels (the W = 8, H = 1 backward on CUDA cores)
+        # these run on the tensor-core kernels
         import ctypes as C
 
         from input_dependent_short_b200 import _lib
 
         p = _lib.DscProblem(B, T, D, W, H, R, 1, 1)
         assert _lib.lib().dsc_lowrank_kernels(C.byref(p), 0) == 0
-        assert _lib.lib().dsc_lowrank_kernels(C.byref(p), 1) == (1 if (W, H) == (8, 1) else 0)
+        assert _lib.lib().dsc_lowrank_kernels(C.byref(p), 1) == 0
     check_full(W_("lr", LOWRANK, B, T, D, W, H, R, dtype=dtype))
 
 
