@@ -100,9 +100,9 @@ DSC_API size_t dsc_bwd_lowrank_workspace_bytes(const dsc_problem *p);
  * use (on the current device's SM count; 148 without a device).  Launches
  * nothing and touches no device memory.  Returns one of:
  *   DSC_LR_TENSOR_CORE  fused, the filter contractions on tcgen05 tensor cores
- *                       (bf16; R a multiple of 8 up to 64, W in {1,2,3,4,8},
- *                       H a divisor of 64, D a multiple of 32*H, and a plan
- *                       that fits the shared memory and tensor memory);
+ *                       (bf16; R a multiple of 8 up to 64, H a divisor of
+ *                       64, D a multiple of 32*H, and a plan that fits the
+ *                       shared memory and tensor memory);
  *   DSC_LR_FUSED        fused, contractions on CUDA cores (fp32, other shapes);
  *   DSC_LR_UNFUSED      filters and their gradient in the caller's workspace;
  * or -1 when the problem is invalid. */

@@ -8,8 +8,8 @@
 // training implementation" (the fused kernels form zU on chip and convolve at
 // once; the filter tensor never reaches HBM).
 //
-// Used for bf16 with R a multiple of 8 up to 64, W in {1, 2, 3, 4, 8}, H a
-// divisor of 64 and D a multiple of 32*H; the CUDA-core kernels cover every
+// Used for bf16 with R a multiple of 8 up to 64, H a divisor of 64 and D a
+// multiple of 32*H (any W from 1 to 8); the CUDA-core kernels cover every
 // other shape.
 #pragma once
 
@@ -97,6 +97,14 @@ __device__ __forceinline__ uint4 lds16(uint32_t a) {
 
 __device__ __forceinline__ uint32_t word_of(const uint4 &v, int i) {
     return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// Packed bf16 products a.lo*b.lo, a.hi*b.hi, each rounded once to bf16 (the
+// exact product of two bf16 values, as fp32 would hold it, rounded to nearest).
+__device__ __forceinline__ uint32_t mul_bf2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
 }
 
 // acc + a.lo*b.lo and acc + a.hi*b.hi straight from packed bf16 words

@@ -10,8 +10,8 @@
 //
 // Block = GB groups = CB = GB*H channels, GB the largest power of two with
 // NBW = W*GB <= 128 filter columns whose block divides D (128/W for W = 1, 2,
-// 4, 8 and 32 for W = 3 unless D is too narrow for that; columns NBW .. 127
-// of the filter and dw tiles stay unused).  A prep kernel
+// 4, 8, 32 for W = 3 and 16 for W = 5 .. 7, unless D is too narrow for that;
+// columns NBW .. 127 of the filter and dw tiles stay unused).  A prep kernel
 // writes each block's U columns tap-major (column k*GB + g) and each z tile
 // (136 rows) in the byte order of their shared-memory images, so per tap k one MMA
 // z[t0+k .. t0+k+127] . U_block[:, k-th GB columns] puts w[t+k, g, k] -- the
@@ -154,6 +154,60 @@ template <int N> __device__ __forceinline__ void st_dw(unsigned char *p, const f
     }
 }
 
+// dw[t, g, k] of groups of several channels: fp32 sums over the thread's
+// channels, then across the PPG parts that share a group.
+template <int W, int VPT, int GPT, int PPG, int RB>
+__device__ __forceinline__ void bwd_dw_groups(const TcMap &m, const unsigned char *xb, const uint4 (&dyv)[VPT][W],
+                                              unsigned char *dwt, float *xch, int part, int t_loc, int s, int g0) {
+    constexpr int WIN = W - 1;
+    constexpr int CT = 8 * VPT;
+    constexpr int GPV = GPT >= VPT ? GPT / VPT : 1;
+    constexpr int CPG = 8 / GPV;
+    const int cs0 = part * CT;
+    float pk[W][GPT];
+#pragma unroll
+    for (int k = 0; k < W; ++k)
+#pragma unroll
+        for (int g = 0; g < GPT; ++g) pk[k][g] = 0.f;
+#pragma unroll
+    for (int v = 0; v < VPT; ++v) {
+        const int cs = cs0 + 8 * v;
+        const int bo = (cs % (RB / 2)) / 8;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            const uint4 xv = *reinterpret_cast<const uint4 *>(xb + tc::swz<RB>(t_loc + WIN - k, bo));
+#pragma unroll
+            for (int wd = 0; wd < 4; ++wd) {
+                const uint32_t dyw = word_of(dyv[v][0], wd), xwd = word_of(xv, wd);
+                const int ga = GPT >= VPT ? v * GPV + (2 * wd) / CPG : (v * GPT) / VPT;
+                const int gb = GPT >= VPT ? v * GPV + (2 * wd + 1) / CPG : (v * GPT) / VPT;
+                pk[k][ga] = fma_bf16_lo(dyw, xwd, pk[k][ga]);
+                pk[k][gb] = fma_bf16_hi(dyw, xwd, pk[k][gb]);
+            }
+        }
+    }
+    if constexpr (PPG == 1) {
+#pragma unroll
+        for (int k = 0; k < W; ++k)
+            st_dw<GPT>(dwt + tc::core_off(t_loc, k * m.GB + g0, TB_NB), pk[k]);
+    } else {
+        // parts p0 .. p0+PPG-1 share the group; part p finishes the taps k = p (mod PPG)
+        float *mine = xch + ((s & 1) * 4 * TC_M + part * TC_M + t_loc) * W;
+#pragma unroll
+        for (int k = 0; k < W; ++k) mine[k] = pk[k][0];
+        epi_bar();
+        const int p0 = part - part % PPG;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            if (k % PPG != part % PPG) continue;
+            float tot = 0.f;
+#pragma unroll
+            for (int q = 0; q < PPG; ++q) tot += xch[((s & 1) * 4 * TC_M + (p0 + q) * TC_M + t_loc) * W + k];
+            st_dw<1>(dwt + tc::core_off(t_loc, k * m.GB + g0, TB_NB), &tot);
+        }
+    }
+}
+
 // One sub-tile of the epilogue for token t_loc, thread part `part`.
 //   VPT vectors of 8 channels; GPT groups among the thread's 8*VPT channels
 //   (1 when the group is wider: PPG parts then share it).
@@ -209,6 +263,16 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
                 }
                 dxv[2 * pp] = lo2(acc2);
                 dxv[2 * pp + 1] = hi2(acc2);
+            } else if constexpr (CPG == 1) {  // a group per channel: the two channels' filters as a pair
+                u64 acc2 = 0ull;
+#pragma unroll
+                for (int k = 0; k < W; ++k) {
+                    const uint32_t word = word_of(dyv[v][k], pp);
+                    const u64 wp = mk2(wt[k][ga], wt[k][gb]), dp = mk2(bf_lo(word), bf_hi(word));
+                    acc2 = k == 0 ? mul2(wp, dp) : fma2(wp, dp, acc2);
+                }
+                dxv[2 * pp] = lo2(acc2);
+                dxv[2 * pp + 1] = hi2(acc2);
             } else {
                 float a0 = 0.f, a1 = 0.f;
 #pragma unroll
@@ -225,48 +289,21 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
             make_uint4(pack_bf2(dxv[0], dxv[1]), pack_bf2(dxv[2], dxv[3]), pack_bf2(dxv[4], dxv[5]),
                        pack_bf2(dxv[6], dxv[7]));
     }
-    // dw[t, g, k] over the thread's channels
-    float pk[W][GPT];
+    if constexpr (GPT == CT) {
+        // one channel per group (H = 1): dw[t, g, k] = dy[t, c] x[t-k, c], rounded once to bf16
 #pragma unroll
-    for (int k = 0; k < W; ++k)
+        for (int v = 0; v < VPT; ++v) {
+            const int bo = ((cs0 + 8 * v) % (RB / 2)) / 8;
 #pragma unroll
-        for (int g = 0; g < GPT; ++g) pk[k][g] = 0.f;
-#pragma unroll
-    for (int v = 0; v < VPT; ++v) {
-        const int cs = cs0 + 8 * v;
-        const int bo = (cs % (RB / 2)) / 8;
-#pragma unroll
-        for (int k = 0; k < W; ++k) {
-            const uint4 xv = *reinterpret_cast<const uint4 *>(xb + tc::swz<RB>(t_loc + WIN - k, bo));
-#pragma unroll
-            for (int wd = 0; wd < 4; ++wd) {
-                const uint32_t dyw = word_of(dyv[v][0], wd), xwd = word_of(xv, wd);
-                const int ga = GPT >= VPT ? v * GPV + (2 * wd) / CPG : (v * GPT) / VPT;
-                const int gb = GPT >= VPT ? v * GPV + (2 * wd + 1) / CPG : (v * GPT) / VPT;
-                pk[k][ga] = fma_bf16_lo(dyw, xwd, pk[k][ga]);
-                pk[k][gb] = fma_bf16_hi(dyw, xwd, pk[k][gb]);
+            for (int k = 0; k < W; ++k) {
+                const uint4 xv = *reinterpret_cast<const uint4 *>(xb + tc::swz<RB>(t_loc + WIN - k, bo));
+                *reinterpret_cast<uint4 *>(dwt + tc::core_off(t_loc, k * m.GB + g0 + 8 * v, TB_NB)) =
+                    make_uint4(mul_bf2(dyv[v][0].x, xv.x), mul_bf2(dyv[v][0].y, xv.y), mul_bf2(dyv[v][0].z, xv.z),
+                               mul_bf2(dyv[v][0].w, xv.w));
             }
         }
-    }
-    if constexpr (PPG == 1) {
-#pragma unroll
-        for (int k = 0; k < W; ++k)
-            st_dw<GPT>(dwt + tc::core_off(t_loc, k * m.GB + g0, TB_NB), pk[k]);
     } else {
-        // parts p0 .. p0+PPG-1 share the group; part p finishes the taps k = p (mod PPG)
-        float *mine = xch + ((s & 1) * 4 * TC_M + part * TC_M + t_loc) * W;
-#pragma unroll
-        for (int k = 0; k < W; ++k) mine[k] = pk[k][0];
-        epi_bar();
-        const int p0 = part - part % PPG;
-#pragma unroll
-        for (int k = 0; k < W; ++k) {
-            if (k % PPG != part % PPG) continue;
-            float tot = 0.f;
-#pragma unroll
-            for (int q = 0; q < PPG; ++q) tot += xch[((s & 1) * 4 * TC_M + (p0 + q) * TC_M + t_loc) * W + k];
-            st_dw<1>(dwt + tc::core_off(t_loc, k * m.GB + g0, TB_NB), &tot);
-        }
+        bwd_dw_groups<W, VPT, GPT, PPG, RB>(m, xb, dyv, dwt, xch, part, t_loc, s, g0);
     }
 }
 
@@ -311,16 +348,12 @@ __device__ __forceinline__ void bwd_subtile_q(const TcMap &m, const unsigned cha
         dxw[pp] = pack_bf2(lo2(acc2), hi2(acc2));
     }
     *reinterpret_cast<uint2 *>(ys + tc::swz<32>(t_loc, chunk) + off) = make_uint2(dxw[0], dxw[1]);
-    // dw[t, g0+i, k] = dy[t, c] x[t-k, c] (one channel per group)
+    // dw[t, g0+i, k] = dy[t, c] x[t-k, c] (one channel per group), rounded once to bf16
 #pragma unroll
     for (int k = 0; k < W; ++k) {
         const uint2 xv = *reinterpret_cast<const uint2 *>(xb + tc::swz<32>(t_loc + WIN - k, chunk) + off);
-        float pk[4];
-        pk[0] = fma_bf16_lo(dyv[0].x, xv.x, 0.f);
-        pk[1] = fma_bf16_hi(dyv[0].x, xv.x, 0.f);
-        pk[2] = fma_bf16_lo(dyv[0].y, xv.y, 0.f);
-        pk[3] = fma_bf16_hi(dyv[0].y, xv.y, 0.f);
-        st_dw<4>(dwt + tc::core_off(t_loc, k * m.GB + g0, TB_NB), pk);
+        *reinterpret_cast<uint2 *>(dwt + tc::core_off(t_loc, k * m.GB + g0, TB_NB)) =
+            make_uint2(mul_bf2(dyv[0].x, xv.x), mul_bf2(dyv[0].y, xv.y));
     }
 }
 
@@ -804,15 +837,16 @@ bool tc_bwd_plan(TcMap &m, int sms) {
         m.CB = (int)(m.GB * m.H);
         if (m.D % m.CB) continue;
         m.nBlkB = (int)(m.D / m.CB);
-        // sub-tiles of 64 channels, or of 32 where the wider ring does not fit
-        // (a group never spans two sub-tiles); 16 for blocks of 16 channels
-        // (W = 8, H = 1)
+        // sub-tiles of 64 channels (32 for W >= 5, whose wider filters take more
+        // registers), or of 32 where the wider ring does not fit (a group never
+        // spans two sub-tiles); 16 for blocks of 16 channels (W >= 5, H = 1)
         if (m.CB == 16) {
             m.SB = 16;
-            if (m.W == 8 && m.H == 1 && bwd_layout(m, sms)) return true;
+            if (m.W >= 5 && m.H == 1 && bwd_layout(m, sms)) return true;
             continue;
         }
-        for (m.SB = m.CB < 64 ? m.CB : 64; m.SB >= 32 && m.SB >= m.H; m.SB /= 2)
+        const int sb_max = m.W >= 5 && m.H <= 32 ? 32 : 64;
+        for (m.SB = m.CB < sb_max ? m.CB : sb_max; m.SB >= 32 && m.SB >= m.H; m.SB /= 2)
             if (bwd_layout(m, sms)) return true;
     }
     return false;
@@ -865,6 +899,10 @@ cudaError_t launch_bwd(const Ctx &c, const TcArgs &a) {
 // Thread channels per sub-tile: CT = 8*VPT (SB = 32 or 64, four parts).
 template <int W, int VPT> cudaError_t bwd_by_h(const Ctx &c, const TcArgs &a) {
     constexpr int CT = 8 * VPT;
+    if constexpr (W >= 5 && VPT == 2) {  // the plan takes 64-channel sub-tiles for W >= 5 only when H = 64
+        if (a.m.H == 64) return launch_bwd<W, VPT, 1, 64 / CT>(c, a);
+        return cudaErrorNotSupported;
+    }
     switch (a.m.H) {
     case 1: if constexpr (CT * W <= 32) return launch_bwd<W, VPT, CT, 1>(c, a); break;
     case 2: if constexpr (CT / 2 * W <= 32) return launch_bwd<W, VPT, CT / 2, 1>(c, a); break;
@@ -878,8 +916,8 @@ template <int W, int VPT> cudaError_t bwd_by_h(const Ctx &c, const TcArgs &a) {
 }
 
 template <int W> cudaError_t bwd_by_vpt(const Ctx &c, const TcArgs &a) {
-    if (a.m.SB == 16) {  // blocks of 16 single-channel groups (W = 8, H = 1)
-        if constexpr (W == 8) return launch_bwd<W, 0, 4, 1>(c, a);
+    if (a.m.SB == 16) {  // blocks of 16 single-channel groups (W >= 5, H = 1)
+        if constexpr (W >= 5) return launch_bwd<W, 0, 4, 1>(c, a);
         return cudaErrorNotSupported;
     }
     return a.m.SB == 32 ? bwd_by_h<W, 1>(c, a) : bwd_by_h<W, 2>(c, a);
@@ -937,6 +975,9 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     case 2: e = bwd_by_vpt<2>(c, a); break;
     case 3: e = bwd_by_vpt<3>(c, a); break;
     case 4: e = bwd_by_vpt<4>(c, a); break;
+    case 5: e = bwd_by_vpt<5>(c, a); break;
+    case 6: e = bwd_by_vpt<6>(c, a); break;
+    case 7: e = bwd_by_vpt<7>(c, a); break;
     case 8: e = bwd_by_vpt<8>(c, a); break;
     }
     if (e != cudaSuccess) return e;

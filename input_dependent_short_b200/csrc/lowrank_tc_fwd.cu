@@ -71,7 +71,7 @@ namespace lrtc {
 bool tc_map(const dsc_problem &p, TcMap &m) {
     if (p.dtype != DSC_BF16) return false;
     if (p.R < 8 || p.R > 64 || p.R % 8) return false;  // 16-byte z rows
-    if (!(p.W == 1 || p.W == 2 || p.W == 3 || p.W == 4 || p.W == 8)) return false;
+    if (p.W < 1 || p.W > 8) return false;
     if (p.H > 64 || (64 % p.H) != 0) return false;
     if (p.D % (TC_GROUPS * p.H)) return false;
     m = TcMap{};
@@ -190,7 +190,7 @@ __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char 
     constexpr int WIN = W - 1;
     constexpr int NT = GPV * W;
     constexpr int CPG = 8 / GPV;
-    constexpr int VBW = W >= 8 ? 1 : (W == 4 ? 2 : 4);
+    constexpr int VBW = W > 4 ? 1 : (W > 2 ? 2 : 4);
     constexpr int VB = VBW < VPT ? VBW : VPT;  // vectors whose x rows are loaded together
     const int cs0 = part * (8 * VPT);  // sub-tile channel of the thread's first vector
     float wt[GPV == 1 ? NGT * W : 2 * NT];
@@ -605,6 +605,9 @@ cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     case 2: return lrtc::fwd_by_gpv<2>(c, a);
     case 3: return lrtc::fwd_by_gpv<3>(c, a);
     case 4: return lrtc::fwd_by_gpv<4>(c, a);
+    case 5: return lrtc::fwd_by_gpv<5>(c, a);
+    case 6: return lrtc::fwd_by_gpv<6>(c, a);
+    case 7: return lrtc::fwd_by_gpv<7>(c, a);
     case 8: return lrtc::fwd_by_gpv<8>(c, a);
     }
     return cudaErrorNotSupported;

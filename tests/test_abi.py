@@ -121,7 +121,10 @@ KERNEL_CHOICE = [
     ((1, 16384, 4096, 2, 1, 64), 0, 0),     # backward with one dw tile
     ((1, 16384, 4096, 8, 1, 16), 0, 0),     # W = 8, H = 1: 16-channel blocks and sub-tiles
     ((1, 16384, 4096, 8, 1, 64), 0, 0),
-    ((2, 100, 4096, 5, 2, 16), 1, 1),       # W = 5
+    ((2, 100, 4096, 5, 2, 16), 0, 0),       # W = 5 .. 7: 16-group blocks
+    ((2, 100, 4096, 7, 1, 32), 0, 0),
+    ((2, 100, 4096, 6, 16, 64), 0, 0),
+    ((2, 100, 4096, 6, 64, 64), 0, 1),      # W >= 5, H = 64, R = 64: the backward's tiles overflow shared memory
     ((2, 100, 4096, 4, 1, 5), 1, 1),        # R not a multiple of 8
     ((2, 100, 4096, 4, 1, 72), 1, 1),       # R above 64
 ]

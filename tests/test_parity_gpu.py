@@ -176,6 +176,12 @@ LOWRANK_SHAPES = [
     # W = 8, H = 1: blocks of 16 channels, sub-tiles of 16 (4 channels a thread)
     (2, 300, 512, 8, 1, 64),
     (1, 200, 2048, 8, 1, 8),
+    # W = 5 .. 7: blocks of 16 groups (80 .. 112 filter columns)
+    (2, 300, 512, 5, 1, 16),
+    (1, 260, 1024, 6, 2, 32),
+    (2, 140, 2048, 7, 8, 24),
+    (1, 200, 4096, 6, 64, 32),
+    (1, 150, 1024, 7, 1, 64),
 ]
 
 
