@@ -90,7 +90,8 @@ def _bind(lib):
     lib.orc_lowrank_grads.argtypes = [P, _In, _In, d, d, d]
     lib.orc_sample.argtypes = [P, C.POINTER(_Filter), _In, _In, C.c_int64, C.c_int64,
                                C.POINTER(C.c_int64), d]
-    for f in ("orc_lowrank_filters", "orc_forward", "orc_backward", "orc_lowrank_grads", "orc_sample"):
+    lib.orc_decode.argtypes = [P, C.POINTER(_Filter), _In, _In, d, d]
+    for f in ("orc_lowrank_filters", "orc_forward", "orc_backward", "orc_lowrank_grads", "orc_sample", "orc_decode"):
         getattr(lib, f).restype = None
     return lib
 
@@ -185,3 +186,17 @@ def sample(P: Problem, kind: int, what: int, idx, *, x=None, dy=None, w=None, z=
     lib.orc_sample(C.byref(P), C.byref(F), _in(x), _in(dy), what, idx.shape[0],
                    q.ctypes.data_as(C.POINTER(C.c_int64)), _dp(out))
     return out
+
+
+def decode(P: Problem, kind: int, x, state, *, w=None, z=None, U=None, ws=None, lib=None):
+    """One decode step (P.T must be 1): x [B,D], state [B,W-1,D] (row j holds
+    x_{t-W+1+j}); head-wise w [B,G,W], low-rank z [B,R] and U [R,G*W], or
+    static ws [D,W].  Returns (y [B,D], the state after the step [B,W-1,D])."""
+    if P.T != 1:
+        raise ValueError("a decode step has T = 1")
+    lib = lib or load()
+    y = _out((P.B, P.D))
+    st = _out((P.B, P.W - 1, P.D))
+    F = _Filter(kind, _in(ws if kind == STATIC else w), _in(z), _in(U))
+    lib.orc_decode(C.byref(P), C.byref(F), _in(x), _in(state), _dp(y), _dp(st))
+    return y, st

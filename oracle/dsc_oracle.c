@@ -273,3 +273,31 @@ void orc_sample(const orc_problem *P, const orc_filter *F, orc_in x, orc_in dy, 
         out[i] = v;
     }
 }
+
+/* Decode step: the definition above evaluated at the newest token t of each
+ * sequence, with its W-1 predecessors taken from a state [B, W-1, D] whose
+ * row j holds x_{t-W+1+j} (zero rows stand for positions before the
+ * sequence start).  P->T is 1: the filters of the new token are head-wise
+ * w [B,1,G,W], low-rank z [B,1,R] with U [R,G*W], or static ws [D,W].
+ *   y[b,c] = r*x[b,c] + w_0 x[b,c] + sum_{k=1}^{W-1} w_k state[b, W-1-k, c]
+ * The state after the step holds x_{t-W+2} .. x_t: rows 1 .. W-2 of the old
+ * state, then x. */
+void orc_decode(const orc_problem *P, const orc_filter *F, orc_in x, orc_in state, double *y_out,
+                double *state_out)
+{
+    const int64_t S = P->W - 1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t b = 0; b < P->B; ++b)
+        for (int64_t c = 0; c < P->D; ++c) {
+            const double xt = val(x, b * P->D + c);
+            double s = P->residual ? xt : 0.0;
+            for (int64_t k = 0; k < P->W; ++k) {
+                const double xk = k == 0 ? xt : val(state, (b * S + (S - k)) * P->D + c);
+                s += tap(P, F, b, 0, c, k) * xk;
+            }
+            y_out[b * P->D + c] = s;
+            for (int64_t j = 0; j + 1 < S; ++j)
+                state_out[(b * S + j) * P->D + c] = val(state, (b * S + j + 1) * P->D + c);
+            if (S > 0) state_out[(b * S + S - 1) * P->D + c] = xt;
+        }
+}

@@ -34,6 +34,11 @@ MUTANTS = {
                                       "for (int64_t t = k; t < P->T; ++t)\n            s += xval(P, dy, b, t, c) * xval(P, x, b, t - (k > 0), c);"),
     "static taps in reverse order": ("if (F->kind == ORC_STATIC) return val(F->w, c * P->W + k);",
                                      "if (F->kind == ORC_STATIC) return val(F->w, c * P->W + (P->W - 1 - k));"),
+    "decode reads the state rows in reverse": ("val(state, (b * S + (S - k)) * P->D + c)",
+                                               "val(state, (b * S + (k - 1)) * P->D + c)"),
+    "decode does not shift the state": ("= val(state, (b * S + j + 1) * P->D + c);",
+                                        "= val(state, (b * S + j) * P->D + c);"),
+    "decode drops the residual": ("double s = P->residual ? xt : 0.0;", "double s = 0.0;"),
 }
 
 
@@ -116,6 +121,15 @@ def _pins(lib):
     dxl, dz, dU, _ = oracle.backward_lowrank(p, x, z, U, dy, lib=lib)
     fl = lambda: np.sum(dy * oracle.forward_lowrank(p, x, z, U, lib=lib))
     check("fd-lowrank", fd(fl, z, dz) and fd(fl, U, dU) and fd(fl, x, dxl))
+
+    # decode steps from a zero state against the forward over the sequence
+    pd = oracle.problem(B, 1, D, W, H, 0, 1)
+    state, ok = np.zeros((B, W - 1, D)), True
+    for t in range(T):
+        yt, state = oracle.decode(pd, oracle.HEADWISE, np.ascontiguousarray(x[:, t]), state,
+                                  w=np.ascontiguousarray(w[:, t]), lib=lib)
+        ok &= np.allclose(yt, y[:, t], atol=1e-12)
+    check("decode", ok and np.array_equal(state[:, -1], x[:, -1]))
     return fails
 
 

@@ -328,3 +328,61 @@ def test_sample_matches_full():
     _, dws = oracle.backward_static(p, x, ws, dy)
     pc = np.array([(c, k) for c in range(D) for k in range(W)])
     np.testing.assert_allclose(oracle.sample(p, oracle.STATIC, oracle.DWS, pc, x=x, dy=dy, w=ws), dws.reshape(-1), atol=1e-11)
+
+
+# ---------------------------------------------------------------- decode ---
+
+DECODE_CASES = [
+    (oracle.HEADWISE, 7, 12, 4, 3, 0, 1),
+    (oracle.HEADWISE, 2, 8, 4, 1, 0, 0),   # T < W: the state still holds zero rows
+    (oracle.HEADWISE, 5, 6, 1, 2, 0, 1),   # W = 1: no state
+    (oracle.LOWRANK, 6, 8, 3, 2, 5, 1),
+    (oracle.LOWRANK, 9, 16, 8, 4, 3, 0),
+    (oracle.STATIC, 6, 5, 4, 1, 0, 1),
+    (oracle.STATIC, 3, 4, 8, 1, 0, 0),
+]
+
+
+@pytest.mark.parametrize("kind,T,D,W,H,R,residual", DECODE_CASES)
+def test_decode_steps_equal_forward(kind, T, D, W, H, R, residual):
+    """T decode steps from a zero state reproduce the (pinned) forward over the
+    T tokens token by token, and the final state holds the last W-1 inputs
+    (zero rows for positions before the start)."""
+    B, G = 2, D // H
+    x = rand(B, T, D)
+    Pf = P(B, T, D, W, H, R, residual)
+    if kind == oracle.HEADWISE:
+        w = rand(B, T, G, W)
+        yref = oracle.forward_headwise(Pf, x, w)
+        filt = lambda t: dict(w=np.ascontiguousarray(w[:, t]))
+    elif kind == oracle.LOWRANK:
+        z, U = rand(B, T, R), rand(R, G * W)
+        yref = oracle.forward_lowrank(Pf, x, z, U)
+        filt = lambda t: dict(z=np.ascontiguousarray(z[:, t]), U=U)
+    else:
+        ws = rand(D, W)
+        yref = oracle.forward_static(Pf, x, ws)
+        filt = lambda t: dict(ws=ws)
+    Pd = P(B, 1, D, W, H, R, residual)
+    state = np.zeros((B, W - 1, D))
+    for t in range(T):
+        y, state = oracle.decode(Pd, kind, np.ascontiguousarray(x[:, t]), state, **filt(t))
+        np.testing.assert_allclose(y, yref[:, t], rtol=0, atol=1e-12)
+    expect = np.zeros((B, W - 1, D))
+    for j in range(W - 1):
+        if T - (W - 1) + j >= 0:
+            expect[:, j] = x[:, T - (W - 1) + j]
+    assert np.array_equal(state, expect)
+
+
+@pytest.mark.parametrize("j", [0, 1, 3])
+def test_decode_delta_filter_reads_the_right_state_row(j):
+    """w_k = delta(k, j): y = x + x_{t-j}, x_{t-j} being state row W-1-j (j >= 1)."""
+    B, D, W = 2, 5, 4
+    x, state = rand(B, D), rand(B, W - 1, D)
+    w = np.zeros((B, D, W))
+    w[:, :, j] = 1.0
+    y, st = oracle.decode(P(B, 1, D, W, 1, 0, 1), oracle.HEADWISE, x, state, w=w)
+    np.testing.assert_array_equal(y, x + (x if j == 0 else state[:, W - 1 - j]))
+    np.testing.assert_array_equal(st[:, :-1], state[:, 1:])
+    np.testing.assert_array_equal(st[:, -1], x)
