@@ -94,6 +94,7 @@ def hbm_peak():
 
 
 KERNEL_SOURCES = {
+    "decode": ("decode.cu", "generic.cu", "common.cuh", "kernels.cuh"),
     "headwise": ("conv_stream.cu", "common.cuh", "kernels.cuh"),
     "static": ("conv_stream.cu", "common.cuh", "kernels.cuh"),
     "lowrank": ("lowrank_tc_fwd.cu", "lowrank_tc_bwd.cu", "lowrank_tc.cuh", "tc.cuh", "lowrank.cu", "common.cuh",
@@ -385,6 +386,184 @@ def run_dsc(args, wl0):
     return result, host, wl
 
 
+# ------------------------------------------------------------------ decode ---
+
+DECODE_METRIC = "decode tokens/s and achieved HBM GB/s (one token per sequence, bf16, W=4) vs B200 roofline"
+
+
+def decode_bytes(wl):
+    """Algorithmic HBM bytes of one decode step: x, y, the state read and
+    written (W-1 rows each), and the filters of the new tokens (head-wise w,
+    low-rank z plus U once, static ws once)."""
+    s = 2 if wl.dtype == "bf16" else 4
+    B, D, W, G, R = wl.B, wl.D, wl.W, wl.G, wl.R
+    base = B * D * s * (2 + 2 * (W - 1))
+    if wl.variant == "headwise":
+        return base + B * G * W * s
+    if wl.variant == "lowrank":
+        return base + B * R * s + R * G * W * s
+    return base + D * W * s
+
+
+class DecodeStep:
+    """Device buffers and the C-ABI call of one decode step."""
+
+    def __init__(self, wl, device):
+        import torch
+
+        import synth
+        from input_dependent_short_b200 import _lib
+        from synth import workloads as wls
+
+        self.wl, self.L = wl, _lib
+        host = wls.make_inputs(wl)
+        B, D, W = wl.B, wl.D, wl.W
+        h = {"x": host["x"].reshape(B, D)}
+        if wl.variant == "headwise":
+            h["w"] = host["w"].reshape(B, wl.G, W)
+        elif wl.variant == "lowrank":
+            h["z"], h["U"] = host["z"].reshape(B, wl.R), host["U"]
+        else:
+            h["ws"] = host["ws"]
+        self.h = {k: synth.to_torch(v, wl.dtype).pin_memory() for k, v in h.items()}
+        self.d = {k: v.to(device) for k, v in self.h.items()}
+        self.state = synth.to_torch(wls.decode_state(wl), wl.dtype).to(device)
+        self.y = torch.empty_like(self.d["x"])
+        self.y_h = torch.empty(self.y.shape, dtype=self.y.dtype).pin_memory()
+        self.p = _lib.DscProblem(B, 1, D, W, wl.H if wl.variant != "static" else 1, wl.R,
+                                 _lib.DSC_BF16 if wl.dtype == "bf16" else _lib.DSC_F32, int(wl.residual))
+        self.nws = _lib.lib().dsc_decode_lowrank_workspace_bytes(self.p) if wl.variant == "lowrank" else 0
+        self.ws = torch.empty(max(self.nws, 16), dtype=torch.uint8, device=device)
+
+    def run(self, stream):
+        d, L = self.d, self.L
+        if self.wl.variant == "headwise":
+            L.call("dsc_decode_headwise", self.p, d["x"].data_ptr(), d["w"].data_ptr(), self.state.data_ptr(),
+                   self.y.data_ptr(), stream)
+        elif self.wl.variant == "lowrank":
+            L.call("dsc_decode_lowrank", self.p, d["x"].data_ptr(), d["z"].data_ptr(), d["U"].data_ptr(),
+                   self.state.data_ptr(), self.y.data_ptr(), self.ws.data_ptr(), self.nws, stream)
+        else:
+            L.call("dsc_decode_static", self.p, d["x"].data_ptr(), d["ws"].data_ptr(), self.state.data_ptr(),
+                   self.y.data_ptr(), stream)
+
+    def h2d(self):  # the new tokens' inputs and filters (U and ws are weights: resident)
+        for k, v in self.h.items():
+            if k not in ("U", "ws"):
+                self.d[k].copy_(v, non_blocking=True)
+
+    def bytes_in(self):
+        return sum(v.numel() * v.element_size() for k, v in self.h.items() if k not in ("U", "ws"))
+
+
+def run_decode(args, wl0):
+    import torch
+    import torch.distributed as dist
+
+    world, rank, local = dist_env()
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    wl = rank_workload(wl0, rank)
+    st = DecodeStep(wl, dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    for _ in range(args.warmup):
+        st.run(stream)
+    torch.cuda.synchronize(dev)
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(K)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    lib = st.L.lib()
+    n0 = lib.dsc_launch_count()
+    with ClockSampler(local) as clocks:
+        start.record()
+        for i in range(K):
+            ev[i][0].record()
+            st.run(stream)
+            ev[i][1].record()
+        end.record()
+        end.synchronize()
+    torch.cuda.synchronize(dev)
+    launches = lib.dsc_launch_count() - n0
+    if world > 1:
+        dist.barrier()
+    ms = max_over_ranks(start.elapsed_time(end), world, dev)
+    call_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(K))
+    # end to end: the new tokens' inputs from pinned host memory, y back to the host
+    Ke = max(3, min(args.e2e_steps, K))
+    for _ in range(2):
+        st.h2d(); st.run(stream); st.y_h.copy_(st.y, non_blocking=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(Ke):
+        st.h2d()
+        st.run(stream)
+        st.y_h.copy_(st.y, non_blocking=True)
+    e1.record()
+    e1.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    nb = decode_bytes(wl)
+    peak, peak_src = hbm_peak()
+    gbs = nb / (call_ms / 1e3) / 1e9
+    result = None
+    if rank == 0:
+        result = {
+            "metric": DECODE_METRIC, "value": job_tokens_per_s(wl.B, world, K, ms), "unit": "tokens/s",
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else "f32",
+            "accumulate": "f32", "data": "synthetic (seeded normals, seed = rank)",
+            "config": {"workload": wl0.name, "variant": wl.variant, "B": wl.B, "D": wl.D, "W": wl.W, "H": wl.H,
+                       "R": wl.R, "residual": wl.residual, "pass": "decode step (one token per sequence)",
+                       "global_batch": wl.B * world, "parallelism": f"dp{world}",
+                       "l2": "step bytes %.0f MB > L2 126 MB, no flush" % (nb / 1e6)},
+            "kernels": {"decode": {"us": call_ms * 1e3, "alg_bytes": nb, "gbs": gbs, "frac": gbs / peak}},
+            "roofline": {"kernel": "k_decode", "bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                         "frac": gbs / peak, "traffic": None, "peak_source": peak_src + " (hbm_gbs, copy)"},
+            "e2e": {"value": job_tokens_per_s(wl.B, world, Ke, e2e_ms), "unit": "tokens/s",
+                    "h2d_bytes_per_step": st.bytes_in(), "d2h_bytes_per_step": st.y.numel() * st.y.element_size(),
+                    "steps": Ke, "ms_per_step": e2e_ms / Ke},
+            "gpu_launches": launches, "clocks": clocks.summary(), "source_digest": source_digest("decode"),
+        }
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return result
+
+
+def decode_reference(wl, seconds=None, steps=None, warmup=0, sequences=64):
+    """The oracle's decode step on `sequences` sequences of the workload: either
+    for about `seconds`, or for `steps` timed steps after `warmup`."""
+    import oracle
+    from synth import workloads as wls
+
+    sub = wl.with_(B=min(wl.B, sequences))
+    host = wls.make_inputs(sub)
+    B, D, W = sub.B, sub.D, sub.W
+    P = oracle.problem(B, 1, D, W, sub.H if sub.variant != "static" else 1, sub.R, sub.residual)
+    kind = {"headwise": oracle.HEADWISE, "lowrank": oracle.LOWRANK, "static": oracle.STATIC}[sub.variant]
+    x, state = host["x"].reshape(B, D), wls.decode_state(sub)
+    kw = {"headwise": lambda: dict(w=host["w"].reshape(B, sub.G, W)),
+          "lowrank": lambda: dict(z=host["z"].reshape(B, sub.R), U=host["U"]),
+          "static": lambda: dict(ws=host["ws"])}[sub.variant]()
+    for _ in range(warmup):
+        oracle.decode(P, kind, x, state, **kw)
+    n, t0 = 0, time.perf_counter()
+    while True:
+        oracle.decode(P, kind, x, state, **kw)
+        n += 1
+        el = time.perf_counter() - t0
+        if (steps is not None and n >= steps) or (seconds is not None and el >= seconds):
+            break
+    return n, B, el
+
+
 # ----------------------------------------------------------- CPU baselines ---
 
 def oracle_pass(wl, t):
@@ -484,6 +663,40 @@ def main():
         ap.error("--warmup must be at least 3")
     from synth import workloads as wls
 
+    if args.workload in wls.DECODE:
+        wl0 = wls.DECODE[args.workload]
+        if args.impl == "reference":
+            world, rank, _ = dist_env()
+            if rank == 0:
+                import oracle
+
+                oracle.build()
+                n, B, el = decode_reference(wl0, steps=args.steps, warmup=args.warmup)
+                v = n * B / el
+                print(json.dumps({
+                    "impl": "reference", "metric": DECODE_METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+                    "steps": args.steps, "warmup": args.warmup, "ms_per_step": el / n * 1e3,
+                    "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                    "data": "synthetic", "config": {"workload": wl0.name, "variant": wl0.variant,
+                                                   "pass": "decode step", "sample_sequences": B},
+                    "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": oracle.max_threads(), "kind": "oracle",
+                                     "sample": f"each step: one decode step of {B} sequences"},
+                    "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}),
+                    flush=True)
+            return
+        res = run_decode(args, wl0)
+        if res is not None:
+            if res["n_gpus"] == 1 and not args.no_cpu_baseline:
+                import oracle
+
+                n, B, el = decode_reference(wl0, seconds=args.cpu_seconds)
+                res["cpu_baseline"] = {"value": n * B / el, "unit": "tokens/s", "cores": oracle.max_threads(),
+                                       "kind": "oracle", "sample": f"{n} decode steps of {B} sequences "
+                                                                   f"(fp64 oracle, {el:.1f} s)"}
+            else:
+                res["cpu_baseline"] = None
+            print(json.dumps(res), flush=True)
+        return
     if args.workload in wls.NAMED:
         wl0 = wls.NAMED[args.workload]
     else:

@@ -155,6 +155,40 @@ DSC_API dsc_status dsc_bwd_static(const dsc_problem *p, const void *x, const voi
 DSC_API dsc_status dsc_bwd_static_noalloc(const dsc_problem *p, const void *x, const void *ws, const void *dy,
                                           void *dx, float *dws, void *stream);
 
+/* ---------------------------------------------------------------- decode ---
+ * Inference step: one new token per sequence.  A causal convolution of width
+ * W needs only the last W-1 inputs of each sequence, kept in a state
+ * [B, W-1, D] (dtype of x) whose row j holds x_{t-W+1+j}, oldest first, with
+ * zero rows for positions before the sequence start.  A step computes
+ *   y[b,c] = r x[b,c] + w_0 x[b,c] + sum_{k=1}^{W-1} w_k state[b, W-1-k, c]
+ * with the new token's filters and then shifts the state in place (rows
+ * 1 .. W-2 move down one row, x becomes the last row).  p->T must be 1;
+ * x, y are [B, D]; for W = 1 there is no state and `state` may be NULL.
+ * Buffers must not overlap.  Steps from a zero state reproduce the training
+ * forward token by token (up to rounding order).
+ * Errors as for the training calls; T != 1 gives DSC_ERR_INVALID_ARG. */
+
+/* Head-wise decode: w [B, G, W] holds the new token's filters. */
+DSC_API dsc_status dsc_decode_headwise(const dsc_problem *p, const void *x, const void *w, void *state, void *y,
+                                       void *stream);
+
+/* Static decode: ws [D, W] as in dsc_fwd_static (p->H is not used). */
+DSC_API dsc_status dsc_decode_static(const dsc_problem *p, const void *x, const void *ws, void *state, void *y,
+                                     void *stream);
+
+/* Scratch of the low-rank decode: the new token's filters, B*G*W fp32. */
+DSC_API size_t dsc_decode_lowrank_workspace_bytes(const dsc_problem *p);
+
+/* Low-rank decode: z [B, R] and U [R, G*W]; w = zU is formed in the
+ * workspace (B*G*W fp32 values for the one token) and then used as above. */
+DSC_API dsc_status dsc_decode_lowrank(const dsc_problem *p, const void *x, const void *z, const void *U, void *state,
+                                      void *y, void *workspace, size_t workspace_bytes, void *stream);
+
+/* State after a prompt x [B, T, D] (p->T = prompt length): row j of
+ * sequence b holds x[b, T-(W-1)+j], zero where that index is negative.  The
+ * prompt's outputs come from the training forward (dsc_fwd_*). */
+DSC_API dsc_status dsc_decode_state(const dsc_problem *p, const void *x, void *state, void *stream);
+
 /* Synchronise `stream`, then return and clear the device status word of the
  * current device: DSC_OK, DSC_ERR_TIMEOUT, or DSC_ERR_CUDA if the stream
  * reported an error. */

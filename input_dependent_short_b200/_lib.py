@@ -36,6 +36,11 @@ _SIGS = {
     "dsc_fwd_lowrank_workspace_bytes": (C.c_size_t, [_P]),
     "dsc_bwd_lowrank_workspace_bytes": (C.c_size_t, [_P]),
     "dsc_lowrank_kernels": (C.c_int, [_P, C.c_int]),
+    "dsc_decode_headwise": (C.c_int, [_P, _v, _v, _v, _v, _v]),
+    "dsc_decode_static": (C.c_int, [_P, _v, _v, _v, _v, _v]),
+    "dsc_decode_lowrank_workspace_bytes": (C.c_size_t, [_P]),
+    "dsc_decode_lowrank": (C.c_int, [_P, _v, _v, _v, _v, _v, _v, C.c_size_t, _v]),
+    "dsc_decode_state": (C.c_int, [_P, _v, _v, _v]),
     "dsc_fwd_lowrank": (C.c_int, [_P, _v, _v, _v, _v, _v, C.c_size_t, _v]),
     "dsc_bwd_lowrank": (C.c_int, [_P, _v, _v, _v, _v, _v, _v, _v, _v, C.c_size_t, _v]),
     "dsc_fwd_static": (C.c_int, [_P, _v, _v, _v, _v]),

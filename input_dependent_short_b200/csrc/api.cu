@@ -247,6 +247,63 @@ dsc_status dsc_bwd_lowrank(const dsc_problem *p, const void *x, const void *z, c
     return done(e);
 }
 
+// ------------------------------------------------------------------ decode ---
+
+static dsc_status validate_decode(const dsc_problem *p, bool lowrank) {
+    dsc_status s = validate(p, lowrank);
+    if (s == DSC_OK && p->T != 1) s = DSC_ERR_INVALID_ARG;
+    return s;
+}
+
+static dsc_status check_state(const dsc_problem *p, const void *state) {
+    return p->W > 1 ? check_ptrs({state}) : DSC_OK;
+}
+
+dsc_status dsc_decode_headwise(const dsc_problem *p, const void *x, const void *w, void *state, void *y,
+                               void *stream) {
+    dsc_status s = validate_decode(p, false);
+    if (s == DSC_OK) s = check_ptrs({x, w, y});
+    if (s == DSC_OK) s = check_state(p, state);
+    if (s != DSC_OK) return s;
+    return done(launch_decode(ctx(stream), *p, 0, x, w, state, y));
+}
+
+dsc_status dsc_decode_static(const dsc_problem *p, const void *x, const void *ws, void *state, void *y,
+                             void *stream) {
+    dsc_status s = validate_decode(p, false);
+    if (s == DSC_OK) s = check_ptrs({x, ws, y});
+    if (s == DSC_OK) s = check_state(p, state);
+    if (s != DSC_OK) return s;
+    return done(launch_decode(ctx(stream), *p, 2, x, ws, state, y));
+}
+
+size_t dsc_decode_lowrank_workspace_bytes(const dsc_problem *p) {
+    if (validate_decode(p, true) != DSC_OK) return 0;
+    return (size_t)p->B * (size_t)(p->D / p->H) * (size_t)p->W * sizeof(float);
+}
+
+dsc_status dsc_decode_lowrank(const dsc_problem *p, const void *x, const void *z, const void *U, void *state, void *y,
+                              void *workspace, size_t workspace_bytes, void *stream) {
+    dsc_status s = validate_decode(p, true);
+    if (s == DSC_OK) s = check_ptrs({x, z, U, y, workspace});
+    if (s == DSC_OK) s = check_state(p, state);
+    if (s != DSC_OK) return s;
+    if (workspace_bytes < dsc_decode_lowrank_workspace_bytes(p)) return DSC_ERR_INVALID_ARG;
+    const Ctx c = ctx(stream);
+    float *wf = static_cast<float *>(workspace);
+    cudaError_t e = launch_lr_filters(c, *p, z, U, wf);  // w[b, g*W+k] = z_b . U[:, g*W+k]
+    if (e == cudaSuccess) e = launch_decode(c, *p, 1, x, wf, state, y);
+    return done(e);
+}
+
+dsc_status dsc_decode_state(const dsc_problem *p, const void *x, void *state, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_ptrs({x});
+    if (s == DSC_OK) s = check_state(p, state);
+    if (s != DSC_OK) return s;
+    return done(launch_decode_state(ctx(stream), *p, x, state));
+}
+
 dsc_status dsc_selftest_timeout(void *stream) {
     return launch_wait_selftest(static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSC_OK : DSC_ERR_CUDA;
 }

@@ -142,6 +142,74 @@ def dsc_bwd_static(x, ws, dy, residual=False):
     return dx, dws
 
 
+# -------------------------------------------------------------------- decode ---
+
+def _dec_problem(x, state, W, H, R, residual):
+    B, D = x.shape
+    if x.dtype not in _DT:
+        raise ValueError(f"unsupported dtype {x.dtype}")
+    if W > 1 and (state is None or state.shape != (B, W - 1, D) or state.dtype != x.dtype):
+        raise ValueError("state must be [B, W-1, D] in the dtype of x")
+    return DscProblem(B, 1, D, W, H, R, _DT[x.dtype], int(bool(residual)))
+
+
+def dsc_decode_headwise(x, w, state, residual=True):
+    """One decode step: x [B,D], the new token's filters w [B,G,W], state
+    [B,W-1,D] (last W-1 inputs, oldest first; updated in place).  Returns y."""
+    dev = _check(x, w, *([state] if state is not None else []), dtype=x.dtype)
+    B, D = x.shape
+    G, W = w.shape[1], w.shape[2]
+    if w.shape[0] != B or D % G:
+        raise ValueError("w must be [B,G,W] with G dividing D")
+    p = _dec_problem(x, state, W, D // G, 0, residual)
+    y = torch.empty_like(x)
+    with torch.cuda.device(dev):
+        call("dsc_decode_headwise", p, _ptr(x), _ptr(w), _ptr(state), _ptr(y), _stream(dev))
+    return y
+
+
+def dsc_decode_static(x, ws, state, residual=False):
+    """One decode step with static filters ws [D,W]; state updated in place."""
+    dev = _check(x, ws, *([state] if state is not None else []), dtype=x.dtype)
+    W = ws.shape[1]
+    if ws.shape[0] != x.shape[1]:
+        raise ValueError("ws must be [D,W]")
+    p = _dec_problem(x, state, W, 1, 0, residual)
+    y = torch.empty_like(x)
+    with torch.cuda.device(dev):
+        call("dsc_decode_static", p, _ptr(x), _ptr(ws), _ptr(state), _ptr(y), _stream(dev))
+    return y
+
+
+def dsc_decode_lowrank(x, z, U, state, H=1, residual=True):
+    """One decode step with low-rank filters w = z U (z [B,R], U [R,G*W]);
+    state updated in place."""
+    dev = _check(x, z, U, *([state] if state is not None else []), dtype=x.dtype)
+    B, D = x.shape
+    R = z.shape[1]
+    if z.shape != (B, R) or U.shape[0] != R or D % H or U.shape[1] % (D // H):
+        raise ValueError("expected z [B,R] and U [R,(D/H)*W]")
+    W = U.shape[1] // (D // H)
+    p = _dec_problem(x, state, W, H, R, residual)
+    n = lib().dsc_decode_lowrank_workspace_bytes(p)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    y = torch.empty_like(x)
+    with torch.cuda.device(dev):
+        call("dsc_decode_lowrank", p, _ptr(x), _ptr(z), _ptr(U), _ptr(state), _ptr(y), _ptr(ws), n, _stream(dev))
+    return y
+
+
+def dsc_decode_state(x, W):
+    """The decode state [B,W-1,D] after a prompt x [B,T,D]."""
+    dev = _check(x)
+    B, T, D = x.shape
+    state = torch.empty(B, W - 1, D, dtype=x.dtype, device=dev) if W > 1 else None
+    p = problem(x, W, 1, 0, False)
+    with torch.cuda.device(dev):
+        call("dsc_decode_state", p, _ptr(x), _ptr(state), _stream(dev))
+    return state
+
+
 def dsc_check(device=None):
     """Synchronise the current stream and raise if a kernel recorded a timeout."""
     dev = torch.device("cuda", torch.cuda.current_device() if device is None else torch.device(device).index)

@@ -20,7 +20,7 @@ from __future__ import annotations
 import math
 from dataclasses import dataclass, replace
 
-from . import BF16, F32, TID_DY, TID_U, TID_W, TID_WS, TID_X, TID_Z, make_tensor
+from . import BF16, F32, TID_DY, TID_STATE, TID_U, TID_W, TID_WS, TID_X, TID_Z, make_tensor
 
 HEADWISE = "headwise"
 LOWRANK = "lowrank"
@@ -91,6 +91,24 @@ def sweep_workloads() -> list:
             out.append(Workload(f"sweep-lowrank W{W} R{R}", LOWRANK, 1, 16384, 4096, W, H=1, R=R))
         out.append(Workload(f"sweep-static W{W}", STATIC, 1, 16384, 4096, W))
     return out
+
+
+# Decode: one new token for each of B sequences (T = 1), the Q/K/V width;
+# the inputs, outputs and state of one step (~200 MB) exceed L2.
+DECODE_QKV_HEADWISE = Workload("decode-qkv-headwise B2048 D6144 W4 H16", HEADWISE, 2048, 1, 6144, 4, H=16)
+DECODE_QKV_LOWRANK = Workload("decode-qkv-lowrank B2048 D6144 W4 H1 R32", LOWRANK, 2048, 1, 6144, 4, H=1, R=32)
+DECODE_STATIC = Workload("decode-static B2048 D6144 W4", STATIC, 2048, 1, 6144, 4)
+
+DECODE = {
+    "decode-qkv-headwise": DECODE_QKV_HEADWISE,
+    "decode-qkv-lowrank": DECODE_QKV_LOWRANK,
+    "decode-static": DECODE_STATIC,
+}
+
+
+def decode_state(wl):
+    """A seeded decode state [B, W-1, D] (the last W-1 inputs of each sequence)."""
+    return make_tensor(wl.seed, TID_STATE, (wl.B, wl.W - 1, wl.D), 1.0, wl.dtype)
 
 
 NAMED = {

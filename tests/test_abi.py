@@ -141,3 +141,20 @@ def test_lowrank_kernel_choice(shape, fwd, bwd):
     assert L.dsc_lowrank_kernels(C.byref(p32), 1) == 1
     bad = P(*shape[:5], R=0)
     assert L.dsc_lowrank_kernels(C.byref(bad), 0) == -1
+
+
+def test_decode_argument_checks():
+    """Decode calls take one token per sequence and reject bad arguments
+    before any CUDA call."""
+    L = _lib.lib()
+    p2 = P(T=2)
+    assert L.dsc_decode_headwise(C.byref(p2), GOOD, GOOD, GOOD, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_decode_static(C.byref(p2), GOOD, GOOD, GOOD, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
+    p = P(T=1)
+    assert L.dsc_decode_headwise(C.byref(p), GOOD, GOOD, None, GOOD, None) == _lib.DSC_ERR_INVALID_ARG  # W > 1: state
+    assert L.dsc_decode_headwise(C.byref(p), GOOD, GOOD, GOOD + 8, GOOD, None) == _lib.DSC_ERR_MISALIGNED
+    lr = P(B=3, T=1, D=16, W=4, H=2, R=4)
+    assert L.dsc_decode_lowrank_workspace_bytes(C.byref(lr)) == 3 * 8 * 4 * 4
+    assert L.dsc_decode_lowrank(C.byref(lr), GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 16, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_decode_lowrank_workspace_bytes(C.byref(P(T=2, R=4))) == 0
+    assert L.dsc_decode_state(C.byref(P(T=5)), None, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
