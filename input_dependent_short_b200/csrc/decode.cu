@@ -76,14 +76,20 @@ __global__ void __launch_bounds__(256) k_decode(const DecArgs a) {
 #pragma unroll
     for (int j = 0; j < S; ++j) load_v<T, V>(sp + j * a.D, st[j], false);
     float y[V];
+    Row<WT, W> taps;  // the W taps of the current channel's filter, reloaded when the filter changes
+    int64_t cur = -1;
 #pragma unroll
     for (int e = 0; e < V; ++e) {
         const int64_t c = c0 + e;
-        const WT *f = MODE == DEC_STATIC ? wp + c * W : wp + (b * a.G + c / a.H) * W;
+        const int64_t fi = MODE == DEC_STATIC ? c : b * a.G + c / a.H;  // filter row of channel c
+        if (fi != cur) {
+            taps.load(wp + fi * W);
+            cur = fi;
+        }
         float acc = a.residual ? xf[e] : 0.f;
-        acc = fmaf(to_f<WT>(__ldg(f)), xf[e], acc);
+        acc = fmaf(taps.get(0), xf[e], acc);
 #pragma unroll
-        for (int k = 1; k < W; ++k) acc = fmaf(to_f<WT>(__ldg(f + k)), st[S - k][e], acc);
+        for (int k = 1; k < W; ++k) acc = fmaf(taps.get(k), st[S - k][e], acc);
         y[e] = acc;
     }
     store_v<T, V>(static_cast<T *>(a.y) + b * a.D + c0, y);

@@ -156,12 +156,12 @@ template <typename T>
 __global__ void __launch_bounds__(256) k_lr_filters(const T *__restrict__ z, const T *__restrict__ U, float *wf,
                                                     int64_t N, int R, int64_t GW) {
     constexpr int TB = 16;
-    __shared__ float zs[TB][256];
+    __shared__ __align__(16) float zs[256][TB];  // [r][token]: one 16-byte load gives four tokens' z_r
     const int64_t n0 = (int64_t)blockIdx.y * TB;
     const int64_t j = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     for (int i = threadIdx.x; i < TB * R; i += blockDim.x) {
         const int tn = i / R, r = i % R;
-        zs[tn][r] = (n0 + tn < N) ? to_f<T>(z[(n0 + tn) * R + r]) : 0.f;
+        zs[r][tn] = (n0 + tn < N) ? to_f<T>(z[(n0 + tn) * R + r]) : 0.f;
     }
     __syncthreads();
     if (j >= GW) return;
@@ -171,7 +171,13 @@ __global__ void __launch_bounds__(256) k_lr_filters(const T *__restrict__ z, con
     for (int r = 0; r < R; ++r) {
         const float u = to_f<T>(U[(int64_t)r * GW + j]);
 #pragma unroll
-        for (int i = 0; i < TB; ++i) acc[i] = fmaf(zs[i][r], u, acc[i]);
+        for (int i = 0; i < TB; i += 4) {
+            const float4 zq = *reinterpret_cast<const float4 *>(&zs[r][i]);
+            acc[i] = fmaf(zq.x, u, acc[i]);
+            acc[i + 1] = fmaf(zq.y, u, acc[i + 1]);
+            acc[i + 2] = fmaf(zq.z, u, acc[i + 2]);
+            acc[i + 3] = fmaf(zq.w, u, acc[i + 3]);
+        }
     }
 #pragma unroll
     for (int i = 0; i < TB; ++i)
