@@ -278,18 +278,22 @@ dsc_status dsc_decode_static(const dsc_problem *p, const void *x, const void *ws
 }
 
 size_t dsc_decode_lowrank_workspace_bytes(const dsc_problem *p) {
-    if (validate_decode(p, true) != DSC_OK) return 0;
+    if (validate_decode(p, true) != DSC_OK || decode_lowrank_fused_ok(*p)) return 0;
     return (size_t)p->B * (size_t)(p->D / p->H) * (size_t)p->W * sizeof(float);
 }
 
 dsc_status dsc_decode_lowrank(const dsc_problem *p, const void *x, const void *z, const void *U, void *state, void *y,
                               void *workspace, size_t workspace_bytes, void *stream) {
     dsc_status s = validate_decode(p, true);
-    if (s == DSC_OK) s = check_ptrs({x, z, U, y, workspace});
+    if (s == DSC_OK) s = check_ptrs({x, z, U, y});
     if (s == DSC_OK) s = check_state(p, state);
     if (s != DSC_OK) return s;
-    if (workspace_bytes < dsc_decode_lowrank_workspace_bytes(p)) return DSC_ERR_INVALID_ARG;
     const Ctx c = ctx(stream);
+    if (decode_lowrank_fused_ok(*p)) return done(launch_decode_lowrank_fused(c, *p, x, z, U, state, y));
+    // other shapes: the token's filters through a scratch
+    s = check_ptrs({workspace});
+    if (s != DSC_OK) return s;
+    if (workspace_bytes < dsc_decode_lowrank_workspace_bytes(p)) return DSC_ERR_INVALID_ARG;
     float *wf = static_cast<float *>(workspace);
     cudaError_t e = launch_lr_filters(c, *p, z, U, wf);  // w[b, g*W+k] = z_b . U[:, g*W+k]
     if (e == cudaSuccess) e = launch_decode(c, *p, 1, x, wf, state, y);

@@ -192,7 +192,7 @@ def dsc_decode_lowrank(x, z, U, state, H=1, residual=True):
     W = U.shape[1] // (D // H)
     p = _dec_problem(x, state, W, H, R, residual)
     n = lib().dsc_decode_lowrank_workspace_bytes(p)
-    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
     y = torch.empty_like(x)
     with torch.cuda.device(dev):
         call("dsc_decode_lowrank", p, _ptr(x), _ptr(z), _ptr(U), _ptr(state), _ptr(y), _ptr(ws), n, _stream(dev))

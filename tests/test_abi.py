@@ -153,8 +153,11 @@ def test_decode_argument_checks():
     p = P(T=1)
     assert L.dsc_decode_headwise(C.byref(p), GOOD, GOOD, None, GOOD, None) == _lib.DSC_ERR_INVALID_ARG  # W > 1: state
     assert L.dsc_decode_headwise(C.byref(p), GOOD, GOOD, GOOD + 8, GOOD, None) == _lib.DSC_ERR_MISALIGNED
-    lr = P(B=3, T=1, D=16, W=4, H=2, R=4)
-    assert L.dsc_decode_lowrank_workspace_bytes(C.byref(lr)) == 3 * 8 * 4 * 4
+    fused = P(B=3, T=1, D=16, W=4, H=2, R=4)  # filters formed in registers: no scratch
+    assert L.dsc_decode_lowrank_workspace_bytes(C.byref(fused)) == 0
+    lr = P(B=3, T=1, D=18, W=4, H=3, R=4)  # D not a multiple of 8: the token's filters through a scratch
+    assert L.dsc_decode_lowrank_workspace_bytes(C.byref(lr)) == 3 * 6 * 4 * 4
     assert L.dsc_decode_lowrank(C.byref(lr), GOOD, GOOD, GOOD, GOOD, GOOD, GOOD, 16, None) == _lib.DSC_ERR_INVALID_ARG
+    assert L.dsc_decode_lowrank(C.byref(lr), GOOD, GOOD, GOOD, GOOD, GOOD, None, 0, None) == _lib.DSC_ERR_INVALID_ARG
     assert L.dsc_decode_lowrank_workspace_bytes(C.byref(P(T=2, R=4))) == 0
     assert L.dsc_decode_state(C.byref(P(T=5)), None, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
