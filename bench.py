@@ -512,6 +512,9 @@ def run_decode(args, wl0):
     nb = decode_bytes(wl)
     peak, peak_src = hbm_peak()
     gbs = nb / (call_ms / 1e3) / 1e9
+    digest = source_digest("decode")
+    kname = "k_decode_lr" if wl.variant == "lowrank" else "k_decode"
+    traffic = ncu_traffic(kname, wl0.name, digest)
     result = None
     if rank == 0:
         result = {
@@ -524,12 +527,12 @@ def run_decode(args, wl0):
                        "global_batch": wl.B * world, "parallelism": f"dp{world}",
                        "l2": "step bytes %.0f MB > L2 126 MB, no flush" % (nb / 1e6)},
             "kernels": {"decode": {"us": call_ms * 1e3, "alg_bytes": nb, "gbs": gbs, "frac": gbs / peak}},
-            "roofline": {"kernel": "k_decode", "bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
-                         "frac": gbs / peak, "traffic": None, "peak_source": peak_src + " (hbm_gbs, copy)"},
+            "roofline": {"kernel": kname, "bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                         "frac": gbs / peak, "traffic": traffic, "peak_source": peak_src + " (hbm_gbs, copy)"},
             "e2e": {"value": job_tokens_per_s(wl.B, world, Ke, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": st.bytes_in(), "d2h_bytes_per_step": st.y.numel() * st.y.element_size(),
                     "steps": Ke, "ms_per_step": e2e_ms / Ke},
-            "gpu_launches": launches, "clocks": clocks.summary(), "source_digest": source_digest("decode"),
+            "gpu_launches": launches, "clocks": clocks.summary(), "source_digest": digest,
         }
     if world > 1:
         dist.barrier()
