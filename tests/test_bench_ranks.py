@@ -60,3 +60,13 @@ def test_algorithmic_bytes_of_the_headline_workload():
     assert fb == N * (4 * D + 2 * GW)
     assert bb == N * (6 * D + 4 * GW)
     assert fb + bb == 1_157_627_904
+
+
+def test_algorithmic_bytes_of_the_decode_workloads():
+    """x and y, the state read and written (W-1 rows each), and the filters."""
+    B, D, W, s = 2048, 6144, 4, 2
+    base = B * D * s * (2 + 2 * (W - 1))
+    assert bench.decode_bytes(wls.DECODE_QKV_HEADWISE) == base + B * 384 * W * s
+    assert bench.decode_bytes(wls.DECODE_QKV_LOWRANK) == base + B * 32 * s + 32 * 6144 * W * s
+    assert bench.decode_bytes(wls.DECODE_STATIC) == base + D * W * s
+    assert bench.decode_bytes(wls.DECODE_QKV_HEADWISE) > 126 * 2 ** 20  # one step's bytes exceed L2
