@@ -94,7 +94,8 @@ def hbm_peak():
 
 
 KERNEL_SOURCES = {
-    "decode": ("decode.cu", "generic.cu", "common.cuh", "kernels.cuh"),
+    "decode": ("decode.cu", "lowrank_tc_dec.cu", "generic.cu", "lowrank_tc.cuh", "tc.cuh", "common.cuh",
+               "kernels.cuh"),
     "headwise": ("conv_stream.cu", "common.cuh", "kernels.cuh"),
     "static": ("conv_stream.cu", "common.cuh", "kernels.cuh"),
     "lowrank": ("lowrank_tc_fwd.cu", "lowrank_tc_bwd.cu", "lowrank_tc.cuh", "tc.cuh", "lowrank.cu", "common.cuh",
@@ -513,7 +514,7 @@ def run_decode(args, wl0):
     peak, peak_src = hbm_peak()
     gbs = nb / (call_ms / 1e3) / 1e9
     digest = source_digest("decode")
-    kname = "k_decode_lr" if wl.variant == "lowrank" else "k_decode"
+    kname = ("k_lr_tc_dec" if wl.dtype == "bf16" else "k_decode_lr") if wl.variant == "lowrank" else "k_decode"
     traffic = ncu_traffic(kname, wl0.name, digest)
     result = None
     if rank == 0:

@@ -95,16 +95,17 @@ DSC_API dsc_status dsc_bwd_headwise(const dsc_problem *p, const void *x, const v
 DSC_API size_t dsc_fwd_lowrank_workspace_bytes(const dsc_problem *p);
 DSC_API size_t dsc_bwd_lowrank_workspace_bytes(const dsc_problem *p);
 
-/* Kernel family a low-rank problem runs on, forward (backward = 0) or
- * backward (backward = 1), as chosen by the same host-side plan the calls
- * use (on the current device's SM count; 148 without a device).  Launches
- * nothing and touches no device memory.  Returns one of:
+/* Kernel family a low-rank problem runs on, forward (backward = 0),
+ * backward (backward = 1) or decode step (backward = 2, p->T = 1), as chosen
+ * by the same host-side plan the calls use (on the current device's SM count;
+ * 148 without a device).  Launches nothing and touches no device memory.
+ * Returns one of:
  *   DSC_LR_TENSOR_CORE  fused, the filter contractions on tcgen05 tensor cores
  *                       (bf16; R a multiple of 8 up to 64, H a divisor of
  *                       64, D a multiple of 32*H, and a plan that fits the
  *                       shared memory and tensor memory);
  *   DSC_LR_FUSED        fused, contractions on CUDA cores (fp32, other shapes);
- *   DSC_LR_UNFUSED      filters and their gradient in the caller's workspace;
+ *   DSC_LR_UNFUSED      filters (and their gradient) in the caller's workspace;
  * or -1 when the problem is invalid. */
 #define DSC_LR_TENSOR_CORE 0
 #define DSC_LR_FUSED 1

@@ -76,6 +76,21 @@ static size_t lr_generic_fwd_bytes(const dsc_problem &p) {
     return (size_t)(p.B * p.T) * (size_t)((p.D / p.H) * p.W) * sizeof(float);
 }
 
+// decode.cu: one decode step (mode 0 head-wise filters [B,G,W] in the input
+// dtype, 1 low-rank filters as fp32 [B,G,W], 2 static [D,W]), the state taken
+// from the last W-1 tokens of a prompt [B,T,D], and the low-rank step with the
+// token's filters formed on chip (tensor cores, or CUDA cores for shapes with
+// D a multiple of the vector width and H dividing or divided by it).
+cudaError_t launch_decode(const Ctx &c, const dsc_problem &p, int mode, const void *x, const void *w, void *state,
+                          void *y);
+cudaError_t launch_decode_state(const Ctx &c, const dsc_problem &p, const void *x, void *state);
+bool decode_lowrank_fused_ok(const dsc_problem &p);
+cudaError_t launch_decode_lowrank_fused(const Ctx &c, const dsc_problem &p, const void *x, const void *z,
+                                        const void *U, void *state, void *y);
+// lowrank_tc_dec.cu: the tensor-core decode's plan and the status word of its bounded waits
+bool decode_lowrank_tc_ok(const dsc_problem &p);
+int take_tc_dec_status(cudaStream_t stream);
+
 }  // namespace dsc
 
 using namespace dsc;
@@ -180,6 +195,11 @@ dsc_status dsc_bwd_static(const dsc_problem *p, const void *x, const void *ws, c
 
 int dsc_lowrank_kernels(const dsc_problem *p, int backward) {
     if (validate(p, true) != DSC_OK) return -1;
+    if (backward == 2) {  // decode step
+        if (p->T != 1) return -1;
+        if (decode_lowrank_tc_ok(*p)) return DSC_LR_TENSOR_CORE;
+        return decode_lowrank_fused_ok(*p) ? DSC_LR_FUSED : DSC_LR_UNFUSED;
+    }
     if (backward ? lowrank_tc_bwd_ok(*p, sm_count()) : lowrank_tc_ok(*p)) return DSC_LR_TENSOR_CORE;
     if (lowrank_fused_ok(*p)) return DSC_LR_FUSED;
     return DSC_LR_UNFUSED;
@@ -316,8 +336,9 @@ dsc_status dsc_check(void *stream) {
     if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return DSC_ERR_CUDA;
     const int st = take_device_status(static_cast<cudaStream_t>(stream));
     const int st_tc = take_tc_status(static_cast<cudaStream_t>(stream));
-    if (st < 0 || st_tc < 0) return DSC_ERR_CUDA;
-    return static_cast<dsc_status>(st ? st : st_tc);
+    const int st_dec = take_tc_dec_status(static_cast<cudaStream_t>(stream));
+    if (st < 0 || st_tc < 0 || st_dec < 0) return DSC_ERR_CUDA;
+    return static_cast<dsc_status>(st ? st : (st_tc ? st_tc : st_dec));
 }
 
 }  // extern "C"

@@ -132,6 +132,8 @@ __global__ void __launch_bounds__(256) k_decode_lr(const DecLrArgs a) {
     const int64_t b_lo = (int64_t)blockIdx.y * SB;
     const T *U = static_cast<const T *>(a.U);
     const T *z = static_cast<const T *>(a.z);
+    // staging: unrolled so that each thread's global loads are in flight together
+#pragma unroll 8
     for (int i = tid; i < a.R * NQ * DL_NV * 4; i += blockDim.x) {
         const int e = i & 3, vv = (i >> 2) % DL_NV, jq = (i >> 2) / DL_NV % NQ, r = (i >> 2) / DL_NV / NQ;
         const int cc = jq * 4 + e;  // tap index within the vector's taps
@@ -143,6 +145,7 @@ __global__ void __launch_bounds__(256) k_decode_lr(const DecLrArgs a) {
         }
         us[i] = u;
     }
+#pragma unroll 8
     for (int i = tid; i < a.R * SB; i += blockDim.x) {
         const int r = i / SB, sq = i % SB;
         zs[i] = b_lo + sq < a.B ? to_f<T>(z[(b_lo + sq) * a.R + r]) : 0.f;
@@ -305,14 +308,22 @@ cudaError_t dl_dispatch(const Ctx &c, const dsc_problem &p, const DecLrArgs &a) 
 
 }  // namespace
 
-bool decode_lowrank_fused_ok(const dsc_problem &p) {
+// lowrank_tc_dec.cu: the tensor-core decode (bf16 shapes the tensor-core map takes).
+bool decode_lowrank_tc_ok(const dsc_problem &p);
+cudaError_t launch_decode_lowrank_tc(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U,
+                                     void *state, void *y);
+
+static bool decode_lowrank_cc_ok(const dsc_problem &p) {
     const int gpv = p.dtype == DSC_BF16 ? dl_gpv<bf16>(p) : dl_gpv<float>(p);
     return gpv > 0 && dl_smem((int)p.R, gpv, (int)p.W) <= (size_t)DL_SMEM_MAX;
 }
 
+bool decode_lowrank_fused_ok(const dsc_problem &p) { return decode_lowrank_tc_ok(p) || decode_lowrank_cc_ok(p); }
+
 cudaError_t launch_decode_lowrank_fused(const Ctx &c, const dsc_problem &p, const void *x, const void *z,
                                         const void *U, void *state, void *y) {
-    if (!decode_lowrank_fused_ok(p)) return cudaErrorNotSupported;
+    if (decode_lowrank_tc_ok(p)) return launch_decode_lowrank_tc(c, p, x, z, U, state, y);
+    if (!decode_lowrank_cc_ok(p)) return cudaErrorNotSupported;
     DecLrArgs a{};
     a.B = p.B;
     a.D = p.D;

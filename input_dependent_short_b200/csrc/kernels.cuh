@@ -86,18 +86,6 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
 
 int resident_blocks(const void *kernel, int threads, size_t smem);
 
-// decode.cu: one decode step (mode 0 head-wise filters [B,G,W] in the input
-// dtype, 1 low-rank filters as fp32 [B,G,W], 2 static [D,W]) and the state
-// taken from the last W-1 tokens of a prompt [B,T,D].
-cudaError_t launch_decode(const Ctx &c, const dsc_problem &p, int mode, const void *x, const void *w, void *state,
-                          void *y);
-cudaError_t launch_decode_state(const Ctx &c, const dsc_problem &p, const void *x, void *state);
-// Low-rank decode with the token's filters formed in registers (shapes with
-// D a multiple of the vector width and H dividing or divided by it).
-bool decode_lowrank_fused_ok(const dsc_problem &p);
-cudaError_t launch_decode_lowrank_fused(const Ctx &c, const dsc_problem &p, const void *x, const void *z,
-                                        const void *U, void *state, void *y);
-
 // Records one kernel launch (api.cu keeps the process-wide count).
 void count_launch();
 

@@ -161,3 +161,8 @@ def test_decode_argument_checks():
     assert L.dsc_decode_lowrank(C.byref(lr), GOOD, GOOD, GOOD, GOOD, GOOD, None, 0, None) == _lib.DSC_ERR_INVALID_ARG
     assert L.dsc_decode_lowrank_workspace_bytes(C.byref(P(T=2, R=4))) == 0
     assert L.dsc_decode_state(C.byref(P(T=5)), None, GOOD, None) == _lib.DSC_ERR_INVALID_ARG
+    # decode kernel family: tensor cores for the Q/K/V decode shape, CUDA cores in fp32, a scratch for ragged D
+    assert L.dsc_lowrank_kernels(C.byref(P(B=2048, T=1, D=6144, W=4, H=1, R=32)), 2) == 0
+    assert L.dsc_lowrank_kernels(C.byref(P(B=2048, T=1, D=6144, W=4, H=1, R=32, dtype=0)), 2) == 1
+    assert L.dsc_lowrank_kernels(C.byref(P(B=3, T=1, D=18, W=4, H=3, R=4)), 2) == 2
+    assert L.dsc_lowrank_kernels(C.byref(P(B=3, T=2, D=64, W=4, H=1, R=8)), 2) == -1

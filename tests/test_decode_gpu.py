@@ -81,7 +81,17 @@ SHAPES = [
     (2, 256, 2, 256, 64),   # one group
     (17, 136, 5, 8, 24),
     (3, 30, 7, 3, 2),       # D not a multiple of 4 or 8
+    (200, 4096, 4, 64, 64), # tiles too large for the tensor-core decode's shared memory: CUDA cores
+    # bf16 low-rank on the tensor-core decode (tiles of 128 sequences, ragged last tile)
+    (300, 512, 4, 1, 32),
+    (129, 2048, 3, 2, 16),
+    (64, 1024, 8, 1, 8),
+    (200, 4096, 4, 64, 32),
+    (5, 256, 1, 8, 16),
+    (130, 1024, 2, 4, 24),
 ]
+
+TC_DECODE = SHAPES[9:]
 
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
@@ -89,6 +99,13 @@ SHAPES = [
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "B{}D{}W{}H{}R{}".format(*s))
 def test_decode_step_matches_oracle(shape, kind, dtype):
     B, D, W, H, R = shape
+    if kind == "lowrank" and dtype == "bf16" and shape in TC_DECODE:
+        import ctypes as C
+
+        from input_dependent_short_b200 import _lib
+
+        p = _lib.DscProblem(B, 1, D, W, H, R, _lib.DSC_BF16, 1)
+        assert _lib.lib().dsc_lowrank_kernels(C.byref(p), 2) == 0  # the tensor-core decode
     residual = 1 if kind != "static" else 0
     t = inputs(kind, B, 1, D, W, H, R, dtype)
     x0 = np.ascontiguousarray(t["x"][:, 0])
@@ -105,7 +122,8 @@ def test_decode_step_matches_oracle(shape, kind, dtype):
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 @pytest.mark.parametrize("kind", ["headwise", "lowrank", "static"])
-@pytest.mark.parametrize("shape", [(2, 12, 64, 4, 16, 8), (3, 5, 24, 8, 2, 16), (1, 9, 4096, 3, 1, 32)],
+@pytest.mark.parametrize("shape", [(2, 12, 64, 4, 16, 8), (3, 5, 24, 8, 2, 16), (1, 9, 4096, 3, 1, 32),
+                                   (130, 6, 1024, 4, 1, 16)],
                          ids=lambda s: "B{}T{}D{}W{}H{}R{}".format(*s))
 def test_decode_steps_and_prompt_match_forward(shape, kind, dtype):
     """A prompt of T0 tokens (its state from dsc_decode_state), then T - T0
