@@ -177,16 +177,20 @@ DSC_API dsc_status dsc_decode_headwise(const dsc_problem *p, const void *x, cons
 DSC_API dsc_status dsc_decode_static(const dsc_problem *p, const void *x, const void *ws, void *state, void *y,
                                      void *stream);
 
-/* Scratch of the low-rank decode: 0 when the fused kernel takes the problem
- * (D a multiple of the 16-byte vector width, H dividing or divided by it,
- * and U's columns of 8 vectors with R rows fitting shared memory), else the
- * new token's filters, B*G*W fp32. */
+/* Scratch of the low-rank decode: 0 when a fused kernel takes the problem,
+ * else the new token's filters, B*G*W fp32.  Fused: the tensor-core kernel
+ * for bf16 shapes of the training tensor-core map (R a multiple of 8 up to
+ * 64, H a divisor of 64, D a multiple of 32*H, tiles fitting shared
+ * memory); otherwise the CUDA-core kernel when D is a multiple of the
+ * 16-byte vector width, H divides or is divided by it, and U's columns of 8
+ * vectors with R rows fit shared memory. */
 DSC_API size_t dsc_decode_lowrank_workspace_bytes(const dsc_problem *p);
 
-/* Low-rank decode: z [B, R] and U [R, G*W].  The fused kernel forms each
- * vector's filters w = zU in registers from U columns staged in shared
- * memory; other shapes form them in the workspace first (`workspace` may be
- * NULL when the size above is 0). */
+/* Low-rank decode: z [B, R] and U [R, G*W].  The fused kernels form the new
+ * token's filters w = zU on chip (in TMEM by one MMA per tile of 128
+ * sequences, or in registers from U columns staged in shared memory); other
+ * shapes form them in the workspace first (`workspace` may be NULL when the
+ * size above is 0). */
 DSC_API dsc_status dsc_decode_lowrank(const dsc_problem *p, const void *x, const void *z, const void *U, void *state,
                                       void *y, void *workspace, size_t workspace_bytes, void *stream);
 
