@@ -91,7 +91,11 @@ def _bind(lib):
     lib.orc_sample.argtypes = [P, C.POINTER(_Filter), _In, _In, C.c_int64, C.c_int64,
                                C.POINTER(C.c_int64), d]
     lib.orc_decode.argtypes = [P, C.POINTER(_Filter), _In, _In, d, d]
-    for f in ("orc_lowrank_filters", "orc_forward", "orc_backward", "orc_lowrank_grads", "orc_sample", "orc_decode"):
+    i64 = C.POINTER(C.c_int64)
+    lib.orc_forward_varlen.argtypes = [P, C.c_int64, _In, _In, i64, C.c_int64, d]
+    lib.orc_backward_varlen.argtypes = [P, C.c_int64, _In, _In, _In, i64, C.c_int64, d, d]
+    for f in ("orc_lowrank_filters", "orc_forward", "orc_backward", "orc_lowrank_grads", "orc_sample", "orc_decode",
+              "orc_forward_varlen", "orc_backward_varlen"):
         getattr(lib, f).restype = None
     return lib
 
@@ -200,3 +204,43 @@ def decode(P: Problem, kind: int, x, state, *, w=None, z=None, U=None, ws=None, 
     F = _Filter(kind, _in(ws if kind == STATIC else w), _in(z), _in(U))
     lib.orc_decode(C.byref(P), C.byref(F), _in(x), _in(state), _dp(y), _dp(st))
     return y, st
+
+
+def _cu(P: Problem, cu_seqlens):
+    cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
+    if P.B != 1 or cu[0] != 0 or cu[-1] != P.T or np.any(np.diff(cu) < 1):
+        raise ValueError("packed sequences: B = 1 and cu_seqlens rising from 0 to T")
+    return cu, cu.ctypes.data_as(C.POINTER(C.c_int64)), len(cu) - 1
+
+
+def forward_varlen(P: Problem, kind: int, x, cu_seqlens, *, w=None, z=None, U=None, ws=None, lib=None):
+    """Packed documents (B = 1, document d = tokens cu[d] .. cu[d+1]-1), no tap
+    crossing a document start.  Head-wise w [1,T,G,W], low-rank z and U (the
+    filters materialised as w = zU), or static ws [D,W].  Returns y [1,T,D]."""
+    lib = lib or load()
+    cu, cp, n = _cu(P, cu_seqlens)
+    if kind == LOWRANK:
+        w, kind = lowrank_filters(P, z, U, lib), HEADWISE
+    y = _out((P.B, P.T, P.D))
+    lib.orc_forward_varlen(C.byref(P), kind, _in(ws if kind == STATIC else w), _in(x), cp, n, _dp(y))
+    return y
+
+
+def backward_varlen(P: Problem, kind: int, x, dy, cu_seqlens, *, w=None, z=None, U=None, ws=None, lib=None):
+    """Gradients of forward_varlen: (dx, dw) for head-wise, (dx, dws) for
+    static, (dx, dz, dU, dw) for low-rank."""
+    lib = lib or load()
+    cu, cp, n = _cu(P, cu_seqlens)
+    lowrank = kind == LOWRANK
+    if lowrank:
+        w, kind = lowrank_filters(P, z, U, lib), HEADWISE
+    dx = _out((P.B, P.T, P.D))
+    dw = _out((P.D, P.W)) if kind == STATIC else _out((P.B, P.T, P.G, P.W))
+    lib.orc_backward_varlen(C.byref(P), kind, _in(ws if kind == STATIC else w), _in(x), _in(dy), cp, n, _dp(dx),
+                            _dp(dw))
+    if not lowrank:
+        return dx, dw
+    dz = _out((P.B, P.T, P.R))
+    dU = _out((P.R, P.G * P.W))
+    lib.orc_lowrank_grads(C.byref(P), _in(z), _in(U), _dp(dw), _dp(dz), _dp(dU))
+    return dx, dz, dU, dw

@@ -301,3 +301,75 @@ void orc_decode(const orc_problem *P, const orc_filter *F, orc_in x, orc_in stat
             if (S > 0) state_out[(b * S + S - 1) * P->D + c] = xt;
         }
 }
+
+/* Variable-length (packed) sequences: one row of P->T tokens (P->B = 1)
+ * holds nseq documents, document d spanning tokens [cu[d], cu[d+1]), with
+ * cu[0] = 0 and cu[nseq] = P->T.  A document is a sequence of its own, so
+ * the definition's zero padding applies at every document start: tap k of
+ * token t contributes only when t-k lies in t's document.  The gradients
+ * follow: dx[s] takes tap k of token s+k only when s+k lies in s's document,
+ * and dw[t,g,k] (and the static dws) takes dy_t x_{t-k} only when t-k does.
+ * Head-wise filters w [1,T,G,W] (low-rank: the materialised w = zU) or
+ * static ws [D,W]. */
+static int64_t doc_of(const int64_t *cu, int64_t nseq, int64_t t)
+{
+    int64_t d = 0;
+    while (d + 1 < nseq && cu[d + 1] <= t) ++d;
+    return d;
+}
+
+void orc_forward_varlen(const orc_problem *P, int64_t kind, orc_in w, orc_in x, const int64_t *cu, int64_t nseq,
+                        double *y_out)
+{
+    orc_filter F = {kind, w, {0, 0}, {0, 0}};
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < P->T; ++t) {
+        const int64_t start = cu[doc_of(cu, nseq, t)];
+        for (int64_t c = 0; c < P->D; ++c) {
+            double s = P->residual ? xval(P, x, 0, t, c) : 0.0;
+            for (int64_t k = 0; k < P->W; ++k)
+                if (t - k >= start) s += tap(P, &F, 0, t, c, k) * xval(P, x, 0, t - k, c);
+            y_out[t * P->D + c] = s;
+        }
+    }
+}
+
+void orc_backward_varlen(const orc_problem *P, int64_t kind, orc_in w, orc_in x, orc_in dy, const int64_t *cu,
+                         int64_t nseq, double *dx_out, double *dw_out)
+{
+    orc_filter F = {kind, w, {0, 0}, {0, 0}};
+    const int64_t G = P->D / P->H;
+#pragma omp parallel for schedule(static)
+    for (int64_t s = 0; s < P->T; ++s) {
+        const int64_t end = cu[doc_of(cu, nseq, s) + 1];
+        for (int64_t c = 0; c < P->D; ++c) {
+            double acc = P->residual ? xval(P, dy, 0, s, c) : 0.0;
+            for (int64_t k = 0; k < P->W; ++k)
+                if (s + k < end) acc += tap(P, &F, 0, s + k, c, k) * xval(P, dy, 0, s + k, c);
+            dx_out[s * P->D + c] = acc;
+        }
+    }
+    if (kind == ORC_STATIC) {
+#pragma omp parallel for schedule(static)
+        for (int64_t c = 0; c < P->D; ++c)
+            for (int64_t k = 0; k < P->W; ++k) {
+                double acc = 0.0;
+                for (int64_t t = 0; t < P->T; ++t)
+                    if (t - k >= cu[doc_of(cu, nseq, t)]) acc += xval(P, dy, 0, t, c) * xval(P, x, 0, t - k, c);
+                dw_out[c * P->W + k] = acc;
+            }
+    } else {
+#pragma omp parallel for schedule(static)
+        for (int64_t t = 0; t < P->T; ++t) {
+            const int64_t start = cu[doc_of(cu, nseq, t)];
+            for (int64_t g = 0; g < G; ++g)
+                for (int64_t k = 0; k < P->W; ++k) {
+                    double acc = 0.0;
+                    if (t - k >= start)
+                        for (int64_t c = g * P->H; c < (g + 1) * P->H; ++c)
+                            acc += xval(P, dy, 0, t, c) * xval(P, x, 0, t - k, c);
+                    dw_out[(t * G + g) * P->W + k] = acc;
+                }
+        }
+    }
+}

@@ -39,6 +39,12 @@ MUTANTS = {
     "decode does not shift the state": ("= val(state, (b * S + j + 1) * P->D + c);",
                                         "= val(state, (b * S + j) * P->D + c);"),
     "decode drops the residual": ("double s = P->residual ? xt : 0.0;", "double s = 0.0;"),
+    "packed forward reaches across a document start": ("if (t - k >= start) s += tap(P, &F, 0, t, c, k)",
+                                                       "if (t - k >= 0) s += tap(P, &F, 0, t, c, k)"),
+    "packed dx reaches past a document end": ("if (s + k < end) acc += tap(P, &F, 0, s + k, c, k)",
+                                              "if (s + k < P->T) acc += tap(P, &F, 0, s + k, c, k)"),
+    "packed dw reaches across a document start": ("if (t - k >= start)\n                        for",
+                                                  "if (t - k >= 0)\n                        for"),
 }
 
 
@@ -130,6 +136,22 @@ def _pins(lib):
                                   w=np.ascontiguousarray(w[:, t]), lib=lib)
         ok &= np.allclose(yt, y[:, t], atol=1e-12)
     check("decode", ok and np.array_equal(state[:, -1], x[:, -1]))
+
+    # packed documents against the documents run one by one
+    lens = (3, 1, 3)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    pp = oracle.problem(1, T, D, W, H, 0, 1)
+    yp = oracle.forward_varlen(pp, oracle.HEADWISE, x[:1], cu, w=w[:1], lib=lib)
+    dxp, dwp = oracle.backward_varlen(pp, oracle.HEADWISE, x[:1], dy[:1], cu, w=w[:1], lib=lib)
+    ok = True
+    for d in range(len(lens)):
+        sl = slice(cu[d], cu[d + 1])
+        pd = oracle.problem(1, lens[d], D, W, H, 0, 1)
+        xs, ws_, dys = (np.ascontiguousarray(a[:1, sl]) for a in (x, w, dy))
+        dxd, dwd = oracle.backward_headwise(pd, xs, ws_, dys, lib=lib)
+        ok &= np.allclose(yp[:, sl], oracle.forward_headwise(pd, xs, ws_, lib=lib), atol=1e-12)
+        ok &= np.allclose(dxp[:, sl], dxd, atol=1e-12) and np.allclose(dwp[:, sl], dwd, atol=1e-12)
+    check("varlen", ok)
     return fails
 
 

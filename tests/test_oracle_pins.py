@@ -386,3 +386,79 @@ def test_decode_delta_filter_reads_the_right_state_row(j):
     np.testing.assert_array_equal(y, x + (x if j == 0 else state[:, W - 1 - j]))
     np.testing.assert_array_equal(st[:, :-1], state[:, 1:])
     np.testing.assert_array_equal(st[:, -1], x)
+
+
+# ------------------------------------------------- variable-length (packed) ---
+
+VARLEN_CASES = [
+    # (kind, document lengths, D, W, H, R, residual)
+    (oracle.HEADWISE, (5, 1, 7, 3), 6, 4, 2, 0, 1),
+    (oracle.HEADWISE, (2, 9), 4, 3, 1, 0, 0),
+    (oracle.LOWRANK, (4, 6, 2), 8, 3, 4, 3, 1),
+    (oracle.STATIC, (3, 3, 5), 5, 4, 1, 0, 1),
+    (oracle.STATIC, (1, 1, 1, 6), 3, 8, 1, 0, 0),
+]
+
+
+def _varlen_inputs(kind, T, D, W, H, R):
+    G = D // H
+    f = {}
+    if kind == oracle.HEADWISE:
+        f["w"] = rand(1, T, G, W)
+    elif kind == oracle.LOWRANK:
+        f["z"], f["U"] = rand(1, T, R), rand(R, G * W)
+    else:
+        f["ws"] = rand(D, W)
+    return rand(1, T, D), rand(1, T, D), f
+
+
+def _plain(kind, P_, x, dy, f):
+    """The (pinned) oracle on one sequence: (y, gradients)."""
+    if kind == oracle.HEADWISE:
+        return oracle.forward_headwise(P_, x, f["w"]), oracle.backward_headwise(P_, x, f["w"], dy)
+    if kind == oracle.LOWRANK:
+        return oracle.forward_lowrank(P_, x, f["z"], f["U"]), oracle.backward_lowrank(P_, x, f["z"], f["U"], dy)
+    return oracle.forward_static(P_, x, f["ws"]), oracle.backward_static(P_, x, f["ws"], dy)
+
+
+@pytest.mark.parametrize("kind,lens,D,W,H,R,residual", VARLEN_CASES)
+def test_varlen_equals_documents_run_separately(kind, lens, D, W, H, R, residual):
+    """Packed documents give, token by token, what each document gives as a
+    sequence of its own; the token reductions (static dws, low-rank dU) are the
+    sums over the documents."""
+    T = sum(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    x, dy, f = _varlen_inputs(kind, T, D, W, H, R)
+    Pp = P(1, T, D, W, H, R, residual)
+    y = oracle.forward_varlen(Pp, kind, x, cu, **f)
+    g = oracle.backward_varlen(Pp, kind, x, dy, cu, **f)
+    total = None
+    for d in range(len(lens)):
+        sl = slice(cu[d], cu[d + 1])
+        fd = {k: (np.ascontiguousarray(v[:, sl]) if k in ("w", "z") else v) for k, v in f.items()}
+        yd, gd = _plain(kind, P(1, lens[d], D, W, H, R, residual), np.ascontiguousarray(x[:, sl]),
+                        np.ascontiguousarray(dy[:, sl]), fd)
+        np.testing.assert_allclose(y[:, sl], yd, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(g[0][:, sl], gd[0], rtol=0, atol=1e-12)  # dx
+        if kind == oracle.HEADWISE:
+            np.testing.assert_allclose(g[1][:, sl], gd[1], rtol=0, atol=1e-12)  # dw
+        elif kind == oracle.LOWRANK:
+            np.testing.assert_allclose(g[1][:, sl], gd[1], rtol=0, atol=1e-12)  # dz
+            total = gd[2] if total is None else total + gd[2]
+        else:
+            total = gd[1] if total is None else total + gd[1]
+    if kind == oracle.LOWRANK:
+        np.testing.assert_allclose(g[2], total, rtol=0, atol=1e-11)  # dU
+    elif kind == oracle.STATIC:
+        np.testing.assert_allclose(g[1], total, rtol=0, atol=1e-11)  # dws
+
+
+@pytest.mark.parametrize("kind", [oracle.HEADWISE, oracle.LOWRANK, oracle.STATIC])
+def test_varlen_one_document_is_the_plain_op(kind):
+    T, D, W, H, R = 9, 6, 4, 3, 2
+    x, dy, f = _varlen_inputs(kind, T, D, W, H, R)
+    Pp = P(1, T, D, W, H, R, 1)
+    y, g = _plain(kind, Pp, x, dy, f)
+    np.testing.assert_array_equal(oracle.forward_varlen(Pp, kind, x, [0, T], **f), y)
+    for a, b in zip(oracle.backward_varlen(Pp, kind, x, dy, [0, T], **f), g):
+        np.testing.assert_array_equal(a, b)
