@@ -70,3 +70,11 @@ def test_algorithmic_bytes_of_the_decode_workloads():
     assert bench.decode_bytes(wls.DECODE_QKV_LOWRANK) == base + B * 32 * s + 32 * 6144 * W * s
     assert bench.decode_bytes(wls.DECODE_STATIC) == base + D * W * s
     assert bench.decode_bytes(wls.DECODE_QKV_HEADWISE) > 126 * 2 ** 20  # one step's bytes exceed L2
+
+
+def test_decode_reference_arm_runs_the_oracle_on_a_sample():
+    """The CPU arm of the decode workloads: the oracle's decode step on a
+    bounded sample of sequences."""
+    wl = wls.DECODE_QKV_LOWRANK.with_(B=8, D=256)
+    n, B, el = bench.decode_reference(wl, steps=2, warmup=1, sequences=4)
+    assert n == 2 and B == 4 and el > 0
