@@ -141,14 +141,16 @@ DSC_API dsc_status dsc_bwd_static(const dsc_problem *p, const void *x, const voi
  * library scratch memory -- plugin or custom-op interfaces that pass an
  * operator only its inputs and outputs, and services that allocate all device
  * memory at start-up and must not call cudaMalloc/cudaFree afterwards.
- * Same arguments, results and errors as dsc_bwd_static, except:
+ * Same arguments, results (bit for bit) and argument errors as
+ * dsc_bwd_static, except:
  *  - its scratch is an array of DSC_NOALLOC_SCRATCH_BYTES inside the library,
  *    one per device, held from library load until process exit; a problem
  *    whose scratch (dsc_bwd_static_workspace_bytes) exceeds that size is
  *    rejected with DSC_ERR_UNSUPPORTED before anything is launched;
  *  - the first call with a given device current looks the array's device
- *    address up (cudaGetSymbolAddress); make that first call before any
- *    stream capture on that device;
+ *    address up (cudaGetSymbolAddress) and keeps it for the life of the
+ *    process; make that first call before any stream capture on that device,
+ *    and do not reset the device (cudaDeviceReset) after it;
  *  - all calls on a device share the one array: calls whose work overlaps on
  *    the GPU (different streams without ordering between them) race and give
  *    wrong results.  Each call writes every scratch element it reads, so the

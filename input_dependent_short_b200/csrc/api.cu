@@ -13,7 +13,7 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 static bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-static dsc_status validate(const dsc_problem *p, bool lowrank) {
+dsc_status validate(const dsc_problem *p, bool lowrank) {
     if (!p) return DSC_ERR_INVALID_ARG;
     if (p->B < 1 || p->T < 1 || p->D < 1 || p->W < 1 || p->W > 8 || p->H < 1) return DSC_ERR_INVALID_ARG;
     if (p->D % p->H) return DSC_ERR_INVALID_ARG;

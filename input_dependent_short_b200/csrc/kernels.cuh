@@ -40,6 +40,10 @@ struct GenArgs {
     float *partial;
 };
 
+// Argument checks shared by the entry points (api.cu): the problem shape and
+// dtype, as documented in dsc.h (DSC_ERR_INVALID_ARG or DSC_ERR_UNSUPPORTED).
+dsc_status validate(const dsc_problem *p, bool lowrank);
+
 struct Ctx {
     cudaStream_t stream;
     int sms;

@@ -23,13 +23,20 @@ constexpr size_t NOALLOC_SCRATCH_FLOATS = DSC_NOALLOC_SCRATCH_BYTES / sizeof(flo
 static __device__ __align__(256) float g_noalloc_scratch[NOALLOC_SCRATCH_FLOATS];
 
 // Device address of the array on the current device.  Looked up on the first
-// call made with each device current, then cached.
+// call made with each device current, then cached for the life of the process
+// (a cudaDeviceReset after that first call is not supported: the module, and
+// the array with it, may be reloaded elsewhere).  A failed CUDA call leaves no
+// sticky last-error behind, so the next entry point does not report it as its
+// own launch failure.
 static float *noalloc_scratch(cudaError_t &err) {
     static std::mutex mu;
     static float *addr[64] = {nullptr};
     int dev = 0;
     err = cudaGetDevice(&dev);
-    if (err != cudaSuccess) return nullptr;
+    if (err != cudaSuccess) {
+        cudaGetLastError();
+        return nullptr;
+    }
     if (dev < 0 || dev >= 64) {
         err = cudaErrorInvalidDevice;
         return nullptr;
@@ -38,7 +45,10 @@ static float *noalloc_scratch(cudaError_t &err) {
     if (!addr[dev]) {
         void *p = nullptr;
         err = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (err != cudaSuccess) return nullptr;
+        if (err != cudaSuccess) {
+            cudaGetLastError();
+            return nullptr;
+        }
         addr[dev] = static_cast<float *>(p);
     }
     return addr[dev];
@@ -48,14 +58,15 @@ static float *noalloc_scratch(cudaError_t &err) {
 
 extern "C" dsc_status dsc_bwd_static_noalloc(const dsc_problem *p, const void *x, const void *ws, const void *dy,
                                              void *dx, float *dws, void *stream) {
-    // Argument checks first, so that a rejected call touches no device state.
-    const size_t need = dsc_bwd_static_workspace_bytes(p);  // 0 for an invalid problem
-    if (need == 0) return DSC_ERR_INVALID_ARG;
+    // The same argument checks as dsc_bwd_static, in the same order and with
+    // the same status codes, so that a rejected call touches no device state.
+    const dsc_status s = dsc::validate(p, false);
+    if (s != DSC_OK) return s;
     for (const void *q : {x, ws, dy, (const void *)dx, (const void *)dws})
         if (!q) return DSC_ERR_INVALID_ARG;
     for (const void *q : {x, ws, dy, (const void *)dx, (const void *)dws})
         if (reinterpret_cast<uintptr_t>(q) & 15u) return DSC_ERR_MISALIGNED;
-    if (need > DSC_NOALLOC_SCRATCH_BYTES) return DSC_ERR_UNSUPPORTED;
+    if (dsc_bwd_static_workspace_bytes(p) > DSC_NOALLOC_SCRATCH_BYTES) return DSC_ERR_UNSUPPORTED;
     cudaError_t err = cudaSuccess;
     float *scratch = dsc::noalloc_scratch(err);
     if (!scratch) return DSC_ERR_CUDA;

@@ -166,3 +166,23 @@ def test_decode_argument_checks():
     assert L.dsc_lowrank_kernels(C.byref(P(B=2048, T=1, D=6144, W=4, H=1, R=32, dtype=0)), 2) == 1
     assert L.dsc_lowrank_kernels(C.byref(P(B=3, T=1, D=18, W=4, H=3, R=4)), 2) == 2
     assert L.dsc_lowrank_kernels(C.byref(P(B=3, T=2, D=64, W=4, H=1, R=8)), 2) == -1
+
+
+def test_noalloc_backward_reports_the_regular_backwards_argument_errors():
+    """dsc_bwd_static_noalloc returns the same status codes as dsc_bwd_static
+    for rejected arguments, before touching any device state: an unsupported
+    length (T > 2^30), an invalid shape, a NULL or misaligned pointer."""
+    L = _lib.lib()
+
+    def both(p, ptrs):
+        a = L.dsc_bwd_static(C.byref(p) if p is not None else None, *ptrs, GOOD, 1 << 40, None)
+        b = L.dsc_bwd_static_noalloc(C.byref(p) if p is not None else None, *ptrs, None)
+        return a, b
+
+    good = [GOOD] * 5
+    assert both(P(T=(1 << 30) + 1), good) == (_lib.DSC_ERR_UNSUPPORTED, _lib.DSC_ERR_UNSUPPORTED)
+    assert both(P(B=(1 << 30) + 1), good) == (_lib.DSC_ERR_UNSUPPORTED, _lib.DSC_ERR_UNSUPPORTED)
+    assert both(P(W=9), good) == (_lib.DSC_ERR_INVALID_ARG, _lib.DSC_ERR_INVALID_ARG)
+    assert both(None, good) == (_lib.DSC_ERR_INVALID_ARG, _lib.DSC_ERR_INVALID_ARG)
+    assert both(P(), [GOOD, GOOD, None, GOOD, GOOD]) == (_lib.DSC_ERR_INVALID_ARG, _lib.DSC_ERR_INVALID_ARG)
+    assert both(P(), [GOOD, GOOD, GOOD, GOOD + 4, GOOD]) == (_lib.DSC_ERR_MISALIGNED, _lib.DSC_ERR_MISALIGNED)
