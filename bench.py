@@ -15,8 +15,12 @@ scaling), the time is the max over ranks of the device-measured time of K
 steps.  Also reported: the roofline of the dominant kernel (the backward)
 against the measured HBM copy bandwidth, the oracle on the host cores as a
 CPU baseline, the same metric end to end with host buffers (H2D of the
-inputs and D2H of all outputs inside the timed region), SM clocks sampled
-during the timed region, and the number of library kernels launched.
+inputs and D2H of all outputs inside the timed region; head-wise batches
+pipelined row by row over three streams), SM clocks sampled during the timed
+region, and the number of library kernels launched.  The default run also
+times the other three training workloads (Q/K/V low-rank, all-linear
+head-wise and low-rank) and reports each under `workloads` with its own
+roofline; `--workloads none` skips them.
 """
 
 from __future__ import annotations
@@ -254,6 +258,32 @@ class Step:
         for k, v in self.out.items():
             self.out_h[k].copy_(v, non_blocking=True)
 
+    # ---- end to end by batch row: rows are independent sequences, so a row's
+    # copies and kernels can overlap another row's.  Only for head-wise filters:
+    # the low-rank dU and the static dws sum over every row of the batch.
+    def row_chunks(self):
+        return self.wl.B if self.wl.variant == "headwise" and self.wl.B > 1 else 1
+
+    def run_row(self, i, stream):
+        """H2D of row i's inputs, its forward and backward (one C-ABI call
+        each, B = 1), D2H of its outputs; all on `stream` (a torch stream)."""
+        import torch
+
+        from input_dependent_short_b200 import ops
+
+        if not hasattr(self, "p1"):
+            x = self.d["x"]
+            self.p1 = ops.problem(x[:1], self.wl.W, self.wl.H, 0, bool(self.wl.residual))
+        with torch.cuda.stream(stream):
+            for k, v in self.h.items():
+                self.d[k][i].copy_(v[i], non_blocking=True)
+            d, o, L, sp = self.d, self.out, self.L, stream.cuda_stream
+            L.call("dsc_fwd_headwise", self.p1, d["x"][i].data_ptr(), d["w"][i].data_ptr(), o["y"][i].data_ptr(), sp)
+            L.call("dsc_bwd_headwise", self.p1, d["x"][i].data_ptr(), d["w"][i].data_ptr(), d["dy"][i].data_ptr(),
+                   o["dx"][i].data_ptr(), o["dw"][i].data_ptr(), sp)
+            for k, v in self.out.items():
+                self.out_h[k][i].copy_(v[i], non_blocking=True)
+
     def bytes_in(self):
         return sum(v.numel() * v.element_size() for v in self.h.values())
 
@@ -314,22 +344,7 @@ def run_dsc(args, wl0):
 
     # end to end: inputs from pinned host memory, every output back to the host
     Ke = max(3, min(args.e2e_steps, K))
-    for _ in range(2):
-        step.h2d(); step.fwd(stream); step.bwd(stream); step.d2h()
-    torch.cuda.synchronize(dev)
-    if world > 1:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(Ke):
-        step.h2d()
-        step.fwd(stream)
-        step.bwd(stream)
-        step.d2h()
-    e1.record()
-    e1.synchronize()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
-
+    e2e_ms, e2e_mode = time_e2e(step, Ke, stream, dev, world)
     tokens = wl.B * wl.T
     fb, bb = step_bytes(wl)
     peak, peak_src = hbm_peak()
@@ -376,15 +391,113 @@ def run_dsc(args, wl0):
             },
             "e2e": {"value": job_tokens_per_s(tokens, world, Ke, e2e_ms), "unit": "tokens/s",
                     "h2d_bytes_per_step": step.bytes_in(), "d2h_bytes_per_step": step.bytes_out(),
-                    "steps": Ke, "ms_per_step": e2e_ms / Ke},
+                    "steps": Ke, "ms_per_step": e2e_ms / Ke, "pipeline": e2e_mode},
             "gpu_launches": launches,
             "clocks": clocks.summary(),
             "source_digest": digest,
         }
+    # the other training workloads, each timed the same way (fewer steps)
+    others = {}
+    if args.workloads:
+        del step
+        torch.cuda.empty_cache()
+        for name in args.workloads.split(","):
+            other = rank_workload(wls.NAMED[name], rank)
+            others[name] = time_workload(other, args.other_steps, args.warmup, dev, world, peak)
+            torch.cuda.empty_cache()
+    if result is not None and others:
+        result["workloads"] = others
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
     return result, host, wl
+
+
+def time_e2e(step, K, stream, dev, world):
+    """Device time of K end-to-end steps: every step copies its inputs from
+    pinned host memory and every output back.  Head-wise batches run row by
+    row, round-robin over three streams, so that one row's H2D, another's
+    kernels and a third's D2H overlap (both copy directions at once)."""
+    import torch
+    import torch.distributed as dist
+
+    n = step.row_chunks()
+    streams = [torch.cuda.Stream(dev) for _ in range(3)] if n > 1 else []
+
+    def one():
+        if n == 1:
+            step.h2d(); step.fwd(stream); step.bwd(stream); step.d2h()
+            return
+        for i in range(n):
+            step.run_row(i, streams[i % 3])
+
+    for _ in range(2):
+        one()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    main = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for s in streams:
+        s.wait_event(e0)
+    for _ in range(K):
+        one()
+    for s in streams:
+        ev = torch.cuda.Event()
+        ev.record(s)
+        main.wait_event(ev)
+    e1.record(main)
+    e1.synchronize()
+    mode = f"{n} batch rows over 3 streams (H2D, kernels and D2H of different rows overlap)" if n > 1 else "serial"
+    return max_over_ranks(e0.elapsed_time(e1), world, dev), mode
+
+
+def time_workload(wl, steps, warmup, dev, world, peak):
+    """Forward + backward of another workload: device time per step, the two
+    calls' HBM fractions and the roofline of its dominant kernel."""
+    import torch
+
+    from synth import workloads as wls
+
+    step = Step(wl, wls.make_inputs(wl), dev)
+    stream = torch.cuda.current_stream(dev).cuda_stream
+    for _ in range(warmup):
+        step.fwd(stream)
+        step.bwd(stream)
+    torch.cuda.synchronize(dev)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(steps)]
+    lib = step.L.lib()
+    n0 = lib.dsc_launch_count()
+    for i in range(steps):
+        ev[i][0].record()
+        step.fwd(stream)
+        ev[i][1].record()
+        step.bwd(stream)
+        ev[i][2].record()
+    torch.cuda.synchronize(dev)
+    launches = lib.dsc_launch_count() - n0
+    fwd_ms = statistics.mean(ev[i][0].elapsed_time(ev[i][1]) for i in range(steps))
+    bwd_ms = statistics.mean(ev[i][1].elapsed_time(ev[i][2]) for i in range(steps))
+    ms = max_over_ranks(statistics.mean(ev[i][0].elapsed_time(ev[i][2]) for i in range(steps)), world, dev)
+    fb, bb = step_bytes(wl)
+    fg, bg = fb / (fwd_ms / 1e3) / 1e9, bb / (bwd_ms / 1e3) / 1e9
+    kname = {"headwise": "k_stream_bwd", "static": "k_stream_bwd",
+             "lowrank": "k_lr_tc_bwd" if wl.dtype == "bf16" else "k_lr_bwd"}[wl.variant]
+    digest = source_digest(wl.variant)
+    out = {
+        "config": {"workload": wl.name, "variant": wl.variant, "B": wl.B, "T": wl.T, "D": wl.D, "W": wl.W,
+                   "H": wl.H, "R": wl.R},
+        "value": job_tokens_per_s(wl.B * wl.T, world, 1, ms), "unit": "tokens/s", "ms_per_step": ms,
+        "steps": steps, "warmup": warmup, "gpu_launches": launches,
+        "kernels": {"fwd": {"us": fwd_ms * 1e3, "alg_bytes": fb, "gbs": fg, "frac": fg / peak},
+                    "bwd": {"us": bwd_ms * 1e3, "alg_bytes": bb, "gbs": bg, "frac": bg / peak}},
+        "roofline": {"kernel": kname, "bound": "hbm", "achieved": bg, "peak": peak, "unit": "GB/s", "frac": bg / peak,
+                     "traffic": ncu_traffic(kname, wl.name, digest), "step_frac": (fb + bb) / (ms / 1e3) / 1e9 / peak},
+        "source_digest": digest,
+    }
+    del step
+    return out
 
 
 # ------------------------------------------------------------------ decode ---
@@ -662,6 +775,10 @@ def main():
     ap.add_argument("--ref-tokens", type=int, default=256)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default=None,
+                    help="comma-separated named workloads also timed in the same run (default: the other three "
+                         "training workloads when --workload is the headline one; 'none' for none)")
+    ap.add_argument("--other-steps", type=int, default=20)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
@@ -709,6 +826,14 @@ def main():
             ap.error(f"unknown workload {args.workload}")
         wl0 = matches[0]
 
+    if args.workloads is None:
+        args.workloads = ("qkv-lowrank,all-linear-headwise,all-linear-lowrank" if args.workload == "qkv-headwise"
+                          else "none")
+    if args.workloads == "none":
+        args.workloads = ""
+    for name in filter(None, args.workloads.split(",")):
+        if name not in wls.NAMED:
+            ap.error(f"unknown workload {name}")
     if args.impl == "reference":
         res = run_reference(args, wl0)
     else:

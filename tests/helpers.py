@@ -31,7 +31,26 @@ def rel_err(got, ref):
     return float(np.max(np.abs(got - ref)) / scale)
 
 
-def assert_close(name, got, ref, dtype):
+def record_error(name, err):
+    """Print a measured error (shown by ``pytest -rP`` / ``-s``) and, when the
+    environment names a file in DSC_ERRLOG, append it there as a JSON line."""
+    import json
+    import os
+
+    print(f"normwise error {name}: {err:.3e}")
+    path = os.environ.get("DSC_ERRLOG")
+    if path:
+        with open(path, "a") as f:
+            f.write(json.dumps({"name": name, "err": err}) + "\n")
+
+
+def assert_close(name, got, ref, dtype, bound=None):
+    """Normwise error of ``got`` against the fp64 ``ref``: at most the stated
+    tolerance of the dtype and, where given, the tighter regression ``bound``
+    (a few times the error the kernels are known to reach)."""
     e = rel_err(got, ref)
+    record_error(name, e)
     assert e <= TOL[dtype], f"{name}: normwise relative error {e:.3e} > {TOL[dtype]:.1e}"
+    if bound is not None:
+        assert e <= bound, f"{name}: normwise relative error {e:.3e} above its regression bound {bound:.1e}"
     return e
