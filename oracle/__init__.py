@@ -94,8 +94,10 @@ def _bind(lib):
     i64 = C.POINTER(C.c_int64)
     lib.orc_forward_varlen.argtypes = [P, C.c_int64, _In, _In, i64, C.c_int64, d]
     lib.orc_backward_varlen.argtypes = [P, C.c_int64, _In, _In, _In, i64, C.c_int64, d, d]
+    lib.orc_forward_chunk.argtypes = [P, C.c_int64, _In, _In, _In, d]
+    lib.orc_backward_chunk.argtypes = [P, C.c_int64, _In, _In, _In, _In, _In, _In, d, d]
     for f in ("orc_lowrank_filters", "orc_forward", "orc_backward", "orc_lowrank_grads", "orc_sample", "orc_decode",
-              "orc_forward_varlen", "orc_backward_varlen"):
+              "orc_forward_varlen", "orc_backward_varlen", "orc_forward_chunk", "orc_backward_chunk"):
         getattr(lib, f).restype = None
     return lib
 
@@ -238,6 +240,61 @@ def backward_varlen(P: Problem, kind: int, x, dy, cu_seqlens, *, w=None, z=None,
     dw = _out((P.D, P.W)) if kind == STATIC else _out((P.B, P.T, P.G, P.W))
     lib.orc_backward_varlen(C.byref(P), kind, _in(ws if kind == STATIC else w), _in(x), _in(dy), cp, n, _dp(dx),
                             _dp(dw))
+    if not lowrank:
+        return dx, dw
+    dz = _out((P.B, P.T, P.R))
+    dU = _out((P.R, P.G * P.W))
+    lib.orc_lowrank_grads(C.byref(P), _in(z), _in(U), _dp(dw), _dp(dz), _dp(dU))
+    return dx, dz, dU, dw
+
+
+def _halo(a, B, W, D):
+    if a is None:
+        return None
+    a = np.ascontiguousarray(a)
+    if a.shape[0] != B or a.shape[1] != W - 1 or a.shape[-1] != D and a.ndim == 3:
+        raise ValueError("halo rows must be [B, W-1, ...]")
+    return a
+
+
+def forward_chunk(P: Problem, kind: int, x, x_prev=None, *, w=None, z=None, U=None, ws=None, lib=None):
+    """One time chunk of longer sequences (context parallelism): x [B,T,D]
+    holds tokens t0 .. t0+T-1, x_prev [B,W-1,D] the W-1 tokens before t0
+    (row j = position t0-W+1+j; None when t0 = 0).  Filters as in
+    forward_varlen (low-rank: materialised w = zU).  Returns y [B,T,D]."""
+    lib = lib or load()
+    if kind == LOWRANK:
+        w, kind = lowrank_filters(P, z, U, lib), HEADWISE
+    y = _out((P.B, P.T, P.D))
+    xp = _halo(x_prev, P.B, P.W, P.D) if P.W > 1 else None
+    lib.orc_forward_chunk(C.byref(P), kind, _in(ws if kind == STATIC else w), _in(x), _in(xp), _dp(y))
+    return y
+
+
+def backward_chunk(P: Problem, kind: int, x, dy, x_prev=None, dy_next=None, *, w=None, w_next=None, z=None,
+                   z_next=None, U=None, ws=None, lib=None):
+    """Gradients of forward_chunk.  dy_next [B,W-1,D] holds dy at positions
+    t0+T .. t0+T+W-2 and w_next [B,W-1,G,W] (head-wise) or z_next [B,W-1,R]
+    (low-rank) the filters of those tokens; None for the last chunk.
+    Returns (dx, dw) head-wise, (dx, dws) static, (dx, dz, dU, dw) low-rank;
+    dU and dws sum over this chunk's tokens only."""
+    lib = lib or load()
+    lowrank = kind == LOWRANK
+    if lowrank:
+        w = lowrank_filters(P, z, U, lib)
+        if dy_next is not None and P.W > 1:
+            Pn = problem(P.B, P.W - 1, P.D, P.W, P.H, P.R, P.residual)
+            w_next = lowrank_filters(Pn, np.ascontiguousarray(z_next), U, lib)
+        kind = HEADWISE
+    xp = _halo(x_prev, P.B, P.W, P.D) if P.W > 1 else None
+    dyn = _halo(dy_next, P.B, P.W, P.D) if P.W > 1 else None
+    wn = np.ascontiguousarray(w_next) if (dyn is not None and kind == HEADWISE) else None
+    if dyn is not None and kind == HEADWISE and wn is None:
+        raise ValueError("dy_next needs the filters of the same tokens")
+    dx = _out((P.B, P.T, P.D))
+    dw = _out((P.D, P.W)) if kind == STATIC else _out((P.B, P.T, P.G, P.W))
+    lib.orc_backward_chunk(C.byref(P), kind, _in(ws if kind == STATIC else w), _in(x), _in(dy), _in(xp), _in(dyn),
+                           _in(wn), _dp(dx), _dp(dw))
     if not lowrank:
         return dx, dw
     dz = _out((P.B, P.T, P.R))

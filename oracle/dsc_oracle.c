@@ -373,3 +373,110 @@ void orc_backward_varlen(const orc_problem *P, int64_t kind, orc_in w, orc_in x,
         }
     }
 }
+
+/* A chunk of longer sequences (context parallelism, the sequence split along
+ * time over ranks): row b holds tokens [t0, t0+T) of sequence b.  The
+ * definition is unchanged; only the values outside the chunk come from its
+ * neighbours instead of being zero:
+ *   xp  [B, W-1, D]: x at positions t0-W+1 .. t0-1 (row j = position
+ *        t0-W+1+j, the decode state's layout), or NULL when t0 = 0;
+ *   dyn [B, W-1, D]: dy at positions t0+T .. t0+T+W-2 (row j = t0+T+j), and
+ *   wn  [B, W-1, G, W]: the head-wise filters of those tokens (low-rank: the
+ *        materialised zU), both NULL for the sequence's last chunk.
+ * With a chunk index u relative to t0 (so u < 0 is in xp, u >= T in dyn):
+ *   y[b,t,c]   = r*x_t + sum_k w(t)_k x_{t-k}
+ *   dx[b,s,c]  = r*dy_s + sum_k w(s+k)_k dy_{s+k}
+ *   dw[b,t,g,k] = sum_{c in g} dy_t x_{t-k};  dws[c,k] = sum_{b,t} dy_t x_{t-k}
+ * where x, dy and w at indices outside the chunk read the halos (terms with
+ * no halo are absent, as in the zero-padded definition). */
+typedef struct {
+    orc_in xp, dyn, wn;
+} orc_halo;
+
+static int x_ext(const orc_problem *P, orc_in x, const orc_halo *h, int64_t b, int64_t u, int64_t c, double *v)
+{
+    if (u >= 0) {
+        *v = xval(P, x, b, u, c);
+        return 1;
+    }
+    if (!h->xp.p) return 0;
+    *v = val(h->xp, (b * (P->W - 1) + (u + P->W - 1)) * P->D + c);
+    return 1;
+}
+
+static int dy_ext(const orc_problem *P, orc_in dy, const orc_halo *h, int64_t b, int64_t u, int64_t c, double *v)
+{
+    if (u < P->T) {
+        *v = xval(P, dy, b, u, c);
+        return 1;
+    }
+    if (!h->dyn.p) return 0;
+    *v = val(h->dyn, (b * (P->W - 1) + (u - P->T)) * P->D + c);
+    return 1;
+}
+
+static double tap_ext(const orc_problem *P, const orc_filter *F, const orc_halo *h, int64_t b, int64_t u, int64_t c,
+                      int64_t k)
+{
+    if (u < P->T || F->kind == ORC_STATIC) return tap(P, F, b, u, c, k);
+    const int64_t G = P->D / P->H;
+    return val(h->wn, ((b * (P->W - 1) + (u - P->T)) * G + c / P->H) * P->W + k);
+}
+
+void orc_forward_chunk(const orc_problem *P, int64_t kind, orc_in w, orc_in x, orc_in xp, double *y_out)
+{
+    orc_filter F = {kind, w, {0, 0}, {0, 0}};
+    orc_halo h = {xp, {0, 0}, {0, 0}};
+    int64_t NT = P->B * P->T;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < NT; ++n) {
+        const int64_t b = n / P->T, t = n % P->T;
+        for (int64_t c = 0; c < P->D; ++c) {
+            double s = P->residual ? xval(P, x, b, t, c) : 0.0, xv;
+            for (int64_t k = 0; k < P->W; ++k)
+                if (x_ext(P, x, &h, b, t - k, c, &xv)) s += tap(P, &F, b, t, c, k) * xv;
+            y_out[n * P->D + c] = s;
+        }
+    }
+}
+
+void orc_backward_chunk(const orc_problem *P, int64_t kind, orc_in w, orc_in x, orc_in dy, orc_in xp, orc_in dyn,
+                        orc_in wn, double *dx_out, double *dw_out)
+{
+    orc_filter F = {kind, w, {0, 0}, {0, 0}};
+    orc_halo h = {xp, dyn, wn};
+    const int64_t NT = P->B * P->T, G = P->D / P->H;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < NT; ++n) {
+        const int64_t b = n / P->T, s = n % P->T;
+        for (int64_t c = 0; c < P->D; ++c) {
+            double acc = P->residual ? xval(P, dy, b, s, c) : 0.0, d;
+            for (int64_t k = 0; k < P->W; ++k)
+                if (dy_ext(P, dy, &h, b, s + k, c, &d)) acc += tap_ext(P, &F, &h, b, s + k, c, k) * d;
+            dx_out[n * P->D + c] = acc;
+        }
+    }
+    if (kind == ORC_STATIC) {
+#pragma omp parallel for schedule(static)
+        for (int64_t c = 0; c < P->D; ++c)
+            for (int64_t k = 0; k < P->W; ++k) {
+                double acc = 0.0, xv;
+                for (int64_t b = 0; b < P->B; ++b)
+                    for (int64_t t = 0; t < P->T; ++t)
+                        if (x_ext(P, x, &h, b, t - k, c, &xv)) acc += xval(P, dy, b, t, c) * xv;
+                dw_out[c * P->W + k] = acc;
+            }
+    } else {
+#pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < NT; ++n) {
+            const int64_t b = n / P->T, t = n % P->T;
+            for (int64_t g = 0; g < G; ++g)
+                for (int64_t k = 0; k < P->W; ++k) {
+                    double acc = 0.0, xv;
+                    for (int64_t c = g * P->H; c < (g + 1) * P->H; ++c)
+                        if (x_ext(P, x, &h, b, t - k, c, &xv)) acc += xval(P, dy, b, t, c) * xv;
+                    dw_out[(n * G + g) * P->W + k] = acc;
+                }
+        }
+    }
+}

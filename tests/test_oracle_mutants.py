@@ -45,6 +45,17 @@ MUTANTS = {
                                               "if (s + k < P->T) acc += tap(P, &F, 0, s + k, c, k)"),
     "packed dw reaches across a document start": ("if (t - k >= start)\n                        for",
                                                   "if (t - k >= 0)\n                        for"),
+    "chunk halo rows read in reverse": ("*v = val(h->xp, (b * (P->W - 1) + (u + P->W - 1)) * P->D + c);",
+                                        "*v = val(h->xp, (b * (P->W - 1) + (-u - 1)) * P->D + c);"),
+    "chunk dx reads dy_next one row late": (
+        "*v = val(h->dyn, (b * (P->W - 1) + (u - P->T)) * P->D + c);",
+        "*v = val(h->dyn, (b * (P->W - 1) + (u - P->T + 1 < P->W - 1 ? u - P->T + 1 : u - P->T)) * P->D + c);"),
+    "chunk dx ignores the next tokens' filters": (
+        "if (u < P->T || F->kind == ORC_STATIC) return tap(P, F, b, u, c, k);",
+        "if (1) return tap(P, F, b, u < P->T ? u : P->T - 1, c, k);"),
+    "chunk dw ignores the halo": (
+        "for (int64_t c = g * P->H; c < (g + 1) * P->H; ++c)\n                        if (x_ext(",
+        "for (int64_t c = g * P->H; c < (g + 1) * P->H; ++c)\n                        if (t - k >= 0 && x_ext("),
 }
 
 
@@ -152,6 +163,36 @@ def _pins(lib):
         ok &= np.allclose(yp[:, sl], oracle.forward_headwise(pd, xs, ws_, lib=lib), atol=1e-12)
         ok &= np.allclose(dxp[:, sl], dxd, atol=1e-12) and np.allclose(dwp[:, sl], dwd, atol=1e-12)
     check("varlen", ok)
+
+    # time chunks with their neighbours' rows as halos against the whole sequence
+    # (a chunk shorter than W-1 makes the halo span two chunks)
+    Wc, lens = 3, (1, 4, 2)
+    pw = oracle.problem(B, T, D, Wc, H, 0, 1)
+    wc = rng.standard_normal((B, T, G, Wc))
+    yw = oracle.forward_headwise(pw, x, wc, lib=lib)
+    dxw, dww = oracle.backward_headwise(pw, x, wc, dy, lib=lib)
+
+    def rows(a, lo, hi):
+        out = np.zeros((B, hi - lo) + a.shape[2:])
+        s_, e_ = max(lo, 0), min(hi, T)
+        if s_ < e_:
+            out[:, s_ - lo:e_ - lo] = a[:, s_:e_]
+        return out
+
+    ok, t0 = True, 0
+    for i, n in enumerate(lens):
+        t1 = t0 + n
+        pc = oracle.problem(B, n, D, Wc, H, 0, 1)
+        xc, dyc, wcc = (np.ascontiguousarray(a[:, t0:t1]) for a in (x, dy, wc))
+        xp = None if i == 0 else rows(x, t0 - Wc + 1, t0)
+        last = i == len(lens) - 1
+        dyn, wn = (None, None) if last else (rows(dy, t1, t1 + Wc - 1), rows(wc, t1, t1 + Wc - 1))
+        yc = oracle.forward_chunk(pc, oracle.HEADWISE, xc, xp, w=wcc, lib=lib)
+        dxc, dwc = oracle.backward_chunk(pc, oracle.HEADWISE, xc, dyc, xp, dyn, w=wcc, w_next=wn, lib=lib)
+        ok &= np.allclose(yc, yw[:, t0:t1], atol=1e-12) and np.allclose(dxc, dxw[:, t0:t1], atol=1e-12)
+        ok &= np.allclose(dwc, dww[:, t0:t1], atol=1e-12)
+        t0 = t1
+    check("chunks", ok)
     return fails
 
 

@@ -462,3 +462,120 @@ def test_varlen_one_document_is_the_plain_op(kind):
     np.testing.assert_array_equal(oracle.forward_varlen(Pp, kind, x, [0, T], **f), y)
     for a, b in zip(oracle.backward_varlen(Pp, kind, x, dy, [0, T], **f), g):
         np.testing.assert_array_equal(a, b)
+
+
+# ------------------------------------------------- sequence chunks (halos) ---
+# Context parallelism splits each sequence along time; a chunk's result needs
+# the W-1 inputs before it (x_prev) and, in the backward, dy and the filters
+# of the W-1 tokens after it.  Pinned against the whole-sequence oracle: the
+# chunks, each with its neighbours' rows as halos, give the whole sequence's
+# outputs row for row, and their token reductions sum to its dU / dws.
+
+CHUNK_CASES = [
+    # kind, B, chunk lengths, D, W, H, R, residual
+    (oracle.HEADWISE, 2, (5, 4, 6), 6, 4, 2, 0, 1),
+    (oracle.HEADWISE, 1, (2, 1, 3, 5), 4, 5, 1, 0, 0),   # chunks shorter than W-1: halos span several chunks
+    (oracle.HEADWISE, 2, (7, 7), 8, 1, 4, 0, 1),         # W = 1: no halo at all
+    (oracle.LOWRANK, 2, (4, 6, 3), 8, 3, 4, 3, 1),
+    (oracle.LOWRANK, 1, (1, 2, 6), 6, 4, 1, 2, 1),
+    (oracle.STATIC, 2, (3, 5, 4), 5, 4, 1, 0, 1),
+    (oracle.STATIC, 1, (2, 2, 2, 3), 3, 6, 1, 0, 0),
+]
+
+
+def _chunk_inputs(kind, B, L, D, W, H, R):
+    G = D // H
+    f = {}
+    if kind == oracle.HEADWISE:
+        f["w"] = rand(B, L, G, W)
+    elif kind == oracle.LOWRANK:
+        f["z"], f["U"] = rand(B, L, R), rand(R, G * W)
+    else:
+        f["ws"] = rand(D, W)
+    return rand(B, L, D), rand(B, L, D), f
+
+
+def _rows(a, lo, hi):
+    """Rows lo .. hi-1 of a [B, L, ...] array, zero where outside [0, L)."""
+    B, L = a.shape[:2]
+    out = np.zeros((B, hi - lo) + a.shape[2:])
+    s, e = max(lo, 0), min(hi, L)
+    if s < e:
+        out[:, s - lo:e - lo] = a[:, s:e]
+    return out
+
+
+@pytest.mark.parametrize("kind,B,lens,D,W,H,R,residual", CHUNK_CASES)
+def test_chunks_with_halos_equal_the_whole_sequence(kind, B, lens, D, W, H, R, residual):
+    L = sum(lens)
+    x, dy, f = _chunk_inputs(kind, B, L, D, W, H, R)
+    Pl = P(B, L, D, W, H, R, residual)
+    y_full, g_full = _plain(kind, Pl, x, dy, f)
+    starts = np.concatenate([[0], np.cumsum(lens)])
+    total = None
+    for i, n in enumerate(lens):
+        t0, t1 = starts[i], starts[i + 1]
+        Pc = P(B, n, D, W, H, R, residual)
+        xc, dyc = np.ascontiguousarray(x[:, t0:t1]), np.ascontiguousarray(dy[:, t0:t1])
+        first, last = i == 0, i == len(lens) - 1
+        x_prev = None if first else _rows(x, t0 - (W - 1), t0)
+        dy_next = None if last else _rows(dy, t1, t1 + W - 1)
+        kw = {}
+        if kind == oracle.HEADWISE:
+            kw = dict(w=np.ascontiguousarray(f["w"][:, t0:t1]),
+                      w_next=None if last else _rows(f["w"], t1, t1 + W - 1))
+        elif kind == oracle.LOWRANK:
+            kw = dict(z=np.ascontiguousarray(f["z"][:, t0:t1]), U=f["U"],
+                      z_next=None if last else _rows(f["z"], t1, t1 + W - 1))
+        else:
+            kw = dict(ws=f["ws"])
+        fwd_kw = {k: v for k, v in kw.items() if k not in ("w_next", "z_next")}
+        yc = oracle.forward_chunk(Pc, kind, xc, x_prev, **fwd_kw)
+        gc = oracle.backward_chunk(Pc, kind, xc, dyc, x_prev, dy_next, **kw)
+        np.testing.assert_array_equal(yc, y_full[:, t0:t1])
+        np.testing.assert_array_equal(gc[0], g_full[0][:, t0:t1])  # dx
+        if kind == oracle.HEADWISE:
+            np.testing.assert_array_equal(gc[1], g_full[1][:, t0:t1])  # dw
+        elif kind == oracle.LOWRANK:
+            np.testing.assert_allclose(gc[1], g_full[1][:, t0:t1], rtol=0, atol=1e-12)  # dz
+            np.testing.assert_array_equal(gc[3], g_full[3][:, t0:t1])  # dw
+            total = gc[2] if total is None else total + gc[2]
+        else:
+            total = gc[1] if total is None else total + gc[1]
+    if kind == oracle.LOWRANK:
+        np.testing.assert_allclose(total, g_full[2], rtol=0, atol=1e-11)  # dU
+    elif kind == oracle.STATIC:
+        np.testing.assert_allclose(total, g_full[1], rtol=0, atol=1e-11)  # dws
+
+
+@pytest.mark.parametrize("kind", [oracle.HEADWISE, oracle.LOWRANK, oracle.STATIC])
+def test_chunk_without_halos_is_the_plain_op(kind):
+    B, T, D, W, H, R = 2, 9, 6, 4, 3, 2
+    x, dy, f = _chunk_inputs(kind, B, T, D, W, H, R)
+    Pp = P(B, T, D, W, H, R, 1)
+    y, g = _plain(kind, Pp, x, dy, f)
+    np.testing.assert_array_equal(oracle.forward_chunk(Pp, kind, x, None, **f), y)
+    for a, b in zip(oracle.backward_chunk(Pp, kind, x, dy, None, None, **f), g):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_chunk_halo_rows_are_read_at_their_positions():
+    """A delta filter on tap j makes y_t = x_t + x_{t-j}: at the chunk's first
+    tokens that reads halo row W-1-j+t, and dx at its last tokens reads dy_next
+    row t+j-T (checked by hand-indexing, W = 4, one channel)."""
+    W, T = 4, 3
+    for j in range(1, W):
+        w = np.zeros((1, T, 1, W))
+        w[..., j] = 1.0
+        x, xp = rand(1, T, 1), rand(1, W - 1, 1)
+        y = oracle.forward_chunk(P(1, T, 1, W), oracle.HEADWISE, x, xp, w=w)
+        for t in range(T):
+            src = x[0, t - j, 0] if t - j >= 0 else xp[0, W - 1 + t - j, 0]
+            assert y[0, t, 0] == x[0, t, 0] + src
+        dy, dyn = rand(1, T, 1), rand(1, W - 1, 1)
+        wn = np.zeros((1, W - 1, 1, W))
+        wn[..., j] = 1.0
+        dx, _ = oracle.backward_chunk(P(1, T, 1, W), oracle.HEADWISE, x, dy, xp, dyn, w=w, w_next=wn)
+        for s in range(T):
+            src = dy[0, s + j, 0] if s + j < T else dyn[0, s + j - T, 0]
+            assert dx[0, s, 0] == dy[0, s, 0] + src
