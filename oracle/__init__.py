@@ -301,3 +301,41 @@ def backward_chunk(P: Problem, kind: int, x, dy, x_prev=None, dy_next=None, *, w
     dU = _out((P.R, P.G * P.W))
     lib.orc_lowrank_grads(C.byref(P), _in(z), _in(U), _dp(dw), _dp(dz), _dp(dU))
     return dx, dz, dU, dw
+
+
+# ------------------------------------------------ the first projection z = hV ---
+# Technical summary, Methodology, "Parameterisation" 1: the filter is a linear
+# map of the current hidden state, factorised at rank R, w(t) = h_t V U with
+# V [d_model, R] and U [R, G*W].  The library's projection calls take h
+# [B,T,d_model] and V and form z = hV themselves; the oracle evaluates the
+# same composition in fp64: z = hV (a plain matrix product), then the pinned
+# low-rank oracle with that z, and the gradients of h and V through the chain
+# rule, dh = dz V^T and dV = sum over tokens of h^T dz.
+
+def _f64(a, dtype_hint=None):
+    import synth
+
+    a = np.asarray(a)
+    if a.dtype == np.uint16:
+        return synth.bf16_bits_to_f32(a).astype(np.float64)
+    return a.astype(np.float64)
+
+
+def projection(h, V) -> np.ndarray:
+    """z [B,T,R] = h [B,T,d_model] . V [d_model,R] in fp64."""
+    return np.einsum("btd,dr->btr", _f64(h), _f64(V))
+
+
+def forward_lowrank_proj(P: Problem, x, h, V, U, lib=None):
+    """Returns (y [B,T,D], z [B,T,R]) with z = hV exact in fp64."""
+    z = np.ascontiguousarray(projection(h, V))
+    return forward_lowrank(P, x, z, U, lib), z
+
+
+def backward_lowrank_proj(P: Problem, x, h, V, U, dy, lib=None):
+    """Returns (dx, dh [B,T,d_model], dV [d_model,R], dU [R,G*W], dz)."""
+    z = np.ascontiguousarray(projection(h, V))
+    dx, dz, dU, _ = backward_lowrank(P, x, z, U, dy, lib)
+    dh = np.einsum("btr,dr->btd", dz, _f64(V))
+    dV = np.einsum("btd,btr->dr", _f64(h), dz)
+    return dx, dh, dV, dU, dz

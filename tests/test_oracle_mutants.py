@@ -210,3 +210,47 @@ def test_pins_catch_mutant(name, tmp_path):
     path.write_text(src.replace(old, new))
     lib = oracle.load(oracle.build(force=True, src=str(path), out=str(tmp_path / "mutant.so")))
     assert _pins(lib), f"no pin caught the mutant '{name}'"
+
+
+# The first projection's oracle is numpy (oracle.forward_lowrank_proj /
+# backward_lowrank_proj); its planted mistakes are swapped-in functions.
+PROJ_MUTANTS = {
+    "projection reads V's rows in reverse": lambda h, V: np.einsum("btd,dr->btr", oracle._f64(h), oracle._f64(V)[::-1]),
+    "projection drops the last model dimension": lambda h, V: np.einsum("btd,dr->btr", oracle._f64(h)[..., :-1],
+                                                                        oracle._f64(V)[:-1]),
+}
+
+
+def _proj_pins_pass(monkeypatch, mutant):
+    if mutant is not None:
+        monkeypatch.setattr(oracle, "projection", mutant)
+    rng = np.random.default_rng(9)
+    B, T, D, W, H, R, dm = 1, 5, 4, 3, 1, 3, 3
+    x, dy, h = rng.standard_normal((B, T, D)), rng.standard_normal((B, T, D)), rng.standard_normal((B, T, dm))
+    V, U = rng.standard_normal((dm, R)), rng.standard_normal((R, (D // H) * W))
+    p = oracle.problem(B, T, D, W, H, R, 1)
+    dx, dh, dV, dU, _ = oracle.backward_lowrank_proj(p, x, h, V, U, dy)
+    ok = True
+    for arg, grad in ((h, dh), (V, dV)):
+        a, g = arg.reshape(-1), grad.reshape(-1)
+        for i in range(a.size):
+            o = a[i]
+            a[i] = o + 0.5
+            lp = np.sum(dy * oracle.forward_lowrank_proj(p, x, h, V, U)[0])
+            a[i] = o - 0.5
+            lm = np.sum(dy * oracle.forward_lowrank_proj(p, x, h, V, U)[0])
+            a[i] = o
+            ok &= abs(lp - lm - g[i]) <= 1e-9 * (1 + abs(g[i]))
+    # identity V reduces to the plain low-rank op
+    y, z = oracle.forward_lowrank_proj(p, x, h, np.eye(dm), U)  # dm == R here
+    ok &= np.array_equal(z, h)
+    return ok
+
+
+def test_projection_pins_pass_unmutated(monkeypatch):
+    assert _proj_pins_pass(monkeypatch, None)
+
+
+@pytest.mark.parametrize("name", sorted(PROJ_MUTANTS))
+def test_projection_pins_catch_mutant(name, monkeypatch):
+    assert not _proj_pins_pass(monkeypatch, PROJ_MUTANTS[name])

@@ -579,3 +579,36 @@ def test_chunk_halo_rows_are_read_at_their_positions():
         for s in range(T):
             src = dy[0, s + j, 0] if s + j < T else dyn[0, s + j - T, 0]
             assert dx[0, s, 0] == dy[0, s, 0] + src
+
+
+# ------------------------------------------------ first projection z = hV ---
+
+@pytest.mark.parametrize("B,T,D,W,H,R,dm", [(1, 6, 4, 3, 1, 2, 5), (2, 5, 6, 2, 3, 3, 4)])
+def test_projection_gradients_by_exact_differences(B, T, D, W, H, R, dm):
+    """L = <dy, y> is linear in h and in V separately (z = hV, y linear in z),
+    so central differences give dh and dV exactly (up to fp64 rounding)."""
+    G = D // H
+    x, dy, h = rand(B, T, D), rand(B, T, D), rand(B, T, dm)
+    V, U = rand(dm, R), rand(R, G * W)
+    Pp = P(B, T, D, W, H, R)
+    dx, dh, dV, dU, dz = oracle.backward_lowrank_proj(Pp, x, h, V, U, dy)
+    loss = lambda: float(np.sum(dy * oracle.forward_lowrank_proj(Pp, x, h, V, U)[0]))  # noqa: E731
+    _loss_grad_check(loss, h, dh)
+    _loss_grad_check(loss, V, dV)
+    _loss_grad_check(loss, U, dU)
+    _loss_grad_check(loss, x, dx)
+
+
+def test_projection_with_identity_V_is_the_plain_lowrank_op():
+    B, T, D, W, H, R = 2, 7, 6, 3, 2, 4
+    G = D // H
+    x, dy, h, U = rand(B, T, D), rand(B, T, D), rand(B, T, R), rand(R, G * W)
+    Pp = P(B, T, D, W, H, R)
+    y, z = oracle.forward_lowrank_proj(Pp, x, h, np.eye(R), U)
+    np.testing.assert_array_equal(z, h)
+    np.testing.assert_array_equal(y, oracle.forward_lowrank(Pp, x, h, U))
+    dx, dh, dV, dU, dz = oracle.backward_lowrank_proj(Pp, x, h, np.eye(R), U, dy)
+    dxl, dzl, dUl, _ = oracle.backward_lowrank(Pp, x, h, U, dy)
+    np.testing.assert_array_equal(dx, dxl)
+    np.testing.assert_array_equal(dh, dzl)
+    np.testing.assert_array_equal(dU, dUl)
