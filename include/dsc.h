@@ -201,6 +201,124 @@ DSC_API dsc_status dsc_decode_lowrank(const dsc_problem *p, const void *x, const
  * prompt's outputs come from the training forward (dsc_fwd_*). */
 DSC_API dsc_status dsc_decode_state(const dsc_problem *p, const void *x, void *state, void *stream);
 
+/* ------------------------------------------------------ packed documents ---
+ * Variable-length batches ("Dynamic Short Convolutions Improve Transformers",
+ * technical summary, Methodology, "Mechanism": the convolution is causal
+ * within a sequence, so every document starts from zero history).
+ * p->B must be 1: the single row of p->T tokens holds n_docs documents,
+ * document d spanning tokens [cu_seqlens[d], cu_seqlens[d+1]).
+ *  - cu_seqlens: DEVICE array of n_docs + 1 int32 offsets rising from
+ *    cu_seqlens[0] = 0 to cu_seqlens[n_docs] = T, every document at least
+ *    one token long; 4-byte aligned (else DSC_ERR_MISALIGNED).  The offsets
+ *    are read on the device only: values outside [0, T] are clamped, so a
+ *    malformed array gives wrong results but no access out of bounds.
+ *  - 1 <= n_docs <= T, else DSC_ERR_INVALID_ARG.
+ * Per document the result is the single-sequence op of the calls above:
+ *   y[t]  = r x_t + sum_{k, t-k >= start(t)} w(t)_k x_{t-k}
+ *   dx[s] = r dy_s + sum_{k, s+k < end(s)} w(s+k)_k dy_{s+k}
+ *   dw[t,g,k] (and dws, dz, dU through it) has no term with t-k < start(t);
+ * dU and dws sum over every document.  Each call runs the plain kernels on
+ * the row, then recomputes the outputs within W-1 tokens of a document
+ * boundary (cost O(n_docs * W * D)).  Arguments, layouts and the remaining
+ * errors as in the plain calls. */
+DSC_API dsc_status dsc_fwd_headwise_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs,
+                                           const void *x, const void *w, void *y, void *stream);
+DSC_API dsc_status dsc_bwd_headwise_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs,
+                                           const void *x, const void *w, const void *dy, void *dx, void *dw,
+                                           void *stream);
+/* workspace: as for dsc_fwd_lowrank. */
+DSC_API dsc_status dsc_fwd_lowrank_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs,
+                                          const void *x, const void *z, const void *U, void *y, void *workspace,
+                                          size_t workspace_bytes, void *stream);
+/* The plain backward's workspace plus 2 * n_docs * (W-1) * G * W fp32 for
+ * the dw rows of the tokens next to a document start. */
+DSC_API size_t dsc_bwd_lowrank_varlen_workspace_bytes(const dsc_problem *p, int64_t n_docs);
+DSC_API dsc_status dsc_bwd_lowrank_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs,
+                                          const void *x, const void *z, const void *U, const void *dy, void *dx,
+                                          void *dz, float *dU, void *workspace, size_t workspace_bytes,
+                                          void *stream);
+DSC_API dsc_status dsc_fwd_static_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs,
+                                         const void *x, const void *ws, void *y, void *stream);
+/* workspace: dsc_bwd_static_workspace_bytes(p). */
+DSC_API dsc_status dsc_bwd_static_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs,
+                                         const void *x, const void *ws, const void *dy, void *dx, float *dws,
+                                         void *workspace, size_t workspace_bytes, void *stream);
+
+/* -------------------------------------------------------- sequence chunks ---
+ * Context parallelism: the sequences are split along time and each call
+ * handles one chunk, tokens [t0, t0 + T) of every sequence (p->T = chunk
+ * length, row b = sequence b).  The convolution reaches W-1 tokens across a
+ * chunk edge, so a chunk takes its neighbours' rows (the halos):
+ *  - x_prev  [B, W-1, D]: x at positions t0-W+1 .. t0-1 (row j = position
+ *    t0-W+1+j, zero rows for positions before the sequence start -- the
+ *    decode state's layout); NULL for a sequence's first chunk;
+ *  - dy_next [B, W-1, D]: dy at positions t0+T .. t0+T+W-2 (row j = position
+ *    t0+T+j, zero rows past the sequence end), with the filters of the same
+ *    tokens: head-wise w_next [B, W-1, G, W], low-rank z_next [B, W-1, R]
+ *    (static filters are the same everywhere); NULL for the last chunk.
+ * Halos are DEVICE pointers in the dtype of x, 16-byte aligned (else
+ * DSC_ERR_MISALIGNED); a dy_next without its filters is DSC_ERR_INVALID_ARG.
+ * Results: the rows [t0, t0+T) of the op on the whole sequences; dU and dws
+ * sum over this chunk's tokens only (sum them over the chunks).
+ * edges_only = 0: the whole call.  edges_only = 1: only the outputs within
+ * W-1 tokens of the chunk's edges are recomputed (and dU / dws corrected);
+ * the output buffers must already hold the plain call's results on the same
+ * inputs (dsc_fwd_headwise etc.), so a caller can run the plain call while
+ * the halos are still being exchanged.  For W = 1 the halos are ignored. */
+DSC_API dsc_status dsc_fwd_headwise_chunk(const dsc_problem *p, const void *x_prev, const void *x, const void *w,
+                                          void *y, int edges_only, void *stream);
+DSC_API dsc_status dsc_bwd_headwise_chunk(const dsc_problem *p, const void *x_prev, const void *dy_next,
+                                          const void *w_next, const void *x, const void *w, const void *dy, void *dx,
+                                          void *dw, int edges_only, void *stream);
+/* workspace: as for dsc_fwd_lowrank (not used when edges_only = 1). */
+DSC_API dsc_status dsc_fwd_lowrank_chunk(const dsc_problem *p, const void *x_prev, const void *x, const void *z,
+                                         const void *U, void *y, void *workspace, size_t workspace_bytes,
+                                         int edges_only, void *stream);
+/* The plain backward's workspace plus 2 * B * (W-1) * G * W fp32. */
+DSC_API size_t dsc_bwd_lowrank_chunk_workspace_bytes(const dsc_problem *p);
+DSC_API dsc_status dsc_bwd_lowrank_chunk(const dsc_problem *p, const void *x_prev, const void *dy_next,
+                                         const void *z_next, const void *x, const void *z, const void *U,
+                                         const void *dy, void *dx, void *dz, float *dU, void *workspace,
+                                         size_t workspace_bytes, int edges_only, void *stream);
+DSC_API dsc_status dsc_fwd_static_chunk(const dsc_problem *p, const void *x_prev, const void *x, const void *ws,
+                                        void *y, int edges_only, void *stream);
+/* workspace: dsc_bwd_static_workspace_bytes(p) (may be NULL when edges_only = 1). */
+DSC_API dsc_status dsc_bwd_static_chunk(const dsc_problem *p, const void *x_prev, const void *dy_next, const void *x,
+                                        const void *ws, const void *dy, void *dx, float *dws, void *workspace,
+                                        size_t workspace_bytes, int edges_only, void *stream);
+
+/* ------------------------------------------------- first projection z = hV ---
+ * The filter generator is a linear map of the current hidden state factorised
+ * at rank R ("Dynamic Short Convolutions Improve Transformers", technical
+ * summary, Methodology, "Parameterisation" 1): w(t) = h_t V U, with h
+ * [B, T, d_model], V [d_model, R] and U [R, G*W].  These calls take h and V
+ * and form z = h V themselves (tensor cores for bf16 with R a multiple of 8
+ * up to 64 and d_model a multiple of 128, CUDA cores otherwise; fp32
+ * accumulation), then run the low-rank convolution on it.  h and V are in
+ * the dtype of x; 1 <= d_model <= 2^30 else DSC_ERR_INVALID_ARG. */
+
+/* Workspace of dsc_fwd_lowrank_proj (that of dsc_fwd_lowrank). */
+DSC_API size_t dsc_fwd_lowrank_proj_workspace_bytes(const dsc_problem *p, int64_t d_model);
+
+/* Forward: z [B,T,R] = h V (written: the backward takes it), then y as
+ * dsc_fwd_lowrank with that z. */
+DSC_API dsc_status dsc_fwd_lowrank_proj(const dsc_problem *p, int64_t d_model, const void *x, const void *h,
+                                        const void *V, const void *U, void *z, void *y, void *workspace,
+                                        size_t workspace_bytes, void *stream);
+
+/* Workspace of dsc_bwd_lowrank_proj: dz, the low-rank backward's workspace
+ * and per-token-range partial sums of dV (never NULL). */
+DSC_API size_t dsc_bwd_lowrank_proj_workspace_bytes(const dsc_problem *p, int64_t d_model);
+
+/* Backward, from the forward's z: dx [B,T,D], dh [B,T,d_model] = dz V^T (dtype
+ * of x), dV [d_model,R] = sum over tokens of h^T dz (fp32) and dU [R,G*W]
+ * (fp32), dz being the low-rank backward's gradient of z (kept in the
+ * workspace).  dV and dU are overwritten; both are deterministic. */
+DSC_API dsc_status dsc_bwd_lowrank_proj(const dsc_problem *p, int64_t d_model, const void *x, const void *h,
+                                        const void *V, const void *z, const void *U, const void *dy, void *dx,
+                                        void *dh, float *dV, float *dU, void *workspace, size_t workspace_bytes,
+                                        void *stream);
+
 /* Synchronise `stream`, then return and clear the device status word of the
  * current device: DSC_OK, DSC_ERR_TIMEOUT, or DSC_ERR_CUDA if the stream
  * reported an error. */

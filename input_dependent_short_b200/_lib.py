@@ -47,6 +47,24 @@ _SIGS = {
     "dsc_bwd_static_workspace_bytes": (C.c_size_t, [_P]),
     "dsc_bwd_static": (C.c_int, [_P, _v, _v, _v, _v, _v, _v, C.c_size_t, _v]),
     "dsc_bwd_static_noalloc": (C.c_int, [_P, _v, _v, _v, _v, _v, _v]),
+    "dsc_fwd_headwise_varlen": (C.c_int, [_P, _v, C.c_int64, _v, _v, _v, _v]),
+    "dsc_bwd_headwise_varlen": (C.c_int, [_P, _v, C.c_int64, _v, _v, _v, _v, _v, _v]),
+    "dsc_fwd_lowrank_varlen": (C.c_int, [_P, _v, C.c_int64, _v, _v, _v, _v, _v, C.c_size_t, _v]),
+    "dsc_bwd_lowrank_varlen_workspace_bytes": (C.c_size_t, [_P, C.c_int64]),
+    "dsc_bwd_lowrank_varlen": (C.c_int, [_P, _v, C.c_int64, _v, _v, _v, _v, _v, _v, _v, _v, C.c_size_t, _v]),
+    "dsc_fwd_static_varlen": (C.c_int, [_P, _v, C.c_int64, _v, _v, _v, _v]),
+    "dsc_bwd_static_varlen": (C.c_int, [_P, _v, C.c_int64, _v, _v, _v, _v, _v, _v, C.c_size_t, _v]),
+    "dsc_fwd_headwise_chunk": (C.c_int, [_P, _v, _v, _v, _v, C.c_int, _v]),
+    "dsc_bwd_headwise_chunk": (C.c_int, [_P, _v, _v, _v, _v, _v, _v, _v, _v, C.c_int, _v]),
+    "dsc_fwd_lowrank_chunk": (C.c_int, [_P, _v, _v, _v, _v, _v, _v, C.c_size_t, C.c_int, _v]),
+    "dsc_bwd_lowrank_chunk_workspace_bytes": (C.c_size_t, [_P]),
+    "dsc_bwd_lowrank_chunk": (C.c_int, [_P, _v, _v, _v, _v, _v, _v, _v, _v, _v, _v, _v, C.c_size_t, C.c_int, _v]),
+    "dsc_fwd_static_chunk": (C.c_int, [_P, _v, _v, _v, _v, C.c_int, _v]),
+    "dsc_bwd_static_chunk": (C.c_int, [_P, _v, _v, _v, _v, _v, _v, _v, _v, C.c_size_t, C.c_int, _v]),
+    "dsc_fwd_lowrank_proj_workspace_bytes": (C.c_size_t, [_P, C.c_int64]),
+    "dsc_fwd_lowrank_proj": (C.c_int, [_P, C.c_int64, _v, _v, _v, _v, _v, _v, _v, C.c_size_t, _v]),
+    "dsc_bwd_lowrank_proj_workspace_bytes": (C.c_size_t, [_P, C.c_int64]),
+    "dsc_bwd_lowrank_proj": (C.c_int, [_P, C.c_int64, _v, _v, _v, _v, _v, _v, _v, _v, _v, _v, _v, C.c_size_t, _v]),
     "dsc_check": (C.c_int, [_v]),
     "dsc_selftest_timeout": (C.c_int, [_v]),
     "dsc_status_string": (C.c_char_p, [C.c_int]),

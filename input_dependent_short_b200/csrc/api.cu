@@ -328,6 +328,299 @@ dsc_status dsc_decode_state(const dsc_problem *p, const void *x, void *state, vo
     return done(launch_decode_state(ctx(stream), *p, x, state));
 }
 
+// ------------------------------------------- packed documents and chunks ---
+
+static size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
+
+static dsc_status check_varlen(const dsc_problem *p, const int32_t *cu, int64_t n_docs) {
+    if (p->B != 1 || n_docs < 1 || n_docs > p->T || !cu) return DSC_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(cu) & 3u) return DSC_ERR_MISALIGNED;
+    // the fix-up grids have one block per (edge row, 256 channels)
+    if (n_docs * (p->W - 1) * ((p->D + 255) / 256) >= ((int64_t)1 << 31)) return DSC_ERR_UNSUPPORTED;
+    return DSC_OK;
+}
+
+static dsc_status check_chunk(const dsc_problem *p) {
+    if (p->B * (p->W - 1) * ((p->D + 255) / 256) >= ((int64_t)1 << 31)) return DSC_ERR_UNSUPPORTED;
+    return DSC_OK;
+}
+
+// Halo pointers of a chunk: present ones must be 16-byte aligned; the filters
+// of the next tokens must come with their dy.
+static dsc_status check_halos(const dsc_problem *p, const void *x_prev, const void *dy_next, const void *f_next,
+                              bool needs_f) {
+    if (p->W < 2) return DSC_OK;
+    for (const void *q : {x_prev, dy_next, f_next})
+        if (q && !aligned16(q)) return DSC_ERR_MISALIGNED;
+    if (dy_next && needs_f && !f_next) return DSC_ERR_INVALID_ARG;
+    return DSC_OK;
+}
+
+static EdgeArgs varlen_edges(const dsc_problem &p, int kind, const int32_t *cu, int64_t n_docs) {
+    EdgeArgs a{};
+    edge_args(p, kind, a);
+    a.cu = cu;
+    a.nseg = n_docs;
+    return a;
+}
+
+static EdgeArgs chunk_edges(const dsc_problem &p, int kind, const void *x_prev, const void *dy_next,
+                            const void *f_next) {
+    EdgeArgs a{};
+    edge_args(p, kind, a);
+    a.cu = nullptr;
+    a.nseg = p.B;
+    if (p.W > 1) {
+        a.x_prev = x_prev;
+        a.dy_next = dy_next;
+        a.f_next = f_next;
+    }
+    return a;
+}
+
+static dsc_status edges_fwd(void *stream, const dsc_problem *p, EdgeArgs a) {
+    if (a.nseg < 1 || p->W < 2) return DSC_OK;
+    if (!a.cu && !a.x_prev) return DSC_OK;  // a sequence's first chunk: the plain call is the whole result
+    return done(launch_edges_fwd(ctx(stream), *p, a));
+}
+
+static dsc_status edges_bwd(void *stream, const dsc_problem *p, EdgeArgs a) {
+    if (a.nseg < 1 || p->W < 2) return DSC_OK;
+    if (!a.cu && !a.x_prev && !a.dy_next) return DSC_OK;
+    return done(launch_edges_bwd(ctx(stream), *p, a));
+}
+
+dsc_status dsc_fwd_headwise_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs, const void *x,
+                                   const void *w, void *y, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_varlen(p, cu_seqlens, n_docs);
+    if (s == DSC_OK) s = dsc_fwd_headwise(p, x, w, y, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = varlen_edges(*p, EDGE_HEADWISE, cu_seqlens, n_docs);
+    a.x = x; a.w = w; a.y = y;
+    return edges_fwd(stream, p, a);
+}
+
+dsc_status dsc_bwd_headwise_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs, const void *x,
+                                   const void *w, const void *dy, void *dx, void *dw, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_varlen(p, cu_seqlens, n_docs);
+    if (s == DSC_OK) s = dsc_bwd_headwise(p, x, w, dy, dx, dw, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = varlen_edges(*p, EDGE_HEADWISE, cu_seqlens, n_docs);
+    a.x = x; a.w = w; a.dy = dy; a.dx = dx; a.dw = dw;
+    return edges_bwd(stream, p, a);
+}
+
+dsc_status dsc_fwd_lowrank_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs, const void *x,
+                                  const void *z, const void *U, void *y, void *workspace, size_t workspace_bytes,
+                                  void *stream) {
+    dsc_status s = validate(p, true);
+    if (s == DSC_OK) s = check_varlen(p, cu_seqlens, n_docs);
+    if (s == DSC_OK) s = dsc_fwd_lowrank(p, x, z, U, y, workspace, workspace_bytes, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = varlen_edges(*p, EDGE_LOWRANK, cu_seqlens, n_docs);
+    a.x = x; a.z = z; a.U = U; a.y = y;
+    return edges_fwd(stream, p, a);
+}
+
+size_t dsc_bwd_lowrank_varlen_workspace_bytes(const dsc_problem *p, int64_t n_docs) {
+    if (validate(p, true) != DSC_OK || n_docs < 1) return 0;
+    return up256(dsc_bwd_lowrank_workspace_bytes(p)) + edge_scratch_bytes(*p, EDGE_LOWRANK, n_docs);
+}
+
+// Low-rank backward with fix-ups: the plain call's workspace first, then the
+// fix-up scratch (dw rows of the fixed tokens and their cross-edge part).
+static dsc_status lowrank_bwd_edges(const dsc_problem *p, EdgeArgs a, const void *x, const void *z, const void *U,
+                                    const void *dy, void *dx, void *dz, float *dU, void *workspace,
+                                    size_t workspace_bytes, size_t main_bytes, bool run_main, void *stream) {
+    const size_t edge = edge_scratch_bytes(*p, EDGE_LOWRANK, a.nseg);
+    const size_t off = run_main ? up256(main_bytes) : 0;
+    if ((off + edge) && (!workspace || workspace_bytes < off + edge)) return DSC_ERR_INVALID_ARG;
+    if ((off + edge) && !aligned16(workspace)) return DSC_ERR_MISALIGNED;
+    if (run_main) {
+        const dsc_status s = dsc_bwd_lowrank(p, x, z, U, dy, dx, dz, dU, main_bytes ? workspace : nullptr, main_bytes,
+                                             stream);
+        if (s != DSC_OK) return s;
+    }
+    a.x = x; a.z = z; a.U = U; a.dy = dy; a.dx = dx; a.dz = dz; a.dU = dU;
+    if (edge) {
+        a.dwfull = reinterpret_cast<float *>(static_cast<char *>(workspace) + off);
+        a.dwdelta = a.dwfull + edge / (2 * sizeof(float));
+    }
+    return edges_bwd(stream, p, a);
+}
+
+dsc_status dsc_bwd_lowrank_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs, const void *x,
+                                  const void *z, const void *U, const void *dy, void *dx, void *dz, float *dU,
+                                  void *workspace, size_t workspace_bytes, void *stream) {
+    dsc_status s = validate(p, true);
+    if (s == DSC_OK) s = check_varlen(p, cu_seqlens, n_docs);
+    if (s == DSC_OK) s = check_ptrs({x, z, U, dy, dx, dz, dU});
+    if (s != DSC_OK) return s;
+    return lowrank_bwd_edges(p, varlen_edges(*p, EDGE_LOWRANK, cu_seqlens, n_docs), x, z, U, dy, dx, dz, dU,
+                             workspace, workspace_bytes, dsc_bwd_lowrank_workspace_bytes(p), true, stream);
+}
+
+dsc_status dsc_fwd_static_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs, const void *x,
+                                 const void *ws, void *y, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_varlen(p, cu_seqlens, n_docs);
+    if (s == DSC_OK) s = dsc_fwd_static(p, x, ws, y, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = varlen_edges(*p, EDGE_STATIC, cu_seqlens, n_docs);
+    a.x = x; a.w = ws; a.y = y;
+    return edges_fwd(stream, p, a);
+}
+
+dsc_status dsc_bwd_static_varlen(const dsc_problem *p, const int32_t *cu_seqlens, int64_t n_docs, const void *x,
+                                 const void *ws, const void *dy, void *dx, float *dws, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_varlen(p, cu_seqlens, n_docs);
+    if (s == DSC_OK) s = dsc_bwd_static(p, x, ws, dy, dx, dws, workspace, workspace_bytes, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = varlen_edges(*p, EDGE_STATIC, cu_seqlens, n_docs);
+    a.x = x; a.w = ws; a.dy = dy; a.dx = dx; a.dws = dws;
+    return edges_bwd(stream, p, a);
+}
+
+dsc_status dsc_fwd_headwise_chunk(const dsc_problem *p, const void *x_prev, const void *x, const void *w, void *y,
+                                  int edges_only, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_chunk(p);
+    if (s == DSC_OK) s = check_ptrs({x, w, y});
+    if (s == DSC_OK) s = check_halos(p, x_prev, nullptr, nullptr, false);
+    if (s == DSC_OK && !edges_only) s = dsc_fwd_headwise(p, x, w, y, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = chunk_edges(*p, EDGE_HEADWISE, x_prev, nullptr, nullptr);
+    a.x = x; a.w = w; a.y = y;
+    return edges_fwd(stream, p, a);
+}
+
+dsc_status dsc_bwd_headwise_chunk(const dsc_problem *p, const void *x_prev, const void *dy_next, const void *w_next,
+                                  const void *x, const void *w, const void *dy, void *dx, void *dw, int edges_only,
+                                  void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_chunk(p);
+    if (s == DSC_OK) s = check_ptrs({x, w, dy, dx, dw});
+    if (s == DSC_OK) s = check_halos(p, x_prev, dy_next, w_next, true);
+    if (s == DSC_OK && !edges_only) s = dsc_bwd_headwise(p, x, w, dy, dx, dw, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = chunk_edges(*p, EDGE_HEADWISE, x_prev, dy_next, w_next);
+    a.x = x; a.w = w; a.dy = dy; a.dx = dx; a.dw = dw;
+    return edges_bwd(stream, p, a);
+}
+
+dsc_status dsc_fwd_lowrank_chunk(const dsc_problem *p, const void *x_prev, const void *x, const void *z, const void *U,
+                                 void *y, void *workspace, size_t workspace_bytes, int edges_only, void *stream) {
+    dsc_status s = validate(p, true);
+    if (s == DSC_OK) s = check_chunk(p);
+    if (s == DSC_OK) s = check_ptrs({x, z, U, y});
+    if (s == DSC_OK) s = check_halos(p, x_prev, nullptr, nullptr, false);
+    if (s == DSC_OK && !edges_only) s = dsc_fwd_lowrank(p, x, z, U, y, workspace, workspace_bytes, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = chunk_edges(*p, EDGE_LOWRANK, x_prev, nullptr, nullptr);
+    a.x = x; a.z = z; a.U = U; a.y = y;
+    return edges_fwd(stream, p, a);
+}
+
+size_t dsc_bwd_lowrank_chunk_workspace_bytes(const dsc_problem *p) {
+    if (validate(p, true) != DSC_OK) return 0;
+    return up256(dsc_bwd_lowrank_workspace_bytes(p)) + edge_scratch_bytes(*p, EDGE_LOWRANK, p->B);
+}
+
+dsc_status dsc_bwd_lowrank_chunk(const dsc_problem *p, const void *x_prev, const void *dy_next, const void *z_next,
+                                 const void *x, const void *z, const void *U, const void *dy, void *dx, void *dz,
+                                 float *dU, void *workspace, size_t workspace_bytes, int edges_only, void *stream) {
+    dsc_status s = validate(p, true);
+    if (s == DSC_OK) s = check_chunk(p);
+    if (s == DSC_OK) s = check_ptrs({x, z, U, dy, dx, dz, dU});
+    if (s == DSC_OK) s = check_halos(p, x_prev, dy_next, z_next, true);
+    if (s != DSC_OK) return s;
+    return lowrank_bwd_edges(p, chunk_edges(*p, EDGE_LOWRANK, x_prev, dy_next, z_next), x, z, U, dy, dx, dz, dU,
+                             workspace, workspace_bytes, dsc_bwd_lowrank_workspace_bytes(p), !edges_only, stream);
+}
+
+dsc_status dsc_fwd_static_chunk(const dsc_problem *p, const void *x_prev, const void *x, const void *ws, void *y,
+                                int edges_only, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_chunk(p);
+    if (s == DSC_OK) s = check_ptrs({x, ws, y});
+    if (s == DSC_OK) s = check_halos(p, x_prev, nullptr, nullptr, false);
+    if (s == DSC_OK && !edges_only) s = dsc_fwd_static(p, x, ws, y, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = chunk_edges(*p, EDGE_STATIC, x_prev, nullptr, nullptr);
+    a.x = x; a.w = ws; a.y = y;
+    return edges_fwd(stream, p, a);
+}
+
+dsc_status dsc_bwd_static_chunk(const dsc_problem *p, const void *x_prev, const void *dy_next, const void *x,
+                                const void *ws, const void *dy, void *dx, float *dws, void *workspace,
+                                size_t workspace_bytes, int edges_only, void *stream) {
+    dsc_status s = validate(p, false);
+    if (s == DSC_OK) s = check_chunk(p);
+    if (s == DSC_OK) s = check_ptrs({x, ws, dy, dx, dws});
+    if (s == DSC_OK) s = check_halos(p, x_prev, dy_next, nullptr, false);
+    if (s == DSC_OK && !edges_only) s = dsc_bwd_static(p, x, ws, dy, dx, dws, workspace, workspace_bytes, stream);
+    if (s != DSC_OK) return s;
+    EdgeArgs a = chunk_edges(*p, EDGE_STATIC, x_prev, dy_next, nullptr);
+    a.x = x; a.w = ws; a.dy = dy; a.dx = dx; a.dws = dws;
+    return edges_bwd(stream, p, a);
+}
+
+// ------------------------------------------------ first projection z = hV ---
+
+static dsc_status check_dmodel(int64_t d_model) {
+    return (d_model < 1 || d_model > ((int64_t)1 << 30)) ? DSC_ERR_INVALID_ARG : DSC_OK;
+}
+
+size_t dsc_fwd_lowrank_proj_workspace_bytes(const dsc_problem *p, int64_t d_model) {
+    if (validate(p, true) != DSC_OK || check_dmodel(d_model) != DSC_OK) return 0;
+    return dsc_fwd_lowrank_workspace_bytes(p);
+}
+
+dsc_status dsc_fwd_lowrank_proj(const dsc_problem *p, int64_t d_model, const void *x, const void *h, const void *V,
+                                const void *U, void *z, void *y, void *workspace, size_t workspace_bytes,
+                                void *stream) {
+    dsc_status s = validate(p, true);
+    if (s == DSC_OK) s = check_dmodel(d_model);
+    if (s == DSC_OK) s = check_ptrs({x, h, V, U, z, y});
+    if (s != DSC_OK) return s;
+    s = done(launch_proj_z(ctx(stream), *p, d_model, h, V, z));
+    if (s != DSC_OK) return s;
+    return dsc_fwd_lowrank(p, x, z, U, y, workspace, workspace_bytes, stream);
+}
+
+// Workspace of the backward with the projection: dz [B,T,R] (input dtype),
+// then the low-rank backward's workspace, then the dV partials.
+static size_t proj_dz_bytes(const dsc_problem &p) {
+    return up256((size_t)(p.B * p.T) * (size_t)p.R * (p.dtype == DSC_BF16 ? 2 : 4));
+}
+
+size_t dsc_bwd_lowrank_proj_workspace_bytes(const dsc_problem *p, int64_t d_model) {
+    if (validate(p, true) != DSC_OK || check_dmodel(d_model) != DSC_OK) return 0;
+    return proj_dz_bytes(*p) + up256(dsc_bwd_lowrank_workspace_bytes(p)) + proj_dV_part_bytes(*p, d_model, sm_count());
+}
+
+dsc_status dsc_bwd_lowrank_proj(const dsc_problem *p, int64_t d_model, const void *x, const void *h, const void *V,
+                                const void *z, const void *U, const void *dy, void *dx, void *dh, float *dV,
+                                float *dU, void *workspace, size_t workspace_bytes, void *stream) {
+    dsc_status s = validate(p, true);
+    if (s == DSC_OK) s = check_dmodel(d_model);
+    if (s == DSC_OK) s = check_ptrs({x, h, V, z, U, dy, dx, dh, dV, dU, workspace});
+    if (s != DSC_OK) return s;
+    if (workspace_bytes < dsc_bwd_lowrank_proj_workspace_bytes(p, d_model)) return DSC_ERR_INVALID_ARG;
+    char *w = static_cast<char *>(workspace);
+    void *dz = w;
+    const size_t main_bytes = dsc_bwd_lowrank_workspace_bytes(p);
+    void *wmain = w + proj_dz_bytes(*p);
+    float *part = reinterpret_cast<float *>(w + proj_dz_bytes(*p) + up256(main_bytes));
+    s = dsc_bwd_lowrank(p, x, z, U, dy, dx, dz, dU, main_bytes ? wmain : nullptr, main_bytes, stream);
+    if (s != DSC_OK) return s;
+    return done(launch_proj_bwd(ctx(stream), *p, d_model, h, V, dz, dh, dV, part));
+}
+
 dsc_status dsc_selftest_timeout(void *stream) {
     return launch_wait_selftest(static_cast<cudaStream_t>(stream)) == cudaSuccess ? DSC_OK : DSC_ERR_CUDA;
 }
@@ -337,8 +630,9 @@ dsc_status dsc_check(void *stream) {
     const int st = take_device_status(static_cast<cudaStream_t>(stream));
     const int st_tc = take_tc_status(static_cast<cudaStream_t>(stream));
     const int st_dec = take_tc_dec_status(static_cast<cudaStream_t>(stream));
-    if (st < 0 || st_tc < 0 || st_dec < 0) return DSC_ERR_CUDA;
-    return static_cast<dsc_status>(st ? st : (st_tc ? st_tc : st_dec));
+    const int st_pj = take_proj_status(static_cast<cudaStream_t>(stream));
+    if (st < 0 || st_tc < 0 || st_dec < 0 || st_pj < 0) return DSC_ERR_CUDA;
+    return static_cast<dsc_status>(st ? st : (st_tc ? st_tc : (st_dec ? st_dec : st_pj)));
 }
 
 }  // extern "C"

@@ -217,6 +217,228 @@ def dsc_check(device=None):
         call("dsc_check", _stream(dev))
 
 
+# ---------------------------------------------------------- packed documents ---
+# Variable-length batches: x [1, T, D] holds several documents back to back,
+# cu_seqlens (int32, on the device) their offsets; no tap crosses a document
+# boundary.
+
+def _cu(cu_seqlens, dev):
+    if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev or cu_seqlens.dim() != 1:
+        raise ValueError("cu_seqlens must be a 1-D int32 tensor on the tensors' device")
+    return cu_seqlens.contiguous(), cu_seqlens.numel() - 1
+
+
+def dsc_fwd_headwise_varlen(x, w, cu_seqlens, residual=True):
+    dev = _check(x, w, dtype=x.dtype)
+    cu, n = _cu(cu_seqlens, dev)
+    p = problem(x, w.shape[3], x.shape[2] // w.shape[2], 0, residual)
+    y = torch.empty_like(x)
+    with torch.cuda.device(dev):
+        call("dsc_fwd_headwise_varlen", p, _ptr(cu), n, _ptr(x), _ptr(w), _ptr(y), _stream(dev))
+    return y
+
+
+def dsc_bwd_headwise_varlen(x, w, dy, cu_seqlens, residual=True):
+    """Returns (dx, dw)."""
+    dev = _check(x, w, dy, dtype=x.dtype)
+    cu, n = _cu(cu_seqlens, dev)
+    p = problem(x, w.shape[3], x.shape[2] // w.shape[2], 0, residual)
+    dx, dw = torch.empty_like(x), torch.empty_like(w)
+    with torch.cuda.device(dev):
+        call("dsc_bwd_headwise_varlen", p, _ptr(cu), n, _ptr(x), _ptr(w), _ptr(dy), _ptr(dx), _ptr(dw), _stream(dev))
+    return dx, dw
+
+
+def dsc_fwd_lowrank_varlen(x, z, U, cu_seqlens, H=1, residual=True):
+    dev = _check(x, z, U, dtype=x.dtype)
+    cu, n = _cu(cu_seqlens, dev)
+    p = _lr_problem(x, z, U, H, residual)
+    y = torch.empty_like(x)
+    nb = lib().dsc_fwd_lowrank_workspace_bytes(p)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
+    with torch.cuda.device(dev):
+        call("dsc_fwd_lowrank_varlen", p, _ptr(cu), n, _ptr(x), _ptr(z), _ptr(U), _ptr(y), _ptr(ws), nb, _stream(dev))
+    return y
+
+
+def dsc_bwd_lowrank_varlen(x, z, U, dy, cu_seqlens, H=1, residual=True):
+    """Returns (dx, dz, dU); dU is fp32."""
+    dev = _check(x, z, U, dy, dtype=x.dtype)
+    cu, n = _cu(cu_seqlens, dev)
+    p = _lr_problem(x, z, U, H, residual)
+    dx, dz = torch.empty_like(x), torch.empty_like(z)
+    dU = torch.empty(U.shape, dtype=torch.float32, device=dev)
+    nb = lib().dsc_bwd_lowrank_varlen_workspace_bytes(p, n)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
+    with torch.cuda.device(dev):
+        call("dsc_bwd_lowrank_varlen", p, _ptr(cu), n, _ptr(x), _ptr(z), _ptr(U), _ptr(dy), _ptr(dx), _ptr(dz),
+             _ptr(dU), _ptr(ws), nb, _stream(dev))
+    return dx, dz, dU
+
+
+def dsc_fwd_static_varlen(x, ws, cu_seqlens, residual=False):
+    dev = _check(x, ws, dtype=x.dtype)
+    cu, n = _cu(cu_seqlens, dev)
+    p = problem(x, ws.shape[1], 1, 0, residual)
+    y = torch.empty_like(x)
+    with torch.cuda.device(dev):
+        call("dsc_fwd_static_varlen", p, _ptr(cu), n, _ptr(x), _ptr(ws), _ptr(y), _stream(dev))
+    return y
+
+
+def dsc_bwd_static_varlen(x, ws, dy, cu_seqlens, residual=False):
+    """Returns (dx, dws); dws is fp32."""
+    dev = _check(x, ws, dy, dtype=x.dtype)
+    cu, n = _cu(cu_seqlens, dev)
+    p = problem(x, ws.shape[1], 1, 0, residual)
+    dx = torch.empty_like(x)
+    dws = torch.empty(ws.shape, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        nb = lib().dsc_bwd_static_workspace_bytes(p)
+        scratch = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        call("dsc_bwd_static_varlen", p, _ptr(cu), n, _ptr(x), _ptr(ws), _ptr(dy), _ptr(dx), _ptr(dws),
+             _ptr(scratch), nb, _stream(dev))
+    return dx, dws
+
+
+# ----------------------------------------------------------- sequence chunks ---
+# Context parallelism: x [B, T, D] is one time chunk of longer sequences.
+# x_prev [B, W-1, D] holds the W-1 inputs before it (None for the first
+# chunk); dy_next [B, W-1, D] and the next tokens' filters (w_next
+# [B, W-1, G, W] or z_next [B, W-1, R]) the W-1 after it (None for the last).
+# edges_only=True recomputes only the outputs next to the chunk's edges in
+# tensors that already hold the plain call's results (passed as `out`).
+
+def _halo_ok(dev, dtype, *hs):
+    for h in hs:
+        if h is not None:
+            _check(h, dtype=dtype)
+            if h.device != dev:
+                raise ValueError("halos must be on the tensors' device")
+
+
+def dsc_fwd_headwise_chunk(x, w, x_prev=None, residual=True, out=None):
+    dev = _check(x, w, dtype=x.dtype)
+    _halo_ok(dev, x.dtype, x_prev)
+    p = problem(x, w.shape[3], x.shape[2] // w.shape[2], 0, residual)
+    y = out if out is not None else torch.empty_like(x)
+    with torch.cuda.device(dev):
+        call("dsc_fwd_headwise_chunk", p, _ptr(x_prev), _ptr(x), _ptr(w), _ptr(y), int(out is not None),
+             _stream(dev))
+    return y
+
+
+def dsc_bwd_headwise_chunk(x, w, dy, x_prev=None, dy_next=None, w_next=None, residual=True, out=None):
+    """Returns (dx, dw)."""
+    dev = _check(x, w, dy, dtype=x.dtype)
+    _halo_ok(dev, x.dtype, x_prev, dy_next, w_next)
+    p = problem(x, w.shape[3], x.shape[2] // w.shape[2], 0, residual)
+    dx, dw = out if out is not None else (torch.empty_like(x), torch.empty_like(w))
+    with torch.cuda.device(dev):
+        call("dsc_bwd_headwise_chunk", p, _ptr(x_prev), _ptr(dy_next), _ptr(w_next), _ptr(x), _ptr(w), _ptr(dy),
+             _ptr(dx), _ptr(dw), int(out is not None), _stream(dev))
+    return dx, dw
+
+
+def dsc_fwd_lowrank_chunk(x, z, U, x_prev=None, H=1, residual=True, out=None):
+    dev = _check(x, z, U, dtype=x.dtype)
+    _halo_ok(dev, x.dtype, x_prev)
+    p = _lr_problem(x, z, U, H, residual)
+    y = out if out is not None else torch.empty_like(x)
+    nb = lib().dsc_fwd_lowrank_workspace_bytes(p)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
+    with torch.cuda.device(dev):
+        call("dsc_fwd_lowrank_chunk", p, _ptr(x_prev), _ptr(x), _ptr(z), _ptr(U), _ptr(y), _ptr(ws), nb,
+             int(out is not None), _stream(dev))
+    return y
+
+
+def dsc_bwd_lowrank_chunk(x, z, U, dy, x_prev=None, dy_next=None, z_next=None, H=1, residual=True, out=None):
+    """Returns (dx, dz, dU); dU (fp32) sums over this chunk's tokens."""
+    dev = _check(x, z, U, dy, dtype=x.dtype)
+    _halo_ok(dev, x.dtype, x_prev, dy_next, z_next)
+    p = _lr_problem(x, z, U, H, residual)
+    if out is not None:
+        dx, dz, dU = out
+    else:
+        dx, dz = torch.empty_like(x), torch.empty_like(z)
+        dU = torch.empty(U.shape, dtype=torch.float32, device=dev)
+    nb = lib().dsc_bwd_lowrank_chunk_workspace_bytes(p)
+    ws = torch.empty(nb, dtype=torch.uint8, device=dev) if nb else None
+    with torch.cuda.device(dev):
+        call("dsc_bwd_lowrank_chunk", p, _ptr(x_prev), _ptr(dy_next), _ptr(z_next), _ptr(x), _ptr(z), _ptr(U),
+             _ptr(dy), _ptr(dx), _ptr(dz), _ptr(dU), _ptr(ws), nb, int(out is not None), _stream(dev))
+    return dx, dz, dU
+
+
+def dsc_fwd_static_chunk(x, ws, x_prev=None, residual=False, out=None):
+    dev = _check(x, ws, dtype=x.dtype)
+    _halo_ok(dev, x.dtype, x_prev)
+    p = problem(x, ws.shape[1], 1, 0, residual)
+    y = out if out is not None else torch.empty_like(x)
+    with torch.cuda.device(dev):
+        call("dsc_fwd_static_chunk", p, _ptr(x_prev), _ptr(x), _ptr(ws), _ptr(y), int(out is not None),
+             _stream(dev))
+    return y
+
+
+def dsc_bwd_static_chunk(x, ws, dy, x_prev=None, dy_next=None, residual=False, out=None):
+    """Returns (dx, dws); dws (fp32) sums over this chunk's tokens."""
+    dev = _check(x, ws, dy, dtype=x.dtype)
+    _halo_ok(dev, x.dtype, x_prev, dy_next)
+    p = problem(x, ws.shape[1], 1, 0, residual)
+    if out is not None:
+        dx, dws = out
+    else:
+        dx = torch.empty_like(x)
+        dws = torch.empty(ws.shape, dtype=torch.float32, device=dev)
+    with torch.cuda.device(dev):
+        nb = lib().dsc_bwd_static_workspace_bytes(p)
+        scratch = torch.empty(max(nb, 16), dtype=torch.uint8, device=dev)
+        call("dsc_bwd_static_chunk", p, _ptr(x_prev), _ptr(dy_next), _ptr(x), _ptr(ws), _ptr(dy), _ptr(dx),
+             _ptr(dws), _ptr(scratch), nb, int(out is not None), _stream(dev))
+    return dx, dws
+
+
+# ---------------------------------------------------- first projection z = hV ---
+
+def _proj_problem(x, h, V, U, H, residual):
+    B, T, D = x.shape
+    dm, R = V.shape
+    if h.shape != (B, T, dm) or U.shape[0] != R or D % H or U.shape[1] % (D // H):
+        raise ValueError("expected h [B,T,d_model], V [d_model,R], U [R,(D/H)*W]")
+    return problem(x, U.shape[1] // (D // H), H, R, residual), dm
+
+
+def dsc_fwd_lowrank_proj(x, h, V, U, H=1, residual=True):
+    """z = hV formed by the library, then y as dsc_fwd_lowrank.  Returns (y, z)."""
+    dev = _check(x, h, V, U, dtype=x.dtype)
+    p, dm = _proj_problem(x, h, V, U, H, residual)
+    y = torch.empty_like(x)
+    z = torch.empty(x.shape[0], x.shape[1], V.shape[1], dtype=x.dtype, device=dev)
+    n = lib().dsc_fwd_lowrank_proj_workspace_bytes(p, dm)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev) if n else None
+    with torch.cuda.device(dev):
+        call("dsc_fwd_lowrank_proj", p, dm, _ptr(x), _ptr(h), _ptr(V), _ptr(U), _ptr(z), _ptr(y), _ptr(ws), n,
+             _stream(dev))
+    return y, z
+
+
+def dsc_bwd_lowrank_proj(x, h, V, z, U, dy, H=1, residual=True):
+    """Returns (dx, dh, dV, dU); dV and dU are fp32."""
+    dev = _check(x, h, V, z, U, dy, dtype=x.dtype)
+    p, dm = _proj_problem(x, h, V, U, H, residual)
+    dx, dh = torch.empty_like(x), torch.empty_like(h)
+    dV = torch.empty(V.shape, dtype=torch.float32, device=dev)
+    dU = torch.empty(U.shape, dtype=torch.float32, device=dev)
+    n = lib().dsc_bwd_lowrank_proj_workspace_bytes(p, dm)
+    ws = torch.empty(n, dtype=torch.uint8, device=dev)
+    with torch.cuda.device(dev):
+        call("dsc_bwd_lowrank_proj", p, dm, _ptr(x), _ptr(h), _ptr(V), _ptr(z), _ptr(U), _ptr(dy), _ptr(dx), _ptr(dh),
+             _ptr(dV), _ptr(dU), _ptr(ws), n, _stream(dev))
+    return dx, dh, dV, dU
+
+
 # ------------------------------------------------------------------ autograd ---
 
 class DynamicShortConvHeadwise(torch.autograd.Function):

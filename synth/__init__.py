@@ -40,7 +40,7 @@ F32 = "f32"
 BF16 = "bf16"
 
 # Tensor ids of the stream keys (one stream per tensor role).
-TID_X, TID_W, TID_Z, TID_U, TID_DY, TID_WS, TID_STATE = 1, 2, 3, 4, 5, 6, 7
+TID_X, TID_W, TID_Z, TID_U, TID_DY, TID_WS, TID_STATE, TID_H, TID_V = 1, 2, 3, 4, 5, 6, 7, 8, 9
 
 _CHUNK = 1 << 21
 

@@ -20,7 +20,7 @@ from __future__ import annotations
 import math
 from dataclasses import dataclass, replace
 
-from . import BF16, F32, TID_DY, TID_STATE, TID_U, TID_W, TID_WS, TID_X, TID_Z, make_tensor
+from . import BF16, F32, TID_DY, TID_H, TID_STATE, TID_U, TID_V, TID_W, TID_WS, TID_X, TID_Z, make_tensor
 
 HEADWISE = "headwise"
 LOWRANK = "lowrank"
@@ -118,3 +118,14 @@ NAMED = {
     "all-linear-headwise": ALL_LINEAR_HEADWISE,
     "all-linear-lowrank": ALL_LINEAR_LOWRANK,
 }
+
+
+def projection_inputs(wl: Workload, d_model: int) -> dict:
+    """The hidden state and first projection of the low-rank filter generator
+    (w(t) = h_t V U): h [B, T, d_model] ~ N(0, 1) and V [d_model, R] ~
+    N(0, 1/d_model), so that z = hV has unit variance like the z of the
+    recipe above."""
+    return {
+        "h": make_tensor(wl.seed, TID_H, (wl.B, wl.T, d_model), 1.0, wl.dtype),
+        "V": make_tensor(wl.seed, TID_V, (d_model, wl.R), 1.0 / math.sqrt(d_model), wl.dtype),
+    }

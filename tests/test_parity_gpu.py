@@ -20,7 +20,7 @@ import synth
 from synth import workloads as wls
 from synth.workloads import HEADWISE, LOWRANK, STATIC, Workload
 
-from helpers import TOL, assert_close, rel_err, to_dev, to_host64
+from helpers import TOL, assert_close, bound, rel_err, to_dev, to_host64
 
 pytestmark = pytest.mark.gpu
 
@@ -87,7 +87,7 @@ def check_full(wl: Workload):
         g = to_host64(got[k])
         assert g.shape == r.shape, k
         assert np.all(np.isfinite(g)), k
-        errs[k] = assert_close(f"{wl.name}:{k}", g, r, wl.dtype)
+        errs[k] = assert_close(f"{wl.name}:{k}", g, r, wl.dtype, bound(k, wl.dtype))
     return errs
 
 
@@ -337,7 +337,7 @@ def sampled_check(wl: Workload, n=384, seed=0):
     for name, what in (("y", oracle.Y), ("dx", oracle.DX)):
         ref = oracle.sample(P, kind, what, np.stack([b, tt, c], 1), **kw)
         g = got[name][torch.as_tensor(b), torch.as_tensor(tt), torch.as_tensor(c)].double().cpu().numpy()
-        errs[name] = assert_close(f"{wl.name}:{name}", g, ref, wl.dtype)
+        errs[name] = assert_close(f"{wl.name}:{name}", g, ref, wl.dtype, bound(name, wl.dtype))
     G = wl.D // wl.H
     if wl.variant == HEADWISE or wl.variant == LOWRANK:
         g_ = rng.integers(0, G, n)
@@ -345,20 +345,20 @@ def sampled_check(wl: Workload, n=384, seed=0):
         if wl.variant == HEADWISE:
             ref = oracle.sample(P, kind, oracle.DW, np.stack([b, tt, g_, k_], 1), **kw)
             gv = got["dw"][torch.as_tensor(b), torch.as_tensor(tt), torch.as_tensor(g_), torch.as_tensor(k_)]
-            errs["dw"] = assert_close(f"{wl.name}:dw", gv.double().cpu().numpy(), ref, wl.dtype)
+            errs["dw"] = assert_close(f"{wl.name}:dw", gv.double().cpu().numpy(), ref, wl.dtype, bound("dw", wl.dtype))
         else:
             r_ = rng.integers(0, wl.R, n)
             ref = oracle.sample(P, kind, oracle.DZ, np.stack([b, tt, r_], 1)[:128], **kw)
             gv = got["dz"][torch.as_tensor(b[:128]), torch.as_tensor(tt[:128]), torch.as_tensor(r_[:128])]
-            errs["dz"] = assert_close(f"{wl.name}:dz", gv.double().cpu().numpy(), ref, wl.dtype)
+            errs["dz"] = assert_close(f"{wl.name}:dz", gv.double().cpu().numpy(), ref, wl.dtype, bound("dz", wl.dtype))
             ref = oracle.sample(P, kind, oracle.DU, np.stack([r_, g_, k_], 1)[:128], **kw)
             gv = got["dU"][torch.as_tensor(r_[:128]), torch.as_tensor(g_[:128] * wl.W + k_[:128])]
-            errs["dU"] = assert_close(f"{wl.name}:dU", gv.double().cpu().numpy(), ref, wl.dtype)
+            errs["dU"] = assert_close(f"{wl.name}:dU", gv.double().cpu().numpy(), ref, wl.dtype, bound("dU", wl.dtype))
     else:
         k_ = rng.integers(0, wl.W, n)
         ref = oracle.sample(P, kind, oracle.DWS, np.stack([c, k_], 1)[:128], **kw)
         gv = got["dws"][torch.as_tensor(c[:128]), torch.as_tensor(k_[:128])]
-        errs["dws"] = assert_close(f"{wl.name}:dws", gv.double().cpu().numpy(), ref, wl.dtype)
+        errs["dws"] = assert_close(f"{wl.name}:dws", gv.double().cpu().numpy(), ref, wl.dtype, bound("dws", wl.dtype))
     for name, v in got.items():
         assert torch.isfinite(v.float()).all(), name
     return errs
