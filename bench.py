@@ -81,11 +81,21 @@ def step_bytes(wl):
     s = 2 if wl.dtype == "bf16" else 4
     N, D, GW, R = wl.B * wl.T, wl.D, (wl.D // wl.H) * wl.W, wl.R
     if wl.variant == "headwise":
-        return N * (2 * D + GW) * s, N * (3 * D + 2 * GW) * s
-    if wl.variant == "lowrank":
+        fb, bb = N * (2 * D + GW) * s, N * (3 * D + 2 * GW) * s
+    elif wl.variant == "lowrank":
         u = R * GW * s
-        return N * (2 * D + R) * s + u, N * (3 * D + 2 * R) * s + u + 4 * R * GW
-    return N * 2 * D * s + D * wl.W * s, N * 3 * D * s + D * wl.W * s + 4 * D * wl.W
+        fb, bb = N * (2 * D + R) * s + u, N * (3 * D + 2 * R) * s + u + 4 * R * GW
+    else:
+        fb, bb = N * 2 * D * s + D * wl.W * s, N * 3 * D * s + D * wl.W * s + 4 * D * wl.W
+    if wl.mode == "proj":  # + h read and z written (forward); h read and dh written, V and dV (backward)
+        dm = wl.d_model
+        fb += N * (dm + R) * s + dm * R * s
+        bb += 2 * N * dm * s + dm * R * (s + 4)
+    elif wl.mode == "chunk":  # + the halo rows
+        S = wl.W - 1
+        fb += wl.B * S * D * s
+        bb += wl.B * S * (2 * D + (wl.G * wl.W if wl.variant == "headwise" else R)) * s
+    return fb, bb
 
 
 def hbm_peak():
@@ -201,15 +211,38 @@ class Step:
         td = torch.bfloat16 if wl.dtype == "bf16" else torch.float32
         import synth
 
+        host = dict(host)
+        if wl.mode == "proj":  # the filters come from h and V: z is an output
+            from synth import workloads as wls
+
+            host.pop("z", None)
+            host.update(wls.projection_inputs(wl, wl.d_model))
         self.h = {k: synth.to_torch(v, wl.dtype).pin_memory() for k, v in host.items()}
         self.d = {k: v.to(device) for k, v in self.h.items()}
         x = self.d["x"]
+        if wl.mode == "varlen":
+            import numpy as np
+
+            from synth import workloads as wls
+
+            lens = wls.doc_lengths(wl.T, wl.doc_mean, wl.seed)
+            self.n_docs = len(lens)
+            self.cu = torch.tensor(np.concatenate([[0], np.cumsum(lens)]), dtype=torch.int32, device=device)
+        if wl.mode == "chunk":
+            from synth import workloads as wls
+
+            self.halo = {k: synth.to_torch(v, wl.dtype).to(device) for k, v in wls.chunk_halos(wl).items()}
         self.out = {"y": torch.empty_like(x), "dx": torch.empty_like(x)}
         if wl.variant == "headwise":
             self.out["dw"] = torch.empty_like(self.d["w"])
             self.p = ops.problem(x, wl.W, wl.H, 0, bool(wl.residual))
         elif wl.variant == "lowrank":
-            self.out["dz"] = torch.empty_like(self.d["z"])
+            if wl.mode == "proj":
+                self.z = torch.empty(wl.B, wl.T, wl.R, dtype=x.dtype, device=device)
+                self.out["dh"] = torch.empty_like(self.d["h"])
+                self.out["dV"] = torch.empty(self.d["V"].shape, dtype=torch.float32, device=device)
+            else:
+                self.out["dz"] = torch.empty_like(self.d["z"])
             self.out["dU"] = torch.empty(self.d["U"].shape, dtype=torch.float32, device=device)
             self.p = ops.problem(x, wl.W, wl.H, wl.R, bool(wl.residual))
         else:
@@ -217,7 +250,16 @@ class Step:
             self.p = ops.problem(x, wl.W, 1, 0, bool(wl.residual))
         lib = _lib.lib()
         self.nfw = self.nbw = 0
-        if wl.variant == "lowrank":
+        if wl.variant == "lowrank" and wl.mode == "proj":
+            self.nfw = lib.dsc_fwd_lowrank_proj_workspace_bytes(self.p, wl.d_model)
+            self.nbw = lib.dsc_bwd_lowrank_proj_workspace_bytes(self.p, wl.d_model)
+        elif wl.variant == "lowrank" and wl.mode == "varlen":
+            self.nfw = lib.dsc_fwd_lowrank_workspace_bytes(self.p)
+            self.nbw = lib.dsc_bwd_lowrank_varlen_workspace_bytes(self.p, self.n_docs)
+        elif wl.variant == "lowrank" and wl.mode == "chunk":
+            self.nfw = lib.dsc_fwd_lowrank_workspace_bytes(self.p)
+            self.nbw = lib.dsc_bwd_lowrank_chunk_workspace_bytes(self.p)
+        elif wl.variant == "lowrank":
             self.nfw = lib.dsc_fwd_lowrank_workspace_bytes(self.p)
             self.nbw = lib.dsc_bwd_lowrank_workspace_bytes(self.p)
         elif wl.variant == "static":
@@ -229,6 +271,8 @@ class Step:
 
     def fwd(self, stream):
         d, o, L = self.d, self.out, self.L
+        if self.wl.mode:
+            return self.fwd_mode(stream)
         if self.wl.variant == "headwise":
             L.call("dsc_fwd_headwise", self.p, d["x"].data_ptr(), d["w"].data_ptr(), o["y"].data_ptr(), stream)
         elif self.wl.variant == "lowrank":
@@ -239,6 +283,8 @@ class Step:
 
     def bwd(self, stream):
         d, o, L = self.d, self.out, self.L
+        if self.wl.mode:
+            return self.bwd_mode(stream)
         if self.wl.variant == "headwise":
             L.call("dsc_bwd_headwise", self.p, d["x"].data_ptr(), d["w"].data_ptr(), d["dy"].data_ptr(),
                    o["dx"].data_ptr(), o["dw"].data_ptr(), stream)
@@ -249,6 +295,58 @@ class Step:
         else:
             L.call("dsc_bwd_static", self.p, d["x"].data_ptr(), d["ws"].data_ptr(), d["dy"].data_ptr(),
                    o["dx"].data_ptr(), o["dws"].data_ptr(), self.bws.data_ptr(), self.nbw, stream)
+
+    # ---- the next rows: packed documents, middle chunks, first projection
+    def fwd_mode(self, stream):
+        d, o, L, wl, P = self.d, self.out, self.L, self.wl, lambda t: t.data_ptr()
+        if wl.mode == "varlen":
+            if wl.variant == "headwise":
+                L.call("dsc_fwd_headwise_varlen", self.p, P(self.cu), self.n_docs, P(d["x"]), P(d["w"]), P(o["y"]), stream)
+            elif wl.variant == "lowrank":
+                L.call("dsc_fwd_lowrank_varlen", self.p, P(self.cu), self.n_docs, P(d["x"]), P(d["z"]), P(d["U"]),
+                       P(o["y"]), P(self.fws), self.nfw, stream)
+            else:
+                L.call("dsc_fwd_static_varlen", self.p, P(self.cu), self.n_docs, P(d["x"]), P(d["ws"]), P(o["y"]), stream)
+        elif wl.mode == "chunk":
+            xp = P(self.halo["x_prev"])
+            if wl.variant == "headwise":
+                L.call("dsc_fwd_headwise_chunk", self.p, xp, P(d["x"]), P(d["w"]), P(o["y"]), 0, stream)
+            elif wl.variant == "lowrank":
+                L.call("dsc_fwd_lowrank_chunk", self.p, xp, P(d["x"]), P(d["z"]), P(d["U"]), P(o["y"]), P(self.fws),
+                       self.nfw, 0, stream)
+            else:
+                L.call("dsc_fwd_static_chunk", self.p, xp, P(d["x"]), P(d["ws"]), P(o["y"]), 0, stream)
+        else:  # proj
+            L.call("dsc_fwd_lowrank_proj", self.p, wl.d_model, P(d["x"]), P(d["h"]), P(d["V"]), P(d["U"]), P(self.z),
+                   P(o["y"]), P(self.fws), self.nfw, stream)
+
+    def bwd_mode(self, stream):
+        d, o, L, wl, P = self.d, self.out, self.L, self.wl, lambda t: t.data_ptr()
+        if wl.mode == "varlen":
+            if wl.variant == "headwise":
+                L.call("dsc_bwd_headwise_varlen", self.p, P(self.cu), self.n_docs, P(d["x"]), P(d["w"]), P(d["dy"]),
+                       P(o["dx"]), P(o["dw"]), stream)
+            elif wl.variant == "lowrank":
+                L.call("dsc_bwd_lowrank_varlen", self.p, P(self.cu), self.n_docs, P(d["x"]), P(d["z"]), P(d["U"]),
+                       P(d["dy"]), P(o["dx"]), P(o["dz"]), P(o["dU"]), P(self.bws), self.nbw, stream)
+            else:
+                L.call("dsc_bwd_static_varlen", self.p, P(self.cu), self.n_docs, P(d["x"]), P(d["ws"]), P(d["dy"]),
+                       P(o["dx"]), P(o["dws"]), P(self.bws), self.nbw, stream)
+        elif wl.mode == "chunk":
+            h = self.halo
+            if wl.variant == "headwise":
+                L.call("dsc_bwd_headwise_chunk", self.p, P(h["x_prev"]), P(h["dy_next"]), P(h["w_next"]), P(d["x"]),
+                       P(d["w"]), P(d["dy"]), P(o["dx"]), P(o["dw"]), 0, stream)
+            elif wl.variant == "lowrank":
+                L.call("dsc_bwd_lowrank_chunk", self.p, P(h["x_prev"]), P(h["dy_next"]), P(h["z_next"]), P(d["x"]),
+                       P(d["z"]), P(d["U"]), P(d["dy"]), P(o["dx"]), P(o["dz"]), P(o["dU"]), P(self.bws), self.nbw, 0,
+                       stream)
+            else:
+                L.call("dsc_bwd_static_chunk", self.p, P(h["x_prev"]), P(h["dy_next"]), P(d["x"]), P(d["ws"]),
+                       P(d["dy"]), P(o["dx"]), P(o["dws"]), P(self.bws), self.nbw, 0, stream)
+        else:  # proj
+            L.call("dsc_bwd_lowrank_proj", self.p, wl.d_model, P(d["x"]), P(d["h"]), P(d["V"]), P(self.z), P(d["U"]),
+                   P(d["dy"]), P(o["dx"]), P(o["dh"]), P(o["dV"]), P(o["dU"]), P(self.bws), self.nbw, stream)
 
     def h2d(self):
         for k, v in self.h.items():
@@ -262,7 +360,8 @@ class Step:
     # copies and kernels can overlap another row's.  Only for head-wise filters:
     # the low-rank dU and the static dws sum over every row of the batch.
     def row_chunks(self):
-        return self.wl.B if self.wl.variant == "headwise" and self.wl.B > 1 else 1
+        plain = self.wl.variant == "headwise" and not self.wl.mode
+        return self.wl.B if plain and self.wl.B > 1 else 1
 
     def run_row(self, i, stream):
         """H2D of row i's inputs, its forward and backward (one C-ABI call
@@ -487,7 +586,9 @@ def time_workload(wl, steps, warmup, dev, world, peak):
     digest = source_digest(wl.variant)
     out = {
         "config": {"workload": wl.name, "variant": wl.variant, "B": wl.B, "T": wl.T, "D": wl.D, "W": wl.W,
-                   "H": wl.H, "R": wl.R},
+                   "H": wl.H, "R": wl.R, **({"mode": wl.mode} if wl.mode else {}),
+                   **({"d_model": wl.d_model} if wl.d_model else {}),
+                   **({"documents": step.n_docs} if wl.mode == "varlen" else {})},
         "value": job_tokens_per_s(wl.B * wl.T, world, 1, ms), "unit": "tokens/s", "ms_per_step": ms,
         "steps": steps, "warmup": warmup, "gpu_launches": launches,
         "kernels": {"fwd": {"us": fwd_ms * 1e3, "alg_bytes": fb, "gbs": fg, "frac": fg / peak},
@@ -686,6 +787,8 @@ def decode_reference(wl, seconds=None, steps=None, warmup=0, sequences=64):
 def oracle_pass(wl, t):
     import oracle
 
+    if wl.mode:
+        return oracle_pass_mode(wl, t)
     if wl.variant == "headwise":
         P = oracle.problem_of(wl)
         oracle.forward_headwise(P, t["x"], t["w"])
@@ -698,6 +801,32 @@ def oracle_pass(wl, t):
         P = oracle.problem(wl.B, wl.T, wl.D, wl.W, 1, 0, wl.residual)
         oracle.forward_static(P, t["x"], t["ws"])
         oracle.backward_static(P, t["x"], t["ws"], t["dy"])
+
+
+def oracle_pass_mode(wl, t):
+    """The oracle's forward + backward of the next rows' workloads (packed
+    documents, a middle chunk with halos, the first projection)."""
+    import numpy as np
+
+    import oracle
+    from synth import workloads as wls
+
+    kind = {"headwise": oracle.HEADWISE, "lowrank": oracle.LOWRANK, "static": oracle.STATIC}[wl.variant]
+    P = oracle.problem(wl.B, wl.T, wl.D, wl.W, wl.H if wl.variant != "static" else 1, wl.R, wl.residual)
+    f = {k: t[k] for k in ("w", "z", "U", "ws") if k in t}
+    if wl.mode == "proj":
+        hv = wls.projection_inputs(wl, wl.d_model)
+        oracle.forward_lowrank_proj(P, t["x"], hv["h"], hv["V"], t["U"])
+        oracle.backward_lowrank_proj(P, t["x"], hv["h"], hv["V"], t["U"], t["dy"])
+    elif wl.mode == "varlen":
+        cu = np.concatenate([[0], np.cumsum(wls.doc_lengths(wl.T, wl.doc_mean, wl.seed))])
+        oracle.forward_varlen(P, kind, t["x"], cu, **f)
+        oracle.backward_varlen(P, kind, t["x"], t["dy"], cu, **f)
+    else:  # chunk
+        h = wls.chunk_halos(wl)
+        nxt = {"headwise": {"w_next": h.get("w_next")}, "lowrank": {"z_next": h.get("z_next")}, "static": {}}
+        oracle.forward_chunk(P, kind, t["x"], h["x_prev"], **f)
+        oracle.backward_chunk(P, kind, t["x"], t["dy"], h["x_prev"], h["dy_next"], **f, **nxt[wl.variant])
 
 
 def sample_of(wl, host, tokens):
@@ -827,8 +956,8 @@ def main():
         wl0 = matches[0]
 
     if args.workloads is None:
-        args.workloads = ("qkv-lowrank,all-linear-headwise,all-linear-lowrank" if args.workload == "qkv-headwise"
-                          else "none")
+        args.workloads = ("qkv-lowrank,all-linear-headwise,all-linear-lowrank,qkv-headwise-varlen,"
+                          "qkv-headwise-chunk,qkv-lowrank-proj" if args.workload == "qkv-headwise" else "none")
     if args.workloads == "none":
         args.workloads = ""
     for name in filter(None, args.workloads.split(",")):

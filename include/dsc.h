@@ -313,7 +313,9 @@ DSC_API size_t dsc_bwd_lowrank_proj_workspace_bytes(const dsc_problem *p, int64_
 /* Backward, from the forward's z: dx [B,T,D], dh [B,T,d_model] = dz V^T (dtype
  * of x), dV [d_model,R] = sum over tokens of h^T dz (fp32) and dU [R,G*W]
  * (fp32), dz being the low-rank backward's gradient of z (kept in the
- * workspace).  dV and dU are overwritten; both are deterministic. */
+ * workspace).  dV and dU are overwritten.  dU is reduced in a fixed order;
+ * dh and dV follow dz, which on some shapes is summed over channel blocks
+ * with atomic fp32 adds, so they can differ in the last bits between runs. */
 DSC_API dsc_status dsc_bwd_lowrank_proj(const dsc_problem *p, int64_t d_model, const void *x, const void *h,
                                         const void *V, const void *z, const void *U, const void *dy, void *dx,
                                         void *dh, float *dV, float *dU, void *workspace, size_t workspace_bytes,

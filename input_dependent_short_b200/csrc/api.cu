@@ -53,8 +53,6 @@ static int sm_count() {
 
 static Ctx ctx(void *stream) { return Ctx{static_cast<cudaStream_t>(stream), sm_count()}; }
 
-static int vec_of(const dsc_problem &p) { return p.dtype == DSC_BF16 ? 8 : 4; }
-
 static dsc_status done(cudaError_t e) { return e == cudaSuccess ? DSC_OK : DSC_ERR_CUDA; }
 
 static GenArgs gen_args(const dsc_problem &p, int wmode) {
@@ -119,7 +117,7 @@ dsc_status dsc_fwd_headwise(const dsc_problem *p, const void *x, const void *w, 
     if (s != DSC_OK) return s;
     const Ctx c = ctx(stream);
     HwArgs a{};
-    if (stream_map(*p, vec_of(*p), a.m)) {
+    if (stream_plan(*p, a.m)) {
         a.x = x; a.w = w; a.y = y;
         return done(launch_hw_fwd(c, *p, a));
     }
@@ -135,7 +133,7 @@ dsc_status dsc_bwd_headwise(const dsc_problem *p, const void *x, const void *w, 
     if (s != DSC_OK) return s;
     const Ctx c = ctx(stream);
     HwArgs a{};
-    if (stream_map(*p, vec_of(*p), a.m)) {
+    if (stream_plan(*p, a.m)) {
         a.x = x; a.w = w; a.dy = dy; a.dx = dx; a.dw = dw;
         return done(launch_hw_bwd(c, *p, a));
     }
@@ -153,7 +151,7 @@ dsc_status dsc_fwd_static(const dsc_problem *p, const void *x, const void *ws, v
     const dsc_problem q = static_view(*p);
     const Ctx c = ctx(stream);
     HwArgs a{};
-    if (stream_map(q, vec_of(q), a.m)) {
+    if (stream_plan(q, a.m)) {
         a.x = x; a.w = ws; a.y = y;
         return done(launch_st_fwd(c, q, a));
     }
@@ -167,7 +165,7 @@ size_t dsc_bwd_static_workspace_bytes(const dsc_problem *p) {
     const dsc_problem q = static_view(*p);
     StreamMap m;
     size_t parts;
-    if (stream_map(q, vec_of(q), m)) parts = st_partial_count(ctx(nullptr), q);
+    if (stream_plan(q, m)) parts = st_partial_count(ctx(nullptr), q);
     else parts = (size_t)(q.B * ((q.T + 63) / 64));
     return parts * (size_t)(q.D * q.W) * sizeof(float);
 }
@@ -181,7 +179,7 @@ dsc_status dsc_bwd_static(const dsc_problem *p, const void *x, const void *ws, c
     const dsc_problem q = static_view(*p);
     const Ctx c = ctx(stream);
     HwArgs a{};
-    if (stream_map(q, vec_of(q), a.m)) {
+    if (stream_plan(q, a.m)) {
         a.x = x; a.w = ws; a.dy = dy; a.dx = dx;
         a.partial = static_cast<float *>(workspace);
         return done(launch_st_bwd(c, q, a, dws));

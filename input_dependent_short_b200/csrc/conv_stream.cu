@@ -81,6 +81,60 @@ __device__ __forceinline__ uint4 lds16(uint32_t a) {
     return r;
 }
 
+// A thread's channel vector: 16 bytes, or 8 bytes for wide filters (W >= 5),
+// where holding the W-1 previous rows and the filter taps of 16 bytes' worth
+// of channels would leave registers for one block of 256 threads per SM.
+template <int VB> struct VIO;
+template <> struct VIO<16> {
+    using U = uint4;
+    __device__ __forceinline__ static U ld(const void *p) { return ld16(p); }
+    __device__ __forceinline__ static void st(void *p, const U &v) { st16(p, v); }
+    __device__ __forceinline__ static U lds(uint32_t a) { return lds16(a); }
+    __device__ __forceinline__ static void cp(uint32_t dst, const void *src) { cp_async16(dst, src); }
+};
+template <> struct VIO<8> {
+    using U = uint2;
+    __device__ __forceinline__ static U ld(const void *p) {
+        U r;
+        asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+        return r;
+    }
+    __device__ __forceinline__ static void st(void *p, const U &v) {
+        asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+    }
+    __device__ __forceinline__ static U lds(uint32_t a) {
+        U r;
+        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(a));
+        return r;
+    }
+    __device__ __forceinline__ static void cp(uint32_t dst, const void *src) { cp_async8(dst, src); }
+};
+
+// VB bytes of T <-> P pairs of fp32 (pair p holds the vector's channels 2p, 2p+1).
+template <typename T, int VB> struct PairsV {
+    static constexpr int P = VB / (2 * (int)sizeof(T));
+    using U = typename VIO<VB>::U;
+    __device__ __forceinline__ static void unpack(const U &u, u64 (&p)[P]) {
+        if constexpr (VB == 16) {
+            Pairs<T>::unpack(u, p);
+        } else if constexpr (sizeof(T) == 2) {
+            p[0] = mk2(bf_lo(u.x), bf_hi(u.x));
+            p[1] = mk2(bf_lo(u.y), bf_hi(u.y));
+        } else {
+            p[0] = mk2(__uint_as_float(u.x), __uint_as_float(u.y));
+        }
+    }
+    __device__ __forceinline__ static U pack(const u64 (&p)[P]) {
+        if constexpr (VB == 16) {
+            return Pairs<T>::pack(p);
+        } else if constexpr (sizeof(T) == 2) {
+            return make_uint2(pack_bf2(lo2(p[0]), hi2(p[0])), pack_bf2(lo2(p[1]), hi2(p[1])));
+        } else {
+            return make_uint2(__float_as_uint(lo2(p[0])), __float_as_uint(hi2(p[0])));
+        }
+    }
+};
+
 constexpr int gcd_c(int a, int b) { return b == 0 ? a : gcd_c(b, a % b); }
 
 // The filter taps a thread needs per token (NW elements of T).  The start of
@@ -147,8 +201,8 @@ __host__ __device__ constexpr int ring_depth(int slots) {
     return slots * 16 * 8 <= 384 ? 8 : (384 / (slots * 16) < 2 ? 2 : 384 / (slots * 16));
 }
 
-template <typename T, int W, int GPT, bool WS, bool BWD> struct StreamCfg {
-    static constexpr int V = VecOf<T>::V;
+template <typename T, int W, int GPT, bool WS, bool BWD, int VB = 16> struct StreamCfg {
+    static constexpr int V = VB / (int)sizeof(T);
     static constexpr int NW = WS ? V * W : GPT * W;  // filter taps per token per thread
     static constexpr int CPG = WS ? 1 : V / GPT;      // channels sharing one filter inside a thread
     static constexpr int WIN = W - 1;
@@ -161,12 +215,17 @@ template <typename T, int W, int GPT, bool WS, bool BWD> struct StreamCfg {
     // Blocks per SM the register budget is sized for: the narrow head-wise
     // filters fit 3 (forward) / 2 (backward) blocks of 256 threads; wider or
     // per-channel (static) filters need more registers per thread.
-    static constexpr int MINB = BWD ? ((!WS && W <= 4) || (WS && W <= 2) ? 2 : 1)
-                                    : ((!WS && W <= 4) ? 3 : (W <= 3 ? 2 : 1));
+    // With 8-byte vectors a thread holds half the state: two blocks per SM,
+    // except the static backward at W >= 6, whose filters, filter-gradient
+    // sums and two windows still need more than the 128 registers that two
+    // blocks leave a thread (one block: no spills).
+    static constexpr int MINB = VB == 8 ? (WS && BWD && W >= 6 ? 1 : 2)
+                                : BWD ? ((!WS && W <= 4) || (WS && W <= 2) ? 2 : 1)
+                                      : ((!WS && W <= 4) ? 3 : (W <= 3 ? 2 : 1));
 };
 
-template <typename T, int W, int GPT, bool WS, bool BWD>
-size_t stream_smem() { return StreamCfg<T, W, GPT, WS, BWD>::SMEM; }
+template <typename T, int W, int GPT, bool WS, bool BWD, int VB>
+size_t stream_smem() { return StreamCfg<T, W, GPT, WS, BWD, VB>::SMEM; }
 
 template <bool B> struct BoolC { static constexpr bool value = B; };
 
@@ -211,16 +270,17 @@ __device__ __forceinline__ void group_reduce(float (&part)[N], int L, int pos) {
 
 // WS = false: head-wise filters w[b,t,g,k] read per token.
 // WS = true : static filters ws[c,k] read once per thread.
-template <typename T, int W, int GPT, bool WS>
-__global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, false>::MINB)) k_stream_fwd(const HwArgs a) {
-    using C = StreamCfg<T, W, GPT, WS, false>;
+template <typename T, int W, int GPT, bool WS, int VB>
+__global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, false, VB>::MINB)) k_stream_fwd(const HwArgs a) {
+    using C = StreamCfg<T, W, GPT, WS, false, VB>;
     using F = typename C::F;
-    using PR = Pairs<T>;
+    using PR = PairsV<T, VB>;
+    using IO = VIO<VB>;
     constexpr int P = PR::P, NS = C::NS, WIN = C::WIN, XW = WIN > 0 ? WIN : 1, CPG = C::CPG;
     extern __shared__ uint4 ring[];
     const StreamMap &m = a.m;
     Pos q;
-    if (!locate<VecOf<T>::V>(m, q) || !q.active) return;
+    if (!locate<C::V>(m, q) || !q.active) return;
     pdl_wait();  // inputs may come from the previous kernel of the stream
     pdl_trigger();
 
@@ -251,7 +311,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
 
     auto issue = [&](int i, int s, bool full) {
         if (full || i < n) {
-            cp_async16(slot(s, 0), xp + i * xstep);
+            IO::cp(slot(s, 0), xp + i * xstep);
             if constexpr (C::WRING) F::copy(slot(s, 1), SUBSTRIDE, wp + i * wstep);
             if constexpr (C::WREG) F::load_direct(wp + i * wstep, wreg[s]);
         }
@@ -262,7 +322,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
 #pragma unroll
     for (int j = 0; j < XW; ++j) {
         const int t = q.t_start - 1 - j;
-        if (WIN > 0 && t >= 0) PR::unpack(ld16(xp - (int64_t)(1 + j) * xstep), xs[j]);
+        if (WIN > 0 && t >= 0) PR::unpack(IO::ld(xp - (int64_t)(1 + j) * xstep), xs[j]);
         else
 #pragma unroll
             for (int pp = 0; pp < P; ++pp) xs[j][pp] = 0ull;
@@ -279,7 +339,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
             issue(i + NS - 1, (u + NS - 1) % NS, FULL);
             cp_wait<NS - 1>();
             u64 xc[P], acc[P];
-            PR::unpack(lds16(slot(u, 0)), xc);
+            PR::unpack(IO::lds(slot(u, 0)), xc);
             uint32_t wv[F::WORDS];
             if constexpr (C::WRING) F::read(slot(u, 1), SUBSTRIDE, wv);
             if constexpr (C::WREG)
@@ -292,7 +352,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
                 for (int k = 1; k < W; ++k) s = fma2(WS ? wsp[pp][k] : tap2<F, W, CPG>(wv, pp, k), xs[k - 1][pp], s);
                 acc[pp] = s;
             }
-            st16(yp + i * xstep, PR::pack(acc));
+            IO::st(yp + i * xstep, PR::pack(acc));
 #pragma unroll
             for (int j = XW - 1; j > 0; --j)
 #pragma unroll
@@ -309,17 +369,18 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
 
 // --------------------------------------------------------------- backward ---
 
-template <typename T, int W, int GPT, bool WS>
-__global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true>::MINB)) k_stream_bwd(const HwArgs a) {
-    using C = StreamCfg<T, W, GPT, WS, true>;
+template <typename T, int W, int GPT, bool WS, int VB>
+__global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true, VB>::MINB)) k_stream_bwd(const HwArgs a) {
+    using C = StreamCfg<T, W, GPT, WS, true, VB>;
     using F = typename C::F;
-    using PR = Pairs<T>;
+    using PR = PairsV<T, VB>;
+    using IO = VIO<VB>;
     constexpr int P = PR::P, NS = C::NS, WIN = C::WIN, XW = WIN > 0 ? WIN : 1, CPG = C::CPG;
     constexpr int PPG = CPG >= 2 ? CPG / 2 : 1;  // channel pairs per filter group (CPG >= 2)
     extern __shared__ uint4 ring[];
     const StreamMap &m = a.m;
     Pos q;
-    if (!locate<VecOf<T>::V>(m, q)) return;  // whole warp out of range; partial warps stay for the shuffles
+    if (!locate<C::V>(m, q)) return;  // whole warp out of range; partial warps stay for the shuffles
     pdl_wait();  // inputs may come from the previous kernel of the stream
     pdl_trigger();
     // Inactive lanes (no channels of their own) stream channel 0 of the same rows: in bounds, never
@@ -347,7 +408,13 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
     constexpr uint32_t SUBSTRIDE = 16u * STREAM_THREADS;
     auto slot = [&](int s, int sub) { return base + (uint32_t)(s * C::SUB + sub) * SUBSTRIDE; };
 
-    u64 wsp[WS ? P : 1][WS ? W : 1];
+    // Static filters: fp32 pairs, or (bf16 with 8-byte vectors, where the
+    // registers are tightest) taps 1 .. W-1 as packed bf16 pairs, unpacked at
+    // each use; exact, the taps being bf16 values.  Tap 0 carries the residual.
+    constexpr bool WPK = WS && VB == 8 && sizeof(T) == 2;
+    u64 wsp[WS && !WPK ? P : 1][WS && !WPK ? W : 1];
+    uint32_t wpk[WPK ? P : 1][WPK ? W : 1];
+    u64 w0p[WPK ? P : 1];
     u64 dws[WS ? P : 1][WS ? W : 1];
     if constexpr (WS) {
         uint32_t wst[F::WORDS];
@@ -356,16 +423,25 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
         for (int pp = 0; pp < P; ++pp)
 #pragma unroll
             for (int k = 0; k < W; ++k) {
-                wsp[pp][k] = k == 0 ? tap2<F, W, CPG>(wst, pp, 0, res) : tap2<F, W, CPG>(wst, pp, k);
+                if constexpr (WPK) {
+                    if (k == 0) w0p[pp] = tap2<F, W, CPG>(wst, pp, 0, res);
+                    else wpk[pp][k] = pack_bf2(F::get(wst, (2 * pp) * W + k), F::get(wst, (2 * pp + 1) * W + k));
+                } else {
+                    wsp[pp][k] = k == 0 ? tap2<F, W, CPG>(wst, pp, 0, res) : tap2<F, W, CPG>(wst, pp, k);
+                }
                 dws[pp][k] = 0ull;
             }
     }
+    auto stap = [&](int pp, int k) -> u64 {
+        if constexpr (WPK) return k == 0 ? w0p[pp] : mk2(bf_lo(wpk[pp][k]), bf_hi(wpk[pp][k]));
+        else return wsp[WS ? pp : 0][WS ? k : 0];
+    };
     uint32_t wreg[C::WREG ? NS : 1][F::WORDS];
 
     auto issue = [&](int i, int s, bool full) {
-        if (full || i < n) cp_async16(slot(s, 0), xp + i * xstep);
+        if (full || i < n) IO::cp(slot(s, 0), xp + i * xstep);
         if (full || i < nl) {
-            cp_async16(slot(s, 1), dyp + i * xstep);
+            IO::cp(slot(s, 1), dyp + i * xstep);
             if constexpr (C::WRING) F::copy(slot(s, 2), SUBSTRIDE, wp + i * wstep);
             if constexpr (C::WREG) F::load_direct(wp + i * wstep, wreg[s]);
         }
@@ -377,7 +453,7 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
 #pragma unroll
     for (int j = 0; j < XW; ++j) {
         const int t = q.t_start - 1 - j;
-        if (WIN > 0 && t >= 0) PR::unpack(ld16(xp - (int64_t)(1 + j) * xstep), xs[j]);
+        if (WIN > 0 && t >= 0) PR::unpack(IO::ld(xp - (int64_t)(1 + j) * xstep), xs[j]);
         else
 #pragma unroll
             for (int pp = 0; pp < P; ++pp) xs[j][pp] = 0ull;
@@ -398,12 +474,12 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
             const bool hx = FULL || i < n, hd = FULL || i < nl;
             u64 xc[P], dyc[P], r0[P];
             uint32_t wv[F::WORDS];
-            if (hx) PR::unpack(lds16(slot(u, 0)), xc);
+            if (hx) PR::unpack(IO::lds(slot(u, 0)), xc);
             else
 #pragma unroll
                 for (int pp = 0; pp < P; ++pp) xc[pp] = 0ull;
             if (hd) {
-                PR::unpack(lds16(slot(u, 1)), dyc);
+                PR::unpack(IO::lds(slot(u, 1)), dyc);
                 if constexpr (C::WRING) F::read(slot(u, 2), SUBSTRIDE, wv);
                 if constexpr (C::WREG)
 #pragma unroll
@@ -418,14 +494,14 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
             // with the residual (rows past the tile are never stored).
 #pragma unroll
             for (int pp = 0; pp < P; ++pp) {
-                r0[pp] = mul2(WS ? wsp[pp][0] : tap2<F, W, CPG>(wv, pp, 0, res), dyc[pp]);
+                r0[pp] = mul2(WS ? stap(pp, 0) : tap2<F, W, CPG>(wv, pp, 0, res), dyc[pp]);
 #pragma unroll
                 for (int k = 1; k < W; ++k)
-                    acc[k - 1][pp] = fma2(WS ? wsp[pp][k] : tap2<F, W, CPG>(wv, pp, k), dyc[pp], acc[k - 1][pp]);
+                    acc[k - 1][pp] = fma2(WS ? stap(pp, k) : tap2<F, W, CPG>(wv, pp, k), dyc[pp], acc[k - 1][pp]);
             }
             if (act && i >= WIN) {  // row i-WIN is complete
-                if constexpr (W > 1) st16(dxp + (i - WIN) * xstep, PR::pack(acc[XW - 1]));
-                else st16(dxp + (i - WIN) * xstep, PR::pack(r0));
+                if constexpr (W > 1) IO::st(dxp + (i - WIN) * xstep, PR::pack(acc[XW - 1]));
+                else IO::st(dxp + (i - WIN) * xstep, PR::pack(r0));
             }
             // dw(i)_k = sum over the group's channels of dy_i * x_{i-k}
             if (FULL || i < n) {
@@ -555,18 +631,34 @@ void finish_map(StreamMap &m, int64_t target_warps) {
     m.n_warps = m.B * m.nTiles * (int64_t)m.nWc;
 }
 
-template <typename T, int W, int GPT, bool WS, bool BWD>
+// The plan: 8-byte vectors for W >= 5 when that mapping exists (two blocks
+// per SM instead of one), else 16-byte vectors; false when neither exists
+// (the generic kernels take the shape).
+bool stream_plan(const dsc_problem &p, StreamMap &m) {
+    const int V16 = p.dtype == DSC_BF16 ? 8 : 4;
+    if (p.W >= 5 && stream_map(p, V16 / 2, m)) {
+        m.vb = 8;
+        return true;
+    }
+    if (stream_map(p, V16, m)) {
+        m.vb = 16;
+        return true;
+    }
+    return false;
+}
+
+template <typename T, int W, int GPT, bool WS, bool BWD, int VB>
 static const void *stream_kernel() {
-    if constexpr (BWD) return (const void *)k_stream_bwd<T, W, GPT, WS>;
-    else return (const void *)k_stream_fwd<T, W, GPT, WS>;
+    if constexpr (BWD) return (const void *)k_stream_bwd<T, W, GPT, WS, VB>;
+    else return (const void *)k_stream_fwd<T, W, GPT, WS, VB>;
 }
 
 // Dynamic shared memory of one instantiation, set up once (thread-safe).
-template <typename T, int W, int GPT, bool WS, bool BWD>
+template <typename T, int W, int GPT, bool WS, bool BWD, int VB>
 static size_t stream_setup(int &per_sm_warps) {
-    static const size_t smem = stream_smem<T, W, GPT, WS, BWD>();
+    static const size_t smem = stream_smem<T, W, GPT, WS, BWD, VB>();
     static const int blocks = [] {
-        const void *k = stream_kernel<T, W, GPT, WS, BWD>();
+        const void *k = stream_kernel<T, W, GPT, WS, BWD, VB>();
         cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         cudaGetLastError();
         return resident_blocks(k, STREAM_THREADS, smem);
@@ -575,29 +667,47 @@ static size_t stream_setup(int &per_sm_warps) {
     return smem;
 }
 
-template <typename T, int W, int GPT, bool WS, bool BWD>
+template <typename T, int W, int GPT, bool WS, bool BWD, int VB>
 static cudaError_t run_stream(const Ctx &c, HwArgs a) {
     int per_sm = 0;
-    const size_t smem = stream_setup<T, W, GPT, WS, BWD>(per_sm);
+    const size_t smem = stream_setup<T, W, GPT, WS, BWD, VB>(per_sm);
     finish_map(a.m, (int64_t)per_sm * c.sms);
     const int64_t blocks = (a.m.n_warps + STREAM_THREADS / 32 - 1) / (STREAM_THREADS / 32);
     cudaError_t e;
-    if constexpr (BWD) e = launch_pdl(k_stream_bwd<T, W, GPT, WS>, dim3((unsigned)blocks), dim3(STREAM_THREADS), smem, c.stream, a);
-    else e = launch_pdl(k_stream_fwd<T, W, GPT, WS>, dim3((unsigned)blocks), dim3(STREAM_THREADS), smem, c.stream, a);
+    if constexpr (BWD)
+        e = launch_pdl(k_stream_bwd<T, W, GPT, WS, VB>, dim3((unsigned)blocks), dim3(STREAM_THREADS), smem, c.stream, a);
+    else
+        e = launch_pdl(k_stream_fwd<T, W, GPT, WS, VB>, dim3((unsigned)blocks), dim3(STREAM_THREADS), smem, c.stream, a);
     return e != cudaSuccess ? e : cudaGetLastError();
 }
 
+// W <= 4: 16-byte vectors only; W >= 5: the vector width of the plan.
 template <typename T, bool WS, bool BWD, int GPT>
 static cudaError_t by_w(const Ctx &c, int W, HwArgs a) {
+    constexpr int V16 = VecOf<T>::V;
+    const bool half = a.m.vb == 8;
     switch (W) {
-    case 1: return run_stream<T, 1, GPT, WS, BWD>(c, a);
-    case 2: return run_stream<T, 2, GPT, WS, BWD>(c, a);
-    case 3: return run_stream<T, 3, GPT, WS, BWD>(c, a);
-    case 4: return run_stream<T, 4, GPT, WS, BWD>(c, a);
-    case 5: return run_stream<T, 5, GPT, WS, BWD>(c, a);
-    case 6: return run_stream<T, 6, GPT, WS, BWD>(c, a);
-    case 7: return run_stream<T, 7, GPT, WS, BWD>(c, a);
-    case 8: return run_stream<T, 8, GPT, WS, BWD>(c, a);
+    case 1: return run_stream<T, 1, GPT, WS, BWD, 16>(c, a);
+    case 2: return run_stream<T, 2, GPT, WS, BWD, 16>(c, a);
+    case 3: return run_stream<T, 3, GPT, WS, BWD, 16>(c, a);
+    case 4: return run_stream<T, 4, GPT, WS, BWD, 16>(c, a);
+    }
+    if (half) {
+        if constexpr (GPT <= V16 / 2) {
+            switch (W) {
+            case 5: return run_stream<T, 5, GPT, WS, BWD, 8>(c, a);
+            case 6: return run_stream<T, 6, GPT, WS, BWD, 8>(c, a);
+            case 7: return run_stream<T, 7, GPT, WS, BWD, 8>(c, a);
+            case 8: return run_stream<T, 8, GPT, WS, BWD, 8>(c, a);
+            }
+        }
+        return cudaErrorInvalidValue;
+    }
+    switch (W) {
+    case 5: return run_stream<T, 5, GPT, WS, BWD, 16>(c, a);
+    case 6: return run_stream<T, 6, GPT, WS, BWD, 16>(c, a);
+    case 7: return run_stream<T, 7, GPT, WS, BWD, 16>(c, a);
+    case 8: return run_stream<T, 8, GPT, WS, BWD, 16>(c, a);
     }
     return cudaErrorInvalidValue;
 }
@@ -634,25 +744,33 @@ cudaError_t launch_st_bwd(const Ctx &c, const dsc_problem &p, HwArgs a, float *d
     return launch_reduce_partials(c, a.partial, st_partial_count(c, p), p.D * p.W, dws);
 }
 
-template <typename T, int W> static int64_t st_tiles_w(const Ctx &c, StreamMap m) {
+template <typename T, int W, int VB> static int64_t st_tiles_w(const Ctx &c, StreamMap m) {
     int per_sm = 0;
-    stream_setup<T, W, 1, true, true>(per_sm);
+    stream_setup<T, W, 1, true, true, VB>(per_sm);
     finish_map(m, (int64_t)per_sm * c.sms);
     return m.B * m.nTiles;
 }
 
 template <typename T> static int64_t st_tiles(const Ctx &c, const dsc_problem &p) {
     StreamMap m;
-    stream_map(p, VecOf<T>::V, m);
+    stream_plan(p, m);
+    if (m.vb == 8) {
+        switch (p.W) {
+        case 5: return st_tiles_w<T, 5, 8>(c, m);
+        case 6: return st_tiles_w<T, 6, 8>(c, m);
+        case 7: return st_tiles_w<T, 7, 8>(c, m);
+        default: return st_tiles_w<T, 8, 8>(c, m);
+        }
+    }
     switch (p.W) {
-    case 1: return st_tiles_w<T, 1>(c, m);
-    case 2: return st_tiles_w<T, 2>(c, m);
-    case 3: return st_tiles_w<T, 3>(c, m);
-    case 4: return st_tiles_w<T, 4>(c, m);
-    case 5: return st_tiles_w<T, 5>(c, m);
-    case 6: return st_tiles_w<T, 6>(c, m);
-    case 7: return st_tiles_w<T, 7>(c, m);
-    default: return st_tiles_w<T, 8>(c, m);
+    case 1: return st_tiles_w<T, 1, 16>(c, m);
+    case 2: return st_tiles_w<T, 2, 16>(c, m);
+    case 3: return st_tiles_w<T, 3, 16>(c, m);
+    case 4: return st_tiles_w<T, 4, 16>(c, m);
+    case 5: return st_tiles_w<T, 5, 16>(c, m);
+    case 6: return st_tiles_w<T, 6, 16>(c, m);
+    case 7: return st_tiles_w<T, 7, 16>(c, m);
+    default: return st_tiles_w<T, 8, 16>(c, m);
     }
 }
 

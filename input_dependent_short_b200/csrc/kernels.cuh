@@ -20,6 +20,7 @@ struct StreamMap {
     int Tt, nTiles, nWc, CW, lanes_used, L, gpt;
     int64_t n_warps;
     int residual;
+    int vb;  // bytes of a thread's channel vector (16, or 8 for W >= 5)
 };
 
 struct HwArgs {
@@ -51,6 +52,7 @@ struct Ctx {
 
 // conv_stream.cu
 bool stream_map(const dsc_problem &p, int V, StreamMap &m);
+bool stream_plan(const dsc_problem &p, StreamMap &m);
 void finish_map(StreamMap &m, int64_t target_warps);
 cudaError_t launch_hw_fwd(const Ctx &c, const dsc_problem &p, HwArgs a);
 cudaError_t launch_hw_bwd(const Ctx &c, const dsc_problem &p, HwArgs a);

@@ -40,6 +40,12 @@ class Workload:
     dtype: str = BF16
     residual: int = 1
     seed: int = 0
+    # "": plain batch rows; "varlen": one row of packed documents (mean length
+    # doc_mean); "chunk": each row a middle time chunk of longer sequences
+    # (halos on both sides); "proj": low-rank filters from h [B,T,d_model] and V
+    mode: str = ""
+    doc_mean: int = 0
+    d_model: int = 0
 
     @property
     def G(self) -> int:
@@ -111,12 +117,26 @@ def decode_state(wl):
     return make_tensor(wl.seed, TID_STATE, (wl.B, wl.W - 1, wl.D), 1.0, wl.dtype)
 
 
+# The next rows on the same Q/K/V shapes: the same tokens as packed
+# documents (variable-length batch), as middle time chunks of longer
+# sequences (context parallelism), and the low-rank filters with their first
+# projection from a d_model = 2048 hidden state.
+QKV_HEADWISE_VARLEN = Workload("qkv-headwise-varlen B1 T16384 D6144 W4 H16 docs~1024", HEADWISE, 1, 16384, 6144, 4,
+                               H=16, mode="varlen", doc_mean=1024)
+QKV_HEADWISE_CHUNK = Workload("qkv-headwise-chunk B8 T2048 D6144 W4 H16 halos", HEADWISE, 8, 2048, 6144, 4, H=16,
+                              mode="chunk")
+QKV_LOWRANK_PROJ = Workload("qkv-lowrank-proj B8 T2048 D6144 W4 H1 R32 d2048", LOWRANK, 8, 2048, 6144, 4, H=1, R=32,
+                            mode="proj", d_model=2048)
+
 NAMED = {
     "tiny": TINY_F32,
     "qkv-headwise": QKV_HEADWISE,
     "qkv-lowrank": QKV_LOWRANK,
     "all-linear-headwise": ALL_LINEAR_HEADWISE,
     "all-linear-lowrank": ALL_LINEAR_LOWRANK,
+    "qkv-headwise-varlen": QKV_HEADWISE_VARLEN,
+    "qkv-headwise-chunk": QKV_HEADWISE_CHUNK,
+    "qkv-lowrank-proj": QKV_LOWRANK_PROJ,
 }
 
 
@@ -129,3 +149,32 @@ def projection_inputs(wl: Workload, d_model: int) -> dict:
         "h": make_tensor(wl.seed, TID_H, (wl.B, wl.T, d_model), 1.0, wl.dtype),
         "V": make_tensor(wl.seed, TID_V, (d_model, wl.R), 1.0 / math.sqrt(d_model), wl.dtype),
     }
+
+
+def doc_lengths(T: int, mean: int, seed: int = 0) -> list:
+    """Seeded document lengths summing to T: geometric with the given mean
+    (a long-tailed mix of short and long documents, as in web text), the
+    last one cut to fit.  The pages' documents (Nemotron-CC) are not
+    available; this stands in for their length mix."""
+    import numpy as np
+
+    rng = np.random.default_rng(1000003 * seed + 17)
+    out, left = [], T
+    while left > 0:
+        n = int(min(left, max(1, rng.geometric(1.0 / mean))))
+        out.append(n)
+        left -= n
+    return out
+
+
+def chunk_halos(wl: Workload) -> dict:
+    """Seeded halo rows of a middle time chunk: x of the W-1 tokens before it,
+    dy and the filters (head-wise w or low-rank z) of the W-1 after it."""
+    dt, S = wl.dtype, max(wl.W - 1, 1)
+    out = {"x_prev": make_tensor(wl.seed + 7919, TID_X, (wl.B, S, wl.D), 1.0, dt),
+           "dy_next": make_tensor(wl.seed + 7919, TID_DY, (wl.B, S, wl.D), 1.0, dt)}
+    if wl.variant == HEADWISE:
+        out["w_next"] = make_tensor(wl.seed + 7919, TID_W, (wl.B, S, wl.G, wl.W), 1.0 / math.sqrt(wl.W), dt)
+    elif wl.variant == LOWRANK:
+        out["z_next"] = make_tensor(wl.seed + 7919, TID_Z, (wl.B, S, wl.R), 1.0, dt)
+    return out

@@ -75,10 +75,14 @@ def test_projection_z_equals_a_separate_projection_then_the_plain_call():
     dx, dh, dV, dU = ops.dsc_bwd_lowrank_proj(x, h, V, z, U, dy)
     dx2, dz2, dU2 = ops.dsc_bwd_lowrank(x, z, U, dy)
     assert torch.equal(dx, dx2) and torch.equal(dU, dU2)
-    # dh = dz V^T and dV = h^T dz against torch's matmul in fp32 on the same dz
+    # dh = dz V^T and dV = h^T dz against torch's fp32 matmul on the dz of the
+    # plain call.  On this shape the backward adds dz over channel blocks with
+    # atomic fp32 adds, so the two calls' bf16 dz can differ by one rounding
+    # in a few elements: hence the bounds (dh also carries its own bf16 output
+    # rounding).
     ref_dh = dz2.float().reshape(-1, 32) @ V.float().t()
     err = (dh.float().reshape(-1, 256) - ref_dh).abs().max() / ref_dh.abs().max()
     assert err.item() < 8e-3
     ref_dV = h.float().reshape(-1, 256).t() @ dz2.float().reshape(-1, 32)
     err = (dV - ref_dV).abs().max() / ref_dV.abs().max()
-    assert err.item() < 1e-4
+    assert err.item() < 2e-3
