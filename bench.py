@@ -495,7 +495,8 @@ def run_dsc(args, wl0):
             "clocks": clocks.summary(),
             "source_digest": digest,
         }
-    # the other training workloads, each timed the same way (fewer steps)
+    # the other training workloads, each timed the same way (fewer steps), with
+    # the oracle on a bounded sample of the same workload beside it (N = 1)
     others = {}
     if args.workloads:
         del step
@@ -503,6 +504,9 @@ def run_dsc(args, wl0):
         for name in args.workloads.split(","):
             other = rank_workload(wls.NAMED[name], rank)
             others[name] = time_workload(other, args.other_steps, args.warmup, dev, world, peak)
+            if world == 1 and not args.no_cpu_baseline:
+                others[name]["cpu_baseline"] = cpu_baseline(other, wls.make_inputs(other.with_(B=1, T=min(other.T, 256))),
+                                                            seconds=args.other_cpu_seconds, tokens=256)
             torch.cuda.empty_cache()
     if result is not None and others:
         result["workloads"] = others
@@ -843,10 +847,10 @@ def sample_of(wl, host, tokens):
     return sub, t
 
 
-def cpu_baseline(wl, host, seconds=10.0):
+def cpu_baseline(wl, host, seconds=10.0, tokens=2048):
     import oracle
 
-    sub, t = sample_of(wl, host, 2048)
+    sub, t = sample_of(wl, host, tokens)
     n = 0
     t0 = time.perf_counter()
     while True:
@@ -908,6 +912,7 @@ def main():
                     help="comma-separated named workloads also timed in the same run (default: the other three "
                          "training workloads when --workload is the headline one; 'none' for none)")
     ap.add_argument("--other-steps", type=int, default=20)
+    ap.add_argument("--other-cpu-seconds", type=float, default=3.0)
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")

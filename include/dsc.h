@@ -90,8 +90,12 @@ DSC_API dsc_status dsc_fwd_headwise(const dsc_problem *p, const void *x, const v
 DSC_API dsc_status dsc_bwd_headwise(const dsc_problem *p, const void *x, const void *w, const void *dy, void *dx, void *dw,
                             void *stream);
 
-/* Bytes of scratch the low-rank forward / backward need for this problem
- * (0 when the fused kernels apply). */
+/* Bytes of scratch the low-rank forward / backward need for this problem.
+ * Forward: a copy of U with each vector's filter columns in tap order
+ * (R*G*W bf16) for the tensor-core kernel with H < 8, 0 for the other fused
+ * kernels, the filters w = zU (B*T*G*W fp32) on the unfused path.  Backward:
+ * operand images of z and U, partial sums of dU and dz (fused), or w and
+ * dw (unfused).  Neither ever holds the filter tensor on the fused paths. */
 DSC_API size_t dsc_fwd_lowrank_workspace_bytes(const dsc_problem *p);
 DSC_API size_t dsc_bwd_lowrank_workspace_bytes(const dsc_problem *p);
 

@@ -205,7 +205,8 @@ int dsc_lowrank_kernels(const dsc_problem *p, int backward) {
 
 size_t dsc_fwd_lowrank_workspace_bytes(const dsc_problem *p) {
     if (validate(p, true) != DSC_OK) return 0;
-    if (lowrank_tc_ok(*p) || lowrank_fused_ok(*p)) return 0;
+    if (lowrank_tc_ok(*p)) return lr_tc_fwd_ws_bytes(*p);
+    if (lowrank_fused_ok(*p)) return 0;
     return lr_generic_fwd_bytes(*p);
 }
 
@@ -222,7 +223,12 @@ dsc_status dsc_fwd_lowrank(const dsc_problem *p, const void *x, const void *z, c
     if (s == DSC_OK) s = check_ptrs({x, z, U, y});
     if (s != DSC_OK) return s;
     const Ctx c = ctx(stream);
-    if (lowrank_tc_ok(*p)) return done(launch_lr_fwd_tc(c, *p, x, z, U, y));
+    if (lowrank_tc_ok(*p)) {
+        const size_t need = lr_tc_fwd_ws_bytes(*p);
+        if (need && (!workspace || workspace_bytes < need)) return DSC_ERR_INVALID_ARG;
+        if (need && !aligned16(workspace)) return DSC_ERR_MISALIGNED;
+        return done(launch_lr_fwd_tc(c, *p, x, z, U, y, workspace, workspace_bytes));
+    }
     if (lowrank_fused_ok(*p)) return done(launch_lr_fwd_fused(c, *p, x, z, U, y));
     // Unfused fallback: filters w = zU in the workspace, then the per-channel kernel.
     if (!workspace) return DSC_ERR_INVALID_ARG;

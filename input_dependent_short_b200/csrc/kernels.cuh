@@ -82,7 +82,9 @@ size_t lr_bwd_fused_ws_bytes(const Ctx &c, const dsc_problem &p);
 
 // lowrank_tc_fwd.cu, lowrank_tc_bwd.cu (tensor-core kernels, bf16)
 bool lowrank_tc_ok(const dsc_problem &p);
-cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U, void *y);
+size_t lr_tc_fwd_ws_bytes(const dsc_problem &p);
+cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U, void *y,
+                             void *ws, size_t ws_bytes);
 int take_tc_status(cudaStream_t stream);
 cudaError_t launch_wait_selftest(cudaStream_t stream);
 bool lowrank_tc_bwd_ok(const dsc_problem &p, int sms);

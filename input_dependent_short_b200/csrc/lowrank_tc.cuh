@@ -52,6 +52,7 @@ struct TcArgs {
     float *dU, *dz_acc, *dU_part;
     bf16 *Up;    // backward: U blocks as shared-memory images (columns tap-major, rows padded to RP)
     bf16 *zimg;  // backward: z tiles (136 rows) as shared-memory images
+    bf16 *Uf;    // forward, H < 8: U [R, G*W] with each 8/H groups' columns tap-major (k*GPV + g)
 };
 
 // Fills the common part of the map; false when the tensor-core kernels do not take the shape.

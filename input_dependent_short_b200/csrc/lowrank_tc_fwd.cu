@@ -238,34 +238,36 @@ __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char 
                     make_uint4(pack_bf2(lo2(yp[0]), hi2(yp[0])), pack_bf2(lo2(yp[1]), hi2(yp[1])),
                                pack_bf2(lo2(yp[2]), hi2(yp[2])), pack_bf2(lo2(yp[3]), hi2(yp[3])));
             } else {
-                // several groups per vector: per-vector loads, the next one in flight while this one computes
+                // several groups per vector: per-vector loads, the next one in flight while this one computes.
+                // The vector's GPV groups have their filters tap-major (column k*GPV + g, from the
+                // permuted U image), so the filters of a channel pair at tap k sit in adjacent
+                // registers and one fma.rn.f32x2 applies a tap to both channels.
                 tc::tmem_wait_ld();
                 float *w = wt + (v & 1) * NT;
                 if (v + 1 < VPT)
                     tmem_ld<NT>(tb + (uint32_t)(((ci0 + 8 * (v + 1)) >> m.lgH) * W),
                                 *reinterpret_cast<float(*)[NT]>(wt + ((v + 1) & 1) * NT));
-                float y[8];
+                u64 y2[4];
 #pragma unroll
                 for (int pp = 0; pp < 4; ++pp) {
                     const int g0 = (2 * pp) / CPG, g1 = (2 * pp + 1) / CPG;
-                    float a0 = 0.f, a1 = 0.f;
 #pragma unroll
                     for (int k = 0; k < W; ++k) {
                         const uint32_t word = word_of(xw[vv][k], pp);
+                        const u64 xp = mk2(bf_lo(word), bf_hi(word));
+                        u64 wp = mk2(w[k * GPV + g0], w[k * GPV + g1]);
                         if (k == 0) {  // tap 0 carries the residual
-                            a0 = (w[g0 * W] + res) * bf_lo(word);
-                            a1 = (w[g1 * W] + res) * bf_hi(word);
+                            wp = add2(wp, mk2(res, res));
+                            y2[pp] = mul2(wp, xp);
                         } else {
-                            a0 = fmaf(w[g0 * W + k], bf_lo(word), a0);
-                            a1 = fmaf(w[g1 * W + k], bf_hi(word), a1);
+                            y2[pp] = fma2(wp, xp, y2[pp]);
                         }
                     }
-                    y[2 * pp] = a0;
-                    y[2 * pp + 1] = a1;
                 }
                 const int cs = cs0 + 8 * v;
                 *reinterpret_cast<uint4 *>(ys + (uint32_t)(cs / (RB / 2)) * ybox + tc::swz<RB>(t_loc, (cs % (RB / 2)) / 8)) =
-                    make_uint4(pack_bf2(y[0], y[1]), pack_bf2(y[2], y[3]), pack_bf2(y[4], y[5]), pack_bf2(y[6], y[7]));
+                    make_uint4(pack_bf2(lo2(y2[0]), hi2(y2[0])), pack_bf2(lo2(y2[1]), hi2(y2[1])),
+                               pack_bf2(lo2(y2[2]), hi2(y2[2])), pack_bf2(lo2(y2[3]), hi2(y2[3])));
             }
         }
     }
@@ -484,6 +486,23 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
     if (warp == 17) tc::tmem_dealloc(tmem, (uint32_t)(2 * m.NFS));
 }
 
+// U with the columns of every GPV = 8/H consecutive groups tap-major: column
+// c*GPV*W + k*GPV + g of the image holds U column (c*GPV + g)*W + k.  With
+// it, the MMA leaves a vector's filters with the taps outermost, so the two
+// channels of a pair find tap k in adjacent registers.
+__global__ void k_fwd_uperm(const bf16 *__restrict__ U, bf16 *__restrict__ Uf, int64_t R, int64_t GW, int W, int GPV) {
+    pdl_wait();
+    pdl_trigger();
+    const int64_t n = R * GW;
+    const int64_t chunk = (int64_t)GPV * W;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / GW, j = i % GW;  // image element (r, j)
+        const int64_t c = j / chunk, q = j % chunk;
+        const int64_t k = q / GPV, g = q % GPV;
+        Uf[i] = U[r * GW + (c * GPV + g) * W + k];
+    }
+}
+
 // Forward plan: the widest channel block whose filters fit half of TMEM
 // (NF <= 256 columns; a buffer takes NFS = NF rounded up to a power of two),
 // narrowed while it still spans 8 or more sub-tiles of 128 channels;
@@ -528,7 +547,8 @@ bool fwd_maps(const TcArgs &a, FwdMaps &f) {
     return make_map(&f.x, a.x, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
            make_map(&f.y, a.y, 3, xd, xs, yb, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE) &&
            make_map(&f.z, a.z, 3, zd, zs, zb, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
-           make_map(&f.u, a.U, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
+           make_map(&f.u, a.Uf ? a.Uf : a.U, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
 }
 
 template <int W, int GPV, int VPT, int NGT>
@@ -593,13 +613,29 @@ bool lowrank_tc_ok(const dsc_problem &p) {
     return lrtc::tc_map(p, m) && lrtc::tc_fwd_plan(m);
 }
 
-cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U, void *y) {
+// Scratch of the tensor-core forward: the permuted U image when several
+// groups share a vector (H < 8), else nothing.
+size_t lr_tc_fwd_ws_bytes(const dsc_problem &p) {
+    if (!lowrank_tc_ok(p) || p.H >= 8) return 0;
+    return ((size_t)p.R * (size_t)((p.D / p.H) * p.W) * 2 + 255) & ~(size_t)255;
+}
+
+cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, const void *z, const void *U, void *y,
+                             void *ws, size_t ws_bytes) {
     lrtc::TcArgs a{};
     if (!lrtc::tc_map(p, a.m) || !lrtc::tc_fwd_plan(a.m)) return cudaErrorNotSupported;
     a.x = static_cast<const bf16 *>(x);
     a.z = static_cast<const bf16 *>(z);
     a.U = static_cast<const bf16 *>(U);
     a.y = static_cast<bf16 *>(y);
+    if (p.H < 8) {
+        if (!ws || ws_bytes < lr_tc_fwd_ws_bytes(p)) return cudaErrorInvalidValue;
+        a.Uf = static_cast<bf16 *>(ws);
+        const int64_t n = p.R * a.m.GW;
+        const cudaError_t e = launch_pdl(lrtc::k_fwd_uperm, dim3((unsigned)min((int64_t)1024, (n + 255) / 256)), dim3(256),
+                                         0, c.stream, a.U, a.Uf, (int64_t)p.R, a.m.GW, (int)p.W, (int)(8 / p.H));
+        if (e != cudaSuccess) return e;
+    }
     switch (a.m.W) {
     case 1: return lrtc::fwd_by_gpv<1>(c, a);
     case 2: return lrtc::fwd_by_gpv<2>(c, a);

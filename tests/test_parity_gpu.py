@@ -385,7 +385,7 @@ def test_sweep_workloads_sampled(wl):
                          ids=["all-linear-shape", "qkv-shape"])
 def test_lowrank_fused_materialises_no_filters(shape):
     """The fused low-rank kernels never hold w = zU or dw in device memory: the
-    forward needs no workspace, the backward's workspace (operand images of z
+    forward's workspace is at most a copy of U, the backward's workspace (operand images of z
     and U, per-range dU partials and an fp32 dz accumulator: O(B*T*R +
     ranges*R*G*W), not O(B*T*G*W)) stays well below the fp32 filter tensor,
     and the peak allocation grows by the outputs and that workspace only.  On
@@ -405,7 +405,8 @@ def test_lowrank_fused_materialises_no_filters(shape):
     L = _lib.lib()
     filters = B * T * (D // H) * W * 4
     ws = L.dsc_bwd_lowrank_workspace_bytes(C.byref(p))
-    assert L.dsc_fwd_lowrank_workspace_bytes(C.byref(p)) == 0
+    wsf = L.dsc_fwd_lowrank_workspace_bytes(C.byref(p))
+    assert wsf <= R * (D // H) * W * 2 + 256  # at most a tap-ordered copy of U
     assert ws < filters / 2
     if (D // H) * W > 4096:
         assert ws < filters / 20
@@ -416,4 +417,4 @@ def test_lowrank_fused_materialises_no_filters(shape):
     dx, dz, dU = o.dsc_bwd_lowrank(x, z, U, dy, H)
     torch.cuda.synchronize()
     outputs = sum(v.numel() * v.element_size() for v in (y, dx, dz, dU))
-    assert torch.cuda.max_memory_allocated() - base <= outputs + ws + (1 << 20)
+    assert torch.cuda.max_memory_allocated() - base <= outputs + ws + wsf + (1 << 20)
