@@ -631,12 +631,16 @@ void finish_map(StreamMap &m, int64_t target_warps) {
     m.n_warps = m.B * m.nTiles * (int64_t)m.nWc;
 }
 
-// The plan: 8-byte vectors for W >= 5 when that mapping exists (two blocks
-// per SM instead of one), else 16-byte vectors; false when neither exists
-// (the generic kernels take the shape).
+// The plan: 8-byte vectors for W >= 5 when that mapping keeps every filter
+// group inside one thread (two blocks per SM instead of one, and no cross-lane
+// reduction), else 16-byte vectors; false when neither exists (the generic
+// kernels take the shape).  Groups that span lanes keep 16-byte vectors:
+// halving the vector would double the lanes of a group and with them the
+// shuffle levels of its dw reduction per byte, which costs more than the
+// second block gains (measured at W = 8, H = 16 and 128).
 bool stream_plan(const dsc_problem &p, StreamMap &m) {
     const int V16 = p.dtype == DSC_BF16 ? 8 : 4;
-    if (p.W >= 5 && stream_map(p, V16 / 2, m)) {
+    if (p.W >= 5 && stream_map(p, V16 / 2, m) && m.L == 1) {
         m.vb = 8;
         return true;
     }

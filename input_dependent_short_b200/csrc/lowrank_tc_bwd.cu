@@ -211,7 +211,7 @@ __device__ __forceinline__ void bwd_dw_groups(const TcMap &m, const unsigned cha
 // One sub-tile of the epilogue for token t_loc, thread part `part`.
 //   VPT vectors of 8 channels; GPT groups among the thread's 8*VPT channels
 //   (1 when the group is wider: PPG parts then share it).
-template <int W, int VPT, int GPT, int PPG, int RB, bool DX = true, bool DWS = true>
+template <int W, int VPT, int GPT, int PPG, int RB>
 __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
                                             unsigned char *dwt, float *xch, int part, int t_loc, int s,
                                             unsigned char *ys, float res, uint32_t release_w) {
@@ -223,35 +223,30 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
     const int ci0 = s * m.SB + cs0;                  // block channel
     const int g0 = ci0 >> m.lgH;                     // block group of the thread's first channel
     // filters w[t+k, g0 .. g0+GPT-1, k] (tap-major TMEM columns k*GB + g)
-    float wt[W][GPT];  // (not read without DX)
-    if constexpr (DX) {
+    float wt[W][GPT];
 #pragma unroll
-        for (int k = 0; k < W; ++k) tmem_ld<GPT>(tb + (uint32_t)(k * m.GB + g0), wt[k]);
-    }
+    for (int k = 0; k < W; ++k) tmem_ld<GPT>(tb + (uint32_t)(k * m.GB + g0), wt[k]);
     const unsigned char *xb = xs;          // x rows t0-WIN .. t0+127
     const unsigned char *yb = xs + boxb;   // dy rows t0 .. t0+127+WIN
-    constexpr int NDY = DX ? W : 1;        // dy rows t .. t+W-1 for dx, row t for dw
     uint4 dyv[VPT][W];
 #pragma unroll
     for (int v = 0; v < VPT; ++v) {
         const int cs = cs0 + 8 * v;
         const int bo = (cs % (RB / 2)) / 8;
 #pragma unroll
-        for (int k = 0; k < NDY; ++k) dyv[v][k] = *reinterpret_cast<const uint4 *>(yb + tc::swz<RB>(t_loc + k, bo));
+        for (int k = 0; k < W; ++k) dyv[v][k] = *reinterpret_cast<const uint4 *>(yb + tc::swz<RB>(t_loc + k, bo));
     }
-    if constexpr (DX) {
-        tc::tmem_wait_ld();
-        if (release_w) {  // the item's last filter read: its TMEM buffer is free for the next MMA
-            tc::fence_before_sync();
-            __syncwarp();
-            if ((threadIdx.x & 31) == 0) tc::mbar_arrive(release_w);
-        }
+    tc::tmem_wait_ld();
+    if (release_w) {  // the item's last filter read: its TMEM buffer is free for the next MMA
+        tc::fence_before_sync();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) tc::mbar_arrive(release_w);
+    }
 #pragma unroll
-        for (int g = 0; g < GPT; ++g) wt[0][g] += res;
-    }
+    for (int g = 0; g < GPT; ++g) wt[0][g] += res;
     // dx
 #pragma unroll
-    for (int v = 0; v < (DX ? VPT : 0); ++v) {
+    for (int v = 0; v < VPT; ++v) {
         float dxv[8];
 #pragma unroll
         for (int pp = 0; pp < 4; ++pp) {
@@ -294,9 +289,7 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
             make_uint4(pack_bf2(dxv[0], dxv[1]), pack_bf2(dxv[2], dxv[3]), pack_bf2(dxv[4], dxv[5]),
                        pack_bf2(dxv[6], dxv[7]));
     }
-    if constexpr (!DWS) {
-        return;
-    } else if constexpr (GPT == CT) {
+    if constexpr (GPT == CT) {
         // one channel per group (H = 1): dw[t, g, k] = dy[t, c] x[t-k, c], rounded once to bf16
 #pragma unroll
         for (int v = 0; v < VPT; ++v) {
@@ -317,7 +310,7 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
 // The same for sub-tiles of 16 channels (blocks of 16 groups, H = 1): the
 // thread's 4 channels are the 8 bytes at `off` in 16-byte chunk `chunk` of
 // each 32-byte row; channel i of the thread is its group g0 + i.
-template <int W, bool DX = true, bool DWS = true>
+template <int W>
 __device__ __forceinline__ void bwd_subtile_q(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
                                               unsigned char *dwt, int part, int t_loc, int s, unsigned char *ys,
                                               float res, uint32_t release_w) {
@@ -325,41 +318,36 @@ __device__ __forceinline__ void bwd_subtile_q(const TcMap &m, const unsigned cha
     const int g0 = s * m.SB + part * 4;  // block group = block channel of the thread's first channel
     const int chunk = part >> 1;
     const uint32_t off = (uint32_t)(part & 1) * 8u;
+    float wt[W][4];
+#pragma unroll
+    for (int k = 0; k < W; ++k) tmem_ld<4>(tb + (uint32_t)(k * m.GB + g0), wt[k]);
     const unsigned char *xb = xs;         // x rows t0-WIN .. t0+127
     const unsigned char *yb = xs + boxb;  // dy rows t0 .. t0+127+WIN
     uint2 dyv[W];
-    if constexpr (DX) {
-        float wt[W][4];
 #pragma unroll
-        for (int k = 0; k < W; ++k) tmem_ld<4>(tb + (uint32_t)(k * m.GB + g0), wt[k]);
-#pragma unroll
-        for (int k = 0; k < W; ++k) dyv[k] = *reinterpret_cast<const uint2 *>(yb + tc::swz<32>(t_loc + k, chunk) + off);
-        tc::tmem_wait_ld();
-        if (release_w) {  // the item's last filter read: its TMEM buffer is free for the next MMA
-            tc::fence_before_sync();
-            __syncwarp();
-            if ((threadIdx.x & 31) == 0) tc::mbar_arrive(release_w);
-        }
-#pragma unroll
-        for (int g = 0; g < 4; ++g) wt[0][g] += res;
-        // dx
-        uint32_t dxw[2];
-#pragma unroll
-        for (int pp = 0; pp < 2; ++pp) {
-            u64 acc2 = 0ull;
-#pragma unroll
-            for (int k = 0; k < W; ++k) {
-                const uint32_t word = pp ? dyv[k].y : dyv[k].x;
-                const u64 wp = mk2(wt[k][2 * pp], wt[k][2 * pp + 1]), dp = mk2(bf_lo(word), bf_hi(word));
-                acc2 = k == 0 ? mul2(wp, dp) : fma2(wp, dp, acc2);
-            }
-            dxw[pp] = pack_bf2(lo2(acc2), hi2(acc2));
-        }
-        *reinterpret_cast<uint2 *>(ys + tc::swz<32>(t_loc, chunk) + off) = make_uint2(dxw[0], dxw[1]);
-    } else {
-        dyv[0] = *reinterpret_cast<const uint2 *>(yb + tc::swz<32>(t_loc, chunk) + off);
+    for (int k = 0; k < W; ++k) dyv[k] = *reinterpret_cast<const uint2 *>(yb + tc::swz<32>(t_loc + k, chunk) + off);
+    tc::tmem_wait_ld();
+    if (release_w) {  // the item's last filter read: its TMEM buffer is free for the next MMA
+        tc::fence_before_sync();
+        __syncwarp();
+        if ((threadIdx.x & 31) == 0) tc::mbar_arrive(release_w);
     }
-    if constexpr (!DWS) return;
+#pragma unroll
+    for (int g = 0; g < 4; ++g) wt[0][g] += res;
+    // dx
+    uint32_t dxw[2];
+#pragma unroll
+    for (int pp = 0; pp < 2; ++pp) {
+        u64 acc2 = 0ull;
+#pragma unroll
+        for (int k = 0; k < W; ++k) {
+            const uint32_t word = pp ? dyv[k].y : dyv[k].x;
+            const u64 wp = mk2(wt[k][2 * pp], wt[k][2 * pp + 1]), dp = mk2(bf_lo(word), bf_hi(word));
+            acc2 = k == 0 ? mul2(wp, dp) : fma2(wp, dp, acc2);
+        }
+        dxw[pp] = pack_bf2(lo2(acc2), hi2(acc2));
+    }
+    *reinterpret_cast<uint2 *>(ys + tc::swz<32>(t_loc, chunk) + off) = make_uint2(dxw[0], dxw[1]);
     // dw[t, g0+i, k] = dy[t, c] x[t-k, c] (one channel per group), rounded once to bf16
 #pragma unroll
     for (int k = 0; k < W; ++k) {
@@ -369,17 +357,11 @@ __device__ __forceinline__ void bwd_subtile_q(const TcMap &m, const unsigned cha
     }
 }
 
-// MODE 0: the whole backward.  MODE 1: dx only (filter MMAs and the dx
-// epilogue).  MODE 2: the filter-gradient side only (dw, dz and dU MMAs).
-// Modes 1 and 2 run back to back where the contractions dominate (H = 1):
-// each keeps a shorter chain of hand-offs per item, at the price of reading
-// dy twice.
-template <int W, int VPT, int GPT, int PPG, int MODE>
+template <int W, int VPT, int GPT, int PPG>
 __global__ void __launch_bounds__(TB_THREADS, 1)
     k_lr_tc_bwd(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tmdy,
                 const __grid_constant__ CUtensorMap tmdx, const TcArgs a) {
     constexpr int WIN = W - 1;
-    constexpr bool DX = MODE != 2, DWS = MODE != 1;
     constexpr int RB = VPT == 0 ? 32 : (VPT == 1 ? 64 : 128);  // box row bytes (16, 32 or 64 channels)
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     const TcMap &m = a.m;
@@ -419,7 +401,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
     if (tid == 0) {
         for (int i = 0; i < TB_MAXOP; ++i) {
             tc::mbar_init(bars.opf(i), 1);
-            tc::mbar_init(bars.ope(i), DWS ? 2 : 1);  // dz and dU MMAs of the item (dx only: filter MMAs)
+            tc::mbar_init(bars.ope(i), 2);  // dz and dU MMAs of the item, from two threads
         }
         for (int i = 0; i < 2; ++i) {
             tc::mbar_init(bars.wf(i), 1);
@@ -478,18 +460,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             for (; nload < NOP && nload < nI; ++nload) load_op(nload);
             int fob = 0, fdb = 0, ftl = 0, fcl = 0;
             uint32_t fdph = 0, foph = 0;
-            for (int li = 0; li < nI && !DWS; ++li) {  // dx only: refill once the filter MMAs are done
-                if (nload < nI) {
-                    wait(bars.ope(fob), foph);
-                    load_op(fob);
-                    ++nload;
-                }
-                if (++fob == NOP) {
-                    fob = 0;
-                    foph ^= 1u;
-                }
-            }
-            for (int li = 0; li < nI && DWS; ++li) {
+            for (int li = 0; li < nI; ++li) {
                 wait(bars.dwf(fdb), fdph);  // item li's dw tile is complete
                 tc::fence_after_sync();
                 const uint32_t zb = sbase + (uint32_t)fob * S.opsize;
@@ -520,7 +491,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                     ++ftl;
                 }
             }
-            if constexpr (DWS) tc::mma_commit(bars.duf());
+            tc::mma_commit(bars.duf());
             for (int b = 0; b < NOP && b < nI; ++b) {  // the last loads have landed
                 const int last = b + ((nI - 1 - b) / NOP) * NOP;
                 tc::mbar_wait(bars.opf(b), (uint32_t)((last / NOP) & 1), TC_WAIT_LIMIT);
@@ -538,9 +509,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                 for (int s = s_begin(li); s < s_end(li); ++s, ++l) {
                     if (l >= NS) wait(bars.xe(slot), xph ^ 1u);
                     const uint32_t xb = sbase + S.ring + (uint32_t)slot * S.slot;
-                    tc::mbar_expect_tx(bars.xf(slot), (uint32_t)((DWS ? 2 : 1) * RB * (TC_M + WIN)));
+                    tc::mbar_expect_tx(bars.xf(slot), (uint32_t)(2 * RB * (TC_M + WIN)));
                     const int c = it.blk * m.CB + s * m.SB;
-                    if constexpr (DWS) tc::tma_load_3d(xb, &tmx, c, it.t0 - WIN, it.b, bars.xf(slot));
+                    tc::tma_load_3d(xb, &tmx, c, it.t0 - WIN, it.b, bars.xf(slot));
                     tc::tma_load_3d(xb + S.boxb, &tmdy, c, it.t0, it.b, bars.xf(slot));
                     if (++slot == NS) {
                         slot = 0;
@@ -558,7 +529,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         // One lane issues each item's per-tap MMAs; the dz / dU MMAs come from
         // warp 19, so the two streams of instructions overlap (a commit tracks
         // only the MMAs of the thread that issues it).
-        if (lane == 0 && DX) {
+        if (lane == 0) {
             const uint32_t id_w = tc::idesc_bf16(TC_M, m.GB, 0, 1);
             int ob = 0;
             uint32_t oph = 0;
@@ -576,7 +547,6 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                         tc::mma_bf16(tmem + (uint32_t)(b * TB_NB + k * m.GB), ad, bd, id_w, ks > 0 ? 1u : 0u);
                     }
                 tc::mma_commit(bars.wf(b));
-                if constexpr (!DWS) tc::mma_commit(bars.ope(ob));  // dx only: the operand buffer is free
                 if (++ob == NOP) {
                     ob = 0;
                     oph ^= 1u;
@@ -585,7 +555,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         }
     } else if (warp == 19) {
         // ---------------------------------------------------- dz MMAs
-        if (lane == 0 && DWS) {
+        if (lane == 0) {
             const uint32_t id_dz = tc::idesc_bf16(TC_M, m.RP, 0, 0);
             int fob = 0, fdb = 0, ftl = 0, fcl = 0;
             uint32_t fdph = 0;
@@ -652,13 +622,13 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         uint32_t xph = 0, dph = 0;
         for (int li = 0; li < nI; ++li) {
             const int b = li & 1;
-            if constexpr (DX) wait(bars.wf(b), (uint32_t)((li >> 1) & 1));
-            if (DWS && li >= DWB) wait(bars.dwe(db), dph ^ 1u);
+            wait(bars.wf(b), (uint32_t)((li >> 1) & 1));
+            if (li >= DWB) wait(bars.dwe(db), dph ^ 1u);
             tc::fence_after_sync();
             const uint32_t tb = tlane + (uint32_t)(b * TB_NB);
             unsigned char *dwt = smem + S.dw + (uint32_t)db * S.dwsize;
             const int sb = s_begin(li), se = s_end(li);
-            if (DWS && (sb > 0 || se < m.nSubB)) {
+            if (sb > 0 || se < m.nSubB) {
                 // part of the block's groups only: the other dw columns must read as zero
                 for (int i = tid; i < TC_M * TB_NB * 2 / 16; i += TB_EPI)
                     *reinterpret_cast<uint4 *>(dwt + 16 * i) = make_uint4(0, 0, 0, 0);
@@ -667,57 +637,51 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
             for (int s = sb; s < se; ++s) {
                 wait(bars.xf(slot), xph);
                 if constexpr (VPT == 0)
-                    bwd_subtile_q<W, DX, DWS>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, part, t_loc,
-                                              s, smem + S.ystage + (uint32_t)ybuf * S.ybox, res,
-                                              s == se - 1 ? bars.we(b) : 0u);
+                    bwd_subtile_q<W>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, part, t_loc, s,
+                                     smem + S.ystage + (uint32_t)ybuf * S.ybox, res, s == se - 1 ? bars.we(b) : 0u);
                 else
-                    bwd_subtile<W, VPT, GPT, PPG, RB, DX, DWS>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb,
-                                                               dwt, xch, part, t_loc, s,
-                                                               smem + S.ystage + (uint32_t)ybuf * S.ybox, res,
-                                                               s == se - 1 ? bars.we(b) : 0u);
+                    bwd_subtile<W, VPT, GPT, PPG, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, xch,
+                                                      part, t_loc, s, smem + S.ystage + (uint32_t)ybuf * S.ybox, res,
+                                                      s == se - 1 ? bars.we(b) : 0u);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars.xe(slot));
-                if constexpr (DX) {
-                    // dx tile -> global by TMA (the staging tile the next sub-tile writes was read
-                    // by the store issued one sub-tile ago, waited for before this barrier)
-                    tc::fence_proxy_async();
-                    if (tid == 0) tc::bulk_wait_read_all();
-                    epi_bar();
-                    if (tid == 0) {
-                        tc::tma_store_3d(&tmdx, sbase + S.ystage + (uint32_t)ybuf * S.ybox, it.blk * m.CB + s * m.SB,
-                                         it.t0, it.b);
-                        tc::bulk_commit();
-                    }
-                    ybuf ^= 1;
+                // dx tile -> global by TMA (the staging tile the next sub-tile writes was read
+                // by the store issued one sub-tile ago, waited for before this barrier)
+                tc::fence_proxy_async();
+                if (tid == 0) tc::bulk_wait_read_all();
+                epi_bar();
+                if (tid == 0) {
+                    tc::tma_store_3d(&tmdx, sbase + S.ystage + (uint32_t)ybuf * S.ybox, it.blk * m.CB + s * m.SB, it.t0,
+                                     it.b);
+                    tc::bulk_commit();
                 }
+                ybuf ^= 1;
                 if (++slot == NS) {
                     slot = 0;
                     xph ^= 1u;
                 }
             }
-            if constexpr (DWS) {
-                tc::fence_proxy_async();  // dw tile (generic stores) -> MMA operand
-                tc::fence_before_sync();
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bars.dwf(db));
-                if (++db == DWB) {
-                    db = 0;
-                    dph ^= 1u;
-                }
-                // the previous tile's dz (its last MMAs have had this whole item to finish)
-                if (li >= 1 && it.cl == 0) dz_out(it.tl - 1, pb, pt0);
+            tc::fence_proxy_async();  // dw tile (generic stores) -> MMA operand
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(bars.dwf(db));
+            if (++db == DWB) {
+                db = 0;
+                dph ^= 1u;
             }
+            // the previous tile's dz (its last MMAs have had this whole item to finish)
+            if (li >= 1 && it.cl == 0) dz_out(it.tl - 1, pb, pt0);
             pb = it.b;
             pt0 = it.t0;
             it.next(m, chunk_lo, ncl);
         }
-        if constexpr (DWS) dz_out(ntl - 1, pb, pt0);
+        dz_out(ntl - 1, pb, pt0);
         // dU of the CTA's blocks over its tile range: TMEM lane = block column k*GB + g
         // (lanes NBW .. 127 hold no filter column)
-        if constexpr (DWS) wait(bars.duf(), 0);
+        wait(bars.duf(), 0);
         tc::fence_after_sync();
         const int k = t_loc / m.GB, gl = t_loc % m.GB;
-        for (int cl = 0; cl < (DWS ? ncl : 0); ++cl) {
+        for (int cl = 0; cl < ncl; ++cl) {
             const int64_t col = (int64_t)(chunk_lo + cl) * m.NBW + gl * W + k;
             for (int r8 = 8 * part; r8 < m.RP; r8 += 32) {  // 8-column chunks, dealt round the parts
                 float v[8];
@@ -738,7 +702,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 
     // teardown: every load and MMA this CTA issued has landed before the
     // shared memory and TMEM are given back (bounded, also after a time-out)
-    if (DWS && warp == 18 && lane == 0) tc::mbar_wait(bars.duf(), 0, TC_WAIT_LIMIT);
+    if (warp == 18 && lane == 0) tc::mbar_wait(bars.duf(), 0, TC_WAIT_LIMIT);
     if (timed_out) atomicExch(&g_dsc_status_tcb, (int)DSC_ERR_TIMEOUT);
     tc::fence_before_sync();
     __syncthreads();
@@ -916,15 +880,10 @@ bool bwd_maps(const TcArgs &a, BwdMaps &f) {
            make_map(&f.dx, a.dx, 3, xd, xs, yb, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE);
 }
 
-// H = 1: every channel has its own filter and the three contractions per
-// item dominate; the dx side and the filter-gradient side run as two passes
-// (modes 1 and 2).  Otherwise one pass (mode 0).
-static bool bwd_split(const TcMap &m) { return m.H == 1; }
-
-template <int W, int VPT, int GPT, int PPG, int MODE = 0>
-cudaError_t launch_bwd_mode(const Ctx &c, const TcArgs &a) {
+template <int W, int VPT, int GPT, int PPG>
+cudaError_t launch_bwd(const Ctx &c, const TcArgs &a) {
     const BwdSmem S(a.m, a.m.NOP, a.m.NSB, a.m.DWB, PPG > 1);
-    static const cudaError_t attr = cudaFuncSetAttribute(k_lr_tc_bwd<W, VPT, GPT, PPG, MODE>,
+    static const cudaError_t attr = cudaFuncSetAttribute(k_lr_tc_bwd<W, VPT, GPT, PPG>,
                                                          cudaFuncAttributeMaxDynamicSharedMemorySize, TB_SMEM);
     if (attr != cudaSuccess) return attr;
     if (S.total > TB_SMEM) return cudaErrorInvalidValue;
@@ -932,22 +891,9 @@ cudaError_t launch_bwd_mode(const Ctx &c, const TcArgs &a) {
     if (!bwd_maps(a, f)) return cudaErrorNotSupported;
     // the whole of TMEM per CTA: enough shared memory that no second CTA shares the SM
     const uint32_t smem = S.total < 120 * 1024 ? 120 * 1024 : S.total;
-    const cudaError_t e = launch_pdl(k_lr_tc_bwd<W, VPT, GPT, PPG, MODE>, dim3((unsigned)(a.m.nGroups * a.m.nRanges)),
+    const cudaError_t e = launch_pdl(k_lr_tc_bwd<W, VPT, GPT, PPG>, dim3((unsigned)(a.m.nGroups * a.m.nRanges)),
                                      dim3(TB_THREADS), smem, c.stream, f.x, f.dy, f.dx, a);
     return e != cudaSuccess ? e : cudaGetLastError();
-}
-
-template <int W, int VPT, int GPT, int PPG>
-cudaError_t launch_bwd(const Ctx &c, const TcArgs &a) {
-    return launch_bwd_mode<W, VPT, GPT, PPG, 0>(c, a);
-}
-
-// H = 1 shapes: one pass, or the two passes of bwd_split.
-template <int W, int VPT, int GPT>
-cudaError_t launch_bwd_h1(const Ctx &c, const TcArgs &a) {
-    if (!bwd_split(a.m)) return launch_bwd_mode<W, VPT, GPT, 1, 0>(c, a);
-    const cudaError_t e = launch_bwd_mode<W, VPT, GPT, 1, 1>(c, a);
-    return e != cudaSuccess ? e : launch_bwd_mode<W, VPT, GPT, 1, 2>(c, a);
 }
 
 // Thread channels per sub-tile: CT = 8*VPT (SB = 32 or 64, four parts).
@@ -958,7 +904,7 @@ template <int W, int VPT> cudaError_t bwd_by_h(const Ctx &c, const TcArgs &a) {
         return cudaErrorNotSupported;
     }
     switch (a.m.H) {
-    case 1: if constexpr (CT * W <= 32) return launch_bwd_h1<W, VPT, CT>(c, a); break;
+    case 1: if constexpr (CT * W <= 32) return launch_bwd<W, VPT, CT, 1>(c, a); break;
     case 2: if constexpr (CT / 2 * W <= 32) return launch_bwd<W, VPT, CT / 2, 1>(c, a); break;
     case 4: return launch_bwd<W, VPT, CT / 4, 1>(c, a);
     case 8: return launch_bwd<W, VPT, CT / 8, 1>(c, a);
@@ -971,7 +917,7 @@ template <int W, int VPT> cudaError_t bwd_by_h(const Ctx &c, const TcArgs &a) {
 
 template <int W> cudaError_t bwd_by_vpt(const Ctx &c, const TcArgs &a) {
     if (a.m.SB == 16) {  // blocks of 16 single-channel groups (W >= 5, H = 1)
-        if constexpr (W >= 5) return launch_bwd_h1<W, 0, 4>(c, a);
+        if constexpr (W >= 5) return launch_bwd<W, 0, 4, 1>(c, a);
         return cudaErrorNotSupported;
     }
     return a.m.SB == 32 ? bwd_by_h<W, 1>(c, a) : bwd_by_h<W, 2>(c, a);
