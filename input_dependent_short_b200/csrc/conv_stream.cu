@@ -432,9 +432,10 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
                 dws[pp][k] = 0ull;
             }
     }
-    auto stap = [&](int pp, int k) -> u64 {
+    auto stap = [&](int pp, int k) -> u64 {  // static filters only
         if constexpr (WPK) return k == 0 ? w0p[pp] : mk2(bf_lo(wpk[pp][k]), bf_hi(wpk[pp][k]));
-        else return wsp[WS ? pp : 0][WS ? k : 0];
+        else if constexpr (WS) return wsp[pp][k];
+        else return 0ull;
     };
     uint32_t wreg[C::WREG ? NS : 1][F::WORDS];
 

@@ -78,3 +78,52 @@ def test_decode_reference_arm_runs_the_oracle_on_a_sample():
     wl = wls.DECODE_QKV_LOWRANK.with_(B=8, D=256)
     n, B, el = bench.decode_reference(wl, steps=2, warmup=1, sequences=4)
     assert n == 2 and B == 4 and el > 0
+
+
+def _dp_rank(rank, world, port, q):
+    """Data parallel: rank r holds batch rows r, r+world, ...; the per-rank
+    token reductions (low-rank dU, static dws), all-reduced, are the whole
+    batch's."""
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import oracle
+
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        rng = np.random.default_rng(3)
+        B, T, D, W, H, R = 4, 9, 6, 3, 2, 3
+        x, dy, z = rng.standard_normal((B, T, D)), rng.standard_normal((B, T, D)), rng.standard_normal((B, T, R))
+        U, ws = rng.standard_normal((R, (D // H) * W)), rng.standard_normal((D, W))
+        rows = list(range(rank, B, world))
+        mine = lambda a: np.ascontiguousarray(a[rows])  # noqa: E731
+        P = oracle.problem(len(rows), T, D, W, H, R, 1)
+        dU = torch.from_numpy(oracle.backward_lowrank(P, mine(x), mine(z), U, mine(dy))[2])
+        dws = torch.from_numpy(oracle.backward_static(oracle.problem(len(rows), T, D, W, 1, 0, 1), mine(x), ws,
+                                                      mine(dy))[1])
+        dist.all_reduce(dU)
+        dist.all_reduce(dws)
+        Pf = oracle.problem(B, T, D, W, H, R, 1)
+        ok = np.allclose(dU.numpy(), oracle.backward_lowrank(Pf, x, z, U, dy)[2], rtol=0, atol=1e-11)
+        ok &= np.allclose(dws.numpy(), oracle.backward_static(oracle.problem(B, T, D, W, 1, 0, 1), x, ws, dy)[1],
+                          rtol=0, atol=1e-11)
+        q.put((rank, bool(ok)))
+    finally:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def test_data_parallel_token_reductions_all_reduce_to_the_whole_batch():
+    world, port = 2, _free_port()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    procs = [ctx.Process(target=_dp_rank, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    out = dict(q.get(timeout=120) for _ in range(world))
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    assert out == {0: True, 1: True}
