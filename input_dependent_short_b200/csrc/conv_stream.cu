@@ -209,7 +209,13 @@ template <typename T, int W, int GPT, bool WS, bool BWD, int VB = 16> struct Str
     using F = FiltRow<T, NW>;
     static constexpr bool WRING = !WS && F::IN_SMEM;  // filter rows through the shared ring
     static constexpr bool WREG = !WS && !F::IN_SMEM;  // filter rows through a register ring
-    static constexpr int SUB = (BWD ? 2 : 1) + (WRING ? F::SLOTS : 0);  // 16-byte slots per token
+    // Ring slots per token (16 bytes x STREAM_THREADS each): the x (and, in
+    // the backward, dy) vectors, then the filter row.  8-byte vectors of one
+    // token share a slot, each row contiguous over the block's threads, so a
+    // warp's 8-byte accesses cover 256 consecutive bytes (no bank conflicts).
+    static constexpr int NV = BWD ? 2 : 1;
+    static constexpr int VSLOTS = VB == 16 ? NV : (NV * 8 + 15) / 16;
+    static constexpr int SUB = VSLOTS + (WRING ? F::SLOTS : 0);  // 16-byte slots per token
     static constexpr int NS = ring_depth(SUB);
     static constexpr size_t SMEM = (size_t)NS * SUB * 16 * STREAM_THREADS;
     // Blocks per SM the register budget is sized for: the narrow head-wise
@@ -294,9 +300,15 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
                         : static_cast<const char *>(a.w) + (row * m.G + q.c0 / m.H) * W * (int64_t)sizeof(T);
     const float res = m.residual ? 1.f : 0.f;
 
-    const uint32_t base = (uint32_t)__cvta_generic_to_shared(ring) + 16u * threadIdx.x;
+    const uint32_t ring0 = (uint32_t)__cvta_generic_to_shared(ring);
+    const uint32_t base = ring0 + 16u * threadIdx.x;
     constexpr uint32_t SUBSTRIDE = 16u * STREAM_THREADS;
     auto slot = [&](int s, int sub) { return base + (uint32_t)(s * C::SUB + sub) * SUBSTRIDE; };
+    // Vector row r (0: x, 1: dy) of ring token s.
+    auto vslot = [&](int s, int r) {
+        if constexpr (VB == 16) return slot(s, r);
+        else return ring0 + 8u * threadIdx.x + (uint32_t)(s * C::SUB) * SUBSTRIDE + (uint32_t)r * (8u * STREAM_THREADS);
+    };
 
     u64 wsp[WS ? P : 1][WS ? W : 1];  // static filters as pairs (tap 0 carries the residual)
     if constexpr (WS) {
@@ -311,8 +323,8 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
 
     auto issue = [&](int i, int s, bool full) {
         if (full || i < n) {
-            IO::cp(slot(s, 0), xp + i * xstep);
-            if constexpr (C::WRING) F::copy(slot(s, 1), SUBSTRIDE, wp + i * wstep);
+            IO::cp(vslot(s, 0), xp + i * xstep);
+            if constexpr (C::WRING) F::copy(slot(s, C::VSLOTS), SUBSTRIDE, wp + i * wstep);
             if constexpr (C::WREG) F::load_direct(wp + i * wstep, wreg[s]);
         }
         cp_commit();
@@ -339,9 +351,9 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, fals
             issue(i + NS - 1, (u + NS - 1) % NS, FULL);
             cp_wait<NS - 1>();
             u64 xc[P], acc[P];
-            PR::unpack(IO::lds(slot(u, 0)), xc);
+            PR::unpack(IO::lds(vslot(u, 0)), xc);
             uint32_t wv[F::WORDS];
-            if constexpr (C::WRING) F::read(slot(u, 1), SUBSTRIDE, wv);
+            if constexpr (C::WRING) F::read(slot(u, C::VSLOTS), SUBSTRIDE, wv);
             if constexpr (C::WREG)
 #pragma unroll
                 for (int k = 0; k < F::WORDS; ++k) wv[k] = wreg[u][k];
@@ -404,9 +416,15 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
     char *dwp = WS ? nullptr : static_cast<char *>(a.dw) + (row * m.G + c0 / m.H) * W * (int64_t)sizeof(T);
     const float res = m.residual ? 1.f : 0.f;
 
-    const uint32_t base = (uint32_t)__cvta_generic_to_shared(ring) + 16u * threadIdx.x;
+    const uint32_t ring0 = (uint32_t)__cvta_generic_to_shared(ring);
+    const uint32_t base = ring0 + 16u * threadIdx.x;
     constexpr uint32_t SUBSTRIDE = 16u * STREAM_THREADS;
     auto slot = [&](int s, int sub) { return base + (uint32_t)(s * C::SUB + sub) * SUBSTRIDE; };
+    // Vector row r (0: x, 1: dy) of ring token s.
+    auto vslot = [&](int s, int r) {
+        if constexpr (VB == 16) return slot(s, r);
+        else return ring0 + 8u * threadIdx.x + (uint32_t)(s * C::SUB) * SUBSTRIDE + (uint32_t)r * (8u * STREAM_THREADS);
+    };
 
     // Static filters: fp32 pairs, or (bf16 with 8-byte vectors, where the
     // registers are tightest) taps 1 .. W-1 as packed bf16 pairs, unpacked at
@@ -440,10 +458,10 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
     uint32_t wreg[C::WREG ? NS : 1][F::WORDS];
 
     auto issue = [&](int i, int s, bool full) {
-        if (full || i < n) IO::cp(slot(s, 0), xp + i * xstep);
+        if (full || i < n) IO::cp(vslot(s, 0), xp + i * xstep);
         if (full || i < nl) {
-            IO::cp(slot(s, 1), dyp + i * xstep);
-            if constexpr (C::WRING) F::copy(slot(s, 2), SUBSTRIDE, wp + i * wstep);
+            IO::cp(vslot(s, 1), dyp + i * xstep);
+            if constexpr (C::WRING) F::copy(slot(s, C::VSLOTS), SUBSTRIDE, wp + i * wstep);
             if constexpr (C::WREG) F::load_direct(wp + i * wstep, wreg[s]);
         }
         cp_commit();
@@ -475,13 +493,13 @@ __global__ void __launch_bounds__(STREAM_THREADS, (StreamCfg<T, W, GPT, WS, true
             const bool hx = FULL || i < n, hd = FULL || i < nl;
             u64 xc[P], dyc[P], r0[P];
             uint32_t wv[F::WORDS];
-            if (hx) PR::unpack(IO::lds(slot(u, 0)), xc);
+            if (hx) PR::unpack(IO::lds(vslot(u, 0)), xc);
             else
 #pragma unroll
                 for (int pp = 0; pp < P; ++pp) xc[pp] = 0ull;
             if (hd) {
-                PR::unpack(IO::lds(slot(u, 1)), dyc);
-                if constexpr (C::WRING) F::read(slot(u, 2), SUBSTRIDE, wv);
+                PR::unpack(IO::lds(vslot(u, 1)), dyc);
+                if constexpr (C::WRING) F::read(slot(u, C::VSLOTS), SUBSTRIDE, wv);
                 if constexpr (C::WREG)
 #pragma unroll
                     for (int k = 0; k < F::WORDS; ++k) wv[k] = wreg[u][k];

@@ -168,6 +168,9 @@ template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dw(co
 #pragma unroll
     for (int k = 0; k < 8; ++k) want[k] = had[k] = 0.f;
     if (live) {
+        // Unrolled so that several channels' loads are in flight at once (the
+        // loop is latency-bound: a few hundred threads, each reading H rows).
+#pragma unroll 8
         for (int64_t c = g * a.H; c < (g + 1) * a.H; ++c) {
             const float d = ldf<T>(a.dy, (b * a.T + t) * a.D + c);
 #pragma unroll

@@ -27,7 +27,10 @@
 //   k_proj_dV  per (128 model rows, token range): h^T x dz over the range,
 //              accumulated in TMEM, written as a per-range partial; a second
 //              kernel sums the partials in a fixed order (deterministic).
-// Operand tiles are TMA boxes of 8 columns (16-byte rows) laid out as the
+// h travels as TMA boxes of 64 model columns (128-byte rows, 128-byte
+// swizzle: one copy per 16 KB stage, full 128-byte requests), read by the MMA
+// through swizzled descriptors (K-major for z, MN-major for dV); the small
+// operands (V, dz) are boxes of 8 columns (16-byte rows) laid out as the
 // MMA's core matrices, as in the convolution kernels.
 #include "lowrank_tc.cuh"
 
@@ -138,9 +141,7 @@ __global__ void __launch_bounds__(PJ_THREADS, 1)
                     if (it >= PJ_NST) wait(empty(s), ph ^ 1u);
                     const uint32_t st = sbase + (uint32_t)s * sbytes;
                     tc::mbar_expect_tx(full(s), abytes + (uint32_t)kz * (PJ_KC * 16));
-                    for (int j = 0; j < PJ_KC / 8; ++j)
-                        tc::tma_load_2d(st + (uint32_t)j * (TC_M * 16), &tmh, kc * PJ_KC + 8 * j, (int)(tile * TC_M),
-                                        full(s));
+                    tc::tma_load_2d(st, &tmh, kc * PJ_KC, (int)(tile * TC_M), full(s));
                     for (int j = 0; j < kz; ++j)
                         tc::tma_load_2d(st + abytes + (uint32_t)j * (PJ_KC * 16), &tmv, 8 * j, kc * PJ_KC, full(s));
                     if (++s == PJ_NST) {
@@ -170,7 +171,7 @@ __global__ void __launch_bounds__(PJ_THREADS, 1)
                     tc::fence_after_sync();
                     const uint32_t st = sbase + (uint32_t)s * sbytes;
                     for (int ks = 0; ks < PJ_KC / 16; ++ks) {
-                        const uint64_t ad = tc::smem_desc(st + (uint32_t)ks * 2u * (TC_M * 16), TC_M * 16, 128);
+                        const uint64_t ad = tc::smem_desc_sw128(st + (uint32_t)ks * 32u, 16, 1024);
                         const uint64_t bd = tc::smem_desc(st + abytes + (uint32_t)ks * 256u, 128, PJ_KC * 16);
                         tc::mma_bf16(tmem + (uint32_t)(b * RP), ad, bd, id, (kc > 0 || ks > 0) ? 1u : 0u);
                     }
@@ -215,8 +216,10 @@ __global__ void __launch_bounds__(PJ_THREADS, 1)
 }
 
 // ---------------------------------------------------------- dh = dz V^T ---
-// Item = (tile of 128 tokens, 256 model columns).  A = dz tile [128 x RP]
-// (K-major), B = V rows [256 x RP] read as V^T (K-major), K = RP.
+// Item = (tile of 128 tokens, PH_NC model columns).  A = dz tile [128 x RP]
+// (K-major), B = V rows [PH_NC x RP] read as V^T (K-major), K = RP.  Two
+// CTAs per SM (TMEM: 2 x 256 columns).
+constexpr int PH_BOX = PH_NC / 64;  // staging boxes of 64 columns
 __global__ void __launch_bounds__(128, 1)
     k_proj_dh(const __grid_constant__ CUtensorMap tmdz, const __grid_constant__ CUtensorMap tmv,
               const __grid_constant__ CUtensorMap tmdh, const ProjArgs a, int nchunks) {
@@ -226,8 +229,8 @@ __global__ void __launch_bounds__(128, 1)
     unsigned char *smem = smem_raw + (sbase - sraw);
     const int RP = a.RP, kz = (int)(a.R / 8);
     const uint32_t abytes = (uint32_t)(TC_M * RP * 2), bbytes = (uint32_t)(PH_NC * RP * 2);
-    const uint32_t stage = abytes + bbytes;       // 4 staging boxes of [128 x 64] bf16 (128-byte swizzle)
-    const uint32_t bar = stage + 4 * TC_M * 128;  // one mbarrier for the loads, one for the MMAs
+    const uint32_t stage = abytes + bbytes;            // PH_BOX staging boxes of [128 x 64] bf16 (128-byte swizzle)
+    const uint32_t bar = stage + PH_BOX * TC_M * 128;  // one mbarrier for the loads, one for the MMAs
     const uint32_t tslot = bar + 16;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int64_t tile = blockIdx.x / nchunks;
@@ -276,19 +279,22 @@ __global__ void __launch_bounds__(128, 1)
     // accumulator row t (TMEM lane) -> bf16 -> swizzled staging box, then TMA stores
     const int t = warp * 32 + lane;
     const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    for (int c = 0; c < PH_NC; c += 8) {
-        float v[8];
-        tc::tmem_ld8(tl + (uint32_t)c, v);
+    for (int c0 = 0; c0 < PH_NC; c0 += 32) {
+        float v[32];
+        lrtc::tmem_ld<32>(tl + (uint32_t)c0, v);
         tc::tmem_wait_ld();
-        unsigned char *box = smem + stage + (uint32_t)(c / 64) * (TC_M * 128);
-        *reinterpret_cast<uint4 *>(box + tc::swz<128>(t, (c % 64) / 8)) =
-            make_uint4(pack_bf2(v[0], v[1]), pack_bf2(v[2], v[3]), pack_bf2(v[4], v[5]), pack_bf2(v[6], v[7]));
+        unsigned char *box = smem + stage + (uint32_t)(c0 / 64) * (TC_M * 128);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(box + tc::swz<128>(t, (c0 % 64) / 8 + q)) =
+                make_uint4(pack_bf2(v[8 * q], v[8 * q + 1]), pack_bf2(v[8 * q + 2], v[8 * q + 3]),
+                           pack_bf2(v[8 * q + 4], v[8 * q + 5]), pack_bf2(v[8 * q + 6], v[8 * q + 7]));
     }
     tc::fence_proxy_async();
     tc::fence_before_sync();
     __syncthreads();
     if (tid == 0) {
-        for (int bx = 0; bx < 4; ++bx)
+        for (int bx = 0; bx < PH_BOX; ++bx)
             if (chunk * PH_NC + bx * 64 < a.d)
                 tc::tma_store_3d(&tmdh, sbase + stage + (uint32_t)bx * (TC_M * 128), chunk * PH_NC + bx * 64,
                                  (int)(tile * TC_M), 0);
@@ -303,8 +309,9 @@ __global__ void __launch_bounds__(128, 1)
 
 // ---------------------------------------------------- dV = sum_t h^T dz ---
 // CTA = (128 model rows, range of token tiles).  Per tile: A = h^T [128 rows
-// x 128 tokens] (MN-major: h boxes of 8 model columns), B = dz tile [128
-// tokens x RP] (MN-major), 8 MMAs of K = 16 tokens into one TMEM accumulator.
+// x 128 tokens] (MN-major: two swizzled h boxes of 64 model columns), B = dz
+// tile [128 tokens x RP] (MN-major), 8 MMAs of K = 16 tokens into one TMEM
+// accumulator.
 __global__ void __launch_bounds__(PJ_THREADS, 1)
     k_proj_dV(const __grid_constant__ CUtensorMap tmh, const __grid_constant__ CUtensorMap tmdz, const ProjArgs a,
               int nchunks) {
@@ -363,8 +370,8 @@ __global__ void __launch_bounds__(PJ_THREADS, 1)
                 const uint32_t st = sbase + (uint32_t)s * sbytes;
                 const int row = (int)((t_lo + tl) * TC_M);
                 tc::mbar_expect_tx(full(s), abytes + (uint32_t)kz * (TC_M * 16));
-                for (int j = 0; j < TC_M / 8; ++j)
-                    tc::tma_load_2d(st + (uint32_t)j * (TC_M * 16), &tmh, chunk * TC_M + 8 * j, row, full(s));
+                for (int j = 0; j < 2; ++j)
+                    tc::tma_load_2d(st + (uint32_t)j * (TC_M * 128), &tmh, chunk * TC_M + 64 * j, row, full(s));
                 for (int j = 0; j < kz; ++j)
                     tc::tma_load_2d(st + abytes + (uint32_t)j * (TC_M * 16), &tmdz, 8 * j, row, full(s));
                 if (++s == PV_NST) {
@@ -387,7 +394,7 @@ __global__ void __launch_bounds__(PJ_THREADS, 1)
                 tc::fence_after_sync();
                 const uint32_t st = sbase + (uint32_t)s * sbytes;
                 for (int ks = 0; ks < TC_M / 16; ++ks) {
-                    const uint64_t ad = tc::smem_desc(st + (uint32_t)ks * 256u, 128, TC_M * 16);
+                    const uint64_t ad = tc::smem_desc_sw128(st + (uint32_t)ks * 2048u, TC_M * 128, 1024);
                     const uint64_t bd = tc::smem_desc(st + abytes + (uint32_t)ks * 256u, 128, TC_M * 16);
                     tc::mma_bf16(tmem, ad, bd, id, (tl > 0 || ks > 0) ? 1u : 0u);
                 }
@@ -436,7 +443,7 @@ __global__ void k_proj_dV_sum(const float *__restrict__ part, int64_t nranges, i
 }
 
 uint32_t z_smem(int RP) { return PJ_NST * (TC_M * PJ_KC * 2 + PJ_KC * RP * 2) + 8 * (2 * PJ_NST + 4) + 16 + 1024; }
-uint32_t dh_smem(int RP) { return TC_M * RP * 2 + PH_NC * RP * 2 + 4 * TC_M * 128 + 16 + 16 + 1024; }
+uint32_t dh_smem(int RP) { return TC_M * RP * 2 + PH_NC * RP * 2 + PH_BOX * TC_M * 128 + 16 + 16 + 1024; }
 uint32_t dV_smem(int RP) { return PV_NST * (TC_M * TC_M * 2 + TC_M * RP * 2) + 8 * (2 * PV_NST + 1) + 16 + 1024; }
 
 bool map2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_in, uint32_t box_out,
@@ -489,7 +496,7 @@ cudaError_t launch_proj_z(const Ctx &c, const dsc_problem &p, int64_t d, const v
     ProjArgs a = proj_args(p, d);
     a.z = static_cast<bf16 *>(z);
     CUtensorMap th, tv;
-    if (!map2d(&th, h, (uint64_t)d, (uint64_t)N, 8, TC_M, CU_TENSOR_MAP_SWIZZLE_NONE) ||
+    if (!map2d(&th, h, (uint64_t)d, (uint64_t)N, 64, TC_M, CU_TENSOR_MAP_SWIZZLE_128B) ||
         !map2d(&tv, V, (uint64_t)p.R, (uint64_t)d, 8, PJ_KC, CU_TENSOR_MAP_SWIZZLE_NONE))
         return cudaErrorNotSupported;
     const uint32_t smem = z_smem(a.RP);
@@ -517,7 +524,7 @@ cudaError_t launch_proj_bwd(const Ctx &c, const dsc_problem &p, int64_t d, const
     CUtensorMap tdz, tvt, tdh, th;
     if (!map2d(&tdz, dz, (uint64_t)p.R, (uint64_t)N, 8, TC_M, CU_TENSOR_MAP_SWIZZLE_NONE) ||
         !map2d(&tvt, V, (uint64_t)p.R, (uint64_t)d, 8, PH_NC, CU_TENSOR_MAP_SWIZZLE_NONE) ||
-        !map2d(&th, h, (uint64_t)d, (uint64_t)N, 8, TC_M, CU_TENSOR_MAP_SWIZZLE_NONE))
+        !map2d(&th, h, (uint64_t)d, (uint64_t)N, 64, TC_M, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorNotSupported;
     {
         const uint64_t dims[3] = {(uint64_t)d, (uint64_t)N, 1};

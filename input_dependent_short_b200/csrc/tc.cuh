@@ -36,6 +36,22 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
     return d;             // base offset 0, absolute LBO mode, layout type 0 (no swizzle)
 }
 
+// Shared-memory matrix descriptor of a tile written by TMA with 128-byte
+// swizzling (rows of 128 bytes, 8-row atoms of 1024 bytes, atom base aligned
+// to 1024 bytes; layout type 2).  K-major: the rows run along M/N, sbo = 1024
+// (the next 8 rows), lbo unused, and a K step of 16 bf16 inside the 128-byte
+// row moves `addr` by 32 bytes.  MN-major: the rows run along K, sbo = 1024
+// (the next 8 K rows), lbo = the byte offset of the next 64 M/N elements.
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version (sm_100)
+    d |= (uint64_t)2 << 61;  // 128-byte swizzle
+    return d;
+}
+
 // Instruction descriptor of kind::f16 with bf16 A/B and an fp32 accumulator.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn_major, int b_mn_major) {
     return (1u << 4)                        // D format: f32
