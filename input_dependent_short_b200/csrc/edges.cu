@@ -22,6 +22,9 @@
 // the difference of the cross-edge terms added.  That costs O(edges * W * D)
 // work (plus one R x (G*W) contraction per fixed token for low-rank), and
 // the roofline kernels keep their inner loops free of per-token edge tests.
+// The fix-up kernels read only the call's inputs before their first store, so
+// they load and compute while the row pass finishes (programmatic dependent
+// launch) and wait for it only to store.
 #include "kernels.cuh"
 
 namespace dsc {
@@ -96,11 +99,11 @@ __device__ __forceinline__ void x_left(const EdgeArgs &a, int64_t b, int64_t s, 
 // ---------------------------------------------------------------- forward ---
 // y of the first W-1 tokens of each segment with a wrong left edge.
 template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_y(const EdgeArgs a, int64_t cblocks) {
+    pdl_trigger();  // the next fix-up kernel may start its loads
     const int64_t row = blockIdx.x / cblocks;
     const int64_t c = (blockIdx.x % cblocks) * ED_THREADS + threadIdx.x;
     const int64_t i = row / (a.W - 1);
     const int j = (int)(row % (a.W - 1));
-    pdl_wait();
     if (c >= a.D || !left_edge(a, i)) return;
     int64_t b, s, e;
     segment(a, i, b, s, e);
@@ -115,17 +118,18 @@ template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_y(con
         else x_left<T>(a, b, s, u, c, xv, unused);
         acc = fmaf(tap<T>(a, b, t, c, k), xv, acc);
     }
+    pdl_wait();  // the row pass, which wrote y here first, is done
     static_cast<T *>(a.y)[(b * a.T + t) * a.D + c] = from_f<T>(acc);
 }
 
 // --------------------------------------------------------------- backward ---
 // dx of the last W-1 tokens of each segment with a wrong right edge.
 template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dx(const EdgeArgs a, int64_t cblocks) {
+    pdl_trigger();  // the next fix-up kernel may start its loads
     const int64_t row = blockIdx.x / cblocks;
     const int64_t c = (blockIdx.x % cblocks) * ED_THREADS + threadIdx.x;
     const int64_t i = row / (a.W - 1);
     const int j = (int)(row % (a.W - 1));
-    pdl_wait();
     if (c >= a.D || !right_edge(a, i)) return;
     int64_t b, s, e;
     segment(a, i, b, s, e);
@@ -141,6 +145,7 @@ template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dx(co
             acc = fmaf(tap_next<T>(a, b, jn, c, k), ldf<T>(a.dy_next, (b * (a.W - 1) + jn) * a.D + c), acc);
         }
     }
+    pdl_wait();  // the row pass, which wrote dx here first, is done
     static_cast<T *>(a.dx)[(b * a.T + t) * a.D + c] = from_f<T>(acc);
 }
 
@@ -153,13 +158,13 @@ template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dx(co
 //              zero-padded pass's (dwdelta); rows with nothing to fix are
 //              zero in both.
 template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dw(const EdgeArgs a) {
+    pdl_trigger();  // the next fix-up kernel may start its loads
     const int64_t idx = (int64_t)blockIdx.x * ED_THREADS + threadIdx.x;
     const int64_t nrows = a.nseg * (a.W - 1);
     if (idx >= nrows * a.G) return;
     const int64_t rowi = idx / a.G, g = idx % a.G;
     const int64_t i = rowi / (a.W - 1);
     const int j = (int)(rowi % (a.W - 1));
-    pdl_wait();
     int64_t b, s, e;
     segment(a, i, b, s, e);
     const int64_t t = s + j;
@@ -190,6 +195,7 @@ template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dw(co
             }
         }
     }
+    pdl_wait();  // the row pass (dw) and the previous call's readers of the scratch are done
     if (a.kind == EDGE_HEADWISE) {
         if (!live) return;
 #pragma unroll
@@ -262,7 +268,6 @@ template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dU(co
 // for the taps that reach across a left edge.  Thread per channel.
 template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dws(const EdgeArgs a) {
     const int64_t c = (int64_t)blockIdx.x * ED_THREADS + threadIdx.x;
-    pdl_wait();
     if (c >= a.D) return;
     float acc[8];
 #pragma unroll
@@ -283,6 +288,7 @@ template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dws(c
             }
         }
     }
+    pdl_wait();  // dws is complete (the row pass and its partial sums)
 #pragma unroll
     for (int k = 1; k < 8; ++k)
         if (k < a.W) a.dws[c * a.W + k] += acc[k];

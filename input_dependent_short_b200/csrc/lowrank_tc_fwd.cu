@@ -490,16 +490,33 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
 // c*GPV*W + k*GPV + g of the image holds U column (c*GPV + g)*W + k.  With
 // it, the MMA leaves a vector's filters with the taps outermost, so the two
 // channels of a pair find tap k in adjacent registers.
+// One thread per chunk of GPV*W columns (a row's chunks are contiguous in
+// both U and the image, GW being a multiple of GPV*W): the chunk is read whole,
+// transposed from group-major to tap-major in registers and written whole,
+// with 16-byte accesses when the chunk is a multiple of 16 bytes.
+constexpr int UPERM_MAX = 64;  // GPV * W <= 8 * 8 columns per chunk
 __global__ void k_fwd_uperm(const bf16 *__restrict__ U, bf16 *__restrict__ Uf, int64_t R, int64_t GW, int W, int GPV) {
     pdl_wait();
     pdl_trigger();
-    const int64_t n = R * GW;
-    const int64_t chunk = (int64_t)GPV * W;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) {
-        const int64_t r = i / GW, j = i % GW;  // image element (r, j)
-        const int64_t c = j / chunk, q = j % chunk;
-        const int64_t k = q / GPV, g = q % GPV;
-        Uf[i] = U[r * GW + (c * GPV + g) * W + k];
+    const int chunk = GPV * W;
+    const int64_t nck = R * (GW / chunk);
+    const bool vec = (chunk * 2) % 16 == 0;
+    for (int64_t ci = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; ci < nck; ci += (int64_t)gridDim.x * blockDim.x) {
+        const bf16 *src = U + ci * chunk;
+        bf16 *dst = Uf + ci * chunk;
+        __align__(16) bf16 in[UPERM_MAX], out[UPERM_MAX];
+        if (vec) {
+            for (int v = 0; v < chunk / 8; ++v) *reinterpret_cast<uint4 *>(in + 8 * v) = ld16(src + 8 * v);
+        } else {
+            for (int q = 0; q < chunk; ++q) in[q] = src[q];
+        }
+        for (int g = 0; g < GPV; ++g)
+            for (int k = 0; k < W; ++k) out[k * GPV + g] = in[g * W + k];
+        if (vec) {
+            for (int v = 0; v < chunk / 8; ++v) st16(dst + 8 * v, *reinterpret_cast<const uint4 *>(out + 8 * v));
+        } else {
+            for (int q = 0; q < chunk; ++q) dst[q] = out[q];
+        }
     }
 }
 
@@ -631,8 +648,8 @@ cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     if (p.H < 8) {
         if (!ws || ws_bytes < lr_tc_fwd_ws_bytes(p)) return cudaErrorInvalidValue;
         a.Uf = static_cast<bf16 *>(ws);
-        const int64_t n = p.R * a.m.GW;
-        const cudaError_t e = launch_pdl(lrtc::k_fwd_uperm, dim3((unsigned)min((int64_t)1024, (n + 255) / 256)), dim3(256),
+        const int64_t n = p.R * (a.m.GW / ((8 / p.H) * p.W));  // chunks
+        const cudaError_t e = launch_pdl(lrtc::k_fwd_uperm, dim3((unsigned)min((int64_t)1024, (n + 127) / 128)), dim3(128),
                                          0, c.stream, a.U, a.Uf, (int64_t)p.R, a.m.GW, (int)p.W, (int)(8 / p.H));
         if (e != cudaSuccess) return e;
     }
