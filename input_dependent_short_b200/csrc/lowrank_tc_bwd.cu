@@ -716,54 +716,84 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
 //     columns j >= NBW zero;
 //   z image of tile i (sequence b, first token t0): element (t, r) at
 //     (r/8)*(136*8) + t*8 + r%8 holding z[b][t0+t][r], zero for r >= R or t0+t >= T.
+// One thread per 16-byte chunk of the images (8 consecutive elements):
+//   U image chunk (blk, jc, r): columns j = 8*jc .. 8*jc+7 of rank row r, one
+//     tap k and 8 consecutive groups (GB is a multiple of 8), gathered with
+//     stride W from U;
+//   z image chunk (tile, rc, t): ranks 8*rc .. 8*rc+7 of token t, one 16-byte
+//     load of z (R is a multiple of 8).
 __global__ void k_bwd_prep(const TcArgs a) {
     pdl_wait();
     pdl_trigger();
     const TcMap &m = a.m;
-    const int64_t ublk = (int64_t)m.RP * TB_NB;
-    const int64_t nU = (int64_t)m.nBlkB * ublk;
-    const int64_t ztile = (int64_t)(m.RP / 8) * TB_ZROWS * 8;
-    const int64_t nZ = m.totalTiles * ztile;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nU + nZ; i += (int64_t)gridDim.x * blockDim.x) {
-        if (i < nU) {
-            const int64_t blk = i / ublk;
-            const int rem = (int)(i % ublk);
-            const int jc = rem / (m.RP * 8), r = (rem % (m.RP * 8)) / 8, e = rem % 8;
-            const int j = jc * 8 + e, k = j / m.GB, g = j % m.GB;
-            a.Up[i] = (r < m.R && k < m.W) ? a.U[(int64_t)r * m.GW + (blk * m.GB + g) * m.W + k] : __float2bfloat16_rn(0.f);
+    const int uper = 16 * m.RP;                  // chunks per U block image
+    const int zper = (m.RP / 8) * TB_ZROWS;      // chunks per z tile image
+    const int64_t nU = (int64_t)m.nBlkB * uper;
+    const int64_t nZ = m.totalTiles * zper;
+    for (int64_t ci = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; ci < nU + nZ; ci += (int64_t)gridDim.x * blockDim.x) {
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (ci < nU) {
+            // thread order (block, rank row, column chunk): a warp's gathers stay
+            // inside the 256-byte run of U that holds a block's row
+            const int64_t blk = ci / uper;
+            const int rem = (int)(ci - blk * uper);
+            const int r = rem >> 4, jc = rem & 15;
+            const int j0 = 8 * jc, k = j0 / m.GB, g0 = j0 - k * m.GB;
+            if (r < m.R && k < m.W) {
+                const bf16 *src = a.U + (int64_t)r * m.GW + (blk * m.GB + g0) * m.W + k;
+                uint32_t w[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    w[e] = (uint32_t)__bfloat16_as_ushort(src[(2 * e) * m.W]) |
+                           ((uint32_t)__bfloat16_as_ushort(src[(2 * e + 1) * m.W]) << 16);
+                v = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            st16(a.Up + ((blk * 16 + jc) * m.RP + r) * 8, v);
         } else {
-            const int64_t i2 = i - nU;
-            const int64_t tile = i2 / ztile;
-            const int rem = (int)(i2 % ztile);
-            const int rc = rem / (TB_ZROWS * 8), t = (rem % (TB_ZROWS * 8)) / 8, e = rem % 8;
-            const int r = rc * 8 + e;
+            const int64_t i2 = ci - nU;
+            const int64_t tile = i2 / zper;
+            const int rem = (int)(i2 - tile * zper);
+            const int rc = rem / TB_ZROWS, t = rem - rc * TB_ZROWS;
             const int64_t b = tile / m.tilesPerSeq;
-            const int64_t tt = (tile % m.tilesPerSeq) * TC_M + t;
-            a.zimg[i2] = (r < m.R && tt < m.T) ? a.z[(b * m.T + tt) * m.R + r] : __float2bfloat16_rn(0.f);
+            const int64_t tt = (tile - b * m.tilesPerSeq) * TC_M + t;
+            if (8 * rc < m.R && tt < m.T) v = ld16(a.z + (b * m.T + tt) * m.R + 8 * rc);
+            st16(a.zimg + i2 * 8, v);
         }
     }
 }
 
+// n is a multiple of 4 and p 16-byte aligned.
 __global__ void k_tc_zero(float *p, int64_t n) {
     pdl_wait();
     pdl_trigger();
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x) p[i] = 0.f;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n / 4; i += (int64_t)gridDim.x * blockDim.x)
+        reinterpret_cast<float4 *>(p)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
 }
 
-// dU = sum of the per-range partials (fixed order); dz = the fp32 accumulator in bf16.
+// dU = sum of the per-range partials (fixed order); dz = the fp32 accumulator in
+// bf16.  Four elements per thread (R and R*GW are multiples of 8).
 __global__ void k_tc_finalize(const TcArgs a) {
     pdl_wait();
     pdl_trigger();
     const TcMap &m = a.m;
-    const int64_t nU = m.nRanges > 1 ? m.R * m.GW : 0;
-    const int64_t nz = m.dzAcc ? m.B * m.T * m.R : 0;
+    const int64_t nU = m.nRanges > 1 ? m.R * m.GW / 4 : 0;
+    const int64_t nz = m.dzAcc ? m.B * m.T * m.R / 4 : 0;
+    const int64_t qs = m.R * m.GW / 4;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nU + nz; i += (int64_t)gridDim.x * blockDim.x) {
         if (i < nU) {
-            float sacc = 0.f;
-            for (int q = 0; q < m.nRanges; ++q) sacc += a.dU_part[(int64_t)q * m.R * m.GW + i];
-            a.dU[i] = sacc;
+            const float4 *part = reinterpret_cast<const float4 *>(a.dU_part);
+            float4 sacc = part[i];
+            for (int q = 1; q < m.nRanges; ++q) {
+                const float4 v = part[(int64_t)q * qs + i];
+                sacc.x += v.x;
+                sacc.y += v.y;
+                sacc.z += v.z;
+                sacc.w += v.w;
+            }
+            reinterpret_cast<float4 *>(a.dU)[i] = sacc;
         } else {
-            a.dz[i - nU] = __float2bfloat16_rn(a.dz_acc[i - nU]);
+            const float4 v = reinterpret_cast<const float4 *>(a.dz_acc)[i - nU];
+            reinterpret_cast<uint2 *>(a.dz)[i - nU] = make_uint2(pack_bf2(v.x, v.y), pack_bf2(v.z, v.w));
         }
     }
 }
@@ -959,14 +989,14 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
         a.dU_part = reinterpret_cast<float *>(w);
         w += (size_t)a.m.nRanges * a.m.R * a.m.GW * 4;
     }
-    const int64_t nprep = (int64_t)a.m.nBlkB * a.m.RP * TB_NB + a.m.totalTiles * (a.m.RP / 8) * TB_ZROWS * 8;
+    const int64_t nprep = (int64_t)a.m.nBlkB * 16 * a.m.RP + a.m.totalTiles * (a.m.RP / 8) * TB_ZROWS;  // chunks
     cudaError_t e = launch_pdl(k_bwd_prep, dim3((unsigned)min((int64_t)2048, (nprep + 255) / 256)), dim3(256), 0,
                                c.stream, a);
     if (e != cudaSuccess) return e;
     if (a.m.dzAcc) {
         a.dz_acc = reinterpret_cast<float *>(w);
         const int64_t n = a.m.B * a.m.T * a.m.R;
-        e = launch_pdl(k_tc_zero, dim3((unsigned)min((int64_t)1024, (n + 255) / 256)), dim3(256), 0, c.stream, a.dz_acc, n);
+        e = launch_pdl(k_tc_zero, dim3((unsigned)min((int64_t)1024, (n / 4 + 255) / 256)), dim3(256), 0, c.stream, a.dz_acc, n);
         if (e != cudaSuccess) return e;
     }
     e = cudaErrorNotSupported;
@@ -982,7 +1012,7 @@ cudaError_t launch_lr_bwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     }
     if (e != cudaSuccess) return e;
     if (a.m.nRanges > 1 || a.m.dzAcc) {
-        const int64_t n = (a.m.nRanges > 1 ? a.m.R * a.m.GW : 0) + (a.m.dzAcc ? a.m.B * a.m.T * a.m.R : 0);
+        const int64_t n = ((a.m.nRanges > 1 ? a.m.R * a.m.GW : 0) + (a.m.dzAcc ? a.m.B * a.m.T * a.m.R : 0)) / 4;
         e = launch_pdl(k_tc_finalize, dim3((unsigned)min((int64_t)2048, (n + 255) / 256)), dim3(256), 0, c.stream, a);
         if (e != cudaSuccess) return e;
     }

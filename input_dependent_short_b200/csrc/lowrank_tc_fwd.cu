@@ -492,32 +492,66 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
 // channels of a pair find tap k in adjacent registers.
 // One thread per chunk of GPV*W columns (a row's chunks are contiguous in
 // both U and the image, GW being a multiple of GPV*W): the chunk is read whole,
-// transposed from group-major to tap-major in registers and written whole,
-// with 16-byte accesses when the chunk is a multiple of 16 bytes.
-constexpr int UPERM_MAX = 64;  // GPV * W <= 8 * 8 columns per chunk
-__global__ void k_fwd_uperm(const bf16 *__restrict__ U, bf16 *__restrict__ Uf, int64_t R, int64_t GW, int W, int GPV) {
+// transposed from group-major to tap-major in registers (GPV and W are
+// compile-time, so the chunk stays in registers) and written whole, with
+// 16-byte accesses when the chunk is a multiple of 16 bytes.
+template <int GPV, int W>
+__global__ void k_fwd_uperm(const bf16 *__restrict__ U, bf16 *__restrict__ Uf, int64_t R, int64_t GW) {
     pdl_wait();
     pdl_trigger();
-    const int chunk = GPV * W;
-    const int64_t nck = R * (GW / chunk);
-    const bool vec = (chunk * 2) % 16 == 0;
+    constexpr int CH = GPV * W;
+    constexpr bool VEC = (CH * 2) % 16 == 0;
+    const int64_t nck = R * (GW / CH);
     for (int64_t ci = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; ci < nck; ci += (int64_t)gridDim.x * blockDim.x) {
-        const bf16 *src = U + ci * chunk;
-        bf16 *dst = Uf + ci * chunk;
-        __align__(16) bf16 in[UPERM_MAX], out[UPERM_MAX];
-        if (vec) {
-            for (int v = 0; v < chunk / 8; ++v) *reinterpret_cast<uint4 *>(in + 8 * v) = ld16(src + 8 * v);
+        const bf16 *src = U + ci * CH;
+        bf16 *dst = Uf + ci * CH;
+        unsigned short in[CH], out[CH];
+        if constexpr (VEC) {
+#pragma unroll
+            for (int v = 0; v < CH / 8; ++v) {
+                const uint4 q = ld16(src + 8 * v);
+                const uint32_t w4[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+                for (int e = 0; e < 8; ++e) in[8 * v + e] = (unsigned short)(w4[e / 2] >> (16 * (e & 1)));
+            }
         } else {
-            for (int q = 0; q < chunk; ++q) in[q] = src[q];
+#pragma unroll
+            for (int q = 0; q < CH; ++q) in[q] = __bfloat16_as_ushort(src[q]);
         }
+#pragma unroll
         for (int g = 0; g < GPV; ++g)
+#pragma unroll
             for (int k = 0; k < W; ++k) out[k * GPV + g] = in[g * W + k];
-        if (vec) {
-            for (int v = 0; v < chunk / 8; ++v) st16(dst + 8 * v, *reinterpret_cast<const uint4 *>(out + 8 * v));
+        if constexpr (VEC) {
+#pragma unroll
+            for (int v = 0; v < CH / 8; ++v) {
+                uint32_t w4[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) w4[e] = (uint32_t)out[8 * v + 2 * e] | ((uint32_t)out[8 * v + 2 * e + 1] << 16);
+                st16(dst + 8 * v, make_uint4(w4[0], w4[1], w4[2], w4[3]));
+            }
         } else {
-            for (int q = 0; q < chunk; ++q) dst[q] = out[q];
+#pragma unroll
+            for (int q = 0; q < CH; ++q) dst[q] = __ushort_as_bfloat16(out[q]);
         }
     }
+}
+
+template <int GPV>
+cudaError_t launch_uperm_w(const Ctx &c, int W, const bf16 *U, bf16 *Uf, int64_t R, int64_t GW) {
+    const int64_t n = R * (GW / (GPV * W));  // chunks
+    const dim3 grid((unsigned)min((int64_t)1024, (n + 127) / 128));
+    switch (W) {
+    case 1: return launch_pdl(k_fwd_uperm<GPV, 1>, grid, dim3(128), 0, c.stream, U, Uf, R, GW);
+    case 2: return launch_pdl(k_fwd_uperm<GPV, 2>, grid, dim3(128), 0, c.stream, U, Uf, R, GW);
+    case 3: return launch_pdl(k_fwd_uperm<GPV, 3>, grid, dim3(128), 0, c.stream, U, Uf, R, GW);
+    case 4: return launch_pdl(k_fwd_uperm<GPV, 4>, grid, dim3(128), 0, c.stream, U, Uf, R, GW);
+    case 5: return launch_pdl(k_fwd_uperm<GPV, 5>, grid, dim3(128), 0, c.stream, U, Uf, R, GW);
+    case 6: return launch_pdl(k_fwd_uperm<GPV, 6>, grid, dim3(128), 0, c.stream, U, Uf, R, GW);
+    case 7: return launch_pdl(k_fwd_uperm<GPV, 7>, grid, dim3(128), 0, c.stream, U, Uf, R, GW);
+    case 8: return launch_pdl(k_fwd_uperm<GPV, 8>, grid, dim3(128), 0, c.stream, U, Uf, R, GW);
+    }
+    return cudaErrorNotSupported;
 }
 
 // Forward plan: the widest channel block whose filters fit half of TMEM
@@ -648,9 +682,10 @@ cudaError_t launch_lr_fwd_tc(const Ctx &c, const dsc_problem &p, const void *x, 
     if (p.H < 8) {
         if (!ws || ws_bytes < lr_tc_fwd_ws_bytes(p)) return cudaErrorInvalidValue;
         a.Uf = static_cast<bf16 *>(ws);
-        const int64_t n = p.R * (a.m.GW / ((8 / p.H) * p.W));  // chunks
-        const cudaError_t e = launch_pdl(lrtc::k_fwd_uperm, dim3((unsigned)min((int64_t)1024, (n + 127) / 128)), dim3(128),
-                                         0, c.stream, a.U, a.Uf, (int64_t)p.R, a.m.GW, (int)p.W, (int)(8 / p.H));
+        const int gpv = (int)(8 / p.H);
+        const cudaError_t e = gpv == 8   ? lrtc::launch_uperm_w<8>(c, (int)p.W, a.U, a.Uf, p.R, a.m.GW)
+                              : gpv == 4 ? lrtc::launch_uperm_w<4>(c, (int)p.W, a.U, a.Uf, p.R, a.m.GW)
+                                         : lrtc::launch_uperm_w<2>(c, (int)p.W, a.U, a.Uf, p.R, a.m.GW);
         if (e != cudaSuccess) return e;
     }
     switch (a.m.W) {

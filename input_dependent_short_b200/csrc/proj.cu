@@ -22,8 +22,9 @@
 //   k_proj_z   persistent; per 128-token tile a K loop over d_model in steps
 //              of 64 (TMA ring of h and V chunks), MMA M=128 N=RP into one of
 //              two TMEM accumulators; 4 epilogue warps store z rows.
-//   k_proj_dh  per (tile, 256 model columns): dz tile x V^T chunk (K = R), the
-//              accumulator staged in shared memory and stored by TMA.
+//   k_proj_dh  persistent; per (tile, 256 model columns): dz tile x V^T chunk
+//              (K = R) into one of two TMEM accumulators, staged in one of two
+//              shared-memory tiles and stored by TMA while the next item runs.
 //   k_proj_dV  per (128 model rows, token range): h^T x dz over the range,
 //              accumulated in TMEM, written as a per-range partial; a second
 //              kernel sums the partials in a fixed order (deterministic).
@@ -216,11 +217,33 @@ __global__ void __launch_bounds__(PJ_THREADS, 1)
 }
 
 // ---------------------------------------------------------- dh = dz V^T ---
-// Item = (tile of 128 tokens, PH_NC model columns).  A = dz tile [128 x RP]
-// (K-major), B = V rows [PH_NC x RP] read as V^T (K-major), K = RP.  Two
-// CTAs per SM (TMEM: 2 x 256 columns).
+// Persistent.  Item = (tile of 128 tokens, PH_NC model columns): A = dz tile
+// [128 x RP] (K-major), B = V rows [PH_NC x RP] read as V^T (K-major), K = RP.
+// Two operand stages, two TMEM accumulators (2 x 256 columns) and two staging
+// tiles, so that one item's store leaves while the next item's MMAs and
+// epilogue run.  Warp 8 (one lane) loads and issues the MMAs; warps 0-7 drain
+// the accumulator (warp w: TMEM lanes 32*(w%4).., columns 128*(w/4)..) into
+// 128-byte-swizzled staging boxes that thread 0 stores by TMA.
 constexpr int PH_BOX = PH_NC / 64;  // staging boxes of 64 columns
-__global__ void __launch_bounds__(128, 1)
+constexpr int PH_EPI = 256;         // epilogue threads
+constexpr int PH_THREADS = PH_EPI + 32;
+
+struct DhSmem {
+    uint32_t abytes, bbytes, stage, stg, bars, tslot, total;
+    __host__ __device__ explicit DhSmem(int RP) {
+        abytes = (uint32_t)(TC_M * RP * 2);
+        bbytes = (uint32_t)(PH_NC * RP * 2);
+        stage = abytes + bbytes;                                                 // multiple of 1024
+        stg = 2 * stage;                                                         // two staging tiles
+        bars = stg + 2 * PH_BOX * TC_M * 128;                                    // opf[2] ope[2] accf[2] acce[2]
+        tslot = bars + 8 * 8;
+        total = tslot + 16 + 1024;
+    }
+};
+
+__device__ __forceinline__ void bulk_wait_read_1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+
+__global__ void __launch_bounds__(PH_THREADS, 1)
     k_proj_dh(const __grid_constant__ CUtensorMap tmdz, const __grid_constant__ CUtensorMap tmv,
               const __grid_constant__ CUtensorMap tmdh, const ProjArgs a, int nchunks) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
@@ -228,83 +251,136 @@ __global__ void __launch_bounds__(128, 1)
     const uint32_t sbase = (sraw + 1023u) & ~1023u;
     unsigned char *smem = smem_raw + (sbase - sraw);
     const int RP = a.RP, kz = (int)(a.R / 8);
-    const uint32_t abytes = (uint32_t)(TC_M * RP * 2), bbytes = (uint32_t)(PH_NC * RP * 2);
-    const uint32_t stage = abytes + bbytes;            // PH_BOX staging boxes of [128 x 64] bf16 (128-byte swizzle)
-    const uint32_t bar = stage + PH_BOX * TC_M * 128;  // one mbarrier for the loads, one for the MMAs
-    const uint32_t tslot = bar + 16;
+    const DhSmem S(RP);
+    auto opf = [&](int s) { return sbase + S.bars + 8u * s; };
+    auto ope = [&](int s) { return sbase + S.bars + 16u + 8u * s; };
+    auto accf = [&](int s) { return sbase + S.bars + 32u + 8u * s; };
+    auto acce = [&](int s) { return sbase + S.bars + 48u + 8u * s; };
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int64_t tile = blockIdx.x / nchunks;
-    const int chunk = (int)(blockIdx.x % nchunks);
+    const int64_t nitems = a.ntiles * nchunks;
+    const int nit = nitems > blockIdx.x ? (int)((nitems - 1 - blockIdx.x) / gridDim.x + 1) : 0;
 
     if (tid == 0) {
-        tc::mbar_init(sbase + bar, 1);
-        tc::mbar_init(sbase + bar + 8, 1);
+        for (int q = 0; q < 2; ++q) {
+            tc::mbar_init(opf(q), 1);
+            tc::mbar_init(ope(q), 1);
+            tc::mbar_init(accf(q), 1);
+            tc::mbar_init(acce(q), 1);
+        }
         tc::fence_mbar_init();
     }
-    // rank columns R .. RP-1 of both operands stay zero (never loaded)
-    for (int i = tid; i < (RP / 8 - kz) * (TC_M + PH_NC); i += 128) {
-        const int j = kz + i / (TC_M + PH_NC), r = i % (TC_M + PH_NC);
+    // rank columns R .. RP-1 of both operands of both stages stay zero (never loaded)
+    for (int i = tid; i < 2 * (RP / 8 - kz) * (TC_M + PH_NC); i += PH_THREADS) {
+        const int st = i / ((RP / 8 - kz) * (TC_M + PH_NC)), i1 = i % ((RP / 8 - kz) * (TC_M + PH_NC));
+        const int j = kz + i1 / (TC_M + PH_NC), r = i1 % (TC_M + PH_NC);
         const uint32_t off = r < TC_M ? (uint32_t)j * (TC_M * 16) + (uint32_t)r * 16
-                                      : abytes + (uint32_t)j * (PH_NC * 16) + (uint32_t)(r - TC_M) * 16;
-        *reinterpret_cast<uint4 *>(smem + off) = make_uint4(0, 0, 0, 0);
+                                      : S.abytes + (uint32_t)j * (PH_NC * 16) + (uint32_t)(r - TC_M) * 16;
+        *reinterpret_cast<uint4 *>(smem + (uint32_t)st * S.stage + off) = make_uint4(0, 0, 0, 0);
     }
     tc::fence_proxy_async();
-    if (warp == 0) tc::tmem_alloc(sbase + tslot, PH_NC);
+    if (warp == 0) tc::tmem_alloc(sbase + S.tslot, 2 * PH_NC);
     tc::fence_before_sync();
     __syncthreads();
     tc::fence_after_sync();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + tslot);
-    bool ok = true;
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + S.tslot);
+    bool timed_out = false;
+    auto wait = [&](uint32_t bar, uint32_t parity) {
+        if (!timed_out && !tc::mbar_wait(bar, parity, TC_WAIT_LIMIT)) timed_out = true;
+    };
     pdl_wait();
     pdl_trigger();
-    if (tid == 0) {
-        tc::mbar_expect_tx(sbase + bar, (uint32_t)kz * (TC_M * 16 + PH_NC * 16));
-        for (int j = 0; j < kz; ++j) {
-            tc::tma_load_2d(sbase + (uint32_t)j * (TC_M * 16), &tmdz, 8 * j, (int)(tile * TC_M), sbase + bar);
-            tc::tma_load_2d(sbase + abytes + (uint32_t)j * (PH_NC * 16), &tmv, 8 * j, chunk * PH_NC, sbase + bar);
+    // item it of this CTA: tile-minor, so that neighbouring CTAs share a V chunk
+    auto item = [&](int it, int64_t &tile, int &chunk) {
+        const int64_t g = blockIdx.x + (int64_t)it * gridDim.x;
+        chunk = (int)(g / a.ntiles);
+        tile = g - (int64_t)chunk * a.ntiles;
+    };
+
+    if (warp == PH_EPI / 32) {
+        if (lane == 0 && nit > 0) {
+            tc::tma_prefetch_desc(&tmdz);
+            tc::tma_prefetch_desc(&tmv);
+            auto load = [&](int it) {
+                const int st = it & 1;
+                int64_t tile;
+                int chunk;
+                item(it, tile, chunk);
+                const uint32_t base = sbase + (uint32_t)st * S.stage;
+                tc::mbar_expect_tx(opf(st), (uint32_t)kz * (TC_M * 16 + PH_NC * 16));
+                for (int j = 0; j < kz; ++j) {
+                    tc::tma_load_2d(base + (uint32_t)j * (TC_M * 16), &tmdz, 8 * j, (int)(tile * TC_M), opf(st));
+                    tc::tma_load_2d(base + S.abytes + (uint32_t)j * (PH_NC * 16), &tmv, 8 * j, chunk * PH_NC, opf(st));
+                }
+            };
+            for (int it = 0; it < 2 && it < nit; ++it) load(it);
+            const uint32_t id = tc::idesc_bf16(TC_M, PH_NC, 0, 0);
+            for (int it = 0; it < nit; ++it) {
+                const int st = it & 1;
+                const uint32_t ph = (uint32_t)((it >> 1) & 1);
+                wait(opf(st), ph);
+                if (it >= 2) wait(acce(st), ph ^ 1u);
+                tc::fence_after_sync();
+                const uint32_t base = sbase + (uint32_t)st * S.stage;
+                for (int ks = 0; ks < RP / 16; ++ks) {
+                    const uint64_t ad = tc::smem_desc(base + (uint32_t)ks * 2u * (TC_M * 16), TC_M * 16, 128);
+                    const uint64_t bd = tc::smem_desc(base + S.abytes + (uint32_t)ks * 2u * (PH_NC * 16), PH_NC * 16, 128);
+                    tc::mma_bf16(tmem + (uint32_t)(st * PH_NC), ad, bd, id, ks > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(accf(st));
+                tc::mma_commit(ope(st));
+                if (it + 2 < nit) {  // refill this stage once its MMAs have read it
+                    wait(ope(st), ph);
+                    load(it + 2);
+                }
+            }
         }
-        ok = tc::mbar_wait(sbase + bar, 0, TC_WAIT_LIMIT);
-        tc::fence_after_sync();
-        const uint32_t id = tc::idesc_bf16(TC_M, PH_NC, 0, 0);
-        for (int ks = 0; ks < RP / 16 && ok; ++ks) {
-            const uint64_t ad = tc::smem_desc(sbase + (uint32_t)ks * 2u * (TC_M * 16), TC_M * 16, 128);
-            const uint64_t bd = tc::smem_desc(sbase + abytes + (uint32_t)ks * 2u * (PH_NC * 16), PH_NC * 16, 128);
-            tc::mma_bf16(tmem, ad, bd, id, ks > 0 ? 1u : 0u);
-        }
-        tc::mma_commit(sbase + bar + 8);
-    }
-    // every thread waits for the MMAs (a time-out on the loads still commits, so this ends)
-    if (!tc::mbar_wait(sbase + bar + 8, 0, TC_WAIT_LIMIT)) ok = false;
-    tc::fence_after_sync();
-    // accumulator row t (TMEM lane) -> bf16 -> swizzled staging box, then TMA stores
-    const int t = warp * 32 + lane;
-    const uint32_t tl = tmem + ((uint32_t)(warp * 32) << 16);
-    for (int c0 = 0; c0 < PH_NC; c0 += 32) {
-        float v[32];
-        lrtc::tmem_ld<32>(tl + (uint32_t)c0, v);
-        tc::tmem_wait_ld();
-        unsigned char *box = smem + stage + (uint32_t)(c0 / 64) * (TC_M * 128);
+    } else {
+        const int q4 = warp & 3, half = warp >> 2;
+        const int t = q4 * 32 + lane;  // token row of the tile = TMEM lane
+        const uint32_t tl = tmem + ((uint32_t)(q4 * 32) << 16);
+        for (int it = 0; it < nit; ++it) {
+            const int st = it & 1;
+            const uint32_t ph = (uint32_t)((it >> 1) & 1);
+            int64_t tile;
+            int chunk;
+            item(it, tile, chunk);
+            wait(accf(st), ph);
+            tc::fence_after_sync();
+            // the store that last used this staging tile (item it-2) has read it;
+            // the one of item it-1 may still be in flight
+            if (tid == 0) bulk_wait_read_1();
+            asm volatile("bar.sync 1, %0;" ::"n"(PH_EPI) : "memory");
+            unsigned char *stg = smem + S.stg + (uint32_t)st * (PH_BOX * TC_M * 128);
+            for (int c0 = half * (PH_NC / 2); c0 < (half + 1) * (PH_NC / 2); c0 += 32) {
+                float v[32];
+                lrtc::tmem_ld<32>(tl + (uint32_t)(st * PH_NC + c0), v);
+                tc::tmem_wait_ld();
+                unsigned char *box = stg + (uint32_t)(c0 / 64) * (TC_M * 128);
 #pragma unroll
-        for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<uint4 *>(box + tc::swz<128>(t, (c0 % 64) / 8 + q)) =
-                make_uint4(pack_bf2(v[8 * q], v[8 * q + 1]), pack_bf2(v[8 * q + 2], v[8 * q + 3]),
-                           pack_bf2(v[8 * q + 4], v[8 * q + 5]), pack_bf2(v[8 * q + 6], v[8 * q + 7]));
+                for (int q = 0; q < 4; ++q)
+                    *reinterpret_cast<uint4 *>(box + tc::swz<128>(t, (c0 % 64) / 8 + q)) =
+                        make_uint4(pack_bf2(v[8 * q], v[8 * q + 1]), pack_bf2(v[8 * q + 2], v[8 * q + 3]),
+                                   pack_bf2(v[8 * q + 4], v[8 * q + 5]), pack_bf2(v[8 * q + 6], v[8 * q + 7]));
+            }
+            tc::fence_before_sync();
+            tc::fence_proxy_async();
+            asm volatile("bar.sync 1, %0;" ::"n"(PH_EPI) : "memory");
+            if (tid == 0) {
+                tc::mbar_arrive(acce(st));
+                for (int bx = 0; bx < PH_BOX; ++bx)
+                    if (chunk * PH_NC + bx * 64 < a.d)
+                        tc::tma_store_3d(&tmdh, sbase + S.stg + (uint32_t)(st * PH_BOX + bx) * (TC_M * 128),
+                                         chunk * PH_NC + bx * 64, (int)(tile * TC_M), 0);
+                tc::bulk_commit();
+            }
+        }
+        if (tid == 0) tc::bulk_wait_all();
     }
-    tc::fence_proxy_async();
+    if (timed_out) record_timeout();
     tc::fence_before_sync();
     __syncthreads();
-    if (tid == 0) {
-        for (int bx = 0; bx < PH_BOX; ++bx)
-            if (chunk * PH_NC + bx * 64 < a.d)
-                tc::tma_store_3d(&tmdh, sbase + stage + (uint32_t)bx * (TC_M * 128), chunk * PH_NC + bx * 64,
-                                 (int)(tile * TC_M), 0);
-        tc::bulk_commit();
-        tc::bulk_wait_all();
-    }
-    if (!ok && tid == 0) record_timeout();
     tc::fence_after_sync();
-    __syncthreads();
-    if (warp == 0) tc::tmem_dealloc(tmem, PH_NC);
+    if (warp == 0) tc::tmem_dealloc(tmem, 2 * PH_NC);
 }
 
 // ---------------------------------------------------- dV = sum_t h^T dz ---
@@ -443,7 +519,7 @@ __global__ void k_proj_dV_sum(const float *__restrict__ part, int64_t nranges, i
 }
 
 uint32_t z_smem(int RP) { return PJ_NST * (TC_M * PJ_KC * 2 + PJ_KC * RP * 2) + 8 * (2 * PJ_NST + 4) + 16 + 1024; }
-uint32_t dh_smem(int RP) { return TC_M * RP * 2 + PH_NC * RP * 2 + PH_BOX * TC_M * 128 + 16 + 16 + 1024; }
+uint32_t dh_smem(int RP) { return DhSmem(RP).total; }
 uint32_t dV_smem(int RP) { return PV_NST * (TC_M * TC_M * 2 + TC_M * RP * 2) + 8 * (2 * PV_NST + 1) + 16 + 1024; }
 
 bool map2d(CUtensorMap *m, const void *base, uint64_t inner, uint64_t outer, uint32_t box_in, uint32_t box_out,
@@ -540,7 +616,8 @@ cudaError_t launch_proj_bwd(const Ctx &c, const dsc_problem &p, int64_t d, const
     if (attr1 != cudaSuccess) return attr1;
     if (attr2 != cudaSuccess) return attr2;
     const int nch = (int)((d + PH_NC - 1) / PH_NC);
-    cudaError_t e = launch_pdl(k_proj_dh, dim3((unsigned)(a.ntiles * nch)), dim3(128), dh_smem(a.RP), c.stream, tdz,
+    const int64_t nitems = a.ntiles * nch;
+    cudaError_t e = launch_pdl(k_proj_dh, dim3((unsigned)(nitems < c.sms ? nitems : c.sms)), dim3(PH_THREADS), dh_smem(a.RP), c.stream, tdz,
                                tvt, tdh, a, nch);
     if (e != cudaSuccess) return e;
     const int nchV = (int)((d + TC_M - 1) / TC_M);
