@@ -210,11 +210,14 @@ __device__ __forceinline__ void bwd_dw_groups(const TcMap &m, const unsigned cha
 
 // One sub-tile of the epilogue for token t_loc, thread part `part`.
 //   VPT vectors of 8 channels; GPT groups among the thread's 8*VPT channels
-//   (1 when the group is wider: PPG parts then share it).
+//   (1 when the group is wider: PPG parts then share it).  With one vector
+//   (VPT = 1) the thread's swizzled row offsets ro[k] (box row t_loc + k; the
+//   x, dy and dx staging boxes share them) are computed once per thread.
 template <int W, int VPT, int GPT, int PPG, int RB>
 __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
                                             unsigned char *dwt, float *xch, int part, int t_loc, int s,
-                                            unsigned char *ys, float res, uint32_t release_w) {
+                                            unsigned char *ys, float res, uint32_t release_w,
+                                            const uint32_t (&ro)[W]) {
     constexpr int WIN = W - 1;
     constexpr int CT = 8 * VPT;                      // the thread's channels
     constexpr int GPV = GPT >= VPT ? GPT / VPT : 1;  // groups inside one vector
@@ -234,7 +237,8 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
         const int cs = cs0 + 8 * v;
         const int bo = (cs % (RB / 2)) / 8;
 #pragma unroll
-        for (int k = 0; k < W; ++k) dyv[v][k] = *reinterpret_cast<const uint4 *>(yb + tc::swz<RB>(t_loc + k, bo));
+        for (int k = 0; k < W; ++k)
+            dyv[v][k] = *reinterpret_cast<const uint4 *>(yb + (VPT == 1 ? ro[k] : tc::swz<RB>(t_loc + k, bo)));
     }
     tc::tmem_wait_ld();
     if (release_w) {  // the item's last filter read: its TMEM buffer is free for the next MMA
@@ -285,19 +289,22 @@ __device__ __forceinline__ void bwd_subtile(const TcMap &m, const unsigned char 
                 dxv[2 * pp + 1] = a1;
             }
         }
-        *reinterpret_cast<uint4 *>(ys + tc::swz<RB>(t_loc, ((cs0 + 8 * v) % (RB / 2)) / 8)) =
+        *reinterpret_cast<uint4 *>(ys + (VPT == 1 ? ro[0] : tc::swz<RB>(t_loc, ((cs0 + 8 * v) % (RB / 2)) / 8))) =
             make_uint4(pack_bf2(dxv[0], dxv[1]), pack_bf2(dxv[2], dxv[3]), pack_bf2(dxv[4], dxv[5]),
                        pack_bf2(dxv[6], dxv[7]));
     }
     if constexpr (GPT == CT) {
         // one channel per group (H = 1): dw[t, g, k] = dy[t, c] x[t-k, c], rounded once to bf16
+        const uint32_t gb16 = (uint32_t)m.GB * 16u;  // bytes between the taps' column blocks of a dw row
 #pragma unroll
         for (int v = 0; v < VPT; ++v) {
             const int bo = ((cs0 + 8 * v) % (RB / 2)) / 8;
+            unsigned char *dwv = dwt + tc::core_off(t_loc, g0 + 8 * v, TB_NB);
 #pragma unroll
             for (int k = 0; k < W; ++k) {
-                const uint4 xv = *reinterpret_cast<const uint4 *>(xb + tc::swz<RB>(t_loc + WIN - k, bo));
-                *reinterpret_cast<uint4 *>(dwt + tc::core_off(t_loc, k * m.GB + g0 + 8 * v, TB_NB)) =
+                const uint4 xv = *reinterpret_cast<const uint4 *>(
+                    xb + (VPT == 1 ? ro[WIN - k] : tc::swz<RB>(t_loc + WIN - k, bo)));
+                *reinterpret_cast<uint4 *>(dwv + (uint32_t)k * gb16) =
                     make_uint4(mul_bf2(dyv[v][0].x, xv.x), mul_bf2(dyv[v][0].y, xv.y), mul_bf2(dyv[v][0].z, xv.z),
                                mul_bf2(dyv[v][0].w, xv.w));
             }
@@ -591,6 +598,9 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
         const float res = m.residual ? 1.f : 0.f;
         const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
         float *xch = reinterpret_cast<float *>(smem + S.xch);
+        uint32_t ro[W];  // swizzled offsets of box rows t_loc .. t_loc+W-1 (one-vector parts)
+#pragma unroll
+        for (int k = 0; k < W; ++k) ro[k] = tc::swz<RB>(t_loc + k, VPT == 1 ? ((part * 8) % (RB / 2)) / 8 : 0);
         // dz of CTA-local tile j (its last block's MMAs are done) leaves TMEM
         auto dz_out = [&](int j, int bseq, int t0) {
             const int tp = j & 1;
@@ -642,7 +652,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                 else
                     bwd_subtile<W, VPT, GPT, PPG, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, dwt, xch,
                                                       part, t_loc, s, smem + S.ystage + (uint32_t)ybuf * S.ybox, res,
-                                                      s == se - 1 ? bars.we(b) : 0u);
+                                                      s == se - 1 ? bars.we(b) : 0u, ro);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars.xe(slot));
                 // dx tile -> global by TMA (the staging tile the next sub-tile writes was read
