@@ -211,12 +211,15 @@ DSC_API dsc_status dsc_decode_state(const dsc_problem *p, const void *x, void *s
  * within a sequence, so every document starts from zero history).
  * p->B must be 1: the single row of p->T tokens holds n_docs documents,
  * document d spanning tokens [cu_seqlens[d], cu_seqlens[d+1]).
- *  - cu_seqlens: DEVICE array of n_docs + 1 int32 offsets rising from
- *    cu_seqlens[0] = 0 to cu_seqlens[n_docs] = T, every document at least
- *    one token long; 4-byte aligned (else DSC_ERR_MISALIGNED).  The offsets
- *    are read on the device only: values outside [0, T] are clamped, so a
- *    malformed array gives wrong results but no access out of bounds.
- *  - 1 <= n_docs <= T, else DSC_ERR_INVALID_ARG.
+ *  - cu_seqlens: DEVICE array of n_docs + 1 int32 offsets, non-decreasing
+ *    from cu_seqlens[0] = 0 to cu_seqlens[n_docs] = T; 4-byte aligned (else
+ *    DSC_ERR_MISALIGNED).  A document may be empty (equal consecutive
+ *    offsets, as in a padded list of documents): it has no tokens and
+ *    changes nothing.  The offsets are read on the device only: values
+ *    outside [0, T] are clamped, so a malformed array gives wrong results
+ *    but no access out of bounds.
+ *  - n_docs >= 1, else DSC_ERR_INVALID_ARG; DSC_ERR_UNSUPPORTED when
+ *    n_docs * (W-1) * ceil(D/256) reaches 2^31 (the fix-up grids).
  * Per document the result is the single-sequence op of the calls above:
  *   y[t]  = r x_t + sum_{k, t-k >= start(t)} w(t)_k x_{t-k}
  *   dx[s] = r dy_s + sum_{k, s+k < end(s)} w(s+k)_k dy_{s+k}

@@ -337,7 +337,7 @@ dsc_status dsc_decode_state(const dsc_problem *p, const void *x, void *state, vo
 static size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
 
 static dsc_status check_varlen(const dsc_problem *p, const int32_t *cu, int64_t n_docs) {
-    if (p->B != 1 || n_docs < 1 || n_docs > p->T || !cu) return DSC_ERR_INVALID_ARG;
+    if (p->B != 1 || n_docs < 1 || !cu) return DSC_ERR_INVALID_ARG;
     if (reinterpret_cast<uintptr_t>(cu) & 3u) return DSC_ERR_MISALIGNED;
     // the fix-up grids have one block per (edge row, 256 channels)
     if (n_docs * (p->W - 1) * ((p->D + 255) / 256) >= ((int64_t)1 << 31)) return DSC_ERR_UNSUPPORTED;

@@ -210,8 +210,8 @@ def decode(P: Problem, kind: int, x, state, *, w=None, z=None, U=None, ws=None, 
 
 def _cu(P: Problem, cu_seqlens):
     cu = np.ascontiguousarray(cu_seqlens, dtype=np.int64)
-    if P.B != 1 or cu[0] != 0 or cu[-1] != P.T or np.any(np.diff(cu) < 1):
-        raise ValueError("packed sequences: B = 1 and cu_seqlens rising from 0 to T")
+    if P.B != 1 or cu[0] != 0 or cu[-1] != P.T or np.any(np.diff(cu) < 0):
+        raise ValueError("packed sequences: B = 1 and cu_seqlens non-decreasing from 0 to T")
     return cu, cu.ctypes.data_as(C.POINTER(C.c_int64)), len(cu) - 1
 
 

@@ -81,6 +81,10 @@ VARLEN_CASES = [
     (LOWRANK, 300, 512, 8, 1, 16, "bf16", (5, 7, 288)),
     (LOWRANK, 200, 96, 3, 4, 5, "f32", (1, 1, 198)),               # CUDA-core fused kernels
     (LOWRANK, 90, 40, 5, 5, 7, "bf16", (40, 50)),                  # unfused path
+    # empty documents (a padded list of documents): at the start, twice in a row, at the end
+    (HEADWISE, 300, 256, 4, 16, 0, "bf16", (0, 1, 2, 0, 0, 3, 50, 127, 1, 116, 0)),
+    (STATIC, 300, 256, 4, 1, 0, "bf16", (0, 60, 0, 0, 240, 0)),
+    (LOWRANK, 600, 1024, 4, 1, 32, "bf16", (0, 127, 0, 1, 128, 0, 0, 2, 3, 339, 0)),
 ]
 
 
@@ -183,8 +187,10 @@ def test_varlen_rejects_bad_arguments():
                                      s) == _lib.DSC_ERR_MISALIGNED
     assert L.dsc_fwd_headwise_varlen(C.byref(p), cu.data_ptr(), 0, x.data_ptr(), w.data_ptr(), x.data_ptr(),
                                      s) == _lib.DSC_ERR_INVALID_ARG
-    assert L.dsc_fwd_headwise_varlen(C.byref(p), cu.data_ptr(), 9, x.data_ptr(), w.data_ptr(), x.data_ptr(),
-                                     s) == _lib.DSC_ERR_INVALID_ARG
+    # more documents than tokens is allowed (empty documents); a count whose fix-up
+    # grid would not fit is refused before anything is read or launched
+    assert L.dsc_fwd_headwise_varlen(C.byref(p), cu.data_ptr(), 1 << 31, x.data_ptr(), w.data_ptr(), x.data_ptr(),
+                                     s) == _lib.DSC_ERR_UNSUPPORTED
 
 
 # --------------------------------------------------------- sequence chunks ---

@@ -454,6 +454,26 @@ def test_varlen_equals_documents_run_separately(kind, lens, D, W, H, R, residual
 
 
 @pytest.mark.parametrize("kind", [oracle.HEADWISE, oracle.LOWRANK, oracle.STATIC])
+def test_varlen_empty_documents_change_nothing(kind):
+    """A document of no tokens (equal consecutive offsets: at the start, twice
+    in a row inside, at the end) has no outputs and no taps, so the packed
+    result is the one without it, exactly; and each non-empty document is
+    still the plain op on its own tokens."""
+    lens = (3, 1, 5, 4)
+    T, D, W, H, R = sum(lens), 6, 4, 3, 2
+    x, dy, f = _varlen_inputs(kind, T, D, W, H, R)
+    Pp = P(1, T, D, W, H, R, 1)
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    cu_e = np.array([0, 0, 3, 4, 4, 4, 9, 13, 13])
+    np.testing.assert_array_equal(oracle.forward_varlen(Pp, kind, x, cu_e, **f), oracle.forward_varlen(Pp, kind, x, cu, **f))
+    for a, b in zip(oracle.backward_varlen(Pp, kind, x, dy, cu_e, **f), oracle.backward_varlen(Pp, kind, x, dy, cu, **f)):
+        np.testing.assert_array_equal(a, b)
+    yd, _ = _plain(kind, P(1, 5, D, W, H, R, 1), np.ascontiguousarray(x[:, 4:9]), np.ascontiguousarray(dy[:, 4:9]),
+                   {k: (np.ascontiguousarray(v[:, 4:9]) if k in ("w", "z") else v) for k, v in f.items()})
+    np.testing.assert_allclose(oracle.forward_varlen(Pp, kind, x, cu_e, **f)[:, 4:9], yd, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("kind", [oracle.HEADWISE, oracle.LOWRANK, oracle.STATIC])
 def test_varlen_one_document_is_the_plain_op(kind):
     T, D, W, H, R = 9, 6, 4, 3, 2
     x, dy, f = _varlen_inputs(kind, T, D, W, H, R)
