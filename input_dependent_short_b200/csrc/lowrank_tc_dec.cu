@@ -8,8 +8,11 @@
 // of CF channels (TMEM lane = sequence), and the step
 //   y[b,c] = r x[b,c] + w_0 x[b,c] + sum_{k>=1} w_k state[b, W-1-k, c]
 // reads x and the W-1 state rows of the tile's sequences from shared memory.
-// The new state (rows 1 .. W-2 of the old one, then x) is written back by the
-// epilogue threads, which hold those rows in registers.
+// The state box is loaded row-major ([row][sequence][channels]: the tensor
+// map lists the state's dimensions as channels, sequence, row), so each row
+// of the tile is one contiguous slab, and the new state (rows 1 .. W-2 of
+// the old one, then x) leaves by W-1 TMA stores straight from those slabs.
+// The ring slot is released once the stores have read it.
 //
 // This is the training forward's kernel structure (lowrank_tc_fwd.cu) with a
 // tile of 128 sequences in place of 128 tokens of one sequence: z [B,R] and
@@ -111,11 +114,10 @@ struct DecWalk {
 };
 
 // Epilogue of one sub-tile for sequence t_loc (row t_loc of the tile): y for
-// VPT vectors of 8 channels, and the sequence's new state rows for them.
+// VPT vectors of 8 channels (the new state leaves by TMA from the slabs).
 template <int W, int GPV, int VPT, int NGT, int RB>
 __device__ __forceinline__ void dec_subtile(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
-                                            int part, int t_loc, int ci0, unsigned char *ys, uint32_t ybox, float res,
-                                            bf16 *st_row, bool live) {
+                                            int part, int t_loc, int ci0, unsigned char *ys, uint32_t ybox, float res) {
     constexpr int S = W - 1;
     constexpr int NT = GPV * W;
     constexpr int CPG = 8 / GPV;
@@ -126,12 +128,11 @@ __device__ __forceinline__ void dec_subtile(const TcMap &m, const unsigned char 
         const int cs = cs0 + 8 * v;
         const unsigned char *bx = xs + (uint32_t)(cs / (RB / 2)) * boxb;
         const int chunk = (cs % (RB / 2)) / 8;
-        // row 0: x; rows 1 .. S: the state rows j = 0 .. S-1 (x_{t-S+j})
+        // slab 0: x; slabs 1 .. S: the state rows j = 0 .. S-1 (x_{t-S+j}); row t_loc of each
         uint4 xw[W];
-        xw[0] = *reinterpret_cast<const uint4 *>(bx + tc::swz<RB>(t_loc, chunk));
+        const uint32_t so = tc::swz<RB>(t_loc, chunk);
 #pragma unroll
-        for (int j = 0; j < S; ++j)
-            xw[1 + j] = *reinterpret_cast<const uint4 *>(bx + RB * TC_M + tc::swz<RB>(t_loc * S + j, chunk));
+        for (int q = 0; q < W; ++q) xw[q] = *reinterpret_cast<const uint4 *>(bx + (uint32_t)q * (RB * TC_M) + so);
         const int ci = ci0 + 8 * v;
         if constexpr (GPV == 1) {  // one group per vector: its W taps, reloaded when the group changes
             if (v == 0 || ((ci >> m.lgH) != ((ci - 8) >> m.lgH))) {
@@ -164,11 +165,6 @@ __device__ __forceinline__ void dec_subtile(const TcMap &m, const unsigned char 
         }
         *reinterpret_cast<uint4 *>(ys + (uint32_t)(cs / (RB / 2)) * ybox + tc::swz<RB>(t_loc, (cs % (RB / 2)) / 8)) =
             make_uint4(pack_bf2(y[0], y[1]), pack_bf2(y[2], y[3]), pack_bf2(y[4], y[5]), pack_bf2(y[6], y[7]));
-        if (live) {  // new state: rows 1 .. S-1 of the old one move down a row, x becomes row S-1
-#pragma unroll
-            for (int j = 0; j + 1 < S; ++j) st16(st_row + (int64_t)j * m.D + 8 * v, xw[2 + j]);
-            if constexpr (S > 0) st16(st_row + (int64_t)(S - 1) * m.D + 8 * v, xw[0]);
-        }
     }
 }
 
@@ -176,7 +172,7 @@ template <int W, int GPV, int VPT, int NGT>
 __global__ void __launch_bounds__(TD_THREADS, 1)
     k_lr_tc_dec(const __grid_constant__ CUtensorMap tmx, const __grid_constant__ CUtensorMap tms,
                 const __grid_constant__ CUtensorMap tmz, const __grid_constant__ CUtensorMap tmu,
-                const __grid_constant__ CUtensorMap tmy, const DecArgsTc a) {
+                const __grid_constant__ CUtensorMap tmy, const __grid_constant__ CUtensorMap tmsr, const DecArgsTc a) {
     constexpr int S = W - 1;
     constexpr int RB = VPT == 1 ? 64 : 128;
     constexpr int NBX = VPT == 4 ? 2 : 1;
@@ -215,7 +211,7 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
         }
         for (int i = 0; i < NS; ++i) {
             tc::mbar_init(bars.xf(i), 1);
-            tc::mbar_init(bars.xe(i), TD_EPI / 32);
+            tc::mbar_init(bars.xe(i), 1);  // thread 0, once the slot's state stores have read it
         }
         tc::fence_mbar_init();
     }
@@ -241,6 +237,7 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
         if (lane == 0) {
             tc::tma_prefetch_desc(&tmx);
             if constexpr (S > 0) tc::tma_prefetch_desc(&tms);
+            if constexpr (S > 0) tc::tma_prefetch_desc(&tmsr);
             tc::tma_prefetch_desc(&tmz);
             tc::tma_prefetch_desc(&tmu);
             DecWalk it;
@@ -282,7 +279,7 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
                     for (int bx = 0; bx < NBX; ++bx) {
                         tc::tma_load_3d(xb + (uint32_t)bx * Sm.boxb, &tmx, c + bx * (RB / 2), it.t0, 0, bars.xf(slot));
                         if constexpr (S > 0)
-                            tc::tma_load_3d(xb + (uint32_t)bx * Sm.boxb + RB * TC_M, &tms, c + bx * (RB / 2), 0, it.t0,
+                            tc::tma_load_3d(xb + (uint32_t)bx * Sm.boxb + RB * TC_M, &tms, c + bx * (RB / 2), it.t0, 0,
                                             bars.xf(slot));
                     }
                     if (++slot == NS) {
@@ -324,36 +321,44 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
         const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
         DecWalk it;
         it.init(ntiles, i_lo);
-        int slot = 0, ybuf = 0;
+        int slot = 0, ybuf = 0, pslot = -1;
         uint32_t xph = 0;
         for (int li = 0; li < nI; ++li, it.next()) {
             const int b = li & 1;
             wait(bars.wf(b), (uint32_t)((li >> 1) & 1));
             tc::fence_after_sync();
             const uint32_t tb = tlane + (uint32_t)(b * d.NFS);
-            const int64_t seq = (int64_t)it.t0 + t_loc;
-            const bool live = seq < a.B;
             const int se = li == nI - 1 ? s_last : d.nSubF;
             for (int s = li == 0 ? s_first : 0; s < se; ++s) {
                 wait(bars.xf(slot), xph);
                 unsigned char *ys = smem + Sm.ystage + (uint32_t)ybuf * NBX * Sm.ybox;
-                const int c0 = it.blk * d.CF + s * d.SF + part * (8 * VPT);
-                bf16 *st_row = a.state + (live ? seq : 0) * S * m.D + c0;
                 dec_subtile<W, GPV, VPT, NGT, RB>(m, smem + Sm.ring + (uint32_t)slot * Sm.slot, Sm.boxb, tb, part,
-                                                  t_loc, s * d.SF + part * (8 * VPT), ys, Sm.ybox, res, st_row, live);
-                __syncwarp();
-                if (lane == 0) tc::mbar_arrive(bars.xe(slot));
+                                                  t_loc, s * d.SF + part * (8 * VPT), ys, Sm.ybox, res);
                 tc::fence_proxy_async();
-                if (tid == 0) tc::bulk_wait_read_all();
+                if (tid == 0) {
+                    // the previous sub-tile's stores (y staging tile, state slabs) have read
+                    // shared memory: its ring slot goes back to the producer
+                    tc::bulk_wait_read_all();
+                    if (pslot >= 0) tc::mbar_arrive(bars.xe(pslot));
+                }
                 asm volatile("bar.sync 1, %0;" ::"n"(TD_EPI) : "memory");
                 if (tid == 0) {
                     const int c = it.blk * d.CF + s * d.SF;
+                    const uint32_t xb = sbase + Sm.ring + (uint32_t)slot * Sm.slot;
 #pragma unroll
-                    for (int bx = 0; bx < NBX; ++bx)
+                    for (int bx = 0; bx < NBX; ++bx) {
                         tc::tma_store_3d(&tmy, sbase + Sm.ystage + (uint32_t)(ybuf * NBX + bx) * Sm.ybox,
                                          c + bx * (RB / 2), it.t0, 0);
+                        // new state row j: old row j+1 (slab j+2) for j < S-1, x (slab 0) for j = S-1;
+                        // rows of sequences past B are clipped by the store
+#pragma unroll
+                        for (int jr = 0; jr < S; ++jr)
+                            tc::tma_store_3d(&tmsr, xb + (uint32_t)bx * Sm.boxb + (uint32_t)(jr + 1 < S ? jr + 2 : 0) * (RB * TC_M),
+                                             c + bx * (RB / 2), it.t0, jr);
+                    }
                     tc::bulk_commit();
                 }
+                pslot = slot;
                 ybuf ^= 1;
                 if (++slot == NS) {
                     slot = 0;
@@ -415,7 +420,7 @@ bool dec_map(const dsc_problem &p, TcMap &m, DecPlan &d) {
 }
 
 struct DecMaps {
-    CUtensorMap x, s, z, u, y;
+    CUtensorMap x, s, z, u, y, sr;  // sr: one state row of a tile, for the stores
 };
 
 bool dec_maps(const DecArgsTc &a, const void *z, const void *U, void *y, DecMaps &f) {
@@ -437,11 +442,16 @@ bool dec_maps(const DecArgsTc &a, const void *z, const void *U, void *y, DecMaps
               make_map(&f.u, U, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
     if (!ok) return false;
     f.s = f.x;  // unused for W = 1
+    f.sr = f.x;
     if (m.W > 1) {
-        const uint64_t sd[3] = {(uint64_t)m.D, (uint64_t)(m.W - 1), (uint64_t)a.B};
-        const uint64_t ss[2] = {(uint64_t)m.D * 2, (uint64_t)((m.W - 1) * m.D * 2)};
-        const uint32_t sb[3] = {(uint32_t)(rb / 2), (uint32_t)(m.W - 1), (uint32_t)TC_M};
-        ok = make_map(&f.s, a.state, 3, sd, ss, sb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B);
+        // the state [B][W-1][D] seen as channels, sequence, row (strides out of order), so that a
+        // box lands row-major: one [128 sequences x SF] slab per row
+        const uint64_t sd[3] = {(uint64_t)m.D, (uint64_t)a.B, (uint64_t)(m.W - 1)};
+        const uint64_t ss[2] = {(uint64_t)((m.W - 1) * m.D * 2), (uint64_t)m.D * 2};
+        const uint32_t sb[3] = {(uint32_t)(rb / 2), (uint32_t)TC_M, (uint32_t)(m.W - 1)};
+        const uint32_t sb1[3] = {(uint32_t)(rb / 2), (uint32_t)TC_M, 1};
+        ok = make_map(&f.s, a.state, 3, sd, ss, sb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
+             make_map(&f.sr, a.state, 3, sd, ss, sb1, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE);
     }
     return ok;
 }
@@ -457,7 +467,7 @@ cudaError_t launch_dec(const Ctx &c, const DecArgsTc &a, const DecMaps &f) {
     const int64_t per = (total + c.sms - 1) / c.sms;
     const int64_t grid = (total + per - 1) / per;
     const uint32_t smem = 2 * a.d.NFS > 256 && S.total < 120 * 1024 ? 120 * 1024 : S.total;
-    k_lr_tc_dec<W, GPV, VPT, NGT><<<(unsigned)grid, TD_THREADS, smem, c.stream>>>(f.x, f.s, f.z, f.u, f.y, a);
+    k_lr_tc_dec<W, GPV, VPT, NGT><<<(unsigned)grid, TD_THREADS, smem, c.stream>>>(f.x, f.s, f.z, f.u, f.y, f.sr, a);
     count_launch();
     return cudaGetLastError();
 }
