@@ -183,10 +183,15 @@ struct ItemWalk {
 
 // Epilogue of one sub-tile: y for VPT vectors of 8 channels of token t.
 // GPV: filter groups inside one vector (8/H for H < 8, else 1).  NGT (only
-// for GPV == 1): groups among the thread's 8*VPT channels.
-template <int W, int GPV, int VPT, int NGT, int RB>
+// for GPV == 1): groups among the thread's 8*VPT channels.  HOFF: the
+// thread's shared-memory offsets (x rows xo[v][k], staging row yo[v]) were
+// computed once per thread (they do not depend on the item or sub-tile).
+constexpr int FWD_HOFF_MAX = 8;  // most hoisted x-row offsets per thread (VPT * W)
+template <int W, int GPV, int VPT, int NGT, int RB, bool HOFF>
 __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char *xs, uint32_t boxb, uint32_t tb,
-                                            int part, int t_loc, int ci0, unsigned char *ys, uint32_t ybox, float res) {
+                                            int part, int t_loc, int ci0, unsigned char *ys, uint32_t ybox, float res,
+                                            const uint32_t (&xo)[HOFF ? VPT : 1][HOFF ? W : 1],
+                                            const uint32_t (&yo)[HOFF ? VPT : 1]) {
     constexpr int WIN = W - 1;
     constexpr int NT = GPV * W;
     constexpr int CPG = 8 / GPV;
@@ -212,8 +217,10 @@ __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char 
             const unsigned char *bx = xs + (uint32_t)(cs / (RB / 2)) * boxb;
             const int chunk = (cs % (RB / 2)) / 8;
 #pragma unroll
-            for (int k = 0; k < W; ++k)
-                xw[vv][k] = *reinterpret_cast<const uint4 *>(bx + tc::swz<RB>(t_loc + WIN - k, chunk));
+            for (int k = 0; k < W; ++k) {
+                if constexpr (HOFF) xw[vv][k] = *reinterpret_cast<const uint4 *>(xs + xo[v0 + vv][k]);
+                else xw[vv][k] = *reinterpret_cast<const uint4 *>(bx + tc::swz<RB>(t_loc + WIN - k, chunk));
+            }
         }
 #pragma unroll
         for (int vv = 0; vv < VB; ++vv) {
@@ -234,7 +241,7 @@ __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char 
                     yp[pp] = acc2;
                 }
                 const int cs = cs0 + 8 * v;
-                *reinterpret_cast<uint4 *>(ys + (uint32_t)(cs / (RB / 2)) * ybox + tc::swz<RB>(t_loc, (cs % (RB / 2)) / 8)) =
+                *reinterpret_cast<uint4 *>(ys + (HOFF ? yo[v] : (uint32_t)(cs / (RB / 2)) * ybox + tc::swz<RB>(t_loc, (cs % (RB / 2)) / 8))) =
                     make_uint4(pack_bf2(lo2(yp[0]), hi2(yp[0])), pack_bf2(lo2(yp[1]), hi2(yp[1])),
                                pack_bf2(lo2(yp[2]), hi2(yp[2])), pack_bf2(lo2(yp[3]), hi2(yp[3])));
             } else {
@@ -265,7 +272,7 @@ __device__ __forceinline__ void fwd_subtile(const TcMap &m, const unsigned char 
                     }
                 }
                 const int cs = cs0 + 8 * v;
-                *reinterpret_cast<uint4 *>(ys + (uint32_t)(cs / (RB / 2)) * ybox + tc::swz<RB>(t_loc, (cs % (RB / 2)) / 8)) =
+                *reinterpret_cast<uint4 *>(ys + (HOFF ? yo[v] : (uint32_t)(cs / (RB / 2)) * ybox + tc::swz<RB>(t_loc, (cs % (RB / 2)) / 8))) =
                     make_uint4(pack_bf2(lo2(y2[0]), hi2(y2[0])), pack_bf2(lo2(y2[1]), hi2(y2[1])),
                                pack_bf2(lo2(y2[2]), hi2(y2[2])), pack_bf2(lo2(y2[3]), hi2(y2[3])));
             }
@@ -420,6 +427,22 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
     } else {
         // ------------------------------------------------------------ epilogue
         const int t_loc = tid & (TC_M - 1), part = tid >> 7, quarter = warp & 3;
+        // the thread's x-row and staging offsets, the same for every item and sub-tile
+        constexpr bool HOFF = VPT * W <= FWD_HOFF_MAX;
+        uint32_t xo[HOFF ? VPT : 1][HOFF ? W : 1], yo[HOFF ? VPT : 1];
+        if constexpr (HOFF) {
+#pragma unroll
+            for (int v = 0; v < VPT; ++v) {
+                const int cs = part * (8 * VPT) + 8 * v;
+                const uint32_t bxo = (uint32_t)(cs / (RB / 2)) * S.boxb;
+#pragma unroll
+                for (int k = 0; k < W; ++k) xo[v][k] = bxo + tc::swz<RB>(t_loc + WIN - k, (cs % (RB / 2)) / 8);
+                yo[v] = (uint32_t)(cs / (RB / 2)) * S.ybox + tc::swz<RB>(t_loc, (cs % (RB / 2)) / 8);
+            }
+        } else {
+            xo[0][0] = 0;
+            yo[0] = 0;
+        }
         const float res = m.residual ? 1.f : 0.f;
         const uint32_t tlane = tmem + ((uint32_t)(quarter * 32) << 16);
         ItemWalk it;
@@ -435,8 +458,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
             for (int s = li == 0 ? s_first : 0; s < se; ++s) {
                 wait(bars.xf(slot), xph);
                 unsigned char *ys = smem + S.ystage + (uint32_t)ybuf * NBX * S.ybox;
-                fwd_subtile<W, GPV, VPT, NGT, RB>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, part, t_loc,
-                                                  s * m.SF + part * (8 * VPT), ys, S.ybox, res);
+                fwd_subtile<W, GPV, VPT, NGT, RB, HOFF>(m, smem + S.ring + (uint32_t)slot * S.slot, S.boxb, tb, part,
+                                                        t_loc, s * m.SF + part * (8 * VPT), ys, S.ybox, res, xo, yo);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars.xe(slot));
                 // y tile -> global by TMA: the staging tile the next sub-tile writes was
