@@ -114,6 +114,11 @@ HEADWISE_SHAPES = [
     (1, 129, 256, 8, 1),    # W = 8 per-channel
     (1, 200, 128, 6, 32),
     (1, 77, 40, 7, 8),      # D = 40: 5 vectors of 8
+    # groups of 16 or more lanes: the backward's reduce-scatter of dw (taps padded to 4 or 8)
+    (1, 90, 256, 5, 128),   # 16 / 32 lanes, W = 5
+    (1, 60, 256, 8, 128),   # 16 / 32 lanes, W = 8
+    (2, 40, 512, 7, 256),   # 32 lanes / generic, W = 7
+    (1, 70, 256, 3, 64),    # 8 / 16 lanes, W = 3
 ]
 
 
