@@ -655,14 +655,17 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                                                       s == se - 1 ? bars.we(b) : 0u, ro);
                 __syncwarp();
                 if (lane == 0) tc::mbar_arrive(bars.xe(slot));
-                // dx tile -> global by TMA (the staging tile the next sub-tile writes was read
-                // by the store issued one sub-tile ago, waited for before this barrier)
+                // dx rows of this lane quarter (32 tokens) -> global by TMA, issued by the
+                // quarter's first thread after a barrier of its 4 warps only; the staging
+                // rows the next sub-tile writes were read by the store this thread issued one
+                // sub-tile ago, waited for before the barrier
                 tc::fence_proxy_async();
-                if (tid == 0) tc::bulk_wait_read_all();
-                epi_bar();
-                if (tid == 0) {
-                    tc::tma_store_3d(&tmdx, sbase + S.ystage + (uint32_t)ybuf * S.ybox, it.blk * m.CB + s * m.SB, it.t0,
-                                     it.b);
+                const bool qlead = warp == quarter && lane == 0;
+                if (qlead) tc::bulk_wait_read_all();
+                asm volatile("bar.sync %0, %1;" ::"r"(2 + quarter), "n"(TB_EPI / 4) : "memory");
+                if (qlead) {
+                    tc::tma_store_3d(&tmdx, sbase + S.ystage + (uint32_t)ybuf * S.ybox + (uint32_t)(quarter * 32 * RB),
+                                     it.blk * m.CB + s * m.SB, it.t0 + quarter * 32, it.b);
                     tc::bulk_commit();
                 }
                 ybuf ^= 1;
@@ -707,7 +710,7 @@ __global__ void __launch_bounds__(TB_THREADS, 1)
                 }
             }
         }
-        if (tid == 0) tc::bulk_wait_all();
+        if (warp == quarter && lane == 0) tc::bulk_wait_all();  // each quarter's own dx stores
     }
 
     // teardown: every load and MMA this CTA issued has landed before the
@@ -912,7 +915,7 @@ bool bwd_maps(const TcArgs &a, BwdMaps &f) {
     const uint64_t xd[3] = {(uint64_t)m.D, (uint64_t)m.T, (uint64_t)m.B};
     const uint64_t xs[2] = {(uint64_t)m.D * 2, (uint64_t)(m.T * m.D * 2)};
     const uint32_t xb[3] = {(uint32_t)(rb / 2), (uint32_t)(TC_M + m.W - 1), 1};
-    const uint32_t yb[3] = {(uint32_t)(rb / 2), (uint32_t)TC_M, 1};
+    const uint32_t yb[3] = {(uint32_t)(rb / 2), 32, 1};  // a lane quarter's 32 rows
     const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
                                   : (rb == 64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
     return make_map(&f.x, a.x, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
