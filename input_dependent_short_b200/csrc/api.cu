@@ -3,7 +3,7 @@
 #include <atomic>
 #include <mutex>
 
-#include "kernels.cuh"
+#include "edges.cuh"
 
 namespace dsc {
 
@@ -365,13 +365,15 @@ static EdgeArgs varlen_edges(const dsc_problem &p, int kind, const int32_t *cu, 
     edge_args(p, kind, a);
     a.cu = cu;
     a.nseg = n_docs;
+    a.early = 1;  // every packed-document call runs the row pass first
     return a;
 }
 
 static EdgeArgs chunk_edges(const dsc_problem &p, int kind, const void *x_prev, const void *dy_next,
-                            const void *f_next) {
+                            const void *f_next, int edges_only) {
     EdgeArgs a{};
     edge_args(p, kind, a);
+    a.early = !edges_only;
     a.cu = nullptr;
     a.nseg = p.B;
     if (p.W > 1) {
@@ -497,7 +499,7 @@ dsc_status dsc_fwd_headwise_chunk(const dsc_problem *p, const void *x_prev, cons
     if (s == DSC_OK) s = check_halos(p, x_prev, nullptr, nullptr, false);
     if (s == DSC_OK && !edges_only) s = dsc_fwd_headwise(p, x, w, y, stream);
     if (s != DSC_OK) return s;
-    EdgeArgs a = chunk_edges(*p, EDGE_HEADWISE, x_prev, nullptr, nullptr);
+    EdgeArgs a = chunk_edges(*p, EDGE_HEADWISE, x_prev, nullptr, nullptr, edges_only);
     a.x = x; a.w = w; a.y = y;
     return edges_fwd(stream, p, a);
 }
@@ -511,7 +513,7 @@ dsc_status dsc_bwd_headwise_chunk(const dsc_problem *p, const void *x_prev, cons
     if (s == DSC_OK) s = check_halos(p, x_prev, dy_next, w_next, true);
     if (s == DSC_OK && !edges_only) s = dsc_bwd_headwise(p, x, w, dy, dx, dw, stream);
     if (s != DSC_OK) return s;
-    EdgeArgs a = chunk_edges(*p, EDGE_HEADWISE, x_prev, dy_next, w_next);
+    EdgeArgs a = chunk_edges(*p, EDGE_HEADWISE, x_prev, dy_next, w_next, edges_only);
     a.x = x; a.w = w; a.dy = dy; a.dx = dx; a.dw = dw;
     return edges_bwd(stream, p, a);
 }
@@ -524,7 +526,7 @@ dsc_status dsc_fwd_lowrank_chunk(const dsc_problem *p, const void *x_prev, const
     if (s == DSC_OK) s = check_halos(p, x_prev, nullptr, nullptr, false);
     if (s == DSC_OK && !edges_only) s = dsc_fwd_lowrank(p, x, z, U, y, workspace, workspace_bytes, stream);
     if (s != DSC_OK) return s;
-    EdgeArgs a = chunk_edges(*p, EDGE_LOWRANK, x_prev, nullptr, nullptr);
+    EdgeArgs a = chunk_edges(*p, EDGE_LOWRANK, x_prev, nullptr, nullptr, edges_only);
     a.x = x; a.z = z; a.U = U; a.y = y;
     return edges_fwd(stream, p, a);
 }
@@ -542,7 +544,7 @@ dsc_status dsc_bwd_lowrank_chunk(const dsc_problem *p, const void *x_prev, const
     if (s == DSC_OK) s = check_ptrs({x, z, U, dy, dx, dz, dU});
     if (s == DSC_OK) s = check_halos(p, x_prev, dy_next, z_next, true);
     if (s != DSC_OK) return s;
-    return lowrank_bwd_edges(p, chunk_edges(*p, EDGE_LOWRANK, x_prev, dy_next, z_next), x, z, U, dy, dx, dz, dU,
+    return lowrank_bwd_edges(p, chunk_edges(*p, EDGE_LOWRANK, x_prev, dy_next, z_next, edges_only), x, z, U, dy, dx, dz, dU,
                              workspace, workspace_bytes, dsc_bwd_lowrank_workspace_bytes(p), !edges_only, stream);
 }
 
@@ -554,7 +556,7 @@ dsc_status dsc_fwd_static_chunk(const dsc_problem *p, const void *x_prev, const 
     if (s == DSC_OK) s = check_halos(p, x_prev, nullptr, nullptr, false);
     if (s == DSC_OK && !edges_only) s = dsc_fwd_static(p, x, ws, y, stream);
     if (s != DSC_OK) return s;
-    EdgeArgs a = chunk_edges(*p, EDGE_STATIC, x_prev, nullptr, nullptr);
+    EdgeArgs a = chunk_edges(*p, EDGE_STATIC, x_prev, nullptr, nullptr, edges_only);
     a.x = x; a.w = ws; a.y = y;
     return edges_fwd(stream, p, a);
 }
@@ -568,7 +570,7 @@ dsc_status dsc_bwd_static_chunk(const dsc_problem *p, const void *x_prev, const 
     if (s == DSC_OK) s = check_halos(p, x_prev, dy_next, nullptr, false);
     if (s == DSC_OK && !edges_only) s = dsc_bwd_static(p, x, ws, dy, dx, dws, workspace, workspace_bytes, stream);
     if (s != DSC_OK) return s;
-    EdgeArgs a = chunk_edges(*p, EDGE_STATIC, x_prev, dy_next, nullptr);
+    EdgeArgs a = chunk_edges(*p, EDGE_STATIC, x_prev, dy_next, nullptr, edges_only);
     a.x = x; a.w = ws; a.dy = dy; a.dx = dx; a.dws = dws;
     return edges_bwd(stream, p, a);
 }

@@ -23,9 +23,12 @@
 // work (plus one R x (G*W) contraction per fixed token for low-rank), and
 // the roofline kernels keep their inner loops free of per-token edge tests.
 // The fix-up kernels read only the call's inputs before their first store, so
-// they load and compute while the row pass finishes (programmatic dependent
-// launch) and wait for it only to store.
-#include "kernels.cuh"
+// when the row pass runs in the same call they load and compute while it
+// finishes (programmatic dependent launch) and wait for it only to store: the
+// row pass itself waited for the stream's earlier kernels before it let them
+// start, so the inputs are complete.  A call that runs the fix-ups alone has
+// no such pass before them, and its first fix-up kernel waits before it reads.
+#include "edges.cuh"
 
 namespace dsc {
 
@@ -99,7 +102,8 @@ __device__ __forceinline__ void x_left(const EdgeArgs &a, int64_t b, int64_t s, 
 // ---------------------------------------------------------------- forward ---
 // y of the first W-1 tokens of each segment with a wrong left edge.
 template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_y(const EdgeArgs a, int64_t cblocks) {
-    pdl_trigger();  // the next fix-up kernel may start its loads
+    if (!a.early) pdl_wait();  // no row pass in this call: inputs may come from the stream's previous kernel
+    pdl_trigger();             // the next fix-up kernel may start its loads
     const int64_t row = blockIdx.x / cblocks;
     const int64_t c = (blockIdx.x % cblocks) * ED_THREADS + threadIdx.x;
     const int64_t i = row / (a.W - 1);
@@ -125,7 +129,8 @@ template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_y(con
 // --------------------------------------------------------------- backward ---
 // dx of the last W-1 tokens of each segment with a wrong right edge.
 template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dx(const EdgeArgs a, int64_t cblocks) {
-    pdl_trigger();  // the next fix-up kernel may start its loads
+    if (!a.early) pdl_wait();  // no row pass in this call: inputs may come from the stream's previous kernel
+    pdl_trigger();             // the next fix-up kernel may start its loads
     const int64_t row = blockIdx.x / cblocks;
     const int64_t c = (blockIdx.x % cblocks) * ED_THREADS + threadIdx.x;
     const int64_t i = row / (a.W - 1);
@@ -158,7 +163,8 @@ template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dx(co
 //              zero-padded pass's (dwdelta); rows with nothing to fix are
 //              zero in both.
 template <typename T> __global__ void __launch_bounds__(ED_THREADS) k_edge_dw(const EdgeArgs a) {
-    pdl_trigger();  // the next fix-up kernel may start its loads
+    if (!a.early) pdl_wait();  // no row pass in this call: inputs may come from the stream's previous kernel
+    pdl_trigger();             // the next fix-up kernel may start its loads
     const int64_t idx = (int64_t)blockIdx.x * ED_THREADS + threadIdx.x;
     const int64_t nrows = a.nseg * (a.W - 1);
     if (idx >= nrows * a.G) return;

@@ -35,6 +35,7 @@ struct TcMap {
     int CF, NF, SF, nSubF, nBlkF, NSF, NOPF;
     int NFS;             // TMEM columns per filter buffer: NF rounded up to a power of two
     int64_t nItemsF;
+    int zsw;             // forward z tile: one TMA box with this row swizzle (2R bytes: R = 16, 32, 64), or 0: 8-column boxes
     // backward: block of CB channels = GB groups -> NBW = W*GB <= 128 filter columns;
     // sub-tiles of SB channels; CTA = (range of tiles) x (group of CPC blocks)
     int CB, GB, NBW, SB, nSubB, nBlkB;

@@ -16,7 +16,8 @@
 //
 // This is the training forward's kernel structure (lowrank_tc_fwd.cu) with a
 // tile of 128 sequences in place of 128 tokens of one sequence: z [B,R] and
-// U [R,G*W] arrive by TMA into the MMA's core-matrix layouts; per sub-tile of
+// U [R,G*W] arrive by TMA into the MMA's operand layouts (z as one swizzled box when
+// R is 16, 32 or 64, as in the forward); per sub-tile of
 // SF channels one TMA box brings x [128 sequences x SF] and one the state
 // [128 sequences x (W-1) rows x SF] (rows of 64 or 128 bytes, swizzled); y
 // leaves through a swizzled staging tile and a TMA store.  Warp roles (576
@@ -256,7 +257,10 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
                     if (i == ob) held = ublk[i];
                 const bool newu = held != it.blk;
                 tc::mbar_expect_tx(bars.opf(ob), (uint32_t)kz * 2048u + (newu ? Sm.ubytes : 0u));
-                for (int j = 0; j < kz; ++j) tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, 0, bars.opf(ob));
+                if (m.zsw) tc::tma_load_3d(zb, &tmz, 0, it.t0, 0, bars.opf(ob));  // one swizzled box
+                else
+                    for (int j = 0; j < kz; ++j)
+                        tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, 0, bars.opf(ob));
                 if (newu) {
 #pragma unroll
                     for (int i = 0; i < TD_MAXOP; ++i)
@@ -302,7 +306,8 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
                 tc::fence_after_sync();
                 const uint32_t zb = sbase + (uint32_t)ob * Sm.opsize, ub = zb + Sm.zbytes;
                 for (int ks = 0; ks < m.RP / 16; ++ks) {
-                    const uint64_t ad = tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
+                    const uint64_t ad = m.zsw ? tc::smem_desc_swz(zb + (uint32_t)ks * 32u, 16, 8u * (uint32_t)m.zsw, m.zsw)
+                                              : tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
                     const uint64_t bd = tc::smem_desc(ub + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
                     tc::mma_bf16(tmem + (uint32_t)(b * d.NFS), ad, bd, id_w, ks > 0 ? 1u : 0u);
                 }
@@ -432,13 +437,16 @@ bool dec_maps(const DecArgsTc &a, const void *z, const void *U, void *y, DecMaps
     const uint32_t xbx[3] = {(uint32_t)(rb / 2), (uint32_t)TC_M, 1};
     const uint64_t zd[3] = {(uint64_t)m.R, (uint64_t)a.B, 1};
     const uint64_t zs[2] = {(uint64_t)m.R * 2, (uint64_t)(a.B * m.R * 2)};
-    const uint32_t zb[3] = {8, (uint32_t)TC_M, 1};
+    const uint32_t zb[3] = {m.zsw ? (uint32_t)m.R : 8u, (uint32_t)TC_M, 1};
+    const CUtensorMapSwizzle zsw = m.zsw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                   : m.zsw == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                   : m.zsw == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
     const uint64_t ud[2] = {(uint64_t)m.GW, (uint64_t)m.R};
     const uint64_t us[1] = {(uint64_t)m.GW * 2};
     const uint32_t ub[2] = {8, (uint32_t)m.RP};
     bool ok = make_map(&f.x, a.x, 3, xd, xs, xbx, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
               make_map(&f.y, y, 3, xd, xs, xbx, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE) &&
-              make_map(&f.z, z, 3, zd, zs, zb, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
+              make_map(&f.z, z, 3, zd, zs, zb, zsw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
               make_map(&f.u, U, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
     if (!ok) return false;
     f.s = f.x;  // unused for W = 1

@@ -21,9 +21,13 @@
 // Every hand-off is an mbarrier (full / empty pairs); nothing waits on the
 // whole block inside the loop.
 //
-// Operand layouts written by TMA (no swizzle, 8-element boxes):
-//   z tile  (A, K-major):  element (t, k) at (k/8)*2048 + t*16 + (k%8)*2
+// Operand layouts written by TMA:
+//   z tile  (A, K-major):  for R = 16, 32 or 64 one box of 128 rows of 2R
+//                          bytes with a 2R-byte swizzle (a few long rows move
+//                          faster than many 16-byte ones); otherwise 8-element
+//                          boxes, element (t, k) at (k/8)*2048 + t*16 + (k%8)*2
 //   U block (B, MN-major): element (k, n) at (n/8)*(RP*16) + k*16 + (n%8)*2
+//                          (no swizzle, 8-element boxes)
 // x sub-tiles: boxes of 64 channels (128-byte rows, 128-byte swizzle) or of
 // 32 channels (64-byte rows, 64-byte swizzle).
 #include "lowrank_tc.cuh"
@@ -82,6 +86,7 @@ bool tc_map(const dsc_problem &p, TcMap &m) {
     m.lgH = 0;
     while ((1 << m.lgH) < m.H) ++m.lgH;
     m.residual = p.residual ? 1 : 0;
+    m.zsw = (m.R == 16 || m.R == 32 || m.R == 64) ? (int)(2 * m.R) : 0;  // then R == RP: no padded k-chunks
     return true;
 }
 
@@ -368,8 +373,12 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
                     if (i == ob) held = ublk[i];
                 const bool newu = held != it.blk;
                 tc::mbar_expect_tx(bars.opf(ob), (uint32_t)kz * 2048u + (newu ? S.ubytes : 0u));
-                for (int j = 0; j < kz; ++j)
-                    tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, it.b, bars.opf(ob));
+                if (m.zsw) {
+                    tc::tma_load_3d(zb, &tmz, 0, it.t0, it.b, bars.opf(ob));
+                } else {
+                    for (int j = 0; j < kz; ++j)
+                        tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, it.b, bars.opf(ob));
+                }
                 if (newu) {
 #pragma unroll
                     for (int i = 0; i < TF_MAXOP; ++i)
@@ -412,7 +421,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
                 tc::fence_after_sync();
                 const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
                 for (int ks = 0; ks < m.RP / 16; ++ks) {
-                    const uint64_t ad = tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
+                    const uint64_t ad = m.zsw ? tc::smem_desc_swz(zb + (uint32_t)ks * 32u, 16, 8u * (uint32_t)m.zsw, m.zsw)
+                                              : tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
                     const uint64_t bd = tc::smem_desc(ub + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
                     tc::mma_bf16(tmem + (uint32_t)(b * m.NFS), ad, bd, id_w, ks > 0 ? 1u : 0u);
                 }
@@ -613,14 +623,17 @@ bool fwd_maps(const TcArgs &a, FwdMaps &f) {
     const uint32_t yb[3] = {(uint32_t)(rb / 2), (uint32_t)TC_M, 1};
     const uint64_t zd[3] = {(uint64_t)m.R, (uint64_t)m.T, (uint64_t)m.B};
     const uint64_t zs[2] = {(uint64_t)m.R * 2, (uint64_t)(m.T * m.R * 2)};
-    const uint32_t zb[3] = {8, (uint32_t)TC_M, 1};
+    const uint32_t zb[3] = {m.zsw ? (uint32_t)m.R : 8u, (uint32_t)TC_M, 1};
+    const CUtensorMapSwizzle zsw = m.zsw == 128 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                   : m.zsw == 64 ? CU_TENSOR_MAP_SWIZZLE_64B
+                                   : m.zsw == 32 ? CU_TENSOR_MAP_SWIZZLE_32B : CU_TENSOR_MAP_SWIZZLE_NONE;
     const uint64_t ud[2] = {(uint64_t)m.GW, (uint64_t)m.R};
     const uint64_t us[1] = {(uint64_t)m.GW * 2};
     const uint32_t ub[2] = {8, (uint32_t)m.RP};
     const CUtensorMapSwizzle sw = rb == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
     return make_map(&f.x, a.x, 3, xd, xs, xb, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B) &&
            make_map(&f.y, a.y, 3, xd, xs, yb, sw, CU_TENSOR_MAP_L2_PROMOTION_NONE) &&
-           make_map(&f.z, a.z, 3, zd, zs, zb, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
+           make_map(&f.z, a.z, 3, zd, zs, zb, zsw, CU_TENSOR_MAP_L2_PROMOTION_L2_128B) &&
            make_map(&f.u, a.Uf ? a.Uf : a.U, 2, ud, us, ub, CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_128B);
 }

@@ -36,6 +36,21 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
     return d;             // base offset 0, absolute LBO mode, layout type 0 (no swizzle)
 }
 
+// Shared-memory descriptor of a K-major operand written by TMA with a 32-,
+// 64- or 128-byte swizzle (`swz` bytes per row): 8-row atoms of `swz`-byte
+// rows, sbo = 8 * swz (the next 8 rows), lbo unused; a K step of 16 bf16
+// inside a row moves `addr` by 32 bytes.  Layout-type field (bits 61-63):
+// 2 = 128-byte, 4 = 64-byte, 6 = 32-byte swizzle.
+__device__ __forceinline__ uint64_t smem_desc_swz(uint32_t addr, uint32_t lbo, uint32_t sbo, int swz) {
+    uint64_t d = 0;
+    d |= (uint64_t)((addr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version (sm_100)
+    d |= (uint64_t)(swz == 128 ? 2 : (swz == 64 ? 4 : 6)) << 61;
+    return d;
+}
+
 // Shared-memory matrix descriptor of a tile written by TMA with 128-byte
 // swizzling (rows of 128 bytes, 8-row atoms of 1024 bytes, atom base aligned
 // to 1024 bytes; layout type 2).  K-major: the rows run along M/N, sbo = 1024
@@ -43,13 +58,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint3
 // row moves `addr` by 32 bytes.  MN-major: the rows run along K, sbo = 1024
 // (the next 8 K rows), lbo = the byte offset of the next 64 M/N elements.
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr, uint32_t lbo, uint32_t sbo) {
-    uint64_t d = 0;
-    d |= (uint64_t)((addr >> 4) & 0x3FFF);
-    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
-    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
-    d |= (uint64_t)1 << 46;  // descriptor version (sm_100)
-    d |= (uint64_t)2 << 61;  // 128-byte swizzle
-    return d;
+    return smem_desc_swz(addr, lbo, sbo, 128);
 }
 
 // Instruction descriptor of kind::f16 with bf16 A/B and an fp32 accumulator.

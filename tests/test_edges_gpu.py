@@ -294,6 +294,37 @@ def test_chunks_match_the_whole_sequence(case, edges_only):
     ops().dsc_check()
 
 
+def test_edges_only_waits_for_the_kernel_that_wrote_its_halos():
+    """The edges-only form may follow, on the same stream, the kernel that
+    wrote its halos; here x_prev and dy_next are the last rows of a long
+    forward's output, launched just before the fix-ups.  The fix-ups must read
+    them only once that kernel is done: each result equals the one-call form
+    run after a synchronize."""
+    o = ops()
+    B, L, D, W, H = 1, 256, 1024, 4, 16
+    G, Tbig = D // H, 1 << 17
+    g = torch.Generator(device="cuda").manual_seed(11)
+
+    def rnd(*shape, scale=1.0):
+        return (torch.randn(*shape, device="cuda", generator=g) * scale).to(torch.bfloat16)
+
+    xc, dyc = rnd(B, L, D), rnd(B, L, D)
+    wc, w_next = rnd(B, L, G, W, scale=0.5), rnd(B, W - 1, G, W, scale=0.5)
+    for _ in range(3):
+        a, wa = rnd(B, Tbig, D), rnd(B, Tbig, G, W, scale=0.5)
+        y = o.dsc_fwd_headwise(xc, wc)
+        x_prev = o.dsc_fwd_headwise(a, wa)[:, Tbig - (W - 1):]
+        y = o.dsc_fwd_headwise_chunk(xc, wc, x_prev, out=y)
+        gr = o.dsc_bwd_headwise(xc, wc, dyc)
+        dy_next = o.dsc_fwd_headwise(a, wa, False)[:, Tbig - (W - 1):]
+        gr = o.dsc_bwd_headwise_chunk(xc, wc, dyc, x_prev, dy_next, w_next, out=gr)
+        torch.cuda.synchronize()
+        assert torch.equal(y, o.dsc_fwd_headwise_chunk(xc, wc, x_prev))
+        full = o.dsc_bwd_headwise_chunk(xc, wc, dyc, x_prev, dy_next, w_next)
+        assert torch.equal(gr[0], full[0]) and torch.equal(gr[1], full[1])
+    ops().dsc_check()
+
+
 def test_chunk_without_halos_is_the_plain_call():
     o = ops()
     wl = Workload("first-last", HEADWISE, 2, 300, 256, 4, H=16, seed=7)
