@@ -24,8 +24,10 @@
 //    halo of dy and w) to finish its last rows; dw(t) needs dy_t and the
 //    x window, and is reduced over the H channels of a group with shuffles
 //    inside the warp (no shared memory, no atomics);
-//  - the grid is sized from the measured residency so that all tiles are in
-//    flight at once (one wave), avoiding a tail of partially filled SMs.
+//  - the grid is sized from the measured residency: a whole number of waves
+//    of resident warps (one, or for the head-wise kernels two or three waves
+//    of shorter tiles, which even out the warps' unequal progress; see
+//    stream_waves).
 #include "kernels.cuh"
 
 namespace dsc {
@@ -698,8 +700,8 @@ bool stream_map(const dsc_problem &p, int V, StreamMap &m) {
     return true;
 }
 
-// Pick the tile length so that all warps are resident at once (exactly one
-// wave): the largest number of time tiles whose warps all fit on the GPU.
+// Pick the tile length for `target_warps` warps (a whole number of waves of
+// resident warps): the largest number of time tiles whose warps fit.
 void finish_map(StreamMap &m, int64_t target_warps) {
     const int64_t cols = m.B * m.nWc;
     int64_t tiles = target_warps / cols;
@@ -751,11 +753,34 @@ static size_t stream_setup(int &per_sm_warps) {
     return smem;
 }
 
+// Waves of tiles.  With one wave (every tile in flight at once) the kernel
+// ends with its slowest warp, and per-warp finish times spread widely: in the
+// Q/K/V head-wise backward from 58 to 138 us around a mean of 104 us, by
+// where the block ran rather than by its data (moving the tensors by half
+// their size left the slow sequences the same).  Several waves of shorter
+// tiles let the SMs whose blocks finish early take new ones; each extra tile
+// costs a ring start-up and, backward, a W-1 token right halo.  Measured per
+// kernel on one box at W = 4: Q/K/V forward -7 % with 3 waves, backward -5 %
+// with 2 (-8 % with 3, but the all-linear backward then +5 %), all-linear
+// forward -4 %, packed-document row -3 %.  They lost elsewhere, so those keep
+// one wave: at W = 2 and W = 8 (+4 to +9 % on the B = 1, T = 16384 widths,
+// where the lighter or register-heavier tokens make a tile's start-up a
+// larger share), with tiles under 32 tokens (forward) or 64 (backward), and
+// in the static kernels, whose filter-gradient partials grow with the tiles.
+template <bool BWD, bool WS> static int stream_waves(StreamMap m, int64_t one_wave) {
+    if constexpr (WS) return 1;
+    if (m.W != 4) return 1;
+    const int f = BWD ? 2 : 3;
+    finish_map(m, one_wave * f);
+    return m.Tt >= (BWD ? 64 : 32) ? f : 1;
+}
+
 template <typename T, int W, int GPT, bool WS, bool BWD, int VB, bool RS = false>
 static cudaError_t run_stream(const Ctx &c, HwArgs a) {
     int per_sm = 0;
     const size_t smem = stream_setup<T, W, GPT, WS, BWD, VB, RS>(per_sm);
-    finish_map(a.m, (int64_t)per_sm * c.sms);
+    const int64_t one_wave = (int64_t)per_sm * c.sms;
+    finish_map(a.m, one_wave * stream_waves<BWD, WS>(a.m, one_wave));
     const int64_t blocks = (a.m.n_warps + STREAM_THREADS / 32 - 1) / (STREAM_THREADS / 32);
     cudaError_t e;
     if constexpr (BWD)
