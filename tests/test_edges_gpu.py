@@ -325,6 +325,68 @@ def test_edges_only_waits_for_the_kernel_that_wrote_its_halos():
     ops().dsc_check()
 
 
+@pytest.mark.parametrize("variant", ["headwise", "static"])
+def test_full_size_chunks_are_bit_exact_with_the_whole_call(variant):
+    """At the Q/K/V size (B=8, T=2048, D=6144, W=4; H=16 head-wise) the whole
+    call and four chunk calls of 512 tokens tile time differently: the whole
+    head-wise call runs several waves of tiles of about 40 tokens, the chunks
+    one wave of shorter ones.  The streaming kernels compute every output
+    element by the same arithmetic in the same order whatever the tiling
+    (the token's taps summed tap by tap), so away from the chunk edges y, dx
+    and the head-wise dw must agree bit for bit at every element, which
+    checks the tile and wave boundaries of the full-size launch.  The W-1
+    rows next to a chunk edge come from the fix-up kernels, which sum in
+    another order: they are compared within the bf16 tolerance, as is the
+    static dws (a sum over tiles, whose order differs)."""
+    o = ops()
+    B, T, D, W, H = 8, 2048, 6144, 4, 16
+    g = torch.Generator(device="cuda").manual_seed(31)
+
+    def rnd(*shape, scale=1.0):
+        return (torch.randn(*shape, device="cuda", generator=g) * scale).to(torch.bfloat16)
+
+    x, dy = rnd(B, T, D), rnd(B, T, D)
+    if variant == "headwise":
+        w = rnd(B, T, D // H, W, scale=0.5)
+        y = o.dsc_fwd_headwise(x, w)
+        dx, dw = o.dsc_bwd_headwise(x, w, dy)
+    else:
+        ws = rnd(D, W, scale=0.5)
+        y = o.dsc_fwd_static(x, ws, True)
+        dx, dws = o.dsc_bwd_static(x, ws, dy, True)
+        dws_sum = torch.zeros_like(dws)
+    n = T // 4
+    for c in range(4):
+        sl = slice(c * n, (c + 1) * n)
+        xc, dyc = x[:, sl].contiguous(), dy[:, sl].contiguous()
+        x_prev = None if c == 0 else x[:, c * n - (W - 1):c * n].contiguous()
+        dy_next = None if c == 3 else dy[:, (c + 1) * n:(c + 1) * n + W - 1].contiguous()
+        lo = 0 if c == 0 else W - 1      # rows after a left edge (fixed up: y, dw)
+        hi = n if c == 3 else n - (W - 1)  # rows before a right edge (fixed up: dx)
+
+        def same(name, got, ref, a, b):
+            assert torch.equal(got[:, a:b], ref[:, a:b]), f"{name} differs in chunk {c}"
+            if a > 0:
+                assert_close(f"{name} chunk {c} left edge", to_host64(got[:, :a]), to_host64(ref[:, :a]), "bf16")
+            if b < n:
+                assert_close(f"{name} chunk {c} right edge", to_host64(got[:, b:]), to_host64(ref[:, b:]), "bf16")
+
+        if variant == "headwise":
+            w_next = None if c == 3 else w[:, (c + 1) * n:(c + 1) * n + W - 1].contiguous()
+            yc = o.dsc_fwd_headwise_chunk(xc, w[:, sl].contiguous(), x_prev)
+            dxc, dwc = o.dsc_bwd_headwise_chunk(xc, w[:, sl].contiguous(), dyc, x_prev, dy_next, w_next)
+            same("dw", dwc, dw[:, sl], lo, n)
+        else:
+            yc = o.dsc_fwd_static_chunk(xc, ws, x_prev, True)
+            dxc, dwsc = o.dsc_bwd_static_chunk(xc, ws, dyc, x_prev, dy_next, True)
+            dws_sum += dwsc
+        same("y", yc, y[:, sl], lo, n)
+        same("dx", dxc, dx[:, sl], 0, hi)
+    if variant == "static":
+        assert_close("full-size static dws, chunked", to_host64(dws_sum), to_host64(dws), "bf16", bound("dws", "bf16"))
+    ops().dsc_check()
+
+
 def test_chunk_without_halos_is_the_plain_call():
     o = ops()
     wl = Workload("first-last", HEADWISE, 2, 300, 256, 4, H=16, seed=7)
