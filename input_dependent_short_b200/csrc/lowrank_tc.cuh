@@ -1,6 +1,7 @@
 // Shared pieces of the tensor-core low-rank kernels (lowrank_tc_fwd.cu,
-// lowrank_tc_bwd.cu): the problem map, the kernel arguments, tensor-map
-// encoding and small device helpers.
+// lowrank_tc_bwd.cu, lowrank_tc_dec.cu): the problem map, the kernel
+// arguments, tensor-map encoding, small device helpers, and the filter-forming
+// pipeline that the training forward and the decode step share.
 //
 // "Dynamic Short Convolutions Improve Transformers", technical summary,
 // Methodology, "Parameterisation" 1 (rank-R factorisation of the filter
@@ -126,6 +127,129 @@ __device__ __forceinline__ float fma_bf16_hi(uint32_t a, uint32_t b, float c) {
         : "=f"(d)
         : "r"(a), "r"(b), "f"(c));
     return d;
+}
+
+// ------------------------------------------------ filter-forming pipeline ---
+// The protocol the training forward (lowrank_tc_fwd.cu) and the decode step
+// (lowrank_tc_dec.cu) share.  A producer thread fills NOP operand buffers (a
+// z tile and a U block each); one thread issues the zU MMAs of consecutive
+// items into two TMEM filter buffers; the sub-tiles the epilogue reads pass
+// through a ring of NS slots.  Each hand-off is a full/empty mbarrier pair:
+// OPF/OPE per operand buffer, WF/WE per filter buffer, XF/XE per slot.
+constexpr int TP_MAXOP = 4;  // most operand buffers
+constexpr int TP_MAXNS = 8;  // most ring slots
+
+struct PipeBars {
+    uint32_t base;
+    static constexpr uint32_t BYTES = (2 * TP_MAXOP + 4 + 2 * TP_MAXNS) * 8;
+    __device__ uint32_t opf(int b) const { return base + 8u * (uint32_t)b; }
+    __device__ uint32_t ope(int b) const { return base + 8u * TP_MAXOP + 8u * (uint32_t)b; }
+    __device__ uint32_t wf(int b) const { return base + 16u * TP_MAXOP + 8u * (uint32_t)b; }
+    __device__ uint32_t we(int b) const { return base + 16u * TP_MAXOP + 16u + 8u * (uint32_t)b; }
+    __device__ uint32_t xf(int s) const { return base + 16u * TP_MAXOP + 32u + 8u * (uint32_t)s; }
+    __device__ uint32_t xe(int s) const { return base + 16u * TP_MAXOP + 32u + 8u * TP_MAXNS + 8u * (uint32_t)s; }
+    // One thread, before the block synchronises: OPF, OPE, WF and XF take one
+    // arrival (a transaction count or an MMA commit); WE and XE take the
+    // counts of their consumers.
+    __device__ void init(int ns, uint32_t we_count, uint32_t xe_count) const {
+        for (int i = 0; i < TP_MAXOP; ++i) {
+            tc::mbar_init(opf(i), 1);
+            tc::mbar_init(ope(i), 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            tc::mbar_init(wf(i), 1);
+            tc::mbar_init(we(i), we_count);
+        }
+        for (int i = 0; i < ns; ++i) {
+            tc::mbar_init(xf(i), 1);
+            tc::mbar_init(xe(i), xe_count);
+        }
+        tc::fence_mbar_init();
+    }
+};
+
+// Zeroes the k-chunks R/8 .. RP/8-1 of every z buffer (the MMA reads them,
+// nothing loads them); a no-op when R = RP.  All threads of the block.
+__device__ __forceinline__ void zero_z_padding(unsigned char *smem, uint32_t opsize, int nop, const TcMap &m, int tid,
+                                               int nthreads) {
+    const int kz = m.R / 8;
+    const int zpad = (m.RP / 8 - kz) * 128;
+    for (int i = tid; i < nop * zpad; i += nthreads) {
+        const int b = i / zpad, r = i % zpad;
+        *reinterpret_cast<uint4 *>(smem + (uint32_t)b * opsize + (uint32_t)kz * 2048 + (uint32_t)r * 16) =
+            make_uint4(0, 0, 0, 0);
+    }
+}
+
+// One item's operands into the buffer at (zb, ub), completing on `bar`: the
+// z tile of rows t0 .. t0+127 of sequence `bseq` (one box of 2R-byte rows
+// with a 2R-byte swizzle for R = 16, 32 or 64, else R/8 boxes of 8 columns in
+// the no-swizzle core-matrix layout) and, when `newu`, the NF columns of U
+// block `blk` as boxes of 8 columns.  The producer thread.
+__device__ __forceinline__ void load_operands(const TcMap &m, const CUtensorMap *tmz, const CUtensorMap *tmu,
+                                              uint32_t zb, uint32_t ub, uint32_t ubytes, int t0, int bseq, int blk,
+                                              int NF, bool newu, uint32_t bar) {
+    const int kz = m.R / 8;
+    tc::mbar_expect_tx(bar, (uint32_t)kz * 2048u + (newu ? ubytes : 0u));
+    if (m.zsw) {
+        tc::tma_load_3d(zb, tmz, 0, t0, bseq, bar);
+    } else {
+        for (int j = 0; j < kz; ++j) tc::tma_load_3d(zb + (uint32_t)j * 2048u, tmz, 8 * j, t0, bseq, bar);
+    }
+    if (newu) {
+        const int col0 = blk * NF;
+        for (int j = 0; j < NF / 8; ++j) tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), tmu, col0 + 8 * j, 0, bar);
+    }
+}
+
+// The zU MMAs of nI consecutive items, issued by one thread: item li waits
+// for its operands (OPF) and for its TMEM buffer li & 1 to be read (WE, from
+// item li-2), forms all NF filter columns of 128 rows with RP/16 MMAs, and
+// commits to WF (filters ready) and OPE (operand buffer free).  `wait` is the
+// kernel's bounded wait.
+template <typename Wait>
+__device__ __forceinline__ void filter_mma_loop(const TcMap &m, const PipeBars &bars, uint32_t sbase, uint32_t opsize,
+                                                uint32_t zbytes, uint32_t tmem, int NF, int NFS, int nI, int NOP,
+                                                Wait &&wait) {
+    const uint32_t id_w = tc::idesc_bf16(TC_M, NF, 0, 1);
+    int ob = 0;
+    uint32_t oph = 0;
+    for (int li = 0; li < nI; ++li) {
+        const int b = li & 1;
+        wait(bars.opf(ob), oph);
+        if (li >= 2) wait(bars.we(b), (uint32_t)(((li - 2) >> 1) & 1));
+        tc::fence_after_sync();
+        const uint32_t zb = sbase + (uint32_t)ob * opsize, ub = zb + zbytes;
+        for (int ks = 0; ks < m.RP / 16; ++ks) {
+            const uint64_t ad = m.zsw ? tc::smem_desc_swz(zb + (uint32_t)ks * 32u, 16, 8u * (uint32_t)m.zsw, m.zsw)
+                                      : tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
+            const uint64_t bd = tc::smem_desc(ub + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
+            tc::mma_bf16(tmem + (uint32_t)(b * NFS), ad, bd, id_w, ks > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(bars.wf(b));
+        tc::mma_commit(bars.ope(ob));
+        if (++ob == NOP) {
+            ob = 0;
+            oph ^= 1u;
+        }
+    }
+}
+
+// Teardown, bounded (also after a time-out): the producer thread waits for
+// the last loads into each of the NS slots (nG sub-tiles in all), the MMA
+// thread for the MMAs that last read each of the NOP operand buffers (nI
+// items), before the shared memory and TMEM are given back.
+__device__ __forceinline__ void drain_loads(const PipeBars &bars, int NS, int nG) {
+    for (int s = 0; s < NS && s < nG; ++s) {
+        const int lastl = s + ((nG - 1 - s) / NS) * NS;
+        tc::mbar_wait(bars.xf(s), (uint32_t)((lastl / NS) & 1), TC_WAIT_LIMIT);
+    }
+}
+__device__ __forceinline__ void drain_mmas(const PipeBars &bars, int NOP, int nI) {
+    for (int b = 0; b < NOP && b < nI; ++b) {
+        const int lastli = b + ((nI - 1 - b) / NOP) * NOP;
+        tc::mbar_wait(bars.ope(b), (uint32_t)((lastli / NOP) & 1), TC_WAIT_LIMIT);
+    }
 }
 
 }  // namespace lrtc

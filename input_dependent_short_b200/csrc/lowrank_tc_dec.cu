@@ -14,7 +14,8 @@
 // the old one, then x) leaves by W-1 TMA stores straight from those slabs.
 // The ring slot is released once the stores have read it.
 //
-// This is the training forward's kernel structure (lowrank_tc_fwd.cu) with a
+// This is the training forward's kernel structure (the pipeline of
+// lowrank_tc.cuh that lowrank_tc_fwd.cu also runs) with a
 // tile of 128 sequences in place of 128 tokens of one sequence: z [B,R] and
 // U [R,G*W] arrive by TMA into the MMA's operand layouts (z as one swizzled box when
 // R is 16, 32 or 64, as in the forward); per sub-tile of
@@ -47,8 +48,8 @@ namespace {
 
 constexpr int TD_EPI = 512;
 constexpr int TD_THREADS = TD_EPI + 64;
-constexpr int TD_MAXNS = 8;
-constexpr int TD_MAXOP = 4;
+constexpr int TD_MAXNS = TP_MAXNS;
+constexpr int TD_MAXOP = TP_MAXOP;
 constexpr int TD_SMEM = 220 * 1024;
 
 // Decode plan: the channel blocks of the training forward (CF channels, NF =
@@ -72,20 +73,10 @@ struct DecSmem {
         opsize = up1024(zbytes + ubytes);
         ystage = (uint32_t)nop * opsize;
         ring = ystage + 2 * (uint32_t)nbx * ybox;
-        bars = ring + (uint32_t)ns * slot;
-        tmem = bars + (2 * TD_MAXOP + 4 + 2 * TD_MAXNS) * 8;
+        bars = ring + (uint32_t)ns * slot;  // PipeBars
+        tmem = bars + PipeBars::BYTES;
         total = tmem + 16 + 1024;
     }
-};
-
-struct DecBars {
-    uint32_t base;
-    __device__ uint32_t opf(int b) const { return base + 8u * (uint32_t)b; }
-    __device__ uint32_t ope(int b) const { return base + 8u * TD_MAXOP + 8u * (uint32_t)b; }
-    __device__ uint32_t wf(int b) const { return base + 16u * TD_MAXOP + 8u * (uint32_t)b; }
-    __device__ uint32_t we(int b) const { return base + 16u * TD_MAXOP + 16u + 8u * (uint32_t)b; }
-    __device__ uint32_t xf(int s) const { return base + 16u * TD_MAXOP + 32u + 8u * (uint32_t)s; }
-    __device__ uint32_t xe(int s) const { return base + 16u * TD_MAXOP + 32u + 8u * TD_MAXNS + 8u * (uint32_t)s; }
 };
 
 struct DecArgsTc {
@@ -197,31 +188,11 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
     const uint32_t sraw = tc::smem_u32(smem_raw);
     const uint32_t sbase = (sraw + 1023u) & ~1023u;
     unsigned char *smem = smem_raw + (sbase - sraw);
-    const DecBars bars{sbase + Sm.bars};
+    const PipeBars bars{sbase + Sm.bars};
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int kz = m.R / 8;
-
-    if (tid == 0) {
-        for (int i = 0; i < TD_MAXOP; ++i) {
-            tc::mbar_init(bars.opf(i), 1);
-            tc::mbar_init(bars.ope(i), 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(bars.wf(i), 1);
-            tc::mbar_init(bars.we(i), TD_EPI / 32);
-        }
-        for (int i = 0; i < NS; ++i) {
-            tc::mbar_init(bars.xf(i), 1);
-            tc::mbar_init(bars.xe(i), 1);  // thread 0, once the slot's state stores have read it
-        }
-        tc::fence_mbar_init();
-    }
-    const int zpad = (m.RP / 8 - kz) * 128;  // padded k-chunks of the z buffers stay zero
-    for (int i = tid; i < NOP * zpad; i += TD_THREADS) {
-        const int b = i / zpad, r = i % zpad;
-        *reinterpret_cast<uint4 *>(smem + (uint32_t)b * Sm.opsize + (uint32_t)kz * 2048 + (uint32_t)r * 16) =
-            make_uint4(0, 0, 0, 0);
-    }
+    // WE: one arrival per epilogue warp; XE: thread 0, once the slot's state stores have read it
+    if (tid == 0) bars.init(NS, TD_EPI / 32, 1);
+    zero_z_padding(smem, Sm.opsize, NOP, m, tid, TD_THREADS);
     tc::fence_proxy_async();
     if (warp == 17) tc::tmem_alloc(sbase + Sm.tmem, (uint32_t)(2 * d.NFS));
     tc::fence_before_sync();
@@ -256,19 +227,12 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
                 for (int i = 0; i < TD_MAXOP; ++i)
                     if (i == ob) held = ublk[i];
                 const bool newu = held != it.blk;
-                tc::mbar_expect_tx(bars.opf(ob), (uint32_t)kz * 2048u + (newu ? Sm.ubytes : 0u));
-                if (m.zsw) tc::tma_load_3d(zb, &tmz, 0, it.t0, 0, bars.opf(ob));  // one swizzled box
-                else
-                    for (int j = 0; j < kz; ++j)
-                        tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, 0, bars.opf(ob));
                 if (newu) {
 #pragma unroll
                     for (int i = 0; i < TD_MAXOP; ++i)
                         if (i == ob) ublk[i] = it.blk;
-                    const int col0 = it.blk * d.NF;
-                    for (int j = 0; j < d.NF / 8; ++j)
-                        tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), &tmu, col0 + 8 * j, 0, bars.opf(ob));
                 }
+                load_operands(m, &tmz, &tmu, zb, ub, Sm.ubytes, it.t0, 0, it.blk, d.NF, newu, bars.opf(ob));
                 if (++ob == NOP) {
                     ob = 0;
                     oph ^= 1u;
@@ -295,30 +259,7 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
         }
     } else if (warp == 17) {
         // ----------------------------------------------------------------- MMA
-        if (lane == 0) {
-            const uint32_t id_w = tc::idesc_bf16(TC_M, d.NF, 0, 1);
-            int ob = 0;
-            uint32_t oph = 0;
-            for (int li = 0; li < nI; ++li) {
-                const int b = li & 1;
-                wait(bars.opf(ob), oph);
-                if (li >= 2) wait(bars.we(b), (uint32_t)(((li - 2) >> 1) & 1));
-                tc::fence_after_sync();
-                const uint32_t zb = sbase + (uint32_t)ob * Sm.opsize, ub = zb + Sm.zbytes;
-                for (int ks = 0; ks < m.RP / 16; ++ks) {
-                    const uint64_t ad = m.zsw ? tc::smem_desc_swz(zb + (uint32_t)ks * 32u, 16, 8u * (uint32_t)m.zsw, m.zsw)
-                                              : tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
-                    const uint64_t bd = tc::smem_desc(ub + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
-                    tc::mma_bf16(tmem + (uint32_t)(b * d.NFS), ad, bd, id_w, ks > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(bars.wf(b));
-                tc::mma_commit(bars.ope(ob));
-                if (++ob == NOP) {
-                    ob = 0;
-                    oph ^= 1u;
-                }
-            }
-        }
+        if (lane == 0) filter_mma_loop(m, bars, sbase, Sm.opsize, Sm.zbytes, tmem, d.NF, d.NFS, nI, NOP, wait);
     } else {
         // ------------------------------------------------------------ epilogue
         const int t_loc = tid & (TC_M - 1), part = tid >> 7, quarter = warp & 3;
@@ -379,18 +320,8 @@ __global__ void __launch_bounds__(TD_THREADS, 1)
 
     // teardown (bounded): the loads and MMAs issued have landed before the
     // shared memory and TMEM are given back
-    if (warp == 16 && lane == 0) {
-        for (int s = 0; s < NS && s < nG; ++s) {
-            const int lastl = s + ((nG - 1 - s) / NS) * NS;
-            tc::mbar_wait(bars.xf(s), (uint32_t)((lastl / NS) & 1), TC_WAIT_LIMIT);
-        }
-    }
-    if (warp == 17 && lane == 0) {
-        for (int b = 0; b < NOP && b < nI; ++b) {
-            const int lastli = b + ((nI - 1 - b) / NOP) * NOP;
-            tc::mbar_wait(bars.ope(b), (uint32_t)((lastli / NOP) & 1), TC_WAIT_LIMIT);
-        }
-    }
+    if (warp == 16 && lane == 0) drain_loads(bars, NS, nG);
+    if (warp == 17 && lane == 0) drain_mmas(bars, NOP, nI);
     if (timed_out) atomicExch(&g_dsc_status_tcd, (int)DSC_ERR_TIMEOUT);
     tc::fence_before_sync();
     __syncthreads();

@@ -130,8 +130,8 @@ namespace {
 
 constexpr int TF_EPI = 512;               // epilogue threads
 constexpr int TF_THREADS = TF_EPI + 64;   // + producer warp + MMA warp
-constexpr int TF_MAXNS = 8;               // most x sub-tiles in flight
-constexpr int TF_MAXOP = 4;               // most operand (z, U) buffers
+constexpr int TF_MAXNS = TP_MAXNS;        // most x sub-tiles in flight
+constexpr int TF_MAXOP = TP_MAXOP;        // most operand (z, U) buffers
 constexpr int TF_SMEM = 220 * 1024;
 
 struct FwdSmem {
@@ -147,20 +147,10 @@ struct FwdSmem {
         opsize = up1024(zbytes + ubytes);
         ystage = (uint32_t)nop * opsize;          // two y staging tiles (TMA store sources)
         ring = ystage + 2 * (uint32_t)nbx * ybox;
-        bars = ring + (uint32_t)ns * slot;        // OPF[MAXOP] OPE[MAXOP] WF[2] WE[2] XF[MAXNS] XE[MAXNS]
-        tmem = bars + (2 * TF_MAXOP + 4 + 2 * TF_MAXNS) * 8;
+        bars = ring + (uint32_t)ns * slot;        // PipeBars
+        tmem = bars + PipeBars::BYTES;
         total = tmem + 16 + 1024;                 // + slack to align the base to 1024 bytes
     }
-};
-
-struct FwdBars {
-    uint32_t base;
-    __device__ uint32_t opf(int b) const { return base + 8u * (uint32_t)b; }
-    __device__ uint32_t ope(int b) const { return base + 8u * TF_MAXOP + 8u * (uint32_t)b; }
-    __device__ uint32_t wf(int b) const { return base + 16u * TF_MAXOP + 8u * (uint32_t)b; }
-    __device__ uint32_t we(int b) const { return base + 16u * TF_MAXOP + 16u + 8u * (uint32_t)b; }
-    __device__ uint32_t xf(int s) const { return base + 16u * TF_MAXOP + 32u + 8u * (uint32_t)s; }
-    __device__ uint32_t xe(int s) const { return base + 16u * TF_MAXOP + 32u + 8u * TF_MAXNS + 8u * (uint32_t)s; }
 };
 
 // Coordinates of consecutive items (block-major, tile-minor: a CTA keeps one
@@ -310,32 +300,10 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
     const uint32_t sraw = tc::smem_u32(smem_raw);
     const uint32_t sbase = (sraw + 1023u) & ~1023u;
     unsigned char *smem = smem_raw + (sbase - sraw);
-    const FwdBars bars{sbase + S.bars};
+    const PipeBars bars{sbase + S.bars};
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int kz = m.R / 8;  // z boxes loaded per item; k-chunks kz .. RP/8-1 stay zero
-
-    if (tid == 0) {
-        for (int i = 0; i < TF_MAXOP; ++i) {
-            tc::mbar_init(bars.opf(i), 1);
-            tc::mbar_init(bars.ope(i), 1);
-        }
-        for (int i = 0; i < 2; ++i) {
-            tc::mbar_init(bars.wf(i), 1);
-            tc::mbar_init(bars.we(i), TF_EPI / 32);
-        }
-        for (int i = 0; i < NS; ++i) {
-            tc::mbar_init(bars.xf(i), 1);
-            tc::mbar_init(bars.xe(i), TF_EPI / 32);
-        }
-        tc::fence_mbar_init();
-    }
-    // zero the padded k-chunks of every z buffer (read by the MMA, never loaded)
-    const int zpad = (m.RP / 8 - kz) * 128;
-    for (int i = tid; i < NOP * zpad; i += TF_THREADS) {
-        const int b = i / zpad, r = i % zpad;
-        *reinterpret_cast<uint4 *>(smem + (uint32_t)b * S.opsize + (uint32_t)kz * 2048 + (uint32_t)r * 16) =
-            make_uint4(0, 0, 0, 0);
-    }
+    if (tid == 0) bars.init(NS, TF_EPI / 32, TF_EPI / 32);  // WE, XE: one arrival per epilogue warp
+    zero_z_padding(smem, S.opsize, NOP, m, tid, TF_THREADS);
     tc::fence_proxy_async();
     if (warp == 17) tc::tmem_alloc(sbase + S.tmem, (uint32_t)(2 * m.NFS));
     tc::fence_before_sync();
@@ -372,21 +340,12 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
                 for (int i = 0; i < TF_MAXOP; ++i)
                     if (i == ob) held = ublk[i];
                 const bool newu = held != it.blk;
-                tc::mbar_expect_tx(bars.opf(ob), (uint32_t)kz * 2048u + (newu ? S.ubytes : 0u));
-                if (m.zsw) {
-                    tc::tma_load_3d(zb, &tmz, 0, it.t0, it.b, bars.opf(ob));
-                } else {
-                    for (int j = 0; j < kz; ++j)
-                        tc::tma_load_3d(zb + (uint32_t)j * 2048u, &tmz, 8 * j, it.t0, it.b, bars.opf(ob));
-                }
                 if (newu) {
 #pragma unroll
                     for (int i = 0; i < TF_MAXOP; ++i)
                         if (i == ob) ublk[i] = it.blk;
-                    const int col0 = it.blk * m.NF;
-                    for (int j = 0; j < m.NF / 8; ++j)
-                        tc::tma_load_2d(ub + (uint32_t)(j * m.RP * 16), &tmu, col0 + 8 * j, 0, bars.opf(ob));
                 }
+                load_operands(m, &tmz, &tmu, zb, ub, S.ubytes, it.t0, it.b, it.blk, m.NF, newu, bars.opf(ob));
                 if (++ob == NOP) {
                     ob = 0;
                     oph ^= 1u;
@@ -410,30 +369,7 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
         }
     } else if (warp == 17) {
         // ----------------------------------------------------------------- MMA
-        if (lane == 0) {
-            const uint32_t id_w = tc::idesc_bf16(TC_M, m.NF, 0, 1);
-            int ob = 0;
-            uint32_t oph = 0;
-            for (int li = 0; li < nI; ++li) {
-                const int b = li & 1;
-                wait(bars.opf(ob), oph);
-                if (li >= 2) wait(bars.we(b), (uint32_t)(((li - 2) >> 1) & 1));
-                tc::fence_after_sync();
-                const uint32_t zb = sbase + (uint32_t)ob * S.opsize, ub = zb + S.zbytes;
-                for (int ks = 0; ks < m.RP / 16; ++ks) {
-                    const uint64_t ad = m.zsw ? tc::smem_desc_swz(zb + (uint32_t)ks * 32u, 16, 8u * (uint32_t)m.zsw, m.zsw)
-                                              : tc::smem_desc(zb + (uint32_t)ks * 4096u, 2048, 128);
-                    const uint64_t bd = tc::smem_desc(ub + (uint32_t)ks * 256u, 128, (uint32_t)(m.RP * 16));
-                    tc::mma_bf16(tmem + (uint32_t)(b * m.NFS), ad, bd, id_w, ks > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(bars.wf(b));
-                tc::mma_commit(bars.ope(ob));
-                if (++ob == NOP) {
-                    ob = 0;
-                    oph ^= 1u;
-                }
-            }
-        }
+        if (lane == 0) filter_mma_loop(m, bars, sbase, S.opsize, S.zbytes, tmem, m.NF, m.NFS, nI, NOP, wait);
     } else {
         // ------------------------------------------------------------ epilogue
         const int t_loc = tid & (TC_M - 1), part = tid >> 7, quarter = warp & 3;
@@ -500,18 +436,8 @@ __global__ void __launch_bounds__(TF_THREADS, 1)
 
     // teardown: every load and MMA this CTA issued has landed before the
     // shared memory and TMEM are given back (bounded, also after a time-out)
-    if (warp == 16 && lane == 0) {
-        for (int s = 0; s < NS && s < nG; ++s) {
-            const int lastl = s + ((nG - 1 - s) / NS) * NS;
-            tc::mbar_wait(bars.xf(s), (uint32_t)((lastl / NS) & 1), TC_WAIT_LIMIT);
-        }
-    }
-    if (warp == 17 && lane == 0) {
-        for (int b = 0; b < NOP && b < nI; ++b) {
-            const int lastli = b + ((nI - 1 - b) / NOP) * NOP;
-            tc::mbar_wait(bars.ope(b), (uint32_t)((lastli / NOP) & 1), TC_WAIT_LIMIT);
-        }
-    }
+    if (warp == 16 && lane == 0) drain_loads(bars, NS, nG);
+    if (warp == 17 && lane == 0) drain_mmas(bars, NOP, nI);
     if (timed_out) atomicExch(&g_dsc_status_tcf, (int)DSC_ERR_TIMEOUT);
     tc::fence_before_sync();
     __syncthreads();
